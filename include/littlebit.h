@@ -1,0 +1,157 @@
+/*
+ * littlebit.h -- C ABI of the B200 (sm_100a) LittleBit linear-layer library.
+ *
+ * The layer (Samsung LittleBit article, aifrontier.co.jp, section 2, the
+ * "latent factorisation", "three scales" and "residual compensation" bullets)
+ * approximates a weight W (d_out x d_in) as
+ *     W  ~=  sum_p  diag(h_p) . U_p . diag(l_p) . V_p^T . diag(g_p)
+ * with U_p in {+-1}^(d_out x s), V_p in {+-1}^(d_in x s), fp16 row scale h
+ * (length d_out), column scale g (length d_in) and latent scale l (length s);
+ * p runs over one path, or two when residual compensation is on, and the
+ * outputs of the paths are added.  W is never formed: the forward is
+ *     y = sum_p  h_p (.) ( U_p ( l_p (.) ( V_p^T ( g_p (.) x ) ) ) ).
+ * Storage per layer is the effective bit width of the LittleBit-2 column
+ * (physicalainews.jp, chapter 1): [s(a+b+16) + 16(a+b)] / (ab) bits per
+ * weight, or [2s(a+b+16) + 32(a+b)] / (ab) with the residual path.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - Pointers named *_dev are CUDA device pointers on the current device;
+ *    everything else is host memory.  The caller owns every buffer it passes.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Device work is enqueued on it and the call returns without
+ *    waiting; the return value reports only what the host can check
+ *    (arguments, alignment, shapes, launch errors).
+ *  - The library keeps one workspace per (device, stream) -- a descriptor
+ *    table and the latent-vector scratch of the forward -- allocated on first
+ *    use with cudaMalloc, grown when needed and freed by littlebit_release().
+ *    Calls enqueued on the same stream are ordered; calls on different streams
+ *    use different workspaces.
+ *  - No entry point falls back to the CPU: without a usable CUDA device the
+ *    call returns LB_ERR_CUDA.
+ */
+#ifndef LITTLEBIT_H
+#define LITTLEBIT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LB_OK = 0,
+  LB_ERR_ARG = 1,         /* null pointer, bad enum, bad count */
+  LB_ERR_ALIGN = 2,       /* a pointer is not aligned as documented */
+  LB_ERR_SHAPE = 3,       /* a dimension is outside what the kernels accept */
+  LB_ERR_CUDA = 4,        /* a CUDA runtime call failed (see littlebit_last_cuda_error) */
+  LB_ERR_TIMEOUT = 5,     /* reserved: a bounded device wait ran out */
+  LB_ERR_UNSUPPORTED = 6  /* a valid request this build does not implement */
+} lb_status;
+
+typedef enum { LB_F16 = 0, LB_BF16 = 1, LB_F32 = 2, LB_I8 = 3 } lb_dtype;
+
+/* Which factor a packed buffer holds (see the layout below). */
+typedef enum { LB_ROLE_V = 0, LB_ROLE_U = 1 } lb_role;
+
+/*
+ * Packed factor layout ("sign-plane tiles")
+ * -----------------------------------------
+ * A factor is viewed as a +-1 matrix F with R rows and K columns, the rows
+ * being the outputs of the pass that reads it and K its contraction:
+ *   LB_ROLE_V:  F[j][i] = V[i][j],  R = s,      K = d_in
+ *   LB_ROLE_U:  F[o][j] = U[o][j],  R = d_out,  K = s
+ * F is cut into tiles of TR x TK = 4096 elements (512 bytes):
+ *   LB_ROLE_V: TR = 16,  TK = 256          LB_ROLE_U: TR = 128, TK = 32
+ * R and K are zero-padded to whole tiles (padding bits are 0).  Tile (rb, kt)
+ * starts at byte 512 * (rb * (Kpad / TK) + kt).  Within a tile, lane
+ * L = 0..31 owns bytes 16L..16L+15 as four little-endian uint32 words
+ * w_0..w_3.  With g = L / 4 and c = L % 4, bit n = 8m + q (m = 0..3,
+ * q = 0..7) of w_r is the sign of element (row, k):
+ *   LB_ROLE_V:  row = 16 rb + g + 8 (r % 2),         k = 256 kt + 32 q + 16 (r / 2) + 4 c + m
+ *   LB_ROLE_U:  row = 128 rb + 16 q + g + 8 (r % 2), k = 32 kt + 16 (r / 2) + 4 c + m
+ * and it is 1 exactly when F[row][k] < 0, i.e. sign(0) is +1.
+ * Why: each lane's 16 bytes are one 128-bit load, and masking a word with
+ * 0x01010101 << q leaves, byte by byte, the int8 A fragment of one
+ * m16n8k32 tensor-core product for rows/columns block q (values 0 or 2^q),
+ * so the decode kernels feed sign bits to the tensor cores with one logic op
+ * per four signs and no unpacking.
+ */
+
+/* Bytes of a packed factor with `rows` x `cols` logical elements (R x K above). */
+size_t littlebit_packed_bytes(lb_role role, int rows, int cols);
+
+/* Effective bits per weight (LittleBit-2 column, chapter 1); host-only math. */
+double littlebit_eff_bits(int d_in, int d_out, int s, int residual);
+
+/*
+ * Pack the signs of a real (or +-1) factor into the layout above.
+ *   src_dev : factor in its natural orientation, n_long x s elements of type
+ *             dt (LB_F16, LB_BF16, LB_F32 or LB_I8); element (a, j) is read at
+ *             src_dev[a * stride_long + j * stride_s] (strides in elements).
+ *             Role V: n_long = d_in (V is d_in x s); role U: n_long = d_out.
+ *   dst_dev : littlebit_packed_bytes(role, R, K) bytes, 16-byte aligned;
+ *             every byte is written (padding bits 0).
+ * A NaN has no sign to keep and is packed as +1 (bit 0).
+ * Errors: LB_ERR_ARG (null, bad dtype/role), LB_ERR_SHAPE (n_long or s < 1),
+ * LB_ERR_ALIGN (dst not 16-byte aligned), LB_ERR_CUDA.
+ */
+lb_status littlebit_pack_signs(const void* src_dev, lb_dtype dt, int n_long, int s,
+                               int64_t stride_long, int64_t stride_s, lb_role role,
+                               void* dst_dev, void* stream);
+
+/* One path of a layer: device pointers, all owned by the caller. */
+typedef struct lb_path {
+  const void* V_bits;    /* packed LB_ROLE_V factor, 16-byte aligned */
+  const void* U_bits;    /* packed LB_ROLE_U factor, 16-byte aligned */
+  const uint16_t* h;     /* fp16 [d_out] row (output) scale */
+  const uint16_t* g;     /* fp16 [d_in]  column (input) scale */
+  const uint16_t* l;     /* fp16 [s]     latent scale */
+} lb_path;
+
+typedef struct lb_layer {
+  int d_in;              /* multiple of 256, >= 256 */
+  int d_out;             /* multiple of 128, >= 128 */
+  int s;                 /* latent rank, 1 .. 1024 */
+  int residual;          /* 0: path[0] only; 1: path[0] + path[1], same s */
+  lb_path path[2];
+} lb_layer;
+
+/*
+ * y = forward(x) for one layer (formula at the top of this file).
+ *   x_dev : batch x d_in row-major activations, y_dev : batch x d_out.
+ *   Decode (1 <= batch <= 16): x and y are fp16 (xdt = LB_F16); two kernel
+ *   launches (latent pass, output pass) with fp32/int32 accumulation.
+ *   Prefill (batch >= 256, multiple of 128): xdt = LB_BF16, y bf16 --
+ *   tensor-core path, see littlebit_linear_forward_many.
+ *   x_dev and y_dev must be 16-byte aligned; every other pointer as in lb_path.
+ * Errors: LB_ERR_ARG, LB_ERR_ALIGN, LB_ERR_SHAPE, LB_ERR_UNSUPPORTED (batch
+ * 17..255 or an unsupported dtype), LB_ERR_CUDA.
+ */
+lb_status littlebit_linear_forward(const lb_layer* layer, const void* x_dev, void* y_dev,
+                                   int batch, lb_dtype xdt, void* stream);
+
+/*
+ * The same forward for n independent layers (each with its own input and
+ * output buffer, e.g. every linear layer of a model stack), done by the same
+ * two launches for the whole list, so that the weights of all layers stream
+ * from HBM back to back.  layers, xs, ys are host arrays of length n.
+ */
+lb_status littlebit_linear_forward_many(const lb_layer* layers, int n, const void* const* xs,
+                                        void* const* ys, int batch, lb_dtype xdt, void* stream);
+
+/* Free every workspace of every device (call with no work in flight). */
+void littlebit_release(void);
+
+/* Human-readable name of a status code (static string). */
+const char* littlebit_status_string(lb_status st);
+
+/* Text of the last CUDA error seen by this thread (static per thread). */
+const char* littlebit_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LITTLEBIT_H */

@@ -1,0 +1,250 @@
+// Host side of the C ABI declared in include/littlebit.h: argument checks,
+// per-(device, stream) workspaces, the device descriptor table and launches.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "lb_internal.h"
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+
+lb_status cuda_fail(cudaError_t e) {
+  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return LB_ERR_CUDA;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Workspace {
+  void* buf = nullptr;
+  size_t cap = 0;
+  std::vector<unsigned char> table;   // last descriptor table uploaded
+};
+
+std::mutex g_mu;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+int g_num_sms[64] = {0};
+
+int num_sms(int dev) {
+  if (dev < 0 || dev >= 64) return 148;
+  if (g_num_sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    g_num_sms[dev] = n;
+  }
+  return g_num_sms[dev];
+}
+
+lb_status check_layer(const lb_layer& L) {
+  if (L.d_in < 256 || L.d_in % 256 != 0) return LB_ERR_SHAPE;
+  if (L.d_out < 128 || L.d_out % 128 != 0) return LB_ERR_SHAPE;
+  if (L.s < 1 || L.s > lb::kMaxRank) return LB_ERR_SHAPE;
+  if (L.residual != 0 && L.residual != 1) return LB_ERR_ARG;
+  for (int p = 0; p <= L.residual; ++p) {
+    const lb_path& P = L.path[p];
+    if (!P.V_bits || !P.U_bits || !P.h || !P.g || !P.l) return LB_ERR_ARG;
+    if (!aligned(P.V_bits, 16) || !aligned(P.U_bits, 16)) return LB_ERR_ALIGN;
+    if (!aligned(P.h, 2) || !aligned(P.g, 2) || !aligned(P.l, 2)) return LB_ERR_ALIGN;
+  }
+  return LB_OK;
+}
+
+// Bytes of per-path scratch for one layer at this batch.
+size_t path_scratch_bytes(const lb_layer& L, int batch) {
+  const int n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
+  size_t b = 0;
+  b += align_up((size_t)n_slices * batch * lb::s16(L.s) * sizeof(float), 256);   // partial
+  b += align_up((size_t)batch * 2 * lb::s32(L.s), 256);                           // planes
+  b += align_up((size_t)batch * sizeof(float), 256);                              // tscale
+  b += align_up((size_t)batch * sizeof(int32_t), 256);                            // tsum
+  return b;
+}
+
+lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
+                         cudaStream_t st) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+
+  // ---- sizes: [table][counters][per-path scratch...]
+  const size_t table_bytes = align_up((size_t)n * sizeof(lb::LayerDesc), 256);
+  const size_t counter_bytes = align_up((size_t)n * 2 * sizeof(unsigned int), 256);
+  size_t total = table_bytes + counter_bytes;
+  int max_s16 = 16;
+  for (int i = 0; i < n; ++i) {
+    total += (size_t)(layers[i].residual + 1) * path_scratch_bytes(layers[i], batch);
+    max_s16 = std::max(max_s16, lb::s16(layers[i].s));
+  }
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  Workspace& ws = g_ws[{dev, st}];
+  if (ws.cap < total) {
+    if (ws.buf) {
+      e = cudaStreamSynchronize(st);
+      if (e != cudaSuccess) return cuda_fail(e);
+      cudaFree(ws.buf);
+      ws.buf = nullptr;
+      ws.cap = 0;
+    }
+    const size_t cap = align_up(total + total / 4, 1 << 20);
+    e = cudaMalloc(&ws.buf, cap);
+    if (e != cudaSuccess) return cuda_fail(e);
+    ws.cap = cap;
+    ws.table.clear();
+    e = cudaMemsetAsync(ws.buf, 0, cap, st);   // counters start at zero
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+
+  // ---- descriptor table
+  unsigned char* base = static_cast<unsigned char*>(ws.buf);
+  unsigned int* counters = reinterpret_cast<unsigned int*>(base + table_bytes);
+  size_t off = table_bytes + counter_bytes;
+  std::vector<lb::LayerDesc> tab(n);
+  int v_items = 0, u_items = 0;
+  for (int i = 0; i < n; ++i) {
+    const lb_layer& L = layers[i];
+    lb::LayerDesc& D = tab[i];
+    std::memset(&D, 0, sizeof(D));
+    D.x = static_cast<const uint16_t*>(xs[i]);
+    D.y = static_cast<uint16_t*>(ys[i]);
+    D.d_in = L.d_in;
+    D.d_out = L.d_out;
+    D.s = L.s;
+    D.npaths = L.residual + 1;
+    D.n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
+    D.v_begin = v_items;
+    D.u_begin = u_items;
+    v_items += D.npaths * D.n_slices;
+    u_items += L.d_out / lb::kUTileRows;
+    for (int p = 0; p < D.npaths; ++p) {
+      lb::PathDesc& P = D.p[p];
+      P.V = static_cast<const uint4*>(L.path[p].V_bits);
+      P.U = static_cast<const uint4*>(L.path[p].U_bits);
+      P.h = L.path[p].h;
+      P.g = L.path[p].g;
+      P.l = L.path[p].l;
+      P.ws.partial = reinterpret_cast<float*>(base + off);
+      off += align_up((size_t)D.n_slices * batch * lb::s16(L.s) * sizeof(float), 256);
+      P.ws.planes = reinterpret_cast<int8_t*>(base + off);
+      off += align_up((size_t)batch * 2 * lb::s32(L.s), 256);
+      P.ws.tscale = reinterpret_cast<float*>(base + off);
+      off += align_up((size_t)batch * sizeof(float), 256);
+      P.ws.tsum = reinterpret_cast<int32_t*>(base + off);
+      off += align_up((size_t)batch * sizeof(int32_t), 256);
+      P.ws.counter = counters + 2 * i + p;
+    }
+  }
+  const size_t tb = (size_t)n * sizeof(lb::LayerDesc);
+  if (ws.table.size() != tb || std::memcmp(ws.table.data(), tab.data(), tb) != 0) {
+    // pageable source: the call returns once the bytes are staged, so `tab`
+    // may go out of scope; stream order protects kernels still reading the table
+    e = cudaMemcpyAsync(ws.buf, tab.data(), tb, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    // the counters' offset depends on the table size, so bytes that earlier
+    // calls used as scratch may now hold counters: start them at zero
+    e = cudaMemsetAsync(counters, 0, counter_bytes, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    ws.table.assign(reinterpret_cast<unsigned char*>(tab.data()),
+                    reinterpret_cast<unsigned char*>(tab.data()) + tb);
+  }
+
+  lb::DecodeArgs a;
+  a.layers = static_cast<const lb::LayerDesc*>(ws.buf);
+  a.n_layers = n;
+  a.batch = batch;
+  a.v_items = v_items;
+  a.u_items = u_items;
+  const int sms = num_sms(dev);
+  e = lb::launch_latent_pass(a, max_s16, sms, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = lb::launch_output_pass(a, sms, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return LB_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t littlebit_packed_bytes(lb_role role, int rows, int cols) {
+  if (rows < 1 || cols < 1) return 0;
+  const int tr = (role == LB_ROLE_V) ? lb::kVTileRows : lb::kUTileRows;
+  const int tk = (role == LB_ROLE_V) ? lb::kVTileK : lb::kUTileK;
+  return (size_t)lb::ceil_div(rows, tr) * lb::ceil_div(cols, tk) * lb::kTileBytes;
+}
+
+double littlebit_eff_bits(int d_in, int d_out, int s, int residual) {
+  const double a = d_in, b = d_out;
+  const double num = residual ? 2.0 * s * (a + b + 16) + 32.0 * (a + b) : (double)s * (a + b + 16) + 16.0 * (a + b);
+  return num / (a * b);
+}
+
+lb_status littlebit_pack_signs(const void* src_dev, lb_dtype dt, int n_long, int s, int64_t stride_long,
+                               int64_t stride_s, lb_role role, void* dst_dev, void* stream) {
+  if (!src_dev || !dst_dev) return LB_ERR_ARG;
+  if (dt != LB_F16 && dt != LB_BF16 && dt != LB_F32 && dt != LB_I8) return LB_ERR_ARG;
+  if (role != LB_ROLE_V && role != LB_ROLE_U) return LB_ERR_ARG;
+  if (n_long < 1 || s < 1) return LB_ERR_SHAPE;
+  if (!aligned(dst_dev, 16)) return LB_ERR_ALIGN;
+  cudaError_t e = lb::launch_pack(src_dev, dt, n_long, s, stride_long, stride_s, role, dst_dev,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LB_OK : cuda_fail(e);
+}
+
+lb_status littlebit_linear_forward_many(const lb_layer* layers, int n, const void* const* xs, void* const* ys,
+                                        int batch, lb_dtype xdt, void* stream) {
+  if (!layers || !xs || !ys || n < 1) return LB_ERR_ARG;
+  if (batch < 1) return LB_ERR_SHAPE;
+  for (int i = 0; i < n; ++i) {
+    const lb_status st = check_layer(layers[i]);
+    if (st != LB_OK) return st;
+    if (!xs[i] || !ys[i]) return LB_ERR_ARG;
+    if (!aligned(xs[i], 16) || !aligned(ys[i], 16)) return LB_ERR_ALIGN;
+  }
+  if (batch <= lb::kMaxBatchDecode) {
+    if (xdt != LB_F16) return LB_ERR_UNSUPPORTED;
+    return decode_forward(layers, n, xs, ys, batch, static_cast<cudaStream_t>(stream));
+  }
+  return LB_ERR_UNSUPPORTED;
+}
+
+lb_status littlebit_linear_forward(const lb_layer* layer, const void* x_dev, void* y_dev, int batch,
+                                   lb_dtype xdt, void* stream) {
+  return littlebit_linear_forward_many(layer, 1, &x_dev, &y_dev, batch, xdt, stream);
+}
+
+void littlebit_release(void) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (auto& kv : g_ws) {
+    if (kv.second.buf) cudaFree(kv.second.buf);
+  }
+  g_ws.clear();
+}
+
+const char* littlebit_status_string(lb_status st) {
+  switch (st) {
+    case LB_OK: return "LB_OK";
+    case LB_ERR_ARG: return "LB_ERR_ARG: invalid argument";
+    case LB_ERR_ALIGN: return "LB_ERR_ALIGN: pointer misaligned";
+    case LB_ERR_SHAPE: return "LB_ERR_SHAPE: unsupported shape";
+    case LB_ERR_CUDA: return "LB_ERR_CUDA: CUDA runtime error";
+    case LB_ERR_TIMEOUT: return "LB_ERR_TIMEOUT: device wait timed out";
+    case LB_ERR_UNSUPPORTED: return "LB_ERR_UNSUPPORTED: not implemented for these arguments";
+  }
+  return "unknown lb_status";
+}
+
+const char* littlebit_last_cuda_error(void) { return g_last_cuda_error; }
+
+}  // extern "C"

@@ -1,0 +1,190 @@
+"""Thin ctypes binding of liblittlebit.so (include/littlebit.h).
+
+Argument marshalling only: every step of the layer runs in the CUDA library.
+Tensors are torch CUDA tensors (torch supplies device memory and streams).
+If the library has not been built, importing this module raises ImportError;
+there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, field
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblittlebit.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -c 'import __graft_entry__ as g; g.build()'` "
+        "(the LittleBit layer has no CPU implementation)"
+    )
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+LB_F16, LB_BF16, LB_F32, LB_I8 = 0, 1, 2, 3
+LB_ROLE_V, LB_ROLE_U = 0, 1
+ROLE = {"V": LB_ROLE_V, "U": LB_ROLE_U}
+STATUS = {0: "LB_OK", 1: "LB_ERR_ARG", 2: "LB_ERR_ALIGN", 3: "LB_ERR_SHAPE", 4: "LB_ERR_CUDA",
+          5: "LB_ERR_TIMEOUT", 6: "LB_ERR_UNSUPPORTED"}
+_DTYPE = {torch.float16: LB_F16, torch.bfloat16: LB_BF16, torch.float32: LB_F32, torch.int8: LB_I8}
+
+
+class LbPath(ctypes.Structure):
+    _fields_ = [("V_bits", ctypes.c_void_p), ("U_bits", ctypes.c_void_p), ("h", ctypes.c_void_p),
+                ("g", ctypes.c_void_p), ("l", ctypes.c_void_p)]
+
+
+class LbLayer(ctypes.Structure):
+    _fields_ = [("d_in", ctypes.c_int), ("d_out", ctypes.c_int), ("s", ctypes.c_int),
+                ("residual", ctypes.c_int), ("path", LbPath * 2)]
+
+
+_lib.littlebit_packed_bytes.restype = ctypes.c_size_t
+_lib.littlebit_packed_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+_lib.littlebit_eff_bits.restype = ctypes.c_double
+_lib.littlebit_eff_bits.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+_lib.littlebit_pack_signs.restype = ctypes.c_int
+_lib.littlebit_pack_signs.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p,
+                                      ctypes.c_void_p]
+_lib.littlebit_linear_forward.restype = ctypes.c_int
+_lib.littlebit_linear_forward.argtypes = [ctypes.POINTER(LbLayer), ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+_lib.littlebit_linear_forward_many.restype = ctypes.c_int
+_lib.littlebit_linear_forward_many.argtypes = [ctypes.POINTER(LbLayer), ctypes.c_int,
+                                               ctypes.POINTER(ctypes.c_void_p),
+                                               ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_void_p]
+_lib.littlebit_release.restype = None
+_lib.littlebit_release.argtypes = []
+_lib.littlebit_status_string.restype = ctypes.c_char_p
+_lib.littlebit_status_string.argtypes = [ctypes.c_int]
+_lib.littlebit_last_cuda_error.restype = ctypes.c_char_p
+_lib.littlebit_last_cuda_error.argtypes = []
+
+
+class LittleBitError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        msg = _lib.littlebit_status_string(code).decode()
+        if code == 4:
+            msg += f" ({_lib.littlebit_last_cuda_error().decode()})"
+        super().__init__(f"{where}: {msg}")
+        self.code = code
+        self.status = STATUS.get(code, str(code))
+
+
+def _check(code: int, where: str) -> None:
+    if code != 0:
+        raise LittleBitError(code, where)
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def library():
+    """The loaded ctypes CDLL (for tests that call the C ABI directly)."""
+    return _lib
+
+
+def packed_bytes(role: str, rows: int, cols: int) -> int:
+    return int(_lib.littlebit_packed_bytes(ROLE[role], rows, cols))
+
+
+def eff_bits(d_in: int, d_out: int, s: int, residual: bool) -> float:
+    return float(_lib.littlebit_eff_bits(d_in, d_out, s, int(bool(residual))))
+
+
+def pack_signs(factor: torch.Tensor, role: str, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Pack the signs of a CUDA factor tensor (V: d_in x s, U: d_out x s)."""
+    if factor.dim() != 2 or not factor.is_cuda:
+        raise ValueError("factor must be a 2-D CUDA tensor")
+    n_long, s = factor.shape
+    rows, cols = (s, n_long) if role == "V" else (n_long, s)
+    nbytes = packed_bytes(role, rows, cols)
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=factor.device)
+    if out.numel() < nbytes:
+        raise ValueError("output buffer too small")
+    _check(_lib.littlebit_pack_signs(ctypes.c_void_p(factor.data_ptr()), _DTYPE[factor.dtype], n_long, s,
+                                     factor.stride(0), factor.stride(1), ROLE[role],
+                                     ctypes.c_void_p(out.data_ptr()), _stream(stream)),
+           "littlebit_pack_signs")
+    return out
+
+
+@dataclass
+class Path:
+    """One path of a layer, all CUDA tensors: packed V/U bytes, fp16 h, g, l."""
+    V_bits: torch.Tensor
+    U_bits: torch.Tensor
+    h: torch.Tensor
+    g: torch.Tensor
+    l: torch.Tensor
+
+
+@dataclass
+class Layer:
+    d_in: int
+    d_out: int
+    s: int
+    paths: list = field(default_factory=list)
+
+    @property
+    def residual(self) -> bool:
+        return len(self.paths) == 2
+
+    def c_struct(self) -> LbLayer:
+        L = LbLayer()
+        L.d_in, L.d_out, L.s, L.residual = self.d_in, self.d_out, self.s, int(self.residual)
+        for i, p in enumerate(self.paths):
+            L.path[i] = LbPath(p.V_bits.data_ptr(), p.U_bits.data_ptr(), p.h.data_ptr(), p.g.data_ptr(),
+                               p.l.data_ptr())
+        return L
+
+
+def forward(layer: Layer, x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = layer(x); x is (batch, d_in) fp16 (decode) on the layer's device."""
+    batch = x.shape[0]
+    if y is None:
+        y = torch.empty((batch, layer.d_out), dtype=x.dtype, device=x.device)
+    L = layer.c_struct()
+    _check(_lib.littlebit_linear_forward(ctypes.byref(L), ctypes.c_void_p(x.data_ptr()),
+                                         ctypes.c_void_p(y.data_ptr()), batch, _DTYPE[x.dtype], _stream(stream)),
+           "littlebit_linear_forward")
+    return y
+
+
+class Stack:
+    """A list of independent layers run by one forward_many call per step.
+
+    Holds the marshalled C structs and pointer arrays so that repeated calls
+    do no Python-side allocation."""
+
+    def __init__(self, layers: list, xs: list, ys: list):
+        assert len(layers) == len(xs) == len(ys) and layers
+        self.layers, self.xs, self.ys = layers, xs, ys
+        self.batch = xs[0].shape[0]
+        self.dtype = _DTYPE[xs[0].dtype]
+        n = len(layers)
+        self._n = n
+        self._arr = (LbLayer * n)(*[L.c_struct() for L in layers])
+        self._xp = (ctypes.c_void_p * n)(*[x.data_ptr() for x in xs])
+        self._yp = (ctypes.c_void_p * n)(*[y.data_ptr() for y in ys])
+
+    def __call__(self, stream=None) -> None:
+        _check(_lib.littlebit_linear_forward_many(self._arr, self._n, self._xp, self._yp, self.batch, self.dtype,
+                                                  _stream(stream)),
+               "littlebit_linear_forward_many")
+
+
+def forward_many(layers: list, xs: list, ys: list, stream=None) -> None:
+    Stack(layers, xs, ys)(stream)
+
+
+def release() -> None:
+    _lib.littlebit_release()

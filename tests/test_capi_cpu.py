@@ -1,0 +1,93 @@
+"""CPU-side checks of the C-ABI library: it loads, exports every entry point
+the header declares, and its host-only functions agree with the oracle."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from oracle import littlebit_oracle as orc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+LIB = os.path.join(ROOT, "latent_binary_factorization_b200", "liblittlebit.so")
+
+
+def _header_functions():
+    funcs = set()
+    for name in os.listdir(os.path.join(ROOT, "include")):
+        if name.endswith(".h"):
+            with open(os.path.join(ROOT, "include", name)) as f:
+                text = f.read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            funcs |= set(re.findall(r"\b(littlebit_\w+)\s*\(", text))
+    return sorted(funcs)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        from latent_binary_factorization_b200 import build_ext
+        build_ext.build()
+    return ctypes.CDLL(LIB)
+
+
+def test_header_declares_entry_points():
+    funcs = _header_functions()
+    for f in ("littlebit_pack_signs", "littlebit_linear_forward", "littlebit_linear_forward_many",
+              "littlebit_packed_bytes", "littlebit_eff_bits"):
+        assert f in funcs
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for f in _header_functions():
+        assert hasattr(lib, f), f"{f} declared in include/ but not exported"
+
+
+def test_host_functions_match_oracle(lib):
+    lib.littlebit_eff_bits.restype = ctypes.c_double
+    lib.littlebit_eff_bits.argtypes = [ctypes.c_int] * 4
+    lib.littlebit_packed_bytes.restype = ctypes.c_size_t
+    lib.littlebit_packed_bytes.argtypes = [ctypes.c_int] * 3
+    for a, b, s, r in [(4096, 4096, 86, 1), (8192, 28672, 620, 0), (512, 512, 32, 0), (4096, 11008, 133, 1)]:
+        assert lib.littlebit_eff_bits(a, b, s, r) == pytest.approx(orc.eff_bits(a, b, s, bool(r)), rel=1e-15)
+    for role, code in (("V", 0), ("U", 1)):
+        for R, K in [(86, 4096), (1, 256), (620, 28672), (4096, 86), (128, 1), (11008, 133)]:
+            assert lib.littlebit_packed_bytes(code, R, K) == orc.packed_nbytes(role, R, K)
+
+
+def test_status_strings(lib):
+    lib.littlebit_status_string.restype = ctypes.c_char_p
+    lib.littlebit_status_string.argtypes = [ctypes.c_int]
+    for code in range(7):
+        assert lib.littlebit_status_string(code).startswith(b"LB_")
+
+
+def test_forward_rejects_bad_arguments_without_device_work(lib):
+    """Argument checks happen on the host before any CUDA call."""
+    from latent_binary_factorization_b200 import littlebit as lb
+    L = lb.LbLayer()
+    L.d_in, L.d_out, L.s, L.residual = 100, 128, 4, 0       # d_in not a multiple of 256
+    f = lb.library().littlebit_linear_forward
+    x = ctypes.c_void_p(16)
+    assert f(ctypes.byref(L), x, x, 1, 0, None) == 3           # LB_ERR_SHAPE
+    L.d_in, L.s = 256, 0
+    assert f(ctypes.byref(L), x, x, 1, 0, None) == 3           # s < 1
+    L.s = 4
+    assert f(ctypes.byref(L), x, x, 1, 0, None) == 1           # null factor pointers
+    for p in range(2):
+        L.path[p] = lb.LbPath(16, 32, 2, 4, 6)
+    L.residual = 2
+    assert f(ctypes.byref(L), x, x, 1, 0, None) == 1           # residual must be 0/1
+    L.residual = 0
+    L.path[0] = lb.LbPath(8, 32, 2, 4, 6)                       # V not 16-byte aligned
+    assert f(ctypes.byref(L), x, x, 1, 0, None) == 2
+    L.path[0] = lb.LbPath(16, 32, 2, 4, 6)
+    assert f(ctypes.byref(L), ctypes.c_void_p(24), x, 1, 0, None) == 2   # x misaligned
+    assert f(ctypes.byref(L), x, x, 0, 0, None) == 3           # batch 0
+    assert f(ctypes.byref(L), x, x, 100, 0, None) == 6         # batch 17..255 unsupported
+    assert f(ctypes.byref(L), x, x, 1, 1, None) == 6           # decode wants fp16
+    pack = lb.library().littlebit_pack_signs
+    assert pack(None, 0, 4, 4, 4, 1, 0, ctypes.c_void_p(16), None) == 1
+    assert pack(ctypes.c_void_p(16), 9, 4, 4, 4, 1, 0, ctypes.c_void_p(16), None) == 1
+    assert pack(ctypes.c_void_p(16), 0, 0, 4, 4, 1, 0, ctypes.c_void_p(16), None) == 3
+    assert pack(ctypes.c_void_p(16), 0, 4, 4, 4, 1, 0, ctypes.c_void_p(8), None) == 2

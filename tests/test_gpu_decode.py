@@ -1,0 +1,191 @@
+"""GPU parity: sign packing (bit-exact) and the decode forward (batch 1..16)
+against the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import littlebit_oracle as orc
+from latent_binary_factorization_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 2e-3      # relative L2 error over the whole output tensor
+MAX_ABS = 1e-2     # max |err| / max |y_ref|
+
+
+@pytest.fixture(scope="module")
+def lbm():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from latent_binary_factorization_b200 import layers, littlebit
+    return littlebit, layers
+
+
+def _check(y_gpu, y_ref, tag=""):
+    y = y_gpu.float().cpu().numpy()
+    e, m = orc.rel_l2(y, y_ref), orc.max_abs_ratio(y, y_ref)
+    assert e <= REL_L2 and m <= MAX_ABS, f"{tag} rel_l2={e:.3e} max_abs_ratio={m:.3e}"
+    return e, m
+
+
+# ----------------------------------------------------------------- packing
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float16, torch.bfloat16, torch.int8])
+@pytest.mark.parametrize("role,n_long,s", [("V", 256, 1), ("V", 512, 33), ("V", 4096, 86), ("V", 768, 16),
+                                           ("U", 128, 1), ("U", 384, 45), ("U", 4096, 188), ("U", 256, 32)])
+def test_pack_bit_exact(lbm, dtype, role, n_long, s):
+    lb, _ = lbm
+    F = synth.real_factor(n_long, s, seed=7, zeros=0.05)      # natural orientation (n_long x s)
+    if dtype == torch.int8:
+        F = np.where(F < 0, -1, 1).astype(np.int8)
+    t = torch.from_numpy(F).to(dtype=dtype, device="cuda") if dtype != torch.int8 else torch.from_numpy(F).cuda()
+    host = t.float().cpu().numpy()        # the values the kernel sees (after dtype rounding)
+    got = lb.pack_signs(t, role).cpu().numpy()
+    want = orc.pack_signs(orc.factor_matrix(role, host), role)
+    assert np.array_equal(got, want)
+
+
+def test_pack_strided_and_signed_zero(lbm):
+    lb, _ = lbm
+    base = torch.randn(300, 512, device="cuda")
+    base[::7, ::3] = 0.0
+    base[1::7, ::5] = -0.0
+    base[2, 2] = float("nan")
+    view = base.t()[:, :300]              # (512 x 300) with strides (1, 512)
+    got = lb.pack_signs(view, "U").cpu().numpy()
+    want = orc.pack_signs(view.cpu().numpy(), "U")
+    assert np.array_equal(got, want)
+
+
+def test_pack_full_size_70b_factor(lbm):
+    """Largest factor of the 70B MLP workload (28672 x 620), role V and U."""
+    lb, _ = lbm
+    gen = torch.Generator(device="cuda").manual_seed(3)
+    S = (1 - 2 * torch.randint(0, 2, (28672, 620), generator=gen, device="cuda", dtype=torch.int8)).to(torch.int8)
+    Sh = S.cpu().numpy()
+    for role in ("V", "U"):
+        got = lb.pack_signs(S, role).cpu().numpy()
+        assert np.array_equal(got, orc.pack_signs(orc.factor_matrix(role, Sh), role)), role
+
+
+# ----------------------------------------------------------------- forward
+
+def _run(lbm, d_in, d_out, s, residual, batch, seed=0):
+    lb, layers = lbm
+    paths = synth.layer(d_in, d_out, s, residual, seed=seed)
+    x = synth.activations(batch, d_in, seed=seed)
+    layer = layers.upload(paths, d_in, d_out, s)
+    y = lb.forward(layer, torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    return y, x, paths
+
+
+def test_tiny_config_against_dense_reconstruction(lbm):
+    """512 -> 512, s = 32, single path, batch 1: also equals dense W x."""
+    y, x, paths = _run(lbm, 512, 512, 32, False, 1, seed=1)
+    _check(y, orc.factored_forward(x, paths), "factored")
+    _check(y, orc.dense_forward(x, paths), "dense")
+
+
+@pytest.mark.parametrize("batch", [1, 2, 3, 4, 5, 8, 13, 16])
+@pytest.mark.parametrize("residual,s", [(False, 188), (True, 86)])
+def test_7b_attention_projection(lbm, batch, residual, s):
+    y, x, paths = _run(lbm, 4096, 4096, s, residual, batch, seed=batch)
+    _check(y, orc.factored_forward(x, paths), f"B={batch}")
+
+
+@pytest.mark.parametrize("d_in,d_out,s,residual,batch", [
+    (256, 128, 1, False, 1),            # smallest shapes, rank 1
+    (256, 128, 1, True, 3),
+    (768, 384, 33, True, 2),            # s just over one 32-block
+    (4096 + 256, 640, 100, False, 1),   # ragged last input slice
+    (8192 + 512, 256, 17, True, 4),     # three slices, last one ragged
+    (4096, 11008, 133, True, 1),        # 7B MLP gate/up at 0.1 BPW
+    (11008, 4096, 135, True, 2),        # 7B MLP down, the quoted rank
+    (1024, 1024, 1024, False, 1),       # maximum rank
+    (512, 256, 511, True, 16),          # ragged rank, full batch
+])
+def test_shapes_and_ragged_edges(lbm, d_in, d_out, s, residual, batch):
+    y, x, paths = _run(lbm, d_in, d_out, s, residual, batch, seed=s)
+    _check(y, orc.factored_forward(x, paths), f"{d_in}x{d_out} s={s}")
+
+
+def test_all_plus_signs_and_zero_input(lbm):
+    lb, layers = lbm
+    d_in, d_out, s = 512, 256, 40
+    paths = synth.layer(d_in, d_out, s, False, seed=5)
+    paths[0]["U"][:] = 1
+    paths[0]["V"][:] = 1
+    layer = layers.upload(paths, d_in, d_out, s)
+    x = synth.activations(2, d_in, seed=5)
+    x[1] = 0
+    y = lb.forward(layer, torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    y_ref = orc.factored_forward(x, paths)
+    _check(y[:1], y_ref[:1], "all +1")
+    assert torch.count_nonzero(y[1]).item() == 0
+
+
+def test_basis_vector_input_gives_weight_column(lbm):
+    lb, layers = lbm
+    d_in, d_out, s = 1024, 512, 64
+    paths = synth.layer(d_in, d_out, s, True, seed=6)
+    layer = layers.upload(paths, d_in, d_out, s)
+    W = sum(orc.dense_weight(p) for p in paths)
+    x = np.zeros((3, d_in), np.float16)
+    cols = [0, 517, 1023]
+    for r, i in enumerate(cols):
+        x[r, i] = 1.0
+    y = lb.forward(layer, torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    _check(y, W[:, cols].T, "basis")
+
+
+def test_forward_many_mixed_stack(lbm):
+    """One forward_many call over layers of different shapes, ranks and path counts."""
+    lb, layers = lbm
+    specs = [(4096, 4096, 86, True), (4096, 11008, 133, True), (11008, 4096, 133, True),
+             (512, 512, 32, False), (8192, 1024, 620, False)]
+    B = 2
+    L, X, Y, refs = [], [], [], []
+    for i, (a, b, s, r) in enumerate(specs):
+        paths = synth.layer(a, b, s, r, seed=100 + i, index=i)
+        x = synth.activations(B, a, seed=100 + i, index=i)
+        L.append(layers.upload(paths, a, b, s))
+        X.append(torch.from_numpy(x).cuda())
+        Y.append(torch.empty(B, b, dtype=torch.float16, device="cuda"))
+        refs.append(orc.factored_forward(x, paths))
+    stack = lb.Stack(L, X, Y)
+    for _ in range(3):            # repeated calls reuse the workspace and counters
+        for y in Y:
+            y.fill_(float("nan"))
+        stack()
+        torch.cuda.synchronize()
+        for i, (y, ref) in enumerate(zip(Y, refs)):
+            _check(y, ref, f"layer {i}")
+
+
+def test_repeatable_and_deterministic(lbm):
+    lb, layers = lbm
+    paths = synth.layer(4096, 4096, 86, True, seed=9)
+    layer = layers.upload(paths, 4096, 4096, 86)
+    x = torch.from_numpy(synth.activations(1, 4096, seed=9)).cuda()
+    y1 = lb.forward(layer, x).clone()
+    y2 = lb.forward(layer, x).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_full_size_70b_mlp_sampled_rows(lbm):
+    """Full-size 70B MLP up projection (8192 -> 28672, single path s = 620,
+    batch 1) in the launch configuration of the stack benchmark; the oracle
+    checks a sample of output rows one by one."""
+    lb, layers = lbm
+    gen = torch.Generator(device="cuda").manual_seed(11)
+    layer, host = layers.random_layer(8192, 28672, 620, False, gen, keep_signs=True)
+    x = torch.randn(1, 8192, generator=gen, device="cuda").half()
+    y = lb.forward(layer, x)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(0).choice(28672, 512, replace=False))
+    y_ref = orc.factored_forward(x.cpu().numpy(), host, rows=rows)
+    _check(y[:, rows], y_ref, "70B sampled")
