@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""Benchmark of the LittleBit layer forward on B200; prints ONE JSON line.
+
+Default workload (one "step" = one forward over a stack of layers, batch 1):
+Llama-2-7B attention projection 4096 -> 4096 at 0.1 BPW with residual
+compensation (s = 86, two paths), replicated as distinct layers (own signs,
+scales, input and output) until the packed bytes exceed 4x the L2 cache, so
+that every step streams its weights from HBM.  The metric is microseconds per
+layer; the roofline object reports the dominant kernel's achieved HBM GB/s.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload (the only other place that runs the oracle).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode µs/layer & % HBM roofline at batch 1; prefill TFLOP/s & % tensor peak"
+FALLBACK_HBM_GBS = 6650.0
+
+# (d_in, d_out, s, residual) per matrix of one model layer
+WORKLOADS = {
+    "7b_attn_0.1bpw_residual": {
+        "desc": "Llama-2-7B attention projection 4096x4096, 0.1 BPW residual (s=86 x 2 paths)",
+        "mats": [(4096, 4096, 86, True)],
+    },
+    "7b_attn_0.1bpw_single": {
+        "desc": "Llama-2-7B attention projection 4096x4096, 0.1 BPW single path (s=188)",
+        "mats": [(4096, 4096, 188, False)],
+    },
+    "70b_mlp_0.1bpw_single": {
+        "desc": "Llama-2-70B MLP layer (8192->28672 gate, up; 28672->8192 down), 0.1 BPW single path s=620",
+        "mats": [(8192, 28672, 620, False), (8192, 28672, 620, False), (28672, 8192, 620, False)],
+    },
+    "70b_mlp_0.1bpw_residual": {
+        "desc": "Llama-2-70B MLP layer, 0.1 BPW residual s=302 x 2 paths",
+        "mats": [(8192, 28672, 302, True), (8192, 28672, 302, True), (28672, 8192, 302, True)],
+    },
+    "7b_layer_0.1bpw_residual": {
+        "desc": "Llama-2-7B layer (4x 4096^2 s=86; 2x 4096->11008 and 11008->4096 s=133), 0.1 BPW residual",
+        "mats": [(4096, 4096, 86, True)] * 4 + [(4096, 11008, 133, True)] * 2 + [(11008, 4096, 133, True)],
+    },
+}
+
+
+def algorithmic_bytes(d_in, d_out, s, residual, batch):
+    """Bytes the method must move for one matrix (packed bits at exactly s(a+b)
+    bits per path, fp16 scales, fp16 input and output)."""
+    paths = 2 if residual else 1
+    per_path = s * (d_in + d_out) / 8 + 2 * (d_in + d_out + s)
+    return paths * per_path + 2 * batch * (d_in + d_out)
+
+
+def kernel_bytes(d_in, d_out, s, residual, batch):
+    """Algorithmic bytes split by kernel: latent pass (V bits, g, l, x) and
+    output pass (U bits, h, y)."""
+    paths = 2 if residual else 1
+    lat = paths * (s * d_in / 8 + 2 * (d_in + s)) + 2 * batch * d_in
+    out = paths * (s * d_out / 8 + 2 * d_out) + 2 * batch * d_out
+    return lat, out
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk.get("hbm_gbs", FALLBACK_HBM_GBS)), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the GPU works."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,utilization.gpu,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        with open(self.tmp.name) as f:
+            rows = [ln.strip().split(", ") for ln in f if ln.strip()]
+        os.unlink(self.tmp.name)
+        samples = []
+        for r in rows:
+            try:
+                samples.append({"sm": float(r[1]), "max": float(r[2]), "util": float(r[3]),
+                                "hw": r[6].strip(), "hwt": r[7].strip(), "swt": r[8].strip(), "pcap": r[9].strip()})
+            except (ValueError, IndexError):
+                continue
+        if not samples:
+            return None
+        load = [s for s in samples if s["util"] > 0] or samples
+        reasons = set()
+        for s in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("pcap", "sw_power_cap")):
+                if s[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s["sm"] for s in load), "sm_max_mhz": max(s["max"] for s in load),
+                "reasons": sorted(reasons), "samples": len(load)}
+
+
+def traffic_record(kernel: str, workload: str):
+    """dram bytes per launch of `kernel` from the committed ncu summary, if it
+    was taken on the current kernel source."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    src = os.path.join(ROOT, "latent_binary_factorization_b200", "csrc", "decode.cu")
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    r = rec.get(workload, {}).get(kernel)
+    if not r or r.get("decode_cu_sha256_16") != digest:
+        return None
+    return r.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def build_stack(mats, n_rep, batch, seed, device):
+    import torch
+    from latent_binary_factorization_b200 import layers as lbl, littlebit as lb
+    gen = torch.Generator(device=device).manual_seed(seed)
+    Ls = []
+    for _ in range(n_rep):
+        for (a, b, s, r) in mats:
+            Ls.append(lbl.random_layer(a, b, s, r, gen, device=device)[0])
+    x_all = torch.randn(sum(L.d_in for L in Ls) * batch, generator=gen, device=device).half()
+    y_all = torch.empty(sum(L.d_out for L in Ls) * batch, dtype=torch.float16, device=device)
+    xs, ys, xo, yo = [], [], 0, 0
+    for L in Ls:
+        xs.append(x_all[xo:xo + batch * L.d_in].view(batch, L.d_in))
+        ys.append(y_all[yo:yo + batch * L.d_out].view(batch, L.d_out))
+        xo += batch * L.d_in
+        yo += batch * L.d_out
+    return lb.Stack(Ls, xs, ys), Ls, x_all, y_all
+
+
+def stack_reps_for_l2(mats, batch, l2_bytes, factor=4.0):
+    per = sum(algorithmic_bytes(*m, batch) for m in mats)
+    return max(1, math.ceil(factor * l2_bytes / per))
+
+
+def time_device(stack, steps, warmup, dist):
+    """K device-timed steps (CUDA events on the launching stream), and the
+    per-kernel split from an event recorded between the two launches."""
+    import torch
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        stack()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if dist:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for k in range(steps):
+        ev[k][0].record(stream)
+        # torch only times events it recorded itself; an event keeps its latest
+        # record, so record it here and let the library re-record it between
+        # its latent-pass and output-pass launches
+        ev[k][1].record(stream)
+        stack(event_between=ev[k][1])
+        ev[k][2].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        torch.distributed.barrier()
+    total_ms = t0.elapsed_time(t1)
+    lat = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+    out = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+    return total_ms, lat, out
+
+
+def time_e2e(stack, x_all, y_all, steps, warmup):
+    """Same forward through the public API with host buffers: H2D of every
+    layer's input from pinned memory, forward, D2H of every output."""
+    import torch
+    stream = torch.cuda.current_stream()
+    xh = torch.empty(x_all.shape, dtype=x_all.dtype, pin_memory=True)
+    xh.copy_(x_all.cpu())
+    yh = torch.empty(y_all.shape, dtype=y_all.dtype, pin_memory=True)
+
+    def step():
+        x_all.copy_(xh, non_blocking=True)
+        stack()
+        yh.copy_(y_all, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1), x_all.numel() * x_all.element_size(), y_all.numel() * y_all.element_size()
+
+
+def measure_workload(name, batch, steps, warmup, device, dist, world, l2, seed=1234, l2_factor=4.0):
+    mats = WORKLOADS[name]["mats"]
+    reps = stack_reps_for_l2(mats, batch, l2, l2_factor)
+    stack, Ls, x_all, y_all = build_stack(mats, reps, batch, seed, device)
+    n_layers = len(Ls)
+    total_ms, lat_ms, out_ms = time_device(stack, steps, warmup, dist)
+    if dist:
+        import torch
+        t = torch.tensor([total_ms, lat_ms, out_ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms, lat_ms, out_ms = t.tolist()
+    alg = sum(algorithmic_bytes(*m, batch) for m in mats) * reps
+    lat_b = sum(kernel_bytes(*m, batch)[0] for m in mats) * reps
+    out_b = sum(kernel_bytes(*m, batch)[1] for m in mats) * reps
+    ms_step = total_ms / steps
+    res = {
+        "workload": name, "desc": WORKLOADS[name]["desc"], "batch": batch, "layers_per_step": n_layers,
+        "model_layers_per_step": reps, "stack_bytes": int(alg), "ms_per_step": ms_step,
+        "us_per_matrix": 1e3 * ms_step / n_layers, "us_per_model_layer": 1e3 * ms_step / reps,
+        "step_gbs": alg / (ms_step * 1e-3) / 1e9,
+        "latent_pass_ms": lat_ms, "output_pass_ms": out_ms,
+        "latent_pass_gbs": lat_b / (lat_ms * 1e-3) / 1e9, "output_pass_gbs": out_b / (out_ms * 1e-3) / 1e9,
+        "latent_bytes": lat_b, "output_bytes": out_b,
+        "world": world,
+    }
+    return res, (stack, x_all, y_all)
+
+
+def run_ours(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = world > 1
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if dist:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    import latent_binary_factorization_b200.littlebit  # noqa: F401  fails loudly without the library
+    props = torch.cuda.get_device_properties(device)
+    l2 = props.L2_cache_size
+    peak, peak_kind = load_peaks()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    main, (stack, x_all, y_all) = measure_workload(args.workload, args.batch, args.steps, args.warmup, device,
+                                                   dist, world, l2, l2_factor=args.l2_factor)
+    e2e_ms, h2d, d2h = time_e2e(stack, x_all, y_all, max(3, args.steps // 4), 2)
+    if dist:
+        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = t.item()
+    del stack, x_all, y_all
+    extras = {}
+    if not args.no_extras:
+        for name, b in (("70b_mlp_0.1bpw_single", 1), ("70b_mlp_0.1bpw_residual", 1),
+                        ("7b_layer_0.1bpw_residual", 1), ("7b_attn_0.1bpw_single", 1),
+                        ("7b_attn_0.1bpw_residual", 4), ("7b_attn_0.1bpw_residual", 16)):
+            if name == args.workload and b == args.batch:
+                continue
+            r, held = measure_workload(name, b, max(5, args.steps // 2), args.warmup, device, dist, world, l2)
+            del held
+            torch.cuda.empty_cache()
+            r["roofline_frac_step"] = r["step_gbs"] / peak
+            extras[f"{name}_b{b}"] = r
+    clocks = sampler.stop()
+
+    n_layers = main["layers_per_step"]
+    lat, out = main["latent_pass_ms"], main["output_pass_ms"]
+    dom = "output_pass" if out >= lat else "latent_pass"
+    dom_bytes = main["output_bytes"] if dom == "output_pass" else main["latent_bytes"]
+    dom_ms = max(lat, out)
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    traffic = traffic_record(dom, args.workload)
+    value = 1e3 * main["ms_per_step"] / (n_layers * world)   # us per layer over all ranks' layers
+    line = {
+        "metric": METRIC,
+        "value": round(value, 5),
+        "unit": "us/layer",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(main["ms_per_step"], 5),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16",
+        "data": "synthetic: fair random signs, scales ~U[0.5,1.5]/sqrt(s), x ~ N(0,1) fp16",
+        "config": {"workload": WORKLOADS[args.workload]["desc"] + f", decode batch {args.batch}, "
+                   f"stack of {n_layers} distinct layers per GPU ({main['stack_bytes'] / 1e6:.0f} MB packed, "
+                   f">= 4x L2; inputs larger than L2, no flush)",
+                   "d_in": WORKLOADS[args.workload]["mats"][0][0], "d_out": WORKLOADS[args.workload]["mats"][0][1],
+                   "s": WORKLOADS[args.workload]["mats"][0][2], "residual": WORKLOADS[args.workload]["mats"][0][3],
+                   "batch": args.batch, "layers_per_gpu": n_layers, "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                     else "fallback", "algorithmic_bytes_per_launch": int(dom_bytes)},
+        "step_roofline": {"achieved": round(main["step_gbs"], 1), "frac": round(main["step_gbs"] / peak, 4),
+                          "latent_pass_gbs": round(main["latent_pass_gbs"], 1),
+                          "output_pass_gbs": round(main["output_pass_gbs"], 1)},
+        "e2e": {"value": round(1e3 * e2e_ms / max(3, args.steps // 4) / (n_layers * world), 5), "unit": "us/layer",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+        "extras": extras,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.workload, args.batch, budget_s=args.cpu_seconds)
+    if dist:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle arm
+# ---------------------------------------------------------------------------
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(workload, batch, budget_s=10.0, n_distinct=4):
+    """Time the fp64 oracle (as it stands) on distinct layers of the workload
+    until about `budget_s` seconds of CPU work; returns us per layer."""
+    from latent_binary_factorization_b200 import synth
+    from oracle import littlebit_oracle as orc
+    mats = WORKLOADS[workload]["mats"]
+    samples = []
+    for i in range(n_distinct):
+        a, b, s, r = mats[i % len(mats)]
+        samples.append((synth.layer(a, b, s, r, seed=77, index=i), synth.activations(batch, a, seed=77, index=i)))
+    orc.factored_forward(samples[0][1], samples[0][0])   # warm
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        paths, x = samples[n % n_distinct]
+        orc.factored_forward(x, paths)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s and n >= 3:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(1e6 * dt / n, 3), "unit": "us/layer", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{n} forwards of {n_distinct} distinct {WORKLOADS[workload]['desc']} layers, batch {batch}, "
+                      f"fp64 numpy, {dt:.1f} s"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from latent_binary_factorization_b200 import synth
+    from oracle import littlebit_oracle as orc
+    mats = WORKLOADS[args.workload]["mats"]
+    per_step = 4
+    samples = []
+    for i in range(per_step):
+        a, b, s, r = mats[i % len(mats)]
+        samples.append((synth.layer(a, b, s, r, seed=88, index=i), synth.activations(args.batch, a, seed=88, index=i)))
+
+    def step():
+        for paths, x in samples:
+            orc.factored_forward(x, paths)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = 1e6 * dt / (args.steps * per_step)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "us/layer", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * dt / args.steps, 3), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOADS[args.workload]["desc"] + f", decode batch {args.batch}; each step = "
+                   f"{per_step} distinct layers on the CPU oracle", "batch": args.batch},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 3), "unit": "us/layer", "kind": "oracle", "cores": _blas_threads(),
+                         "sample": f"{per_step} layers per step x {args.steps} steps"},
+        "e2e": {"value": round(value, 3), "unit": "us/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="7b_attn_0.1bpw_residual")
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--l2-factor", type=float, default=4.0,
+                    help="stack size as a multiple of the L2 cache (>= 1 keeps inputs larger than L2)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -46,7 +46,7 @@ typedef enum {
   LB_ERR_ALIGN = 2,       /* a pointer is not aligned as documented */
   LB_ERR_SHAPE = 3,       /* a dimension is outside what the kernels accept */
   LB_ERR_CUDA = 4,        /* a CUDA runtime call failed (see littlebit_last_cuda_error) */
-  LB_ERR_TIMEOUT = 5,     /* reserved: a bounded device wait ran out */
+  LB_ERR_TIMEOUT = 5,     /* a bounded device wait ran out (littlebit_device_status) */
   LB_ERR_UNSUPPORTED = 6  /* a valid request this build does not implement */
 } lb_status;
 
@@ -105,8 +105,8 @@ lb_status littlebit_pack_signs(const void* src_dev, lb_dtype dt, int n_long, int
 typedef struct lb_path {
   const void* V_bits;    /* packed LB_ROLE_V factor, 16-byte aligned */
   const void* U_bits;    /* packed LB_ROLE_U factor, 16-byte aligned */
-  const uint16_t* h;     /* fp16 [d_out] row (output) scale */
-  const uint16_t* g;     /* fp16 [d_in]  column (input) scale */
+  const uint16_t* h;     /* fp16 [d_out] row (output) scale, 16-byte aligned */
+  const uint16_t* g;     /* fp16 [d_in]  column (input) scale, 16-byte aligned */
   const uint16_t* l;     /* fp16 [s]     latent scale */
 } lb_path;
 
@@ -140,6 +140,25 @@ lb_status littlebit_linear_forward(const lb_layer* layer, const void* x_dev, voi
  */
 lb_status littlebit_linear_forward_many(const lb_layer* layers, int n, const void* const* xs,
                                         void* const* ys, int batch, lb_dtype xdt, void* stream);
+
+/*
+ * littlebit_linear_forward_many, and in addition records `event_between`
+ * (a cudaEvent_t passed as void*, or NULL) on `stream` between the latent-pass
+ * launch and the output-pass launch, so that a caller can time the two
+ * kernels separately with CUDA events.
+ */
+lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, const void* const* xs,
+                                              void* const* ys, int batch, lb_dtype xdt, void* stream,
+                                              void* event_between);
+
+/*
+ * Waits for `stream`, then returns in *status the device-side error bits that
+ * the forward kernels enqueued on it have raised since the last call, and
+ * clears them.  Bit (1 << LB_ERR_TIMEOUT) means a bounded wait for a bulk copy
+ * into shared memory gave up (the outputs of that call are not valid).
+ * *status is 0 when nothing was raised.  Errors: LB_ERR_ARG, LB_ERR_CUDA.
+ */
+lb_status littlebit_device_status(void* stream, unsigned int* status);
 
 /* Free every workspace of every device (call with no work in flight). */
 void littlebit_release(void);

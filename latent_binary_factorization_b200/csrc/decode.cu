@@ -4,27 +4,38 @@
 // (Samsung LittleBit article, section 2: two binary matrix products plus
 // elementwise scaling, residual paths added).
 //
-// Both binary products run on the int8 tensor cores (mma.sync m16n8k32,
-// u8 x s8 -> s32) without unpacking the signs.  The packed layout stores, for
-// each lane of a 512-byte tile, the four 32-bit A-fragment registers of eight
-// m16n8k32 products at once: bit q of every byte belongs to product q.  So
-// `word & (0x01010101 << q)` is that product's A register with entries
-// {0, 2^q}; one logic op per four signs, and the product's sum carries a known
-// factor 2^q that is shifted out once per output (exact integer arithmetic).
-// The B operand is the vector (g*x for the latent pass, t' = l*t for the
-// output pass) quantised to 16 bits, v = scale * (256*hi + lo), hi and lo being
-// two int8 columns; for a +-1 sign b = 1 - 2*bit,
-//     sum_k sign_k v_k = sum_k v_k - 2 * sum_k bit_k v_k.
-// Columns 2r and 2r+1 of the 8-column product hold batch row r's hi and lo
+// Arithmetic.  Both binary products run on the int8 tensor cores
+// (mma.sync m16n8k32, u8 x s8 -> s32) without unpacking the signs.  The packed
+// layout stores, for each lane of a 512-byte tile, the four 32-bit A-fragment
+// registers of eight m16n8k32 products at once: bit q of every byte belongs to
+// product q.  So `word & (0x01010101 << q)` is that product's A register with
+// entries {0, 2^q}; one logic op per four signs, and the product's sum carries
+// a known factor 2^q that is shifted out exactly in integer arithmetic.  The B
+// operand is the vector (g*x for the latent pass, t' = l*t for the output
+// pass) quantised to 16 bits, v = step * (256*hi + lo), hi and lo being two
+// int8 columns; for a +-1 sign s = 1 - 2*bit,
+//     sum_k s_k v_k = sum_k v_k - 2 * sum_k bit_k v_k.
+// Columns 2r and 2r+1 of an 8-column product hold batch row r's hi and lo
 // bytes, so one product serves four batch rows.
 //
-// Latent pass: CTA = (layer, path, 4096-input slice); each warp owns 4 tiles of
-// the slice and walks all 16-row latent blocks; the slice's exact integer sums
-// are combined in shared memory and written as one fp32 partial per latent
-// row.  The CTA that finishes a path's last slice (atomic ticket, no waiting)
-// sums the partials in slice order, multiplies by l and quantises t'.
-// Output pass: warp = (layer, 128 output rows); walks the role-U tiles of both
-// paths, scales by the quantisation step and h, adds the paths, writes fp16.
+// Data movement.  Sign tiles stream from HBM into a per-warp ring of shared
+// memory stages with bulk async copies (cp.async.bulk, completion counted on
+// an mbarrier per stage); the warp issues the copy for chunk c + stages as soon
+// as it has read chunk c, so a few KB per warp stay in flight without holding
+// registers.  Every wait is bounded: after kSpinLimit polls the kernel sets
+// LB_ERR_TIMEOUT in the status word and stops waiting.
+//
+// Latent pass: CTA item = (layer, path, 4096-input slice, 128-row chunk); warp
+// w owns tiles 4w..4w+3 of the slice and walks the chunk's 16-row latent
+// blocks; exact integer sums are combined in shared memory and written as one
+// fp32 partial per latent row.  The CTA that finishes a path's last item
+// (atomic ticket, no waiting) sums the partials in slice order, multiplies by
+// l and quantises t'.
+// Output pass: warp item = (layer, 128 output rows); each warp owns a
+// contiguous item range and streams it as chunks of up to 4 K-tiles, across
+// path, item and layer boundaries; the bulk copies also bring the chunk's t'
+// bytes and, for the last chunk of a path, the 128 h values and the
+// quantisation step.  Paths are added in fp32 and y is written in fp16.
 #include <cuda_fp16.h>
 
 #include "lb_internal.h"
@@ -32,34 +43,74 @@
 namespace lb {
 namespace {
 
-__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+// ------------------------------------------------------------------ PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+// global -> shared bulk copy (no multicast); 16-byte aligned, size % 16 == 0
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for phase `parity` of `bar`; false after kSpinLimit polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (int i = 0; i < kSpinLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+__device__ __forceinline__ uint4 ld_nc(const void* p) {
   uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
 }
 
-__device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
   asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ float2 h2x2(uint32_t v) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&v));
+}
 __device__ __forceinline__ float h2f(uint16_t v) { return __half2float(__ushort_as_half(v)); }
 __device__ __forceinline__ uint16_t f2h(float v) { return __half_as_ushort(__float2half_rn(v)); }
-
-__device__ __forceinline__ const LayerDesc& find_layer(const DecodeArgs& a, int item, bool latent) {
-  int lo = 0, hi = a.n_layers - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    const int begin = latent ? a.layers[mid].v_begin : a.layers[mid].u_begin;
-    if (begin <= item) lo = mid; else hi = mid - 1;
-  }
-  return a.layers[lo];
-}
 
 // quantise to v = 256*hi + lo; returns v and writes the two int8 bytes
 __device__ __forceinline__ int quantise(float u, float inv, int8_t& hi, int8_t& lo) {
@@ -71,194 +122,356 @@ __device__ __forceinline__ int quantise(float u, float inv, int8_t& hi, int8_t& 
   return v;
 }
 
-template <int NB>
-__device__ __forceinline__ void block_reduce_max_sum(float (&mx)[4 * NB], int (&sm)[4 * NB],
-                                                     float (*s_mx)[16], int (*s_sm)[16], int B) {
+// Block-wide max / sum of N values per thread (all threads get the result).
+template <int N>
+__device__ __forceinline__ void block_max(float (&v)[N], float (*s_buf)[16]) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
-  for (int b = 0; b < 4 * NB; ++b) {
+  for (int i = 0; i < N; ++i) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      mx[b] = fmaxf(mx[b], __shfl_xor_sync(0xffffffffu, mx[b], o));
-      sm[b] += __shfl_xor_sync(0xffffffffu, sm[b], o);
-    }
-    if (lane == 0 && b < B) { s_mx[warp][b] = mx[b]; s_sm[warp][b] = sm[b]; }
+    for (int o = 16; o > 0; o >>= 1) v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], o));
+    if (lane == 0) s_buf[warp][i] = v[i];
   }
   __syncthreads();
 #pragma unroll
-  for (int b = 0; b < 4 * NB; ++b) {
-    if (b < B) {
-      float m = s_mx[0][b];
-      int ssum = s_sm[0][b];
+  for (int i = 0; i < N; ++i) {
+    float m = s_buf[0][i];
 #pragma unroll
-      for (int w = 1; w < kVWarps; ++w) { m = fmaxf(m, s_mx[w][b]); ssum += s_sm[w][b]; }
-      mx[b] = m;
-      sm[b] = ssum;
-    }
+    for (int w = 1; w < kVWarps; ++w) m = fmaxf(m, s_buf[w][i]);
+    v[i] = m;
   }
   __syncthreads();
+}
+
+template <int N>
+__device__ __forceinline__ void block_sum(int (&v)[N], int (*s_buf)[16]) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
+    if (lane == 0) s_buf[warp][i] = v[i];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    int m = s_buf[0][i];
+#pragma unroll
+    for (int w = 1; w < kVWarps; ++w) m += s_buf[w][i];
+    v[i] = m;
+  }
+  __syncthreads();
+}
+
+// Index of the layer whose item range holds `item` (binary search, once per
+// warp or CTA; later items are reached by walking forward).
+__device__ __forceinline__ int find_layer(const DecodeArgs& a, int item, bool latent) {
+  int lo = 0, hi = a.n_layers - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    const int begin = latent ? a.layers[mid].v_begin : a.layers[mid].u_begin;
+    if (begin <= item) lo = mid; else hi = mid - 1;
+  }
+  return lo;
 }
 
 // ---------------------------------------------------------------------------
 // latent pass:  t_j (partial over one slice) = sum_i V[i][j] g_i x_i
 // ---------------------------------------------------------------------------
+
+struct VItem {
+  int li, p, sl, rc;
+};
+
+// decode `item` into (layer, path, slice, row chunk); li walks forward
+__device__ __forceinline__ VItem decode_v(const DecodeArgs& a, int item, int& li) {
+  while (li + 1 < a.n_layers && a.layers[li + 1].v_begin <= item) ++li;
+  const LayerDesc& L = a.layers[li];
+  int rel = item - L.v_begin;
+  const int per_path = L.n_slices * L.n_rchunks;
+  VItem it;
+  it.li = li;
+  it.p = rel / per_path;
+  rel -= it.p * per_path;
+  it.sl = rel / L.n_rchunks;
+  it.rc = rel - it.sl * L.n_rchunks;
+  return it;
+}
+
+// Walks one warp's sequence of bulk-copy chunks (one per 16-row block it owns).
+struct VFeed {
+  int item, li, rb, rb_hi, row_stride;   // row_stride: bytes from one 16-row block to the next
+  uint32_t bytes;                        // this warp's tiles per row block * 512
+  const unsigned char* base;             // this warp's first tile at row block 0
+
+  __device__ __forceinline__ void set(const DecodeArgs& a, int warp) {
+    const VItem it = decode_v(a, item, li);
+    const LayerDesc& L = a.layers[li];
+    const int k0 = it.sl * kVSlice, klen = min(kVSlice, L.d_in - k0);
+    const int nt = max(0, min(kVTilesPerWarp, klen / kVTileK - kVTilesPerWarp * warp));
+    row_stride = (L.d_in / kVTileK) * kTileBytes;
+    rb = it.rc * kVRowChunk;
+    rb_hi = min((L.s + 15) >> 4, rb + kVRowChunk);
+    bytes = (uint32_t)nt * kTileBytes;
+    base = reinterpret_cast<const unsigned char*>(L.p[it.p].V) +
+           (size_t)(k0 / kVTileK + kVTilesPerWarp * warp) * kTileBytes;
+  }
+  __device__ __forceinline__ void normalize(const DecodeArgs& a, int warp, int end) {
+    while (item < end && (bytes == 0 || rb >= rb_hi)) {
+      if (++item < end) set(a, warp);
+    }
+  }
+  __device__ __forceinline__ void advance(const DecodeArgs& a, int warp, int end) {
+    ++rb;
+    normalize(a, warp, end);
+  }
+  __device__ __forceinline__ const unsigned char* src() const { return base + (size_t)rb * row_stride; }
+};
+
 template <int NB>
-__global__ void __launch_bounds__(kVWarps * 32) latent_pass_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_kernel(const DecodeArgs a) {
   constexpr int NCOL = 8 * NB;
-  extern __shared__ __align__(16) unsigned char smem[];
-  int8_t* bpl = reinterpret_cast<int8_t*>(smem);                         // [kVSlice/32][NCOL][32]
-  int* acc = reinterpret_cast<int*>(smem + (size_t)kVSlice * NCOL);      // [B][S16] (or fp32 t')
+  extern __shared__ __align__(1024) unsigned char smem[];
+  unsigned char* ring = smem;                                                         // [warps][stages][2 KB]
+  int8_t* bpl = reinterpret_cast<int8_t*>(smem + kVWarps * kVStages * kChunkBytes);  // [128][NCOL][32]
+  int* acc = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(bpl) + (size_t)kVSlice * NCOL);  // [16][128]
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(acc + kMaxBatchDecode * kVRowChunk * 16);               // [warps][stages]
+  float* tp = reinterpret_cast<float*>(bpl);   // finalize: [B][S16] fp32 (bpl is free then)
   __shared__ float s_mx[kVWarps][16];
   __shared__ int s_sm[kVWarps][16];
   __shared__ int s_last;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
   const int B = a.batch;
+  const int i_begin = (int)((long long)a.v_items * blockIdx.x / gridDim.x);
+  const int i_end = (int)((long long)a.v_items * (blockIdx.x + 1) / gridDim.x);
+  if (i_begin >= i_end) return;   // uniform over the CTA
 
-  for (int item = blockIdx.x; item < a.v_items; item += gridDim.x) {
-    const LayerDesc& L = find_layer(a, item, true);
-    const int rel = item - L.v_begin;
-    const int p = rel / L.n_slices, sl = rel - p * L.n_slices;
-    const PathDesc& P = L.p[p];
+  unsigned char* my_ring = ring + (size_t)warp * kVStages * kChunkBytes;
+  uint64_t* my_bar = mbar + warp * kVStages;
+  if (lane == 0) {
+    for (int st = 0; st < kVStages; ++st) mbar_init(&my_bar[st], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  // prime this warp's ring
+  const int li0 = find_layer(a, i_begin, true);
+  VFeed feed;
+  feed.item = i_begin;
+  feed.li = li0;
+  feed.set(a, warp);
+  feed.normalize(a, warp, i_end);
+#pragma unroll 1
+  for (int st = 0; st < kVStages; ++st) {
+    if (feed.item < i_end) {
+      if (lane == 0) {
+        mbar_expect_tx(&my_bar[st], feed.bytes);
+        bulk_g2s(my_ring + st * kChunkBytes, feed.src(), feed.bytes, &my_bar[st]);
+      }
+      feed.advance(a, warp, i_end);
+    }
+  }
+  uint32_t consumed = 0;
+  bool dead = false;
+
+  int li = li0;
+  int prev_li = -1, prev_p = -1, prev_sl = -1;   // slice whose B operand is staged
+  float step[4 * NB];
+  int vs[4 * NB];
+  uint32_t bf[NB == 1 ? kVTilesPerWarp * 8 : 1][2];
+
+  for (int item = i_begin; item < i_end; ++item) {
+    const VItem it = decode_v(a, item, li);
+    const LayerDesc& L = a.layers[li];
+    const PathDesc& P = L.p[it.p];
     const int d_in = L.d_in, s = L.s;
     const int S16 = (s + 15) & ~15;
-    const int k0 = sl * kVSlice;
-    const int klen = min(kVSlice, d_in - k0);          // multiple of 256
-    const int n_kt_all = d_in / kVTileK;
-
-    // ---- 1. u = g * x on the slice: per-row max |u| and the quantisation step
-    float mx[4 * NB];
-    int vs[4 * NB];
-#pragma unroll
-    for (int b = 0; b < 4 * NB; ++b) { mx[b] = 0.f; vs[b] = 0; }
-    for (int k = tid; k < klen; k += kVWarps * 32) {
-      const float gk = h2f(P.g[k0 + k]);
-#pragma unroll
-      for (int b = 0; b < 4 * NB; ++b)
-        if (b < B) mx[b] = fmaxf(mx[b], fabsf(gk * h2f(L.x[(size_t)b * d_in + k0 + k])));
-    }
-    block_reduce_max_sum<NB>(mx, vs, s_mx, s_sm, B);
-    float inv[4 * NB], step[4 * NB];
-#pragma unroll
-    for (int b = 0; b < 4 * NB; ++b) {
-      inv[b] = mx[b] > 0.f ? kQMax / mx[b] : 0.f;
-      step[b] = mx[b] > 0.f ? mx[b] / kQMax : 0.f;
-    }
-    // ---- 2. quantised planes into the B-operand staging area; sum of v
-    for (int k = tid; k < klen; k += kVWarps * 32) {
-      const float gk = h2f(P.g[k0 + k]);
-      int8_t* col = bpl + (size_t)(k >> 5) * NCOL * 32 + (k & 31);
-#pragma unroll
-      for (int b = 0; b < 4 * NB; ++b) {
-        int8_t hi = 0, lo = 0;
-        if (b < B) vs[b] += quantise(gk * h2f(L.x[(size_t)b * d_in + k0 + k]), inv[b], hi, lo);
-        const int n = (b >> 2) * 8 + (b & 3) * 2;   // column of (row b, hi); lo is n + 1
-        col[n * 32] = hi;
-        col[(n + 1) * 32] = lo;
-      }
-    }
-    block_reduce_max_sum<NB>(mx, vs, s_mx, s_sm, B);   // mx unchanged; vs = slice sum of v
-    for (int i = tid; i < B * S16; i += kVWarps * 32) acc[i] = 0;
-    __syncthreads();
-
-    // ---- 3. warp w: tiles 4w..4w+3 of the slice, all 16-row latent blocks
+    const int k0 = it.sl * kVSlice;
+    const int klen = min(kVSlice, d_in - k0);   // multiple of 256
     const int nt = max(0, min(kVTilesPerWarp, klen / kVTileK - kVTilesPerWarp * warp));
-    const int kt0 = k0 / kVTileK + kVTilesPerWarp * warp;   // first global K-tile of this warp
-    uint32_t bf[NB == 1 ? kVTilesPerWarp * 8 : 1][2];
-    if constexpr (NB == 1) {
+    const int rb_lo = it.rc * kVRowChunk, rb_hi = min(S16 >> 4, rb_lo + kVRowChunk);
+    const int nrow = 16 * (rb_hi - rb_lo);
+
+    if (it.li != prev_li || it.p != prev_p || it.sl != prev_sl) {
+      // ---- u = g * x on the slice, quantised per batch row to 16 bits and
+      //      staged as int8 hi/lo B-operand columns (all loads issue up front)
+      constexpr int kChunks = kVSlice / 8 / (kVWarps * 32);
+      const int nchunk = klen / 8;
+      uint4 gq[kChunks];
 #pragma unroll
-      for (int t = 0; t < kVTilesPerWarp; ++t)
+      for (int i = 0; i < kChunks; ++i) {
+        const int ch = tid + i * kVWarps * 32;
+        gq[i] = ch < nchunk ? ld_nc(P.g + k0 + 8 * ch) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int kb = (kVTilesPerWarp * warp + t) * 8 + q;
-          const int8_t* base = bpl + ((size_t)kb * NCOL + g) * 32 + 4 * c;
-          bf[t * 8 + q][0] = *reinterpret_cast<const uint32_t*>(base);
-          bf[t * 8 + q][1] = *reinterpret_cast<const uint32_t*>(base + 16);
+      for (int bg = 0; bg < NB; ++bg) {
+        uint4 xq[4][kChunks];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int i = 0; i < kChunks; ++i) {
+            const int ch = tid + i * kVWarps * 32, b = 4 * bg + r;
+            xq[r][i] = (b < B && ch < nchunk) ? ld_nc(L.x + (size_t)b * d_in + k0 + 8 * ch)
+                                               : make_uint4(0, 0, 0, 0);
+          }
+        float mx[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int i = 0; i < kChunks; ++i) {
+            const uint32_t* xw = &xq[r][i].x;
+            const uint32_t* gw = &gq[i].x;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 xf = h2x2(xw[e]), gf = h2x2(gw[e]);
+              mx[r] = fmaxf(mx[r], fmaxf(fabsf(xf.x * gf.x), fabsf(xf.y * gf.y)));
+            }
+          }
+        block_max<4>(mx, s_mx);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float inv = mx[r] > 0.f ? kQMax / mx[r] : 0.f;
+          step[4 * bg + r] = mx[r] > 0.f ? mx[r] / kQMax : 0.f;
+          int vsum = 0;
+#pragma unroll
+          for (int i = 0; i < kChunks; ++i) {
+            const int ch = tid + i * kVWarps * 32;
+            const uint32_t* xw = &xq[r][i].x;
+            const uint32_t* gw = &gq[i].x;
+            uint32_t hi[2] = {0u, 0u}, lo[2] = {0u, 0u};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 xf = h2x2(xw[e]), gf = h2x2(gw[e]);
+              int8_t h0, l0, h1, l1;
+              vsum += quantise(xf.x * gf.x, inv, h0, l0) + quantise(xf.y * gf.y, inv, h1, l1);
+              const int sh = 16 * (e & 1);
+              hi[e >> 1] |= ((uint32_t)(uint8_t)h0 | ((uint32_t)(uint8_t)h1 << 8)) << sh;
+              lo[e >> 1] |= ((uint32_t)(uint8_t)l0 | ((uint32_t)(uint8_t)l1 << 8)) << sh;
+            }
+            if (ch < nchunk) {
+              const int k = 8 * ch;
+              int8_t* col = bpl + ((size_t)(k >> 5) * NCOL + bg * 8 + 2 * r) * 32 + (k & 31);
+              *reinterpret_cast<uint2*>(col) = make_uint2(hi[0], hi[1]);
+              *reinterpret_cast<uint2*>(col + 32) = make_uint2(lo[0], lo[1]);
+            }
+          }
+          vs[4 * bg + r] = vsum;
         }
-    }
-    const int n_rb = S16 / 16;
-    const uint4* vt = P.V + (size_t)lane;
-    uint4 cur[kVTilesPerWarp], nxt[kVTilesPerWarp];
-#pragma unroll
-    for (int t = 0; t < kVTilesPerWarp; ++t)
-      cur[t] = (t < nt) ? ld_stream(vt + ((size_t)0 * n_kt_all + kt0 + t) * 32) : make_uint4(0, 0, 0, 0);
-    for (int rb = 0; rb < n_rb; ++rb) {
-      if (rb + 1 < n_rb) {
+      }
+      block_sum<4 * NB>(vs, s_sm);   // ends with __syncthreads: bpl complete
+      if constexpr (NB == 1) {
 #pragma unroll
         for (int t = 0; t < kVTilesPerWarp; ++t)
-          nxt[t] = (t < nt) ? ld_stream(vt + ((size_t)(rb + 1) * n_kt_all + kt0 + t) * 32)
-                            : make_uint4(0, 0, 0, 0);
-      }
-      int d[8][NB][4];
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) d[q][nb][0] = d[q][nb][1] = d[q][nb][2] = d[q][nb][3] = 0;
-#pragma unroll
-      for (int t = 0; t < kVTilesPerWarp; ++t) {
-        if (t < nt) {
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const uint32_t m = 0x01010101u << q;
-            const uint32_t a0 = cur[t].x & m, a1 = cur[t].y & m, a2 = cur[t].z & m, a3 = cur[t].w & m;
+            const int kb = (kVTilesPerWarp * warp + t) * 8 + q;
+            const int8_t* base = bpl + ((size_t)kb * NCOL + g) * 32 + 4 * c;
+            bf[t * 8 + q][0] = *reinterpret_cast<const uint32_t*>(base);
+            bf[t * 8 + q][1] = *reinterpret_cast<const uint32_t*>(base + 16);
+          }
+      }
+      prev_li = it.li;
+      prev_p = it.p;
+      prev_sl = it.sl;
+    }
+    for (int i = tid; i < B * kVRowChunk * 16; i += kVWarps * 32) acc[i] = 0;
+    __syncthreads();
+
+    // ---- this warp's tiles for every 16-row block of the chunk
+    if (nt > 0) {
+      for (int rb = rb_lo; rb < rb_hi; ++rb) {
+        const int slot = consumed % kVStages;
+        if (!dead && !mbar_wait(&my_bar[slot], (consumed / kVStages) & 1)) {
+          dead = true;
+          atomicOr(a.status, 1u << LB_ERR_TIMEOUT);
+        }
+        const unsigned char* stage = my_ring + slot * kChunkBytes;
+        uint4 cur[kVTilesPerWarp];
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-              uint32_t b0, b1;
-              if constexpr (NB == 1) {
-                b0 = bf[t * 8 + q][0];
-                b1 = bf[t * 8 + q][1];
-              } else {
-                const int kb = (kVTilesPerWarp * warp + t) * 8 + q;
-                const int8_t* base = bpl + ((size_t)kb * NCOL + nb * 8 + g) * 32 + 4 * c;
-                b0 = *reinterpret_cast<const uint32_t*>(base);
-                b1 = *reinterpret_cast<const uint32_t*>(base + 16);
+        for (int t = 0; t < kVTilesPerWarp; ++t)
+          cur[t] = t < nt ? *reinterpret_cast<const uint4*>(stage + t * kTileBytes + lane * 16)
+                          : make_uint4(0, 0, 0, 0);
+        int d[8][NB][4];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) d[q][nb][0] = d[q][nb][1] = d[q][nb][2] = d[q][nb][3] = 0;
+#pragma unroll
+        for (int t = 0; t < kVTilesPerWarp; ++t) {
+          if (t < nt) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const uint32_t m = 0x01010101u << q;
+              const uint32_t a0 = cur[t].x & m, a1 = cur[t].y & m, a2 = cur[t].z & m, a3 = cur[t].w & m;
+#pragma unroll
+              for (int nb = 0; nb < NB; ++nb) {
+                uint32_t b0, b1;
+                if constexpr (NB == 1) {
+                  b0 = bf[t * 8 + q][0];
+                  b1 = bf[t * 8 + q][1];
+                } else {
+                  const int kb = (kVTilesPerWarp * warp + t) * 8 + q;
+                  const int8_t* base = bpl + ((size_t)kb * NCOL + nb * 8 + g) * 32 + 4 * c;
+                  b0 = *reinterpret_cast<const uint32_t*>(base);
+                  b1 = *reinterpret_cast<const uint32_t*>(base + 16);
+                }
+                mma_u8s8(d[q][nb], a0, a1, a2, a3, b0, b1);
               }
-              mma_u8s8(d[q][nb], a0, a1, a2, a3, b0, b1);
             }
           }
         }
-      }
-      // fold: sum_q (256*D_hi + D_lo) / 2^q, Horner from q = 7 down (exact)
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-        int r0 = 256 * d[7][nb][0] + d[7][nb][1];
-        int r1 = 256 * d[7][nb][2] + d[7][nb][3];
-#pragma unroll
-        for (int q = 6; q >= 0; --q) {
-          r0 = (r0 >> 1) + 256 * d[q][nb][0] + d[q][nb][1];
-          r1 = (r1 >> 1) + 256 * d[q][nb][2] + d[q][nb][3];
+        // the stage has been read (its words fed the products): refill it
+        __syncwarp();
+        if (feed.item < i_end) {
+          if (lane == 0) {
+            mbar_expect_tx(&my_bar[slot], feed.bytes);
+            bulk_g2s(my_ring + slot * kChunkBytes, feed.src(), feed.bytes, &my_bar[slot]);
+          }
+          feed.advance(a, warp, i_end);
         }
-        const int b = 4 * nb + c;
-        if (b < B && nt > 0) {
-          atomicAdd(&acc[b * S16 + 16 * rb + g], r0);
-          atomicAdd(&acc[b * S16 + 16 * rb + g + 8], r1);
+        ++consumed;
+        // fold: sum_q (256*D_hi + D_lo) / 2^q, Horner from q = 7 down (exact)
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          int r0 = 256 * d[7][nb][0] + d[7][nb][1];
+          int r1 = 256 * d[7][nb][2] + d[7][nb][3];
+#pragma unroll
+          for (int q = 6; q >= 0; --q) {
+            r0 = (r0 >> 1) + 256 * d[q][nb][0] + d[q][nb][1];
+            r1 = (r1 >> 1) + 256 * d[q][nb][2] + d[q][nb][3];
+          }
+          const int b = 4 * nb + c;
+          if (b < B) {
+            const int row = 16 * (rb - rb_lo) + g;
+            atomicAdd(&acc[b * (kVRowChunk * 16) + row], r0);
+            atomicAdd(&acc[b * (kVRowChunk * 16) + row + 8], r1);
+          }
         }
       }
-#pragma unroll
-      for (int t = 0; t < kVTilesPerWarp; ++t) cur[t] = nxt[t];
     }
     __syncthreads();
 
-    // ---- 4. slice partial: step * (sum v - 2 * sum bit*v)
-    float* part = P.ws.partial + (size_t)sl * B * S16;
-    for (int i = tid; i < B * S16; i += kVWarps * 32) {
-      const int b = i / S16;
+    // ---- partial of this slice for the chunk's rows: step * (sum v - 2 * sum bit*v)
+    float* part = P.ws.partial + (size_t)it.sl * B * S16 + 16 * rb_lo;
+    for (int i = tid; i < B * nrow; i += kVWarps * 32) {
+      const int b = i / nrow, r = i - b * nrow;
       float st = 0.f;
       int vsum = 0;
 #pragma unroll
       for (int bb = 0; bb < 4 * NB; ++bb)
         if (bb == b) { st = step[bb]; vsum = vs[bb]; }
-      part[i] = st * (float)(vsum - 2 * acc[i]);
+      part[(size_t)b * S16 + r] = st * (float)(vsum - 2 * acc[b * (kVRowChunk * 16) + r]);
     }
     __threadfence();
     __syncthreads();
-    if (tid == 0) s_last = (atomicAdd(P.ws.counter, 1u) == (unsigned)(L.n_slices - 1));
+    if (tid == 0)
+      s_last = (atomicAdd(P.ws.counter, 1u) == (unsigned)(L.n_slices * L.n_rchunks - 1));
     __syncthreads();
 
     if (s_last) {
-      // ---- 5. last slice of this path: t' = l * sum of partials, quantised
+      // ---- last item of this path: t' = l * (sum of slice partials), quantised
       __threadfence();
-      float* tp = reinterpret_cast<float*>(acc);
       float mt[4 * NB];
       int ts[4 * NB];
 #pragma unroll
@@ -275,7 +488,7 @@ __global__ void __launch_bounds__(kVWarps * 32) latent_pass_kernel(const DecodeA
         for (int bb = 0; bb < 4 * NB; ++bb)
           if (bb == b) mt[bb] = fmaxf(mt[bb], fabsf(t));
       }
-      block_reduce_max_sum<NB>(mt, ts, s_mx, s_sm, B);
+      block_max<4 * NB>(mt, s_mx);
       const int S32 = (s + 31) & ~31;
       for (int i = tid; i < B * S32; i += kVWarps * 32) {
         const int b = i / S32, j = i - b * S32;
@@ -290,20 +503,25 @@ __global__ void __launch_bounds__(kVWarps * 32) latent_pass_kernel(const DecodeA
           for (int bb = 0; bb < 4 * NB; ++bb)
             if (bb == b) ts[bb] += v;
         }
-        P.ws.planes[(size_t)(b * 2) * S32 + j] = hi;
-        P.ws.planes[(size_t)(b * 2 + 1) * S32 + j] = lo;
+        int8_t* pl = P.ws.planes + ((size_t)((j >> 5) * B + b) * 2) * 32 + (j & 31);
+        pl[0] = hi;
+        pl[32] = lo;
       }
-      block_reduce_max_sum<NB>(mt, ts, s_mx, s_sm, B);
+      block_sum<4 * NB>(ts, s_sm);
       if (tid < B) {
         float m = 0.f;
         int sum = 0;
 #pragma unroll
         for (int bb = 0; bb < 4 * NB; ++bb)
           if (bb == tid) { m = mt[bb]; sum = ts[bb]; }
-        P.ws.tscale[tid] = m > 0.f ? m / kQMax : 0.f;
-        P.ws.tsum[tid] = sum;
+        TStat st;
+        st.step = m > 0.f ? m / kQMax : 0.f;
+        st.sum = sum;
+        st.pad[0] = st.pad[1] = 0;
+        P.ws.tstat[tid] = st;
       }
       if (tid == 0) *P.ws.counter = 0u;
+      prev_li = -1;   // tp overwrote the staged B operand
     }
     __syncthreads();
   }
@@ -312,43 +530,132 @@ __global__ void __launch_bounds__(kVWarps * 32) latent_pass_kernel(const DecodeA
 // ---------------------------------------------------------------------------
 // output pass:  y_o = sum_p h_p[o] * sum_j U_p[o][j] t'_p[j]
 // ---------------------------------------------------------------------------
+
+template <int NB>
+struct OutCfg {
+  static constexpr int kStages = NB <= 2 ? 6 : 4;
+};
+
+// stage: [4 tiles: 2048][t' bytes: 4 K-tiles x B x 64][h: 256][tstat: 16 B]
+__host__ __device__ __forceinline__ int out_planes_off() { return kChunkBytes; }
+__host__ __device__ __forceinline__ int out_h_off(int B) { return kChunkBytes + kChunkTiles * B * 64; }
+__host__ __device__ __forceinline__ int out_tstat_off(int B) { return out_h_off(B) + kUTileRows * 2; }
+__host__ __device__ __forceinline__ int out_stage_bytes(int B) {
+  return (out_tstat_off(B) + 16 * B + 127) & ~127;
+}
+
+// Position in a warp's stream of output-pass chunks (up to 4 K-tiles of one
+// (item, path)), with the fields of the current layer cached.
+struct OutCursor {
+  int li, item, p, kt0;
+  int n_kt, npaths, u_begin, u_end;
+
+  __device__ __forceinline__ void enter(const DecodeArgs& a, int l) {
+    li = l;
+    const LayerDesc& L = a.layers[l];
+    n_kt = (L.s + 31) >> 5;
+    npaths = L.npaths;
+    u_begin = L.u_begin;
+    u_end = (l + 1 < a.n_layers) ? a.layers[l + 1].u_begin : a.u_items;
+  }
+  __device__ __forceinline__ int ntile() const { return min(kChunkTiles, n_kt - kt0); }
+  __device__ __forceinline__ bool path_end() const { return kt0 + kChunkTiles >= n_kt; }
+  __device__ __forceinline__ void advance(const DecodeArgs& a) {
+    kt0 += kChunkTiles;
+    if (kt0 >= n_kt) {
+      kt0 = 0;
+      if (++p == npaths) {
+        p = 0;
+        if (++item == u_end && item < a.u_items) enter(a, li + 1);
+      }
+    }
+  }
+};
+
+__device__ __forceinline__ void out_issue(const DecodeArgs& a, const OutCursor& cu, unsigned char* stage,
+                                          uint64_t* bar, int B) {
+  const LayerDesc& L = a.layers[cu.li];
+  const PathDesc& P = L.p[cu.p];
+  const int ob = cu.item - cu.u_begin;
+  const int nt = cu.ntile();
+  const uint32_t tb = (uint32_t)nt * kTileBytes, pb = (uint32_t)nt * B * 64;
+  const bool last = cu.path_end();
+  const uint32_t total = tb + pb + (last ? kUTileRows * 2 + 16 * B : 0);
+  mbar_expect_tx(bar, total);
+  bulk_g2s(stage, reinterpret_cast<const unsigned char*>(P.U) + ((size_t)ob * cu.n_kt + cu.kt0) * kTileBytes,
+           tb, bar);
+  bulk_g2s(stage + out_planes_off(), P.ws.planes + (size_t)cu.kt0 * B * 64, pb, bar);
+  if (last) {
+    bulk_g2s(stage + out_h_off(B), P.h + (size_t)ob * kUTileRows, kUTileRows * 2, bar);
+    bulk_g2s(stage + out_tstat_off(B), P.ws.tstat, 16 * B, bar);
+  }
+}
+
 template <int NB>
 __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeArgs a) {
+  constexpr int S = OutCfg<NB>::kStages;
+  extern __shared__ __align__(1024) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
   const int B = a.batch;
-  for (int item = blockIdx.x * kUWarps + warp; item < a.u_items; item += gridDim.x * kUWarps) {
-    const LayerDesc& L = find_layer(a, item, false);
-    const int ob = item - L.u_begin;
-    const int s = L.s, S32 = (s + 31) & ~31, n_kt = S32 / kUTileK;
-    float yacc[8][2][NB];
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) yacc[q][0][nb] = yacc[q][1][nb] = 0.f;
+  const int sb = out_stage_bytes(B);
+  unsigned char* my_ring = smem + (size_t)warp * S * sb;
+  uint64_t* my_bar = reinterpret_cast<uint64_t*>(smem + (size_t)kUWarps * S * sb) + warp * S;
 
-    for (int p = 0; p < L.npaths; ++p) {
-      const PathDesc& P = L.p[p];
-      int d[8][NB][4];
+  const long long W = (long long)gridDim.x * kUWarps, gw = (long long)blockIdx.x * kUWarps + warp;
+  const int i_begin = (int)(a.u_items * gw / W), i_end = (int)(a.u_items * (gw + 1) / W);
+  if (i_begin >= i_end) return;   // no CTA-wide barriers in this kernel
+
+  if (lane == 0) {
+    for (int st = 0; st < S; ++st) mbar_init(&my_bar[st], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  OutCursor fd;
+  fd.enter(a, find_layer(a, i_begin, false));
+  fd.item = i_begin;
+  fd.p = 0;
+  fd.kt0 = 0;
+  OutCursor cs = fd;
+#pragma unroll 1
+  for (int st = 0; st < S; ++st) {
+    if (fd.item < i_end) {
+      if (lane == 0) out_issue(a, fd, my_ring + st * sb, &my_bar[st], B);
+      fd.advance(a);
+    }
+  }
+
+  float yacc[8][2][NB];
+  int d[8][NB][4];
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
+  for (int q = 0; q < 8; ++q)
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb) d[q][nb][0] = d[q][nb][1] = d[q][nb][2] = d[q][nb][3] = 0;
-      const uint4* ut = P.U + (size_t)ob * n_kt * 32 + lane;
-      uint4 w = ld_stream(ut);
-      for (int kt = 0; kt < n_kt; ++kt) {
-        const uint4 cur = w;
-        if (kt + 1 < n_kt) w = ld_stream(ut + (size_t)(kt + 1) * 32);
+    for (int nb = 0; nb < NB; ++nb) {
+      yacc[q][0][nb] = yacc[q][1][nb] = 0.f;
+      d[q][nb][0] = d[q][nb][1] = d[q][nb][2] = d[q][nb][3] = 0;
+    }
+  uint32_t consumed = 0;
+  bool dead = false;
+
+  while (cs.item < i_end) {
+    const int slot = consumed % S;
+    if (!dead && !mbar_wait(&my_bar[slot], (consumed / S) & 1)) {
+      dead = true;
+      atomicOr(a.status, 1u << LB_ERR_TIMEOUT);
+    }
+    const unsigned char* stage = my_ring + slot * sb;
+    const int nt = cs.ntile();
+#pragma unroll
+    for (int t = 0; t < kChunkTiles; ++t) {
+      if (t < nt) {
+        const uint4 cur = *reinterpret_cast<const uint4*>(stage + t * kTileBytes + lane * 16);
         uint32_t b0[NB], b1[NB];
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
           const int b = 4 * nb + (g >> 1);
-          if (b < B) {
-            const int8_t* pl = P.ws.planes + (size_t)(b * 2 + (g & 1)) * S32 + kt * 32 + 4 * c;
-            b0[nb] = *reinterpret_cast<const uint32_t*>(pl);
-            b1[nb] = *reinterpret_cast<const uint32_t*>(pl + 16);
-          } else {
-            b0[nb] = b1[nb] = 0u;
-          }
+          const unsigned char* pl = stage + out_planes_off() + ((t * B + b) * 2 + (g & 1)) * 32 + 4 * c;
+          b0[nb] = b < B ? *reinterpret_cast<const uint32_t*>(pl) : 0u;
+          b1[nb] = b < B ? *reinterpret_cast<const uint32_t*>(pl + 16) : 0u;
         }
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -358,54 +665,87 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
           for (int nb = 0; nb < NB; ++nb) mma_u8s8(d[q][nb], a0, a1, a2, a3, b0[nb], b1[nb]);
         }
       }
-      // epilogue of this path: rows 128ob + 16q + g (+8), batch row 4nb + c
+    }
+    if (cs.path_end()) {
+      // path finished: rows 128*ob + 16q + g (+8), batch row 4nb + c
+      const uint16_t* hs = reinterpret_cast<const uint16_t*>(stage + out_h_off(B));
+      const TStat* tst = reinterpret_cast<const TStat*>(stage + out_tstat_off(B));
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb) {
         const int b = 4 * nb + c;
         if (b < B) {
-          const float st = P.ws.tscale[b];
-          const int tsum = P.ws.tsum[b];
+          const float st = tst[b].step;
+          const int tsum = tst[b].sum;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const int c0 = ((d[q][nb][0] >> q) << 8) + (d[q][nb][1] >> q);
             const int c1 = ((d[q][nb][2] >> q) << 8) + (d[q][nb][3] >> q);
-            const int o0 = ob * kUTileRows + 16 * q + g;
-            yacc[q][0][nb] += h2f(P.h[o0]) * (st * (float)(tsum - 2 * c0));
-            yacc[q][1][nb] += h2f(P.h[o0 + 8]) * (st * (float)(tsum - 2 * c1));
+            yacc[q][0][nb] += h2f(hs[16 * q + g]) * (st * (float)(tsum - 2 * c0));
+            yacc[q][1][nb] += h2f(hs[16 * q + g + 8]) * (st * (float)(tsum - 2 * c1));
           }
         }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) d[q][nb][0] = d[q][nb][1] = d[q][nb][2] = d[q][nb][3] = 0;
       }
-    }
+      if (cs.p == cs.npaths - 1) {
+        const LayerDesc& L = a.layers[cs.li];
+        const int ob = cs.item - cs.u_begin;
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      const int b = 4 * nb + c;
-      if (b < B) {
-        uint16_t* yr = L.y + (size_t)b * L.d_out + ob * kUTileRows + g;
+        for (int nb = 0; nb < NB; ++nb) {
+          const int b = 4 * nb + c;
+          if (b < B) {
+            uint16_t* yr = L.y + (size_t)b * L.d_out + ob * kUTileRows + g;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          yr[16 * q] = f2h(yacc[q][0][nb]);
-          yr[16 * q + 8] = f2h(yacc[q][1][nb]);
+            for (int q = 0; q < 8; ++q) {
+              yr[16 * q] = f2h(yacc[q][0][nb]);
+              yr[16 * q + 8] = f2h(yacc[q][1][nb]);
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q) yacc[q][0][nb] = yacc[q][1][nb] = 0.f;
         }
       }
     }
+    // the stage has been read: refill it with the chunk `S` ahead
+    __syncwarp();
+    if (fd.item < i_end) {
+      if (lane == 0) out_issue(a, fd, my_ring + slot * sb, &my_bar[slot], B);
+      fd.advance(a);
+    }
+    ++consumed;
+    cs.advance(a);
   }
 }
 
+// ------------------------------------------------------------------ launchers
+
+size_t latent_smem(int nb) {
+  return (size_t)kVWarps * kVStages * kChunkBytes + (size_t)kVSlice * 8 * nb +
+         (size_t)kMaxBatchDecode * kVRowChunk * 16 * 4 + (size_t)kVWarps * kVStages * 8;
+}
+
 template <int NB>
-size_t smem_bytes(int batch, int max_s16) {
-  return (size_t)kVSlice * 8 * NB + (size_t)batch * max_s16 * 4;
+size_t output_smem(int batch) {
+  return (size_t)kUWarps * OutCfg<NB>::kStages * out_stage_bytes(batch) + (size_t)kUWarps * OutCfg<NB>::kStages * 8;
 }
 
 template <int NB>
 cudaError_t launch_latent(const DecodeArgs& a, int max_s16, int num_sms, cudaStream_t st) {
-  const size_t smem = smem_bytes<NB>(a.batch, max_s16);
-  cudaError_t e = cudaFuncSetAttribute(latent_pass_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e != cudaSuccess) return e;
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, latent_pass_kernel<NB>, kVWarps * 32, smem);
-  if (e != cudaSuccess) return e;
-  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const size_t smem = latent_smem(NB);
+  if ((size_t)a.batch * max_s16 * 4 > (size_t)kVSlice * 8 * NB) return cudaErrorInvalidValue;   // t' fits bpl
+  static bool attr_set = false;
+  cudaError_t e;
+  if (!attr_set) {
+    e = cudaFuncSetAttribute(latent_pass_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, latent_pass_kernel<NB>, kVWarps * 32, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  }
   const int grid = max(1, min(a.v_items, per_sm * num_sms));
   latent_pass_kernel<NB><<<grid, kVWarps * 32, smem, st>>>(a);
   return cudaGetLastError();
@@ -413,22 +753,25 @@ cudaError_t launch_latent(const DecodeArgs& a, int max_s16, int num_sms, cudaStr
 
 template <int NB>
 cudaError_t launch_output(const DecodeArgs& a, int num_sms, cudaStream_t st) {
+  const size_t smem = output_smem<NB>(a.batch);
+  const size_t smem_max = output_smem<NB>(4 * NB);
+  static bool attr_set = false;
+  cudaError_t e;
+  if (!attr_set) {
+    e = cudaFuncSetAttribute(output_pass_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
   int per_sm = 0;
-  cudaError_t e =
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, output_pass_kernel<NB>, kUWarps * 32, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, output_pass_kernel<NB>, kUWarps * 32, smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
   const int grid = max(1, min((a.u_items + kUWarps - 1) / kUWarps, per_sm * num_sms));
-  output_pass_kernel<NB><<<grid, kUWarps * 32, 0, st>>>(a);
+  output_pass_kernel<NB><<<grid, kUWarps * 32, smem, st>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
-
-size_t latent_pass_smem(int batch, int max_s16) {
-  const int nb = (batch + 3) / 4;
-  return (size_t)kVSlice * 8 * nb + (size_t)batch * max_s16 * 4;
-}
 
 cudaError_t launch_latent_pass(const DecodeArgs& a, int max_s16, int num_sms, cudaStream_t st) {
   switch ((a.batch + 3) / 4) {

@@ -15,34 +15,50 @@ constexpr int kVTileRows = 16, kVTileK = 256;   // role-V tile
 constexpr int kUTileRows = 128, kUTileK = 32;   // role-U tile
 constexpr int kTileBytes = 512;
 
-// Latent pass (V^T) work unit: one CTA reduces kVSliceTiles role-V K-tiles
-// (kVSlice inputs) for every latent row of one path; warp w owns tiles
-// kVTilesPerWarp*w .. kVTilesPerWarp*w + kVTilesPerWarp - 1 of the slice.
+// Latent pass (V^T) work item: (layer, path, input slice, row chunk).  One CTA
+// of kVWarps warps covers kVSlice inputs; warp w owns the kVTilesPerWarp
+// K-tiles 4w..4w+3 of the slice and walks the kVRowChunk 16-row latent blocks
+// of the chunk.  Per 16-row block a warp's tiles are contiguous (2 KB), one
+// bulk copy.
 constexpr int kVWarps = 4;
 constexpr int kVTilesPerWarp = 4;
 constexpr int kVSliceTiles = kVWarps * kVTilesPerWarp;   // 16 tiles
 constexpr int kVSlice = kVSliceTiles * kVTileK;          // 4096 inputs
-// Output pass (U) work unit: one warp owns one 128-row block of one layer.
+constexpr int kVRowChunk = 8;                            // 16-row blocks per item
+constexpr int kVStages = 4;                              // bulk-copy ring per warp
+constexpr int kChunkTiles = 4;                           // tiles per bulk copy
+constexpr int kChunkBytes = kChunkTiles * kTileBytes;    // 2048
+
+// Output pass (U) work item: (layer, 128 output rows), one warp.
 constexpr int kUWarps = 4;
+
 // Quantisation of the int8 B operand: v = 256*hi + lo with hi, lo in [-128, 127]
 // needs |v| <= 32639.
 constexpr float kQMax = 32639.f;
+
+// Bounded waits: iterations of mbarrier.try_wait before a wait gives up.
+constexpr int kSpinLimit = 1 << 22;
 
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 inline int s16(int s) { return ceil_div(s, 16) * 16; }
 inline int s32(int s) { return ceil_div(s, 32) * 32; }
 
+// Quantised t' of one path, per batch row b: t'_j ~= step_b * (256*hi + lo).
+struct TStat {
+  float step;   // quantisation step
+  int sum;      // sum over j < s of (256*hi + lo)
+  int pad[2];
+};
+
 // Per-path scratch written by the latent pass and read by the output pass.
 //   partial : [n_slices][batch][s16] fp32  sums of one input slice
-//   planes  : [batch][2][s32] int8          t' = l*t quantised, hi and lo bytes
-//   tscale  : [batch] fp32                  t' ~= tscale * (256*hi + lo)
-//   tsum    : [batch] int32                 sum over j of (256*hi + lo)
-//   counter : slices of this path finished (reset to 0 by the last one)
+//   planes  : [s32/32][batch][2][32] int8   hi and lo bytes of t', K-tile major
+//   tstat   : [batch] TStat
+//   counter : items of this path finished (reset to 0 by the last one)
 struct PathScratch {
   float* partial;
   int8_t* planes;
-  float* tscale;
-  int32_t* tsum;
+  TStat* tstat;
   unsigned int* counter;
 };
 
@@ -61,21 +77,21 @@ struct LayerDesc {
   uint16_t* y;        // [batch][d_out] fp16
   int d_in, d_out, s, npaths;
   int n_slices;       // ceil(d_in / kVSlice)
+  int n_rchunks;      // ceil(s16 / 16 / kVRowChunk)
   int v_begin;        // first latent-pass work item of this layer
   int u_begin;        // first output-pass work item of this layer
-  int pad;
 };
 
 struct DecodeArgs {
   const LayerDesc* layers;  // device table
+  unsigned int* status;     // device error word (LB_ERR_TIMEOUT bit on a wait timeout)
   int n_layers;
   int batch;
-  int v_items;              // total latent-pass items (layer, path, slice)
+  int v_items;              // total latent-pass items
   int u_items;              // total output-pass items (layer, 128-row block)
 };
 
 // Launchers (decode.cu).  The batch selects the template (4 rows per n-block).
-size_t latent_pass_smem(int batch, int max_s16);
 cudaError_t launch_latent_pass(const DecodeArgs& a, int max_s16, int num_sms, cudaStream_t st);
 cudaError_t launch_output_pass(const DecodeArgs& a, int num_sms, cudaStream_t st);
 

@@ -55,32 +55,33 @@ lb_status check_layer(const lb_layer& L) {
     const lb_path& P = L.path[p];
     if (!P.V_bits || !P.U_bits || !P.h || !P.g || !P.l) return LB_ERR_ARG;
     if (!aligned(P.V_bits, 16) || !aligned(P.U_bits, 16)) return LB_ERR_ALIGN;
-    if (!aligned(P.h, 2) || !aligned(P.g, 2) || !aligned(P.l, 2)) return LB_ERR_ALIGN;
+    if (!aligned(P.h, 16) || !aligned(P.g, 16) || !aligned(P.l, 2)) return LB_ERR_ALIGN;
   }
   return LB_OK;
 }
 
 // Bytes of per-path scratch for one layer at this batch.
+size_t partial_bytes(const lb_layer& L, int batch) {
+  return align_up((size_t)lb::ceil_div(L.d_in, lb::kVSlice) * batch * lb::s16(L.s) * sizeof(float), 256);
+}
+size_t planes_bytes(const lb_layer& L, int batch) { return align_up((size_t)batch * 2 * lb::s32(L.s), 256); }
+size_t tstat_bytes(int batch) { return align_up((size_t)batch * sizeof(lb::TStat), 256); }
 size_t path_scratch_bytes(const lb_layer& L, int batch) {
-  const int n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
-  size_t b = 0;
-  b += align_up((size_t)n_slices * batch * lb::s16(L.s) * sizeof(float), 256);   // partial
-  b += align_up((size_t)batch * 2 * lb::s32(L.s), 256);                           // planes
-  b += align_up((size_t)batch * sizeof(float), 256);                              // tscale
-  b += align_up((size_t)batch * sizeof(int32_t), 256);                            // tsum
-  return b;
+  return partial_bytes(L, batch) + planes_bytes(L, batch) + tstat_bytes(batch);
 }
 
+constexpr size_t kStatusBytes = 256;   // device status word at the start of a workspace
+
 lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
-                         cudaStream_t st) {
+                         cudaStream_t st, cudaEvent_t between) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
 
-  // ---- sizes: [table][counters][per-path scratch...]
+  // ---- sizes: [status][table][counters][per-path scratch...]
   const size_t table_bytes = align_up((size_t)n * sizeof(lb::LayerDesc), 256);
   const size_t counter_bytes = align_up((size_t)n * 2 * sizeof(unsigned int), 256);
-  size_t total = table_bytes + counter_bytes;
+  size_t total = kStatusBytes + table_bytes + counter_bytes;
   int max_s16 = 16;
   for (int i = 0; i < n; ++i) {
     total += (size_t)(layers[i].residual + 1) * path_scratch_bytes(layers[i], batch);
@@ -108,8 +109,9 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
 
   // ---- descriptor table
   unsigned char* base = static_cast<unsigned char*>(ws.buf);
-  unsigned int* counters = reinterpret_cast<unsigned int*>(base + table_bytes);
-  size_t off = table_bytes + counter_bytes;
+  lb::LayerDesc* table = reinterpret_cast<lb::LayerDesc*>(base + kStatusBytes);
+  unsigned int* counters = reinterpret_cast<unsigned int*>(base + kStatusBytes + table_bytes);
+  size_t off = kStatusBytes + table_bytes + counter_bytes;
   std::vector<lb::LayerDesc> tab(n);
   int v_items = 0, u_items = 0;
   for (int i = 0; i < n; ++i) {
@@ -123,9 +125,10 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
     D.s = L.s;
     D.npaths = L.residual + 1;
     D.n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
+    D.n_rchunks = lb::ceil_div(lb::s16(L.s) / 16, lb::kVRowChunk);
     D.v_begin = v_items;
     D.u_begin = u_items;
-    v_items += D.npaths * D.n_slices;
+    v_items += D.npaths * D.n_slices * D.n_rchunks;
     u_items += L.d_out / lb::kUTileRows;
     for (int p = 0; p < D.npaths; ++p) {
       lb::PathDesc& P = D.p[p];
@@ -135,13 +138,11 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
       P.g = L.path[p].g;
       P.l = L.path[p].l;
       P.ws.partial = reinterpret_cast<float*>(base + off);
-      off += align_up((size_t)D.n_slices * batch * lb::s16(L.s) * sizeof(float), 256);
+      off += partial_bytes(L, batch);
       P.ws.planes = reinterpret_cast<int8_t*>(base + off);
-      off += align_up((size_t)batch * 2 * lb::s32(L.s), 256);
-      P.ws.tscale = reinterpret_cast<float*>(base + off);
-      off += align_up((size_t)batch * sizeof(float), 256);
-      P.ws.tsum = reinterpret_cast<int32_t*>(base + off);
-      off += align_up((size_t)batch * sizeof(int32_t), 256);
+      off += planes_bytes(L, batch);
+      P.ws.tstat = reinterpret_cast<lb::TStat*>(base + off);
+      off += tstat_bytes(batch);
       P.ws.counter = counters + 2 * i + p;
     }
   }
@@ -149,7 +150,7 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   if (ws.table.size() != tb || std::memcmp(ws.table.data(), tab.data(), tb) != 0) {
     // pageable source: the call returns once the bytes are staged, so `tab`
     // may go out of scope; stream order protects kernels still reading the table
-    e = cudaMemcpyAsync(ws.buf, tab.data(), tb, cudaMemcpyHostToDevice, st);
+    e = cudaMemcpyAsync(table, tab.data(), tb, cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return cuda_fail(e);
     // the counters' offset depends on the table size, so bytes that earlier
     // calls used as scratch may now hold counters: start them at zero
@@ -160,7 +161,8 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   }
 
   lb::DecodeArgs a;
-  a.layers = static_cast<const lb::LayerDesc*>(ws.buf);
+  a.layers = table;
+  a.status = reinterpret_cast<unsigned int*>(base);
   a.n_layers = n;
   a.batch = batch;
   a.v_items = v_items;
@@ -168,6 +170,10 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   const int sms = num_sms(dev);
   e = lb::launch_latent_pass(a, max_s16, sms, st);
   if (e != cudaSuccess) return cuda_fail(e);
+  if (between) {
+    e = cudaEventRecord(between, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   e = lb::launch_output_pass(a, sms, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return LB_OK;
@@ -202,8 +208,9 @@ lb_status littlebit_pack_signs(const void* src_dev, lb_dtype dt, int n_long, int
   return e == cudaSuccess ? LB_OK : cuda_fail(e);
 }
 
-lb_status littlebit_linear_forward_many(const lb_layer* layers, int n, const void* const* xs, void* const* ys,
-                                        int batch, lb_dtype xdt, void* stream) {
+lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, const void* const* xs,
+                                              void* const* ys, int batch, lb_dtype xdt, void* stream,
+                                              void* event_between) {
   if (!layers || !xs || !ys || n < 1) return LB_ERR_ARG;
   if (batch < 1) return LB_ERR_SHAPE;
   for (int i = 0; i < n; ++i) {
@@ -214,14 +221,39 @@ lb_status littlebit_linear_forward_many(const lb_layer* layers, int n, const voi
   }
   if (batch <= lb::kMaxBatchDecode) {
     if (xdt != LB_F16) return LB_ERR_UNSUPPORTED;
-    return decode_forward(layers, n, xs, ys, batch, static_cast<cudaStream_t>(stream));
+    return decode_forward(layers, n, xs, ys, batch, static_cast<cudaStream_t>(stream),
+                          static_cast<cudaEvent_t>(event_between));
   }
   return LB_ERR_UNSUPPORTED;
+}
+
+lb_status littlebit_linear_forward_many(const lb_layer* layers, int n, const void* const* xs, void* const* ys,
+                                        int batch, lb_dtype xdt, void* stream) {
+  return littlebit_linear_forward_many_timed(layers, n, xs, ys, batch, xdt, stream, nullptr);
 }
 
 lb_status littlebit_linear_forward(const lb_layer* layer, const void* x_dev, void* y_dev, int batch,
                                    lb_dtype xdt, void* stream) {
   return littlebit_linear_forward_many(layer, 1, &x_dev, &y_dev, batch, xdt, stream);
+}
+
+lb_status littlebit_device_status(void* stream, unsigned int* status) {
+  if (!status) return LB_ERR_ARG;
+  *status = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto it = g_ws.find({dev, st});
+  if (it == g_ws.end() || !it->second.buf) return LB_OK;
+  e = cudaMemcpy(status, it->second.buf, sizeof(unsigned int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaMemset(it->second.buf, 0, sizeof(unsigned int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return LB_OK;
 }
 
 void littlebit_release(void) {

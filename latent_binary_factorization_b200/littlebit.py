@@ -58,6 +58,13 @@ _lib.littlebit_linear_forward_many.argtypes = [ctypes.POINTER(LbLayer), ctypes.c
                                                ctypes.POINTER(ctypes.c_void_p),
                                                ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_int,
                                                ctypes.c_void_p]
+_lib.littlebit_linear_forward_many_timed.restype = ctypes.c_int
+_lib.littlebit_linear_forward_many_timed.argtypes = [ctypes.POINTER(LbLayer), ctypes.c_int,
+                                                     ctypes.POINTER(ctypes.c_void_p),
+                                                     ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_int,
+                                                     ctypes.c_void_p, ctypes.c_void_p]
+_lib.littlebit_device_status.restype = ctypes.c_int
+_lib.littlebit_device_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint)]
 _lib.littlebit_release.restype = None
 _lib.littlebit_release.argtypes = []
 _lib.littlebit_status_string.restype = ctypes.c_char_p
@@ -176,14 +183,28 @@ class Stack:
         self._xp = (ctypes.c_void_p * n)(*[x.data_ptr() for x in xs])
         self._yp = (ctypes.c_void_p * n)(*[y.data_ptr() for y in ys])
 
-    def __call__(self, stream=None) -> None:
-        _check(_lib.littlebit_linear_forward_many(self._arr, self._n, self._xp, self._yp, self.batch, self.dtype,
-                                                  _stream(stream)),
-               "littlebit_linear_forward_many")
+    def __call__(self, stream=None, event_between: torch.cuda.Event | None = None) -> None:
+        if event_between is None:
+            _check(_lib.littlebit_linear_forward_many(self._arr, self._n, self._xp, self._yp, self.batch,
+                                                      self.dtype, _stream(stream)),
+                   "littlebit_linear_forward_many")
+        else:
+            _check(_lib.littlebit_linear_forward_many_timed(self._arr, self._n, self._xp, self._yp, self.batch,
+                                                            self.dtype, _stream(stream),
+                                                            ctypes.c_void_p(event_between.cuda_event)),
+                   "littlebit_linear_forward_many_timed")
 
 
 def forward_many(layers: list, xs: list, ys: list, stream=None) -> None:
     Stack(layers, xs, ys)(stream)
+
+
+def device_status(stream=None) -> int:
+    """Wait for the stream and return (and clear) the device error bits its
+    forward kernels raised; 0 means none."""
+    out = ctypes.c_uint(0)
+    _check(_lib.littlebit_device_status(_stream(stream), ctypes.byref(out)), "littlebit_device_status")
+    return int(out.value)
 
 
 def release() -> None:

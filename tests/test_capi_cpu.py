@@ -75,13 +75,17 @@ def test_forward_rejects_bad_arguments_without_device_work(lib):
     L.s = 4
     assert f(ctypes.byref(L), x, x, 1, 0, None) == 1           # null factor pointers
     for p in range(2):
-        L.path[p] = lb.LbPath(16, 32, 2, 4, 6)
+        L.path[p] = lb.LbPath(16, 32, 64, 48, 6)
     L.residual = 2
     assert f(ctypes.byref(L), x, x, 1, 0, None) == 1           # residual must be 0/1
     L.residual = 0
-    L.path[0] = lb.LbPath(8, 32, 2, 4, 6)                       # V not 16-byte aligned
+    L.path[0] = lb.LbPath(8, 32, 64, 48, 6)                      # V not 16-byte aligned
     assert f(ctypes.byref(L), x, x, 1, 0, None) == 2
-    L.path[0] = lb.LbPath(16, 32, 2, 4, 6)
+    L.path[0] = lb.LbPath(16, 32, 64, 40, 6)                     # g not 16-byte aligned
+    assert f(ctypes.byref(L), x, x, 1, 0, None) == 2
+    L.path[0] = lb.LbPath(16, 32, 66, 48, 6)                     # h not 16-byte aligned
+    assert f(ctypes.byref(L), x, x, 1, 0, None) == 2
+    L.path[0] = lb.LbPath(16, 32, 64, 48, 6)
     assert f(ctypes.byref(L), ctypes.c_void_p(24), x, 1, 0, None) == 2   # x misaligned
     assert f(ctypes.byref(L), x, x, 0, 0, None) == 3           # batch 0
     assert f(ctypes.byref(L), x, x, 100, 0, None) == 6         # batch 17..255 unsupported

@@ -165,6 +165,15 @@ def test_forward_many_mixed_stack(lbm):
             _check(y, ref, f"layer {i}")
 
 
+def test_device_status_clean_after_forward(lbm):
+    lb, layers = lbm
+    paths = synth.layer(2048, 1024, 200, True, seed=4)
+    layer = layers.upload(paths, 2048, 1024, 200)
+    x = torch.from_numpy(synth.activations(3, 2048, seed=4)).cuda()
+    lb.forward(layer, x)
+    assert lb.device_status() == 0
+
+
 def test_repeatable_and_deterministic(lbm):
     lb, layers = lbm
     paths = synth.layer(4096, 4096, 86, True, seed=9)
