@@ -152,6 +152,30 @@ lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, con
                                               void* event_between);
 
 /*
+ * The decode forward of littlebit_linear_forward (one layer, 1 <= batch <= 16,
+ * fp16 x and y) for callers that cannot let the library allocate device
+ * memory: for example a process whose device memory is reserved up front by
+ * its own allocator, or a latency-critical loop that cannot absorb the
+ * device-wide synchronisation of cudaMalloc/cudaFree.  The pages describe no
+ * such interface; it has no counterpart in them.
+ *   - Allocates nothing.  Its scratch is one fixed 1 MiB device array inside
+ *     the library, held by every GPU that loads the library until the process
+ *     exits.  A layer whose latent-pass scratch (ceil(d_in/4096) * batch *
+ *     16*ceil(s/16) fp32 partials, plus t' bytes, per path) does not fit
+ *     returns LB_ERR_SHAPE.
+ *   - The first call on a device, with that device current, looks up the
+ *     array's device address (cudaGetSymbolAddress); make that first call
+ *     before any stream capture.
+ *   - Every call shares the array and the array keeps the last call's
+ *     contents; the call clears what must start at zero itself.  Calls whose
+ *     work overlaps on the GPU (other streams, other host threads) race on it
+ *     and give wrong results: serialise them.
+ * Arguments, alignment and other errors as littlebit_linear_forward.
+ */
+lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_dev, void* y_dev,
+                                           int batch, lb_dtype xdt, void* stream);
+
+/*
  * Waits for `stream`, then returns in *status the device-side error bits that
  * the forward kernels enqueued on it have raised since the last call, and
  * clears them.  Bit (1 << LB_ERR_TIMEOUT) means a bounded wait for a bulk copy
