@@ -32,7 +32,7 @@
 // (atomic ticket, no waiting) sums the partials in slice order, multiplies by
 // l and quantises t'.
 // Output pass: warp item = (layer, 128 output rows); each warp owns a
-// contiguous item range and streams it as chunks of up to 4 K-tiles, across
+// contiguous item range and streams it as chunks of up to 8 K-tiles, across
 // path, item and layer boundaries; the bulk copies also bring the chunk's t'
 // bytes and, for the last chunk of a path, the 128 h values and the
 // quantisation step.  Paths are added in fp32 and y is written in fp16.
@@ -71,14 +71,17 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// try_wait may suspend the warp for up to this long before reporting "not yet"
+constexpr uint32_t kWaitHintNs = 1000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitHintNs)
       : "memory");
   return ok != 0;
 }
@@ -104,6 +107,15 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
       "{%0,%1,%2,%3};"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D = A*B (accumulator starts at zero)
+__device__ __forceinline__ void mma_u8s8_zc(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
 
 __device__ __forceinline__ float2 h2x2(uint32_t v) {
@@ -387,39 +399,40 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_ker
           atomicOr(a.status, 1u << LB_ERR_TIMEOUT);
         }
         const unsigned char* stage = my_ring + slot * kChunkBytes;
-        uint4 cur[kVTilesPerWarp];
-#pragma unroll
-        for (int t = 0; t < kVTilesPerWarp; ++t)
-          cur[t] = t < nt ? *reinterpret_cast<const uint4*>(stage + t * kTileBytes + lane * 16)
-                          : make_uint4(0, 0, 0, 0);
         int d[8][NB][4];
+        // tile t of this warp's slice part, products q = 0..7 into d[q]
+        auto tile = [&](int t, bool first) {
+          const uint4 cur = *reinterpret_cast<const uint4*>(stage + t * kTileBytes + lane * 16);
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t m = 0x01010101u << q;
+            const uint32_t a0 = cur.x & m, a1 = cur.y & m, a2 = cur.z & m, a3 = cur.w & m;
 #pragma unroll
-          for (int nb = 0; nb < NB; ++nb) d[q][nb][0] = d[q][nb][1] = d[q][nb][2] = d[q][nb][3] = 0;
-#pragma unroll
-        for (int t = 0; t < kVTilesPerWarp; ++t) {
-          if (t < nt) {
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const uint32_t m = 0x01010101u << q;
-              const uint32_t a0 = cur[t].x & m, a1 = cur[t].y & m, a2 = cur[t].z & m, a3 = cur[t].w & m;
-#pragma unroll
-              for (int nb = 0; nb < NB; ++nb) {
-                uint32_t b0, b1;
-                if constexpr (NB == 1) {
-                  b0 = bf[t * 8 + q][0];
-                  b1 = bf[t * 8 + q][1];
-                } else {
-                  const int kb = (kVTilesPerWarp * warp + t) * 8 + q;
-                  const int8_t* base = bpl + ((size_t)kb * NCOL + nb * 8 + g) * 32 + 4 * c;
-                  b0 = *reinterpret_cast<const uint32_t*>(base);
-                  b1 = *reinterpret_cast<const uint32_t*>(base + 16);
-                }
-                mma_u8s8(d[q][nb], a0, a1, a2, a3, b0, b1);
+            for (int nb = 0; nb < NB; ++nb) {
+              uint32_t b0, b1;
+              if constexpr (NB == 1) {
+                b0 = bf[t * 8 + q][0];
+                b1 = bf[t * 8 + q][1];
+              } else {
+                const int kb = (kVTilesPerWarp * warp + t) * 8 + q;
+                const int8_t* base = bpl + ((size_t)kb * NCOL + nb * 8 + g) * 32 + 4 * c;
+                b0 = *reinterpret_cast<const uint32_t*>(base);
+                b1 = *reinterpret_cast<const uint32_t*>(base + 16);
               }
+              if (first) mma_u8s8_zc(d[q][nb], a0, a1, a2, a3, b0, b1);
+              else mma_u8s8(d[q][nb], a0, a1, a2, a3, b0, b1);
             }
           }
+        };
+        if (nt == kVTilesPerWarp) {
+          tile(0, true);
+#pragma unroll
+          for (int t = 1; t < kVTilesPerWarp; ++t) tile(t, false);
+        } else {
+          tile(0, true);   // nt >= 1 here
+#pragma unroll
+          for (int t = 1; t < kVTilesPerWarp; ++t)
+            if (t < nt) tile(t, false);
         }
         // the stage has been read (its words fed the products): refill it
         __syncwarp();
@@ -431,16 +444,21 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_ker
           feed.advance(a, warp, i_end);
         }
         ++consumed;
-        // fold: sum_q (256*D_hi + D_lo) / 2^q, Horner from q = 7 down (exact)
+        // fold: sum_q D_q / 2^q per plane, as 2^-7 * sum_q D_q * 2^(7-q) (Horner
+        // from q = 0; every term is a multiple of 2^7 because D_q is a multiple
+        // of 2^q), then 256 * hi + lo
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
-          int r0 = 256 * d[7][nb][0] + d[7][nb][1];
-          int r1 = 256 * d[7][nb][2] + d[7][nb][3];
+          int h0 = d[0][nb][0], l0 = d[0][nb][1], h1 = d[0][nb][2], l1 = d[0][nb][3];
 #pragma unroll
-          for (int q = 6; q >= 0; --q) {
-            r0 = (r0 >> 1) + 256 * d[q][nb][0] + d[q][nb][1];
-            r1 = (r1 >> 1) + 256 * d[q][nb][2] + d[q][nb][3];
+          for (int q = 1; q < 8; ++q) {
+            h0 = 2 * h0 + d[q][nb][0];
+            l0 = 2 * l0 + d[q][nb][1];
+            h1 = 2 * h1 + d[q][nb][2];
+            l1 = 2 * l1 + d[q][nb][3];
           }
+          const int r0 = 2 * h0 + (l0 >> 7);
+          const int r1 = 2 * h1 + (l1 >> 7);
           const int b = 4 * nb + c;
           if (b < B) {
             const int row = 16 * (rb - rb_lo) + g;
@@ -463,15 +481,18 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_ker
         if (bb == b) { st = step[bb]; vsum = vs[bb]; }
       part[(size_t)b * S16 + r] = st * (float)(vsum - 2 * acc[b * (kVRowChunk * 16) + r]);
     }
-    __threadfence();
     __syncthreads();
-    if (tid == 0)
+    if (tid == 0) {
+      // the barrier orders every thread's partial before this release; the
+      // last arriver's acquire then sees all slices of the path
+      __threadfence();
       s_last = (atomicAdd(P.ws.counter, 1u) == (unsigned)(L.n_slices * L.n_rchunks - 1));
+      __threadfence();
+    }
     __syncthreads();
 
     if (s_last) {
       // ---- last item of this path: t' = l * (sum of slice partials), quantised
-      __threadfence();
       float mt[4 * NB];
       int ts[4 * NB];
 #pragma unroll
@@ -531,25 +552,40 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_ker
 // output pass:  y_o = sum_p h_p[o] * sum_j U_p[o][j] t'_p[j]
 // ---------------------------------------------------------------------------
 
+constexpr int kUChunkTiles = 8;                           // K-tiles per bulk copy
+constexpr int kUChunkBytes = kUChunkTiles * kTileBytes;   // 4 KB
+
 template <int NB>
 struct OutCfg {
-  static constexpr int kStages = NB <= 2 ? 6 : 4;
+  static constexpr int kStages = NB == 1 ? 3 : 2;
 };
 
-// stage: [4 tiles: 2048][t' bytes: 4 K-tiles x B x 64][h: 256][tstat: 16 B]
-__host__ __device__ __forceinline__ int out_planes_off() { return kChunkBytes; }
-__host__ __device__ __forceinline__ int out_h_off(int B) { return kChunkBytes + kChunkTiles * B * 64; }
+// stage: [8 tiles: 4 KB][t' bytes: 8 K-tiles x B x 64][h: 256][tstat: 16 B per row]
+__host__ __device__ __forceinline__ int out_planes_off() { return kUChunkBytes; }
+__host__ __device__ __forceinline__ int out_h_off(int B) { return kUChunkBytes + kUChunkTiles * B * 64; }
 __host__ __device__ __forceinline__ int out_tstat_off(int B) { return out_h_off(B) + kUTileRows * 2; }
 __host__ __device__ __forceinline__ int out_stage_bytes(int B) {
   return (out_tstat_off(B) + 16 * B + 127) & ~127;
 }
 
-// Position in a warp's stream of output-pass chunks (up to 4 K-tiles of one
-// (item, path)), with the fields of the current layer cached.
+// Position in a warp's stream of output-pass chunks (up to 8 K-tiles of one
+// (item, path)), with the current layer's fields and the path's base
+// pointers cached so that issuing a chunk needs no descriptor loads.
 struct OutCursor {
   int li, item, p, kt0;
   int n_kt, npaths, u_begin, u_end;
+  const unsigned char* U;   // path p's tiles
+  const int8_t* planes;     // path p's t' bytes
+  const uint16_t* h;
+  const TStat* tstat;
 
+  __device__ __forceinline__ void set_path(const DecodeArgs& a) {
+    const PathDesc& P = a.layers[li].p[p];
+    U = reinterpret_cast<const unsigned char*>(P.U);
+    planes = P.ws.planes;
+    h = P.h;
+    tstat = P.ws.tstat;
+  }
   __device__ __forceinline__ void enter(const DecodeArgs& a, int l) {
     li = l;
     const LayerDesc& L = a.layers[l];
@@ -558,36 +594,54 @@ struct OutCursor {
     u_begin = L.u_begin;
     u_end = (l + 1 < a.n_layers) ? a.layers[l + 1].u_begin : a.u_items;
   }
-  __device__ __forceinline__ int ntile() const { return min(kChunkTiles, n_kt - kt0); }
-  __device__ __forceinline__ bool path_end() const { return kt0 + kChunkTiles >= n_kt; }
+  __device__ __forceinline__ int ntile() const { return min(kUChunkTiles, n_kt - kt0); }
+  __device__ __forceinline__ bool path_end() const { return kt0 + kUChunkTiles >= n_kt; }
   __device__ __forceinline__ void advance(const DecodeArgs& a) {
-    kt0 += kChunkTiles;
+    kt0 += kUChunkTiles;
     if (kt0 >= n_kt) {
       kt0 = 0;
       if (++p == npaths) {
         p = 0;
         if (++item == u_end && item < a.u_items) enter(a, li + 1);
       }
+      set_path(a);
     }
   }
 };
 
-__device__ __forceinline__ void out_issue(const DecodeArgs& a, const OutCursor& cu, unsigned char* stage,
-                                          uint64_t* bar, int B) {
-  const LayerDesc& L = a.layers[cu.li];
-  const PathDesc& P = L.p[cu.p];
+__device__ __forceinline__ void out_issue(const OutCursor& cu, unsigned char* stage, uint64_t* bar, int B) {
   const int ob = cu.item - cu.u_begin;
   const int nt = cu.ntile();
   const uint32_t tb = (uint32_t)nt * kTileBytes, pb = (uint32_t)nt * B * 64;
   const bool last = cu.path_end();
-  const uint32_t total = tb + pb + (last ? kUTileRows * 2 + 16 * B : 0);
-  mbar_expect_tx(bar, total);
-  bulk_g2s(stage, reinterpret_cast<const unsigned char*>(P.U) + ((size_t)ob * cu.n_kt + cu.kt0) * kTileBytes,
-           tb, bar);
-  bulk_g2s(stage + out_planes_off(), P.ws.planes + (size_t)cu.kt0 * B * 64, pb, bar);
+  mbar_expect_tx(bar, tb + pb + (last ? kUTileRows * 2 + 16 * B : 0));
+  bulk_g2s(stage, cu.U + ((size_t)ob * cu.n_kt + cu.kt0) * kTileBytes, tb, bar);
+  bulk_g2s(stage + out_planes_off(), cu.planes + (size_t)cu.kt0 * B * 64, pb, bar);
   if (last) {
-    bulk_g2s(stage + out_h_off(B), P.h + (size_t)ob * kUTileRows, kUTileRows * 2, bar);
-    bulk_g2s(stage + out_tstat_off(B), P.ws.tstat, 16 * B, bar);
+    bulk_g2s(stage + out_h_off(B), cu.h + (size_t)ob * kUTileRows, kUTileRows * 2, bar);
+    bulk_g2s(stage + out_tstat_off(B), cu.tstat, 16 * B, bar);
+  }
+}
+
+// One K-tile of one path: eight m16n8k32 products (row block q = 0..7).
+// `pl` points at this thread's t' bytes of tile t (batch row g/2, plane g%2);
+// `pl_step` = B * 64 bytes from one tile's t' bytes to the next.
+template <int NB>
+__device__ __forceinline__ void out_tile(int (&d)[8][NB][4], const unsigned char* stage, int t, int lane,
+                                         const unsigned char* pl, bool (&bval)[NB]) {
+  const uint4 cur = *reinterpret_cast<const uint4*>(stage + t * kTileBytes + lane * 16);
+  uint32_t b0[NB], b1[NB];
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    b0[nb] = bval[nb] ? *reinterpret_cast<const uint32_t*>(pl + nb * 256) : 0u;
+    b1[nb] = bval[nb] ? *reinterpret_cast<const uint32_t*>(pl + nb * 256 + 16) : 0u;
+  }
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const uint32_t m = 0x01010101u << q;
+    const uint32_t a0 = cur.x & m, a1 = cur.y & m, a2 = cur.z & m, a3 = cur.w & m;
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) mma_u8s8(d[q][nb], a0, a1, a2, a3, b0[nb], b1[nb]);
   }
 }
 
@@ -616,11 +670,12 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
   fd.item = i_begin;
   fd.p = 0;
   fd.kt0 = 0;
+  fd.set_path(a);
   OutCursor cs = fd;
 #pragma unroll 1
   for (int st = 0; st < S; ++st) {
     if (fd.item < i_end) {
-      if (lane == 0) out_issue(a, fd, my_ring + st * sb, &my_bar[st], B);
+      if (lane == 0) out_issue(fd, my_ring + st * sb, &my_bar[st], B);
       fd.advance(a);
     }
   }
@@ -635,36 +690,29 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
       d[q][nb][0] = d[q][nb][1] = d[q][nb][2] = d[q][nb][3] = 0;
     }
   uint32_t consumed = 0;
+  int slot = 0;
   bool dead = false;
+  // this thread's B-operand column: batch row 4nb + g/2, plane g%2
+  const int pl_off = out_planes_off() + ((g >> 1) * 2 + (g & 1)) * 32 + 4 * c;
+  const int pl_step = B * 64;
+  bool bval[NB];
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) bval[nb] = 4 * nb + (g >> 1) < B;
 
   while (cs.item < i_end) {
-    const int slot = consumed % S;
     if (!dead && !mbar_wait(&my_bar[slot], (consumed / S) & 1)) {
       dead = true;
       atomicOr(a.status, 1u << LB_ERR_TIMEOUT);
     }
     const unsigned char* stage = my_ring + slot * sb;
     const int nt = cs.ntile();
+    const unsigned char* pl = stage + pl_off;
+    if (nt == kUChunkTiles) {
 #pragma unroll
-    for (int t = 0; t < kChunkTiles; ++t) {
-      if (t < nt) {
-        const uint4 cur = *reinterpret_cast<const uint4*>(stage + t * kTileBytes + lane * 16);
-        uint32_t b0[NB], b1[NB];
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-          const int b = 4 * nb + (g >> 1);
-          const unsigned char* pl = stage + out_planes_off() + ((t * B + b) * 2 + (g & 1)) * 32 + 4 * c;
-          b0[nb] = b < B ? *reinterpret_cast<const uint32_t*>(pl) : 0u;
-          b1[nb] = b < B ? *reinterpret_cast<const uint32_t*>(pl + 16) : 0u;
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint32_t m = 0x01010101u << q;
-          const uint32_t a0 = cur.x & m, a1 = cur.y & m, a2 = cur.z & m, a3 = cur.w & m;
-#pragma unroll
-          for (int nb = 0; nb < NB; ++nb) mma_u8s8(d[q][nb], a0, a1, a2, a3, b0[nb], b1[nb]);
-        }
-      }
+      for (int t = 0; t < kUChunkTiles; ++t) out_tile<NB>(d, stage, t, lane, pl + t * pl_step, bval);
+    } else {
+#pragma unroll 1
+      for (int t = 0; t < nt; ++t) out_tile<NB>(d, stage, t, lane, pl + t * pl_step, bval);
     }
     if (cs.path_end()) {
       // path finished: rows 128*ob + 16q + g (+8), batch row 4nb + c
@@ -675,13 +723,14 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
         const int b = 4 * nb + c;
         if (b < B) {
           const float st = tst[b].step;
-          const int tsum = tst[b].sum;
+          const float base = st * (float)tst[b].sum;
+          const float m2 = -2.f * st;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const int c0 = ((d[q][nb][0] >> q) << 8) + (d[q][nb][1] >> q);
             const int c1 = ((d[q][nb][2] >> q) << 8) + (d[q][nb][3] >> q);
-            yacc[q][0][nb] += h2f(hs[16 * q + g]) * (st * (float)(tsum - 2 * c0));
-            yacc[q][1][nb] += h2f(hs[16 * q + g + 8]) * (st * (float)(tsum - 2 * c1));
+            yacc[q][0][nb] = fmaf(h2f(hs[16 * q + g]), fmaf(m2, (float)c0, base), yacc[q][0][nb]);
+            yacc[q][1][nb] = fmaf(h2f(hs[16 * q + g + 8]), fmaf(m2, (float)c1, base), yacc[q][1][nb]);
           }
         }
 #pragma unroll
@@ -709,10 +758,11 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
     // the stage has been read: refill it with the chunk `S` ahead
     __syncwarp();
     if (fd.item < i_end) {
-      if (lane == 0) out_issue(a, fd, my_ring + slot * sb, &my_bar[slot], B);
+      if (lane == 0) out_issue(fd, my_ring + slot * sb, &my_bar[slot], B);
       fd.advance(a);
     }
     ++consumed;
+    if (++slot == S) slot = 0;
     cs.advance(a);
   }
 }

@@ -36,7 +36,8 @@ constexpr int kUWarps = 4;
 // needs |v| <= 32639.
 constexpr float kQMax = 32639.f;
 
-// Bounded waits: iterations of mbarrier.try_wait before a wait gives up.
+// Bounded waits: polls of mbarrier.try_wait (each may suspend up to ~1 us)
+// before a wait gives up (a few seconds in total).
 constexpr int kSpinLimit = 1 << 22;
 
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
