@@ -133,9 +133,10 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(load)}
 
 
-def traffic_record(kernel: str, workload: str):
-    """dram bytes per launch of `kernel` from the committed ncu summary, if it
-    was taken on the current kernel source."""
+def traffic_record(kernel: str, workload: str, model_layers: int):
+    """dram bytes per launch of `kernel` from the committed ncu summary (bytes
+    per model layer x the model layers of this launch), if it was taken on the
+    current kernel source."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
@@ -148,7 +149,7 @@ def traffic_record(kernel: str, workload: str):
     r = rec.get(workload, {}).get(kernel)
     if not r or r.get("decode_cu_sha256_16") != digest:
         return None
-    return r.get("dram_bytes_per_launch")
+    return int(r["dram_bytes_per_model_layer"] * model_layers)
 
 
 # ---------------------------------------------------------------------------
@@ -313,7 +314,7 @@ def run_ours(args):
     dom_bytes = main["output_bytes"] if dom == "output_pass" else main["latent_bytes"]
     dom_ms = max(lat, out)
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
-    traffic = traffic_record(dom, args.workload)
+    traffic = traffic_record(dom, args.workload, main["model_layers_per_step"])
     value = 1e3 * main["ms_per_step"] / (n_layers * world)   # us per layer over all ranks' layers
     line = {
         "metric": METRIC,
