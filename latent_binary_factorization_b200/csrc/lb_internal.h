@@ -96,6 +96,11 @@ struct DecodeArgs {
 cudaError_t launch_latent_pass(const DecodeArgs& a, int max_s16, int num_sms, cudaStream_t st);
 cudaError_t launch_output_pass(const DecodeArgs& a, int num_sms, cudaStream_t st);
 
+// prefill.cu: one layer, M rows (multiple of 128), x fp16 or bf16 (y the same)
+size_t prefill_workspace_bytes(int M, int d_in, int d_out, int s, int npaths);
+cudaError_t launch_prefill(const LayerDesc& L, int M, const void* x, int x_bf16, void* y, unsigned char* ws,
+                           unsigned int* status, cudaStream_t st);
+
 // pack.cu
 cudaError_t launch_pack(const void* src, lb_dtype dt, int n_long, int s, int64_t stride_long,
                         int64_t stride_s, lb_role role, void* dst, cudaStream_t st);

@@ -179,6 +179,59 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   return LB_OK;
 }
 
+// Prefill (batch >= 128, multiple of 128): the tensor-core path, one layer
+// after the other on the stream, sharing one workspace.
+lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
+                          int x_bf16, cudaStream_t st) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  size_t need = 0;
+  for (int i = 0; i < n; ++i)
+    need = std::max(need, lb::prefill_workspace_bytes(batch, layers[i].d_in, layers[i].d_out, layers[i].s,
+                                                      layers[i].residual + 1));
+  need += kStatusBytes;
+  std::lock_guard<std::mutex> lock(g_mu);
+  Workspace& ws = g_ws[{dev, st}];
+  if (ws.cap < need) {
+    if (ws.buf) {
+      e = cudaStreamSynchronize(st);
+      if (e != cudaSuccess) return cuda_fail(e);
+      cudaFree(ws.buf);
+      ws.buf = nullptr;
+      ws.cap = 0;
+    }
+    const size_t cap = align_up(need + need / 4, 1 << 20);
+    e = cudaMalloc(&ws.buf, cap);
+    if (e != cudaSuccess) return cuda_fail(e);
+    ws.cap = cap;
+    e = cudaMemsetAsync(ws.buf, 0, cap, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  ws.table.clear();   // the decode table region is overwritten below
+  unsigned char* base = static_cast<unsigned char*>(ws.buf);
+  unsigned int* status = reinterpret_cast<unsigned int*>(base);
+  for (int i = 0; i < n; ++i) {
+    const lb_layer& L = layers[i];
+    lb::LayerDesc D;
+    std::memset(&D, 0, sizeof(D));
+    D.d_in = L.d_in;
+    D.d_out = L.d_out;
+    D.s = L.s;
+    D.npaths = L.residual + 1;
+    for (int p = 0; p < D.npaths; ++p) {
+      D.p[p].V = static_cast<const uint4*>(L.path[p].V_bits);
+      D.p[p].U = static_cast<const uint4*>(L.path[p].U_bits);
+      D.p[p].h = L.path[p].h;
+      D.p[p].g = L.path[p].g;
+      D.p[p].l = L.path[p].l;
+    }
+    e = lb::launch_prefill(D, batch, xs[i], x_bf16, ys[i], base + kStatusBytes, status, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return LB_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -223,6 +276,10 @@ lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, con
     if (xdt != LB_F16) return LB_ERR_UNSUPPORTED;
     return decode_forward(layers, n, xs, ys, batch, static_cast<cudaStream_t>(stream),
                           static_cast<cudaEvent_t>(event_between));
+  }
+  if (batch % 128 == 0) {
+    if (xdt != LB_F16 && xdt != LB_BF16) return LB_ERR_UNSUPPORTED;
+    return prefill_forward(layers, n, xs, ys, batch, xdt == LB_BF16 ? 1 : 0, static_cast<cudaStream_t>(stream));
   }
   return LB_ERR_UNSUPPORTED;
 }

@@ -1,0 +1,100 @@
+"""GPU parity of the prefill forward (batch >= 128, tcgen05 tensor cores)
+against the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import littlebit_oracle as orc
+from latent_binary_factorization_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 2e-3
+MAX_ABS = 1e-2
+
+
+@pytest.fixture(scope="module")
+def lbm():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from latent_binary_factorization_b200 import layers, littlebit
+    return littlebit, layers
+
+
+def _x(M, d_in, seed, dtype):
+    if dtype == torch.bfloat16:
+        xf = synth.activations(M, d_in, seed=seed, dtype="bf16")         # float32, bf16-exact
+        return torch.from_numpy(xf).to(torch.bfloat16), xf.astype(np.float64)
+    xh = synth.activations(M, d_in, seed=seed)
+    return torch.from_numpy(xh), xh.astype(np.float64)
+
+
+def _check(y, y_ref, tag):
+    a = y.float().cpu().numpy()
+    e, m = orc.rel_l2(a, y_ref), orc.max_abs_ratio(a, y_ref)
+    assert e <= REL_L2 and m <= MAX_ABS, f"{tag}: rel_l2={e:.3e} max_abs_ratio={m:.3e}"
+    return e
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("d_in,d_out,s,residual,M", [
+    (512, 512, 32, False, 128),      # tiny config, one tile
+    (512, 512, 32, True, 256),
+    (1024, 384, 100, True, 256),     # ragged N tile of GEMM2 (384 = 256 + 128), ragged rank
+    (768, 640, 1, False, 128),       # rank 1
+    (256, 128, 45, True, 384),       # smallest shapes
+])
+def test_prefill_small_full_output(lbm, dtype, d_in, d_out, s, residual, M):
+    lb, layers = lbm
+    paths = synth.layer(d_in, d_out, s, residual, seed=s + M)
+    layer = layers.upload(paths, d_in, d_out, s)
+    xt, x64 = _x(M, d_in, seed=s, dtype=dtype)
+    y = lb.forward(layer, xt.cuda())
+    torch.cuda.synchronize()
+    assert y.dtype == dtype
+    _check(y, orc.factored_forward(x64, paths), f"{d_in}x{d_out} s={s} M={M}")
+    assert lb.device_status() == 0
+
+
+@pytest.mark.parametrize("d_in,d_out,s", [(4096, 4096, 290), (4096, 11008, 431), (11008, 4096, 431)])
+def test_prefill_7b_0p3bpw_full_size_sampled_tokens(lbm, d_in, d_out, s):
+    """Llama-2-7B linear layers at 0.3 BPW with residual, M = 2048 bf16 tokens;
+    the oracle checks 64 sampled token rows over all outputs."""
+    lb, layers = lbm
+    paths = synth.layer(d_in, d_out, s, True, seed=d_out)
+    layer = layers.upload(paths, d_in, d_out, s)
+    xt, x64 = _x(2048, d_in, seed=7, dtype=torch.bfloat16)
+    y = lb.forward(layer, xt.cuda())
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(1).choice(2048, 64, replace=False))
+    _check(y[rows], orc.factored_forward(x64[rows], paths), f"7B {d_in}x{d_out}")
+
+
+def test_prefill_matches_decode_on_same_rows(lbm):
+    """The tensor-core prefill and the decode kernels agree row by row."""
+    lb, layers = lbm
+    paths = synth.layer(2048, 1024, 133, True, seed=3)
+    layer = layers.upload(paths, 2048, 1024, 133)
+    xt, _ = _x(128, 2048, seed=3, dtype=torch.float16)
+    y_pre = lb.forward(layer, xt.cuda())
+    y_dec = torch.cat([lb.forward(layer, xt[i:i + 16].cuda()) for i in range(0, 128, 16)])
+    torch.cuda.synchronize()
+    a, b = y_pre.float().cpu().numpy(), y_dec.float().cpu().numpy()
+    assert orc.rel_l2(a, b) <= 2 * REL_L2
+
+
+def test_prefill_forward_many(lbm):
+    lb, layers = lbm
+    specs = [(1024, 1024, 64, True), (1024, 2048, 100, False), (2048, 512, 77, True)]
+    L, X, Y, refs = [], [], [], []
+    for i, (a, b, s, r) in enumerate(specs):
+        paths = synth.layer(a, b, s, r, seed=50 + i, index=i)
+        xt, x64 = _x(256, a, seed=50 + i, dtype=torch.bfloat16)
+        L.append(layers.upload(paths, a, b, s))
+        X.append(xt.cuda())
+        Y.append(torch.empty(256, b, dtype=torch.bfloat16, device="cuda"))
+        refs.append(orc.factored_forward(x64, paths))
+    lb.Stack(L, X, Y)()
+    torch.cuda.synchronize()
+    for i, (y, ref) in enumerate(zip(Y, refs)):
+        _check(y, ref, f"layer {i}")
