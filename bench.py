@@ -267,6 +267,44 @@ def measure_workload(name, batch, steps, warmup, device, dist, world, l2, seed=1
     return res, (stack, x_all, y_all)
 
 
+PREFILL_MATS = [(4096, 4096, 290, True)] * 4 + [(4096, 11008, 431, True)] * 2 + [(11008, 4096, 431, True)]
+
+
+def measure_prefill(n_layers, M, steps, warmup, device, dist, seed=4321):
+    """Llama-2-7B full linear stack at 0.3 BPW residual (4096^2 at s=290;
+    4096<->11008 at s=431), M bf16 tokens per matrix, one forward_many per step."""
+    import torch
+    from latent_binary_factorization_b200 import layers as lbl, littlebit as lb
+    gen = torch.Generator(device=device).manual_seed(seed)
+    Ls, X, Y = [], [], []
+    for _ in range(n_layers):
+        for (a, b, s, r) in PREFILL_MATS:
+            Ls.append(lbl.random_layer(a, b, s, r, gen, device=device)[0])
+            X.append(torch.randn(M, a, generator=gen, device=device).to(torch.bfloat16))
+            Y.append(torch.empty(M, b, dtype=torch.bfloat16, device=device))
+    stack = lb.Stack(Ls, X, Y)
+    for _ in range(warmup):
+        stack()
+    torch.cuda.synchronize()
+    if dist:
+        torch.distributed.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        stack()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    if dist:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = t.item()
+    flops = sum(2 * M * s * (a + b) * (2 if r else 1) for a, b, s, r in PREFILL_MATS) * n_layers
+    del stack, Ls, X, Y
+    torch.cuda.empty_cache()
+    return ms, flops
+
+
 def run_ours(args):
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -306,6 +344,22 @@ def run_ours(args):
             torch.cuda.empty_cache()
             r["roofline_frac_step"] = r["step_gbs"] / peak
             extras[f"{name}_b{b}"] = r
+    prefill = None
+    if not args.no_prefill:
+        pms, pflops = measure_prefill(args.prefill_layers, 2048, max(3, args.steps // 20), 3, device, dist)
+        pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+            os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+        burst, sustained = float(pk.get("bf16_tflops", 1590.0)), float(pk.get("bf16_tflops_sustained", 1400.0))
+        tf = pflops / (pms * 1e-3) / 1e12 * world
+        prefill = {"workload": f"Llama-2-7B full linear stack at 0.3 BPW residual (4x 4096^2 s=290; 4096<->11008 "
+                               f"s=431), {args.prefill_layers} layers, M=2048 bf16 tokens per matrix",
+                   "ms_per_step": round(pms, 4), "tflops": round(tf, 1), "unit": "TFLOP/s",
+                   "algorithmic_flops_per_step": pflops,
+                   "roofline": {"bound": "tensor", "achieved": round(tf / world, 1), "peak": burst,
+                                "unit": "TFLOP/s", "frac": round(tf / world / burst, 4),
+                                "frac_of_sustained": round(tf / world / sustained, 4),
+                                "peak_source": "measured (MEASURED_PEAKS.json bf16_tflops, burst)",
+                                "note": "step-level: operand preparation + both tcgen05 GEMMs"}}
     clocks = sampler.stop()
 
     n_layers = main["layers_per_step"]
@@ -347,6 +401,7 @@ def run_ours(args):
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
         "extras": extras,
+        "prefill": prefill,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload, args.batch, budget_s=args.cpu_seconds)
@@ -446,6 +501,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill (tensor-core) measurement")
+    ap.add_argument("--prefill-layers", type=int, default=32)
     ap.add_argument("--l2-factor", type=float, default=4.0,
                     help="stack size as a multiple of the L2 cache (>= 1 keeps inputs larger than L2)")
     args = ap.parse_args()
