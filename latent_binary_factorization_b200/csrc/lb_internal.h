@@ -96,10 +96,12 @@ struct DecodeArgs {
 cudaError_t launch_latent_pass(const DecodeArgs& a, int max_s16, int num_sms, cudaStream_t st);
 cudaError_t launch_output_pass(const DecodeArgs& a, int num_sms, cudaStream_t st);
 
-// prefill.cu: one layer, M rows (multiple of 128), x fp16 or bf16 (y the same)
-size_t prefill_workspace_bytes(int M, int d_in, int d_out, int s, int npaths);
-cudaError_t launch_prefill(const LayerDesc& L, int M, const void* x, int x_bf16, void* y, unsigned char* ws,
-                           unsigned int* status, cudaStream_t st);
+// prefill.cu: layers of M rows (multiple of 128), x fp16 or bf16 (y the same)
+int prefill_sp(int s, int npaths);
+size_t prefill_layer_bytes(int M, int d_in, int d_out, int s, int npaths);
+size_t prefill_table_bytes(int n_layers);
+cudaError_t launch_prefill_group(const LayerDesc* Ls, const void* const* xs, void* const* ys, int n, int M,
+                                 int x_bf16, unsigned char* ws, unsigned int* status, int num_sms, cudaStream_t st);
 
 // pack.cu
 cudaError_t launch_pack(const void* src, lb_dtype dt, int n_long, int s, int64_t stride_long,

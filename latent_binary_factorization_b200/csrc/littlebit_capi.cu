@@ -179,18 +179,35 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   return LB_OK;
 }
 
-// Prefill (batch >= 128, multiple of 128): the tensor-core path, one layer
-// after the other on the stream, sharing one workspace.
+// Prefill (batch >= 128, multiple of 128): the tensor-core path.  Layers are
+// taken in groups whose operand buffers fit kPrefillGroupBytes; each group is
+// one set of operand preparations plus two grouped GEMM launches.
+constexpr size_t kPrefillGroupBytes = (size_t)4 << 30;
+
 lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
                           int x_bf16, cudaStream_t st) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
-  size_t need = 0;
-  for (int i = 0; i < n; ++i)
-    need = std::max(need, lb::prefill_workspace_bytes(batch, layers[i].d_in, layers[i].d_out, layers[i].s,
-                                                      layers[i].residual + 1));
-  need += kStatusBytes;
+  // plan the groups
+  std::vector<int> starts;
+  size_t need = 0, cur = 0;
+  int cnt = 0;
+  for (int i = 0; i < n; ++i) {
+    const size_t b = lb::prefill_layer_bytes(batch, layers[i].d_in, layers[i].d_out, layers[i].s,
+                                             layers[i].residual + 1);
+    if (cnt == 0 || cur + b > kPrefillGroupBytes || cnt == 4096) {
+      if (cnt) need = std::max(need, cur + lb::prefill_table_bytes(cnt));
+      starts.push_back(i);
+      cur = 0;
+      cnt = 0;
+    }
+    cur += b;
+    ++cnt;
+  }
+  need = std::max(need, cur + lb::prefill_table_bytes(cnt)) + kStatusBytes;
+  starts.push_back(n);
+
   std::lock_guard<std::mutex> lock(g_mu);
   Workspace& ws = g_ws[{dev, st}];
   if (ws.cap < need) {
@@ -201,7 +218,7 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
       ws.buf = nullptr;
       ws.cap = 0;
     }
-    const size_t cap = align_up(need + need / 4, 1 << 20);
+    const size_t cap = align_up(need + need / 8, 1 << 20);
     e = cudaMalloc(&ws.buf, cap);
     if (e != cudaSuccess) return cuda_fail(e);
     ws.cap = cap;
@@ -211,9 +228,10 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
   ws.table.clear();   // the decode table region is overwritten below
   unsigned char* base = static_cast<unsigned char*>(ws.buf);
   unsigned int* status = reinterpret_cast<unsigned int*>(base);
+  std::vector<lb::LayerDesc> descs(n);
   for (int i = 0; i < n; ++i) {
     const lb_layer& L = layers[i];
-    lb::LayerDesc D;
+    lb::LayerDesc& D = descs[i];
     std::memset(&D, 0, sizeof(D));
     D.d_in = L.d_in;
     D.d_out = L.d_out;
@@ -226,7 +244,12 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
       D.p[p].g = L.path[p].g;
       D.p[p].l = L.path[p].l;
     }
-    e = lb::launch_prefill(D, batch, xs[i], x_bf16, ys[i], base + kStatusBytes, status, st);
+  }
+  const int sms = num_sms(dev);
+  for (size_t gi = 0; gi + 1 < starts.size(); ++gi) {
+    const int i0 = starts[gi], cnt_g = starts[gi + 1] - starts[gi];
+    e = lb::launch_prefill_group(descs.data() + i0, xs + i0, ys + i0, cnt_g, batch, x_bf16, base + kStatusBytes,
+                                 status, sms, st);
     if (e != cudaSuccess) return cuda_fail(e);
   }
   return LB_OK;

@@ -36,7 +36,6 @@ constexpr int kBK = 64;           // K per stage
 constexpr int kStages = 4;
 constexpr int kABytes = kBM * kBK * 2;   // 16 KB
 constexpr int kBBytes = kBN * kBK * 2;   // 32 KB
-constexpr int kGemmThreads = 128;
 
 __host__ __device__ __forceinline__ size_t tiled_off(int r, int k, int R) {
   return ((size_t)(k >> 6) * (R >> 3) + (r >> 3)) * 1024 + ((k & 63) >> 3) * 128 + (r & 7) * 16 + (k & 7) * 2;
@@ -132,15 +131,19 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 
 // ------------------------------------------------------------------ operand preparation
 
-// x (M x K, fp16 or bf16, row-major, leading dimension K) -> fp16 core-matrix tiles
+// x (M x K, fp16 or bf16, row-major) -> fp16 core-matrix tiles.  Thread t
+// writes the 16-byte chunk t of the output; eight consecutive threads read
+// one 128-byte run of a row.
 __global__ void __launch_bounds__(256) prep_x_kernel(const uint16_t* __restrict__ x, int is_bf16, int M, int K,
                                                      unsigned char* __restrict__ out) {
-  const long long n16 = (long long)M * K / 8;   // 16-byte chunks
+  const long long n16 = (long long)M * K / 8;
+  const int rgs = M >> 3;
   for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < n16;
        t += (long long)gridDim.x * blockDim.x) {
-    // chunk t covers row r, columns 8c .. 8c+7 in row-major order
-    const int r = (int)(t / (K / 8));
-    const int k = (int)(t % (K / 8)) * 8;
+    const int kc = (int)(t & 7), rr = (int)((t >> 3) & 7);
+    const long long blk = t >> 6;               // (K-block, row-group) block of 1 KB
+    const int rg = (int)(blk % rgs), kb = (int)(blk / rgs);
+    const int r = 8 * rg + rr, k = 64 * kb + 8 * kc;
     uint4 v = *reinterpret_cast<const uint4*>(x + (size_t)r * K + k);
     if (is_bf16) {
       uint32_t* w = &v.x;
@@ -151,222 +154,297 @@ __global__ void __launch_bounds__(256) prep_x_kernel(const uint16_t* __restrict_
         w[e] = *reinterpret_cast<const uint32_t*>(&h);
       }
     }
-    *reinterpret_cast<uint4*>(out + tiled_off(r, k, M)) = v;
+    *reinterpret_cast<uint4*>(out + blk * 1024 + kc * 128 + rr * 16) = v;
   }
 }
 
-// B1 (P*Sp rows x d_in): row j' = p*Sp + j holds V_p[i][j] * g_p[i] (0 for j >= s)
+// B1 (P*Sp rows x d_in): row p*Sp + j holds V_p[i][j] * g_p[i].  One thread per
+// 16-byte lane of a packed role-V tile: its four words hold, for each q, four
+// consecutive i of one row, i.e. one 8-byte piece of B1.  Rows j >= s inside
+// the packed tiles get +-g (finite; GEMM1's epilogue zeroes them through l);
+// rows from the tiles' end up to Sp are zero.
 __global__ void __launch_bounds__(256) prep_b1_kernel(const LayerDesc L, int Sp, unsigned char* __restrict__ out) {
   const int R = L.npaths * Sp, K = L.d_in;
-  const int n_kt = K / kVTileK;
-  const long long n16 = (long long)R * K / 8;
-  for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < n16;
+  const int n_kt = K / kVTileK, n_rb = (L.s + 15) >> 4;
+  const long long lanes = (long long)L.npaths * n_rb * n_kt * 32;
+  const long long zero_rows = (long long)L.npaths * (Sp - 16 * n_rb);
+  const long long zeros = zero_rows * (K / 8);
+  for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < lanes + zeros;
        t += (long long)gridDim.x * blockDim.x) {
-    const int jr = (int)(t / (K / 8));
-    const int i0 = (int)(t % (K / 8)) * 8;
-    const int p = jr / Sp, j = jr - p * Sp;
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
-    if (j < L.s) {
-      const unsigned char* V = reinterpret_cast<const unsigned char*>(L.p[p].V);
+    if (t < lanes) {
+      const int lane = (int)(t & 31);
+      const long long tile = t >> 5;
+      const int p = (int)(tile / ((long long)n_rb * n_kt));
+      const int tt = (int)(tile - (long long)p * n_rb * n_kt);
+      const int rb = tt / n_kt, kt = tt - rb * n_kt;
+      const uint4 w4 = *reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned char*>(L.p[p].V) +
+                                                        (size_t)tt * kTileBytes + 16 * lane);
+      const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
       const uint16_t* g = L.p[p].g;
-      const int rb = j >> 4, jj = j & 15, gg = jj & 7, rlo = jj >> 3;
+      const int gg = lane >> 2, c = lane & 3;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int i = i0 + e;
-        const int kk = i & 255, q = kk >> 5, rem = kk & 31;
-        const int rhi = rem >> 4, c = (rem & 15) >> 2, m = rem & 3;
-        const int lane = 4 * gg + c, r = 2 * rhi + rlo;
-        const unsigned char byte = V[((size_t)rb * n_kt + (i >> 8)) * kTileBytes + 16 * lane + 4 * r + m];
-        const uint32_t bit = (byte >> q) & 1u;
-        const uint32_t val = (uint32_t)g[i] ^ (bit << 15);
-        w[e >> 1] |= val << (16 * (e & 1));
+      for (int r = 0; r < 4; ++r) {
+        const int jr = p * Sp + 16 * rb + gg + 8 * (r & 1);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int i0 = 256 * kt + 32 * q + 16 * (r >> 1) + 4 * c;
+          const uint2 gv = *reinterpret_cast<const uint2*>(g + i0);
+          const uint32_t bits = (wv[r] >> q) & 0x01010101u;   // byte m: bit of i0 + m
+          const uint32_t s0 = (bits & 1u) << 15, s1 = ((bits >> 8) & 1u) << 31;
+          const uint32_t s2 = ((bits >> 16) & 1u) << 15, s3 = ((bits >> 24) & 1u) << 31;
+          *reinterpret_cast<uint2*>(out + tiled_off(jr, i0, R)) = make_uint2(gv.x ^ (s0 | s1), gv.y ^ (s2 | s3));
+        }
       }
+    } else {
+      const long long z = t - lanes;
+      const int row_i = (int)(z / (K / 8)), k = (int)(z % (K / 8)) * 8;
+      const int per = Sp - 16 * n_rb;
+      const int p = row_i / per, jr = p * Sp + 16 * n_rb + (row_i - p * per);
+      *reinterpret_cast<uint4*>(out + tiled_off(jr, k, R)) = make_uint4(0u, 0u, 0u, 0u);
     }
-    *reinterpret_cast<uint4*>(out + tiled_off(jr, i0, R)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
-// B2 (d_out rows x P*Sp): column j' = p*Sp + j of row o holds U_p[o][j] * h_p[o]
+// B2 (d_out rows x P*Sp): row o, column p*Sp + j holds U_p[o][j] * h_p[o].  One
+// thread per 16-byte lane of a packed role-U tile: for each q its word gives
+// four consecutive j of one row.  Columns from the tiles' end up to Sp are zero.
 __global__ void __launch_bounds__(256) prep_b2_kernel(const LayerDesc L, int Sp, unsigned char* __restrict__ out) {
   const int R = L.d_out, K = L.npaths * Sp;
-  const int n_kt = (L.s + 31) >> 5;
-  const long long n16 = (long long)R * K / 8;
-  for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < n16;
+  const int n_kt = (L.s + 31) >> 5, n_ob = R / kUTileRows;
+  const long long lanes = (long long)L.npaths * n_ob * n_kt * 32;
+  const int zcols = Sp - 32 * n_kt;                       // zero columns per path
+  const long long zeros = (long long)L.npaths * R * (zcols / 8);
+  for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < lanes + zeros;
        t += (long long)gridDim.x * blockDim.x) {
-    const int o = (int)(t / (K / 8));
-    const int j0 = (int)(t % (K / 8)) * 8;
-    const int ob = o >> 7, oo = o & 127, q = oo >> 4, rr = oo & 15, gg = rr & 7, rlo = rr >> 3;
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (t < lanes) {
+      const int lane = (int)(t & 31);
+      const long long tile = t >> 5;
+      const int p = (int)(tile / ((long long)n_ob * n_kt));
+      const int tt = (int)(tile - (long long)p * n_ob * n_kt);
+      const int ob = tt / n_kt, kt = tt - ob * n_kt;
+      const uint4 w4 = *reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned char*>(L.p[p].U) +
+                                                        (size_t)tt * kTileBytes + 16 * lane);
+      const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+      const uint16_t* h = L.p[p].h;
+      const int gg = lane >> 2, c = lane & 3;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int jr = j0 + e, p = jr / Sp, j = jr - p * Sp;
-      if (j < L.s) {
-        const unsigned char* U = reinterpret_cast<const unsigned char*>(L.p[p].U);
-        const int kk = j & 31, rhi = kk >> 4, c = (kk & 15) >> 2, m = kk & 3;
-        const int lane = 4 * gg + c, r = 2 * rhi + rlo;
-        const unsigned char byte = U[((size_t)ob * n_kt + (j >> 5)) * kTileBytes + 16 * lane + 4 * r + m];
-        const uint32_t bit = (byte >> q) & 1u;
-        const uint32_t val = (uint32_t)L.p[p].h[o] ^ (bit << 15);
-        w[e >> 1] |= val << (16 * (e & 1));
+      for (int r = 0; r < 4; ++r) {
+        const int j0 = p * Sp + 32 * kt + 16 * (r >> 1) + 4 * c;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int o = kUTileRows * ob + 16 * q + gg + 8 * (r & 1);
+          const uint32_t hv = (uint32_t)h[o] * 0x00010001u;
+          const uint32_t bits = (wv[r] >> q) & 0x01010101u;
+          const uint32_t s0 = (bits & 1u) << 15, s1 = ((bits >> 8) & 1u) << 31;
+          const uint32_t s2 = ((bits >> 16) & 1u) << 15, s3 = ((bits >> 24) & 1u) << 31;
+          *reinterpret_cast<uint2*>(out + tiled_off(o, j0, R)) = make_uint2(hv ^ (s0 | s1), hv ^ (s2 | s3));
+        }
       }
+    } else {
+      const long long z = t - lanes;
+      const int per = R * (zcols / 8);
+      const int p = (int)(z / per);
+      const int zz = (int)(z - (long long)p * per);
+      const int o = zz / (zcols / 8), j = p * Sp + 32 * n_kt + (zz % (zcols / 8)) * 8;
+      *reinterpret_cast<uint4*>(out + tiled_off(o, j, R)) = make_uint4(0u, 0u, 0u, 0u);
     }
-    *reinterpret_cast<uint4*>(out + tiled_off(o, j0, R)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
-// ------------------------------------------------------------------ tcgen05 GEMM
+// ------------------------------------------------------------------ grouped persistent tcgen05 GEMM
+//
+// One launch computes every tile of a list of problems D = A * B^T (M x N,
+// fp32 in tensor memory).  Warp 0 lane 0 streams A/B stages with bulk copies,
+// warp 1 lane 0 issues tcgen05.mma, warps 2..5 drain the accumulator; two
+// 256-column accumulators alternate so a tile's epilogue overlaps the next
+// tile's products.
 
-struct GemmArgs {
+struct GemmProblem {
   const unsigned char* A;   // core-matrix tiles, M rows x K
   const unsigned char* B;   // core-matrix tiles, N rows x K
-  int M, N, K;
-  int mode;                 // 0: T' = l * acc -> fp16 tiles; 1: y = acc -> row-major
-  // mode 0
+  int M, N, K, mode;        // mode 0: T' = l * acc -> fp16 tiles; 1: y = acc -> row-major
   const uint16_t* l0;
   const uint16_t* l1;
   int s, Sp;
-  unsigned char* T;         // core-matrix tiles, M rows x N (N = P*Sp)
-  // mode 1
-  void* Y;                  // row-major M x N
+  unsigned char* T;         // mode 0 output, core-matrix tiles M x N
+  void* Y;                  // mode 1 output, row-major M x N
   int y_bf16;
+  int tiles_n, tile_begin;
+};
+
+struct GroupArgs {
+  const GemmProblem* probs;
+  int n_probs, total_tiles;
   unsigned int* status;
 };
 
-__global__ void __launch_bounds__(kGemmThreads, 1) umma_gemm_kernel(const GemmArgs g) {
+constexpr int kGroupThreads = 192;
+
+struct TileInfo {
+  const GemmProblem* P;
+  int m0, n0, n_len, nk;
+};
+
+__device__ __forceinline__ TileInfo tile_info(const GroupArgs& ga, int tile) {
+  int lo = 0, hi = ga.n_probs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (ga.probs[mid].tile_begin <= tile) lo = mid; else hi = mid - 1;
+  }
+  TileInfo ti;
+  ti.P = ga.probs + lo;
+  const int local = tile - ti.P->tile_begin;
+  const int mt = local / ti.P->tiles_n, nt = local - mt * ti.P->tiles_n;
+  ti.m0 = mt * kBM;
+  ti.n0 = nt * kBN;
+  ti.n_len = min(kBN, ti.P->N - ti.n0);
+  ti.nk = ti.P->K / kBK;
+  return ti;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su(b)) : "memory");
+}
+
+__global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const GroupArgs ga) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  unsigned char* sA = smem;                                   // [stages][16 KB]
-  unsigned char* sB = smem + kStages * kABytes;               // [stages][32 KB]
+  unsigned char* sA = smem;
+  unsigned char* sB = smem + kStages * kABytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * kBBytes);
   uint64_t* empty = full + kStages;
-  uint64_t* done = empty + kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* accf = empty + kStages;
+  uint64_t* acce = accf + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kBM, n0 = blockIdx.y * kBN;
-  const int n_len = min(kBN, g.N - n0);   // multiple of 16
-  const int nk = g.K / kBK;
-
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su(tmem_slot)),
-                 "r"(kBN)
+                 "r"(2 * kBN)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (threadIdx.x == 32) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
     }
-    mbar_init(done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&accf[i], 1);
+      mbar_init(&acce[i], 4);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  bool ok = true;
+  bool dead = false;
 
   if (threadIdx.x == 0) {
-    // ---- producer: one bulk copy per operand per stage
-    const uint32_t bbytes = (uint32_t)n_len * kBK * 2;
-    for (int kb = 0; kb < nk && ok; ++kb) {
-      const int st = kb % kStages;
-      if (kb >= kStages) ok = mbar_wait(&empty[st], ((kb / kStages) - 1) & 1);
-      if (!ok) break;
-      mbar_expect_tx(&full[st], kABytes + bbytes);
-      bulk_g2s(sA + st * kABytes, g.A + ((size_t)kb * (g.M >> 3) + (m0 >> 3)) * 1024, kABytes, &full[st]);
-      bulk_g2s(sB + st * kBBytes, g.B + ((size_t)kb * (g.N >> 3) + (n0 >> 3)) * 1024, bbytes, &full[st]);
+    // ---- producer
+    uint32_t it = 0;
+    for (int tile = blockIdx.x; tile < ga.total_tiles; tile += gridDim.x) {
+      const TileInfo ti = tile_info(ga, tile);
+      const uint32_t bbytes = (uint32_t)ti.n_len * kBK * 2;
+      const int Mg = ti.P->M >> 3, Ng = ti.P->N >> 3;
+      for (int kb = 0; kb < ti.nk; ++kb, ++it) {
+        const int st = it % kStages;
+        if (it >= kStages && !dead && !mbar_wait(&empty[st], ((it / kStages) - 1) & 1)) dead = true;
+        mbar_expect_tx(&full[st], kABytes + bbytes);
+        bulk_g2s(sA + st * kABytes, ti.P->A + ((size_t)kb * Mg + (ti.m0 >> 3)) * 1024, kABytes, &full[st]);
+        bulk_g2s(sB + st * kBBytes, ti.P->B + ((size_t)kb * Ng + (ti.n0 >> 3)) * 1024, bbytes, &full[st]);
+      }
     }
   } else if (threadIdx.x == 32) {
-    // ---- MMA issuer: 4 x (M=128, N=n_len, K=16) per stage
-    const uint32_t idesc = umma_idesc_f16(kBM, n_len);
-    for (int kb = 0; kb < nk && ok; ++kb) {
-      const int st = kb % kStages;
-      ok = mbar_wait(&full[st], (kb / kStages) & 1);
-      if (!ok) break;
+    // ---- MMA issuer
+    uint32_t it = 0, nt = 0;
+    for (int tile = blockIdx.x; tile < ga.total_tiles; tile += gridDim.x, ++nt) {
+      const TileInfo ti = tile_info(ga, tile);
+      const int ab = nt & 1;
+      if (nt >= 2 && !dead && !mbar_wait(&acce[ab], ((nt >> 1) - 1) & 1)) dead = true;
       tc_fence_after();
-      const uint32_t a0 = su(sA + st * kABytes), b0 = su(sB + st * kBBytes);
+      const uint32_t d = tmem + (uint32_t)(ab * kBN);
+      const uint32_t idesc = umma_idesc_f16(kBM, ti.n_len);
+      for (int kb = 0; kb < ti.nk; ++kb, ++it) {
+        const int st = it % kStages;
+        if (!dead && !mbar_wait(&full[st], (it / kStages) & 1)) dead = true;
+        tc_fence_after();
+        const uint32_t a0 = su(sA + st * kABytes), b0 = su(sB + st * kBBytes);
 #pragma unroll
-      for (int ks = 0; ks < kBK / 16; ++ks) {
-        const uint64_t ad = umma_desc(a0 + ks * 256, 128, 1024);
-        const uint64_t bd = umma_desc(b0 + ks * 256, 128, 1024);
-        umma_f16(tmem, ad, bd, idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < kBK / 16; ++ks)
+          umma_f16(d, umma_desc(a0 + ks * 256, 128, 1024), umma_desc(b0 + ks * 256, 128, 1024), idesc,
+                   (kb > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(&empty[st]);
       }
-      umma_commit(&empty[st]);   // stage free once these products are done
+      umma_commit(&accf[ab]);
     }
-    umma_commit(done);
+  } else if (warp >= 2) {
+    // ---- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
+    const int quarter = warp & 3;
+    uint32_t nt = 0;
+    for (int tile = blockIdx.x; tile < ga.total_tiles; tile += gridDim.x, ++nt) {
+      const TileInfo ti = tile_info(ga, tile);
+      const int ab = nt & 1;
+      if (!dead && !mbar_wait(&accf[ab], (nt >> 1) & 1)) dead = true;
+      dead = __any_sync(0xffffffffu, dead);
+      tc_fence_after();
+      const GemmProblem& P = *ti.P;
+      const int row = ti.m0 + 32 * quarter + lane;
+      const uint32_t taddr = tmem + (uint32_t)(ab * kBN) + ((uint32_t)(32 * quarter) << 16);
+      for (int c0 = 0; c0 < ti.n_len; c0 += 16) {
+        float v[16];
+        tmem_ld16(taddr + (uint32_t)c0, v);
+        uint32_t w[8];
+        if (P.mode == 0) {
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            float lv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int n = ti.n0 + c0 + e + u;
+              const int p = n / P.Sp, j = n - p * P.Sp;
+              const uint16_t* l = p == 0 ? P.l0 : P.l1;
+              lv[u] = j < P.s ? __half2float(__ushort_as_half(l[j])) : 0.f;
+            }
+            const __half2 hh = __floats2half2_rn(lv[0] * v[e], lv[1] * v[e + 1]);
+            w[e >> 1] = *reinterpret_cast<const uint32_t*>(&hh);
+          }
+          *reinterpret_cast<uint4*>(P.T + tiled_off(row, ti.n0 + c0, P.M)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(P.T + tiled_off(row, ti.n0 + c0 + 8, P.M)) =
+              make_uint4(w[4], w[5], w[6], w[7]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            if (P.y_bf16) {
+              const __nv_bfloat162 bb = __floats2bfloat162_rn(v[e], v[e + 1]);
+              w[e >> 1] = *reinterpret_cast<const uint32_t*>(&bb);
+            } else {
+              const __half2 hh = __floats2half2_rn(v[e], v[e + 1]);
+              w[e >> 1] = *reinterpret_cast<const uint32_t*>(&hh);
+            }
+          }
+          uint16_t* yr = static_cast<uint16_t*>(P.Y) + (size_t)row * P.N + ti.n0 + c0;
+          *reinterpret_cast<uint4*>(yr) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(yr + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[ab]);
+    }
+    if (dead && lane == 0) atomicOr(ga.status, 1u << LB_ERR_TIMEOUT);
   }
+  if ((threadIdx.x == 0 || threadIdx.x == 32) && dead) atomicOr(ga.status, 1u << LB_ERR_TIMEOUT);
   __syncwarp();
-
-  // ---- epilogue: warp w owns TMEM lanes 32w..32w+31 = tile rows
-  if (!mbar_wait(done, 0)) ok = false;
-  ok = __all_sync(0xffffffffu, ok);   // tcgen05.ld below needs the whole warp
-  if (!ok) {
-    if (lane == 0) atomicOr(g.status, 1u << LB_ERR_TIMEOUT);
-  } else {
-    tc_fence_after();
-    const int row = m0 + warp * 32 + lane;
-    const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
-    for (int c0 = 0; c0 < n_len; c0 += 16) {
-      float v[16];
-      tmem_ld16(taddr + (uint32_t)c0, v);
-      if (g.mode == 0) {
-        // T'[row][n] = l(n) * acc, n = n0 + c0 + e; two fp16 x 8 chunks
-        uint32_t w[8];
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          float lv[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int n = n0 + c0 + e + u;
-            const int p = n / g.Sp, j = n - p * g.Sp;
-            const uint16_t* l = p == 0 ? g.l0 : g.l1;
-            lv[u] = j < g.s ? __half2float(__ushort_as_half(l[j])) : 0.f;
-          }
-          const __half2 h = __floats2half2_rn(lv[0] * v[e], lv[1] * v[e + 1]);
-          w[e >> 1] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-        *reinterpret_cast<uint4*>(g.T + tiled_off(row, n0 + c0, g.M)) = make_uint4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<uint4*>(g.T + tiled_off(row, n0 + c0 + 8, g.M)) = make_uint4(w[4], w[5], w[6], w[7]);
-      } else {
-        uint32_t w[8];
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          if (g.y_bf16) {
-            const __nv_bfloat162 b = __floats2bfloat162_rn(v[e], v[e + 1]);
-            w[e >> 1] = *reinterpret_cast<const uint32_t*>(&b);
-          } else {
-            const __half2 h = __floats2half2_rn(v[e], v[e + 1]);
-            w[e >> 1] = *reinterpret_cast<const uint32_t*>(&h);
-          }
-        }
-        uint16_t* yr = static_cast<uint16_t*>(g.Y) + (size_t)row * g.N + n0 + c0;
-        *reinterpret_cast<uint4*>(yr) = make_uint4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<uint4*>(yr + 8) = make_uint4(w[4], w[5], w[6], w[7]);
-      }
-    }
-  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kBN) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kBN) : "memory");
   }
 }
 
-size_t gemm_smem() { return (size_t)kStages * (kABytes + kBBytes) + (2 * kStages + 1) * 8 + 16; }
-
-cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(umma_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem());
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
-  dim3 grid(g.M / kBM, (g.N + kBN - 1) / kBN);
-  umma_gemm_kernel<<<grid, kGemmThreads, gemm_smem(), st>>>(g);
-  return cudaGetLastError();
-}
+size_t group_smem() { return (size_t)kStages * (kABytes + kBBytes) + (2 * kStages + 4) * 8 + 16; }
 
 int grid_for(long long work, int per_block) {
   long long b = (work + per_block - 1) / per_block;
@@ -376,59 +454,74 @@ int grid_for(long long work, int per_block) {
 
 }  // namespace
 
-// One layer, M rows: prepare the three operands, then GEMM1 and GEMM2.
-// ws must hold prefill_workspace_bytes(...) bytes, 1 KB aligned.
-size_t prefill_workspace_bytes(int M, int d_in, int d_out, int s, int npaths) {
-  const int Sp = npaths == 2 ? s32(s) : ceil_div(s, 64) * 64;
-  const size_t NK = (size_t)npaths * Sp;
-  const size_t x16 = (size_t)M * d_in * 2, b1 = NK * d_in * 2, b2 = (size_t)d_out * NK * 2, t = (size_t)M * NK * 2;
-  return ((x16 + 1023) & ~1023ull) + ((b1 + 1023) & ~1023ull) + ((b2 + 1023) & ~1023ull) + ((t + 1023) & ~1023ull);
+int prefill_sp(int s, int npaths) { return npaths == 2 ? s32(s) : ceil_div(s, 64) * 64; }
+
+size_t prefill_layer_bytes(int M, int d_in, int d_out, int s, int npaths) {
+  const size_t NK = (size_t)npaths * prefill_sp(s, npaths);
+  auto a1k = [](size_t v) { return (v + 1023) & ~(size_t)1023; };
+  return a1k((size_t)M * d_in * 2) + a1k(NK * d_in * 2) + a1k((size_t)d_out * NK * 2) + a1k((size_t)M * NK * 2);
 }
 
-cudaError_t launch_prefill(const LayerDesc& L, int M, const void* x, int x_bf16, void* y, unsigned char* ws,
-                           unsigned int* status, cudaStream_t st) {
-  const int P = L.npaths;
-  const int Sp = P == 2 ? s32(L.s) : ceil_div(L.s, 64) * 64;
-  const int NK = P * Sp;
-  unsigned char* X16 = ws;
-  unsigned char* B1 = X16 + (((size_t)M * L.d_in * 2 + 1023) & ~1023ull);
-  unsigned char* B2 = B1 + (((size_t)NK * L.d_in * 2 + 1023) & ~1023ull);
-  unsigned char* T = B2 + (((size_t)L.d_out * NK * 2 + 1023) & ~1023ull);
+size_t prefill_table_bytes(int n_layers) { return ((size_t)2 * n_layers * sizeof(GemmProblem) + 1023) & ~(size_t)1023; }
 
-  prep_x_kernel<<<grid_for((long long)M * L.d_in / 8, 256), 256, 0, st>>>(static_cast<const uint16_t*>(x), x_bf16, M,
-                                                                          L.d_in, X16);
-  prep_b1_kernel<<<grid_for((long long)NK * L.d_in / 8, 256), 256, 0, st>>>(L, Sp, B1);
-  prep_b2_kernel<<<grid_for((long long)L.d_out * NK / 8, 256), 256, 0, st>>>(L, Sp, B2);
+// Prepare the operands of a group of layers and run GEMM1 and GEMM2 for all of
+// them, one grouped launch each.  `ws` holds, first, a table of 2n problems
+// (prefill_table_bytes(n)), then each layer's buffers (prefill_layer_bytes).
+cudaError_t launch_prefill_group(const LayerDesc* Ls, const void* const* xs, void* const* ys, int n, int M,
+                                 int x_bf16, unsigned char* ws, unsigned int* status, int num_sms, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(umma_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)group_smem());
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  GemmProblem* table_dev = reinterpret_cast<GemmProblem*>(ws);
+  unsigned char* buf = ws + prefill_table_bytes(n);
+  // host copies of the two problem lists
+  static thread_local GemmProblem host[2 * 4096];
+  if (n > 4096) return cudaErrorInvalidValue;
+  int tiles1 = 0, tiles2 = 0;
+  for (int i = 0; i < n; ++i) {
+    const LayerDesc& L = Ls[i];
+    const int P = L.npaths, Sp = prefill_sp(L.s, P), NK = P * Sp;
+    auto a1k = [](size_t v) { return (v + 1023) & ~(size_t)1023; };
+    unsigned char* X16 = buf;
+    unsigned char* B1 = X16 + a1k((size_t)M * L.d_in * 2);
+    unsigned char* B2 = B1 + a1k((size_t)NK * L.d_in * 2);
+    unsigned char* T = B2 + a1k((size_t)L.d_out * NK * 2);
+    buf = T + a1k((size_t)M * NK * 2);
+
+    prep_x_kernel<<<grid_for((long long)M * L.d_in / 8, 256), 256, 0, st>>>(static_cast<const uint16_t*>(xs[i]),
+                                                                            x_bf16, M, L.d_in, X16);
+    const long long l1 = (long long)P * ((L.s + 15) >> 4) * (L.d_in / kVTileK) * 32 +
+                         (long long)P * (Sp - 16 * ((L.s + 15) >> 4)) * (L.d_in / 8);
+    prep_b1_kernel<<<grid_for(l1, 256), 256, 0, st>>>(L, Sp, B1);
+    const long long l2 = (long long)P * (L.d_out / kUTileRows) * ((L.s + 31) >> 5) * 32 +
+                         (long long)P * L.d_out * ((Sp - 32 * ((L.s + 31) >> 5)) / 8);
+    prep_b2_kernel<<<grid_for(l2, 256), 256, 0, st>>>(L, Sp, B2);
+
+    GemmProblem& g1 = host[i];
+    g1 = GemmProblem{};
+    g1.A = X16; g1.B = B1; g1.M = M; g1.N = NK; g1.K = L.d_in; g1.mode = 0;
+    g1.l0 = L.p[0].l; g1.l1 = P == 2 ? L.p[1].l : L.p[0].l; g1.s = L.s; g1.Sp = Sp; g1.T = T;
+    g1.tiles_n = ceil_div(NK, kBN); g1.tile_begin = tiles1;
+    tiles1 += (M / kBM) * g1.tiles_n;
+    GemmProblem& g2 = host[n + i];
+    g2 = GemmProblem{};
+    g2.A = T; g2.B = B2; g2.M = M; g2.N = L.d_out; g2.K = NK; g2.mode = 1; g2.Y = ys[i]; g2.y_bf16 = x_bf16;
+    g2.tiles_n = ceil_div(L.d_out, kBN); g2.tile_begin = tiles2;
+    tiles2 += (M / kBM) * g2.tiles_n;
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-
-  GemmArgs g1 = {};
-  g1.A = X16;
-  g1.B = B1;
-  g1.M = M;
-  g1.N = NK;
-  g1.K = L.d_in;
-  g1.mode = 0;
-  g1.l0 = L.p[0].l;
-  g1.l1 = P == 2 ? L.p[1].l : L.p[0].l;
-  g1.s = L.s;
-  g1.Sp = Sp;
-  g1.T = T;
-  g1.status = status;
-  e = launch_gemm(g1, st);
+  e = cudaMemcpyAsync(table_dev, host, sizeof(GemmProblem) * 2 * n, cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return e;
-
-  GemmArgs g2 = {};
-  g2.A = T;
-  g2.B = B2;
-  g2.M = M;
-  g2.N = L.d_out;
-  g2.K = NK;
-  g2.mode = 1;
-  g2.Y = y;
-  g2.y_bf16 = x_bf16;
-  g2.status = status;
-  return launch_gemm(g2, st);
+  GroupArgs g1a{table_dev, n, tiles1, status};
+  umma_group_kernel<<<min(tiles1, num_sms), kGroupThreads, group_smem(), st>>>(g1a);
+  GroupArgs g2a{table_dev + n, n, tiles2, status};
+  umma_group_kernel<<<min(tiles2, num_sms), kGroupThreads, group_smem(), st>>>(g2a);
+  return cudaGetLastError();
 }
 
 }  // namespace lb
