@@ -190,6 +190,11 @@ __device__ __forceinline__ int find_layer(const DecodeArgs& a, int item, bool la
 // ---------------------------------------------------------------------------
 // latent pass:  t_j (partial over one slice) = sum_i V[i][j] g_i x_i
 // ---------------------------------------------------------------------------
+// CTA item = (layer, path, 2048-input slice, 8 latent row blocks).  The CTA
+// quantises g*x of the slice once into shared memory as B fragments; warp w
+// takes row blocks 2w, 2w+1 and accumulates their eight products per K-block
+// over the whole slice (one B fragment load feeds both blocks), then folds the
+// 2^q factors once and writes one fp32 partial per latent row.
 
 struct VItem {
   int li, p, sl, rc;
@@ -210,48 +215,79 @@ __device__ __forceinline__ VItem decode_v(const DecodeArgs& a, int item, int& li
   return it;
 }
 
-// Walks one warp's sequence of bulk-copy chunks (one per 16-row block it owns).
+// Row blocks a warp processes at once: two share each B-fragment load; with
+// more than four batch rows the accumulators would not fit, so one.
+template <int NB>
+struct VCfg {
+  static constexpr int kRPW = NB == 1 ? 2 : 1;
+};
+
+// One warp's sequence of bulk-copy chunks: per item, per group of kRPW row
+// blocks, per 4 K-tiles of the slice.
+template <int NB>
 struct VFeed {
-  int item, li, rb, rb_hi, row_stride;   // row_stride: bytes from one 16-row block to the next
-  uint32_t bytes;                        // this warp's tiles per row block * 512
-  const unsigned char* base;             // this warp's first tile at row block 0
+  static constexpr int RPW = VCfg<NB>::kRPW;
+  int item, li, grp, kc;
+  int rb0, n_rb, n_kt_all, kt0, nkt;   // current item
+  const unsigned char* V;
 
   __device__ __forceinline__ void set(const DecodeArgs& a, int warp) {
     const VItem it = decode_v(a, item, li);
     const LayerDesc& L = a.layers[li];
-    const int k0 = it.sl * kVSlice, klen = min(kVSlice, L.d_in - k0);
-    const int nt = max(0, min(kVTilesPerWarp, klen / kVTileK - kVTilesPerWarp * warp));
-    row_stride = (L.d_in / kVTileK) * kTileBytes;
-    rb = it.rc * kVRowChunk;
-    rb_hi = min((L.s + 15) >> 4, rb + kVRowChunk);
-    bytes = (uint32_t)nt * kTileBytes;
-    base = reinterpret_cast<const unsigned char*>(L.p[it.p].V) +
-           (size_t)(k0 / kVTileK + kVTilesPerWarp * warp) * kTileBytes;
+    const int k0 = it.sl * kVSlice;
+    nkt = min(kVSliceTiles, (L.d_in - k0) / kVTileK);
+    n_kt_all = L.d_in / kVTileK;
+    kt0 = k0 / kVTileK;
+    n_rb = (L.s + 15) >> 4;
+    rb0 = it.rc * kVRowChunk + 2 * warp;
+    V = reinterpret_cast<const unsigned char*>(L.p[it.p].V);
+    grp = 0;
+    kc = 0;
   }
+  __device__ __forceinline__ int rb() const { return rb0 + grp * RPW; }
+  __device__ __forceinline__ bool valid() const { return rb() < n_rb; }
   __device__ __forceinline__ void normalize(const DecodeArgs& a, int warp, int end) {
-    while (item < end && (bytes == 0 || rb >= rb_hi)) {
+    while (item < end && !valid()) {
       if (++item < end) set(a, warp);
     }
   }
   __device__ __forceinline__ void advance(const DecodeArgs& a, int warp, int end) {
-    ++rb;
+    if (++kc * kChunkTiles >= nkt) {
+      kc = 0;
+      if (++grp * RPW >= 2) {
+        if (++item < end) set(a, warp);
+      }
+    }
     normalize(a, warp, end);
   }
-  __device__ __forceinline__ const unsigned char* src() const { return base + (size_t)rb * row_stride; }
+  // issue this chunk: up to RPW row blocks x ntile K-tiles into `stage`
+  __device__ __forceinline__ void issue(unsigned char* stage, uint64_t* bar) const {
+    const int ntile = min(kChunkTiles, nkt - kc * kChunkTiles);
+    const uint32_t bytes = (uint32_t)ntile * kTileBytes;
+    int nrb = 0;
+#pragma unroll
+    for (int r = 0; r < RPW; ++r)
+      if (rb() + r < n_rb) ++nrb;
+    mbar_expect_tx(bar, bytes * nrb);
+#pragma unroll
+    for (int r = 0; r < RPW; ++r)
+      if (rb() + r < n_rb)
+        bulk_g2s(stage + r * kChunkBytes,
+                 V + ((size_t)(rb() + r) * n_kt_all + kt0 + kc * kChunkTiles) * kTileBytes, bytes, bar);
+  }
 };
 
 template <int NB>
 __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_kernel(const DecodeArgs a) {
   constexpr int NCOL = 8 * NB;
+  constexpr int RPW = VCfg<NB>::kRPW;
+  constexpr int kStageBytes = RPW * kChunkBytes;
   extern __shared__ __align__(1024) unsigned char smem[];
-  unsigned char* ring = smem;                                                         // [warps][stages][2 KB]
-  int8_t* bpl = reinterpret_cast<int8_t*>(smem + kVWarps * kVStages * kChunkBytes);  // [128][NCOL][32]
-  int* acc = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(bpl) + (size_t)kVSlice * NCOL);  // [16][128]
-  uint64_t* mbar = reinterpret_cast<uint64_t*>(acc + kMaxBatchDecode * kVRowChunk * 16);               // [warps][stages]
-  float* tp = reinterpret_cast<float*>(bpl);   // finalize: [B][S16] fp32 (bpl is free then)
+  unsigned char* ring = smem;                                                          // [warps][stages][RPW x 2 KB]
+  uint2* bst = reinterpret_cast<uint2*>(smem + kVWarps * kVStages * kStageBytes);    // [64][NCOL][4] (b0, b1)
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(bst) + (size_t)kVSlice * NCOL);
   __shared__ float s_mx[kVWarps][16];
   __shared__ int s_sm[kVWarps][16];
-  __shared__ int s_last;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
   const int B = a.batch;
@@ -259,7 +295,7 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_ker
   const int i_end = (int)((long long)a.v_items * (blockIdx.x + 1) / gridDim.x);
   if (i_begin >= i_end) return;   // uniform over the CTA
 
-  unsigned char* my_ring = ring + (size_t)warp * kVStages * kChunkBytes;
+  unsigned char* my_ring = ring + (size_t)warp * kVStages * kStageBytes;
   uint64_t* my_bar = mbar + warp * kVStages;
   if (lane == 0) {
     for (int st = 0; st < kVStages; ++st) mbar_init(&my_bar[st], 1);
@@ -267,9 +303,8 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_ker
   }
   __syncwarp();
 
-  // prime this warp's ring
   const int li0 = find_layer(a, i_begin, true);
-  VFeed feed;
+  VFeed<NB> feed;
   feed.item = i_begin;
   feed.li = li0;
   feed.set(a, warp);
@@ -277,39 +312,36 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_ker
 #pragma unroll 1
   for (int st = 0; st < kVStages; ++st) {
     if (feed.item < i_end) {
-      if (lane == 0) {
-        mbar_expect_tx(&my_bar[st], feed.bytes);
-        bulk_g2s(my_ring + st * kChunkBytes, feed.src(), feed.bytes, &my_bar[st]);
-      }
+      if (lane == 0) feed.issue(my_ring + st * kStageBytes, &my_bar[st]);
       feed.advance(a, warp, i_end);
     }
   }
   uint32_t consumed = 0;
+  int slot = 0;
   bool dead = false;
 
   int li = li0;
   int prev_li = -1, prev_p = -1, prev_sl = -1;   // slice whose B operand is staged
   float step[4 * NB];
   int vs[4 * NB];
-  uint32_t bf[NB == 1 ? kVTilesPerWarp * 8 : 1][2];
 
   for (int item = i_begin; item < i_end; ++item) {
     const VItem it = decode_v(a, item, li);
     const LayerDesc& L = a.layers[li];
     const PathDesc& P = L.p[it.p];
     const int d_in = L.d_in, s = L.s;
-    const int S16 = (s + 15) & ~15;
+    const int S16 = (s + 15) & ~15, n_rb = S16 >> 4;
     const int k0 = it.sl * kVSlice;
     const int klen = min(kVSlice, d_in - k0);   // multiple of 256
-    const int nt = max(0, min(kVTilesPerWarp, klen / kVTileK - kVTilesPerWarp * warp));
-    const int rb_lo = it.rc * kVRowChunk, rb_hi = min(S16 >> 4, rb_lo + kVRowChunk);
-    const int nrow = 16 * (rb_hi - rb_lo);
+    const int nkt = klen / kVTileK;
 
     if (it.li != prev_li || it.p != prev_p || it.sl != prev_sl) {
-      // ---- u = g * x on the slice, quantised per batch row to 16 bits and
-      //      staged as int8 hi/lo B-operand columns (all loads issue up front)
-      constexpr int kChunks = kVSlice / 8 / (kVWarps * 32);
+      // ---- u = g * x on the slice, quantised per batch row to 16 bits, staged
+      //      as (b0, b1) B-fragment pairs: column n = 2*(row%4) (+1 for lo) of
+      //      n-block row/4, K-block kb = k/32, thread column c
+      constexpr int kChunks = kVSlice / 8 / (kVWarps * 32);   // 8-input chunks per thread
       const int nchunk = klen / 8;
+      __syncthreads();   // previous users of the staging area are done
       uint4 gq[kChunks];
 #pragma unroll
       for (int i = 0; i < kChunks; ++i) {
@@ -362,189 +394,187 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_ker
               lo[e >> 1] |= ((uint32_t)(uint8_t)l0 | ((uint32_t)(uint8_t)l1 << 8)) << sh;
             }
             if (ch < nchunk) {
-              const int k = 8 * ch;
-              int8_t* col = bpl + ((size_t)(k >> 5) * NCOL + bg * 8 + 2 * r) * 32 + (k & 31);
-              *reinterpret_cast<uint2*>(col) = make_uint2(hi[0], hi[1]);
-              *reinterpret_cast<uint2*>(col + 32) = make_uint2(lo[0], lo[1]);
+              // inputs 8ch..8ch+7: K-block kb, within-block offset kk0 (0, 8, 16, 24);
+              // kk < 16 -> b0 bytes of columns c = kk/4, else b1 bytes of c = (kk-16)/4
+              const int kb = ch >> 2, kk0 = (ch & 3) * 8;
+              const int cc = (kk0 & 15) >> 2, half = kk0 >> 4;
+              uint32_t* base_hi = reinterpret_cast<uint32_t*>(bst + ((size_t)kb * NCOL + bg * 8 + 2 * r) * 4);
+              uint32_t* base_lo = reinterpret_cast<uint32_t*>(bst + ((size_t)kb * NCOL + bg * 8 + 2 * r + 1) * 4);
+              base_hi[2 * cc + half] = hi[0];
+              base_hi[2 * (cc + 1) + half] = hi[1];
+              base_lo[2 * cc + half] = lo[0];
+              base_lo[2 * (cc + 1) + half] = lo[1];
             }
           }
           vs[4 * bg + r] = vsum;
         }
       }
-      block_sum<4 * NB>(vs, s_sm);   // ends with __syncthreads: bpl complete
-      if constexpr (NB == 1) {
-#pragma unroll
-        for (int t = 0; t < kVTilesPerWarp; ++t)
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int kb = (kVTilesPerWarp * warp + t) * 8 + q;
-            const int8_t* base = bpl + ((size_t)kb * NCOL + g) * 32 + 4 * c;
-            bf[t * 8 + q][0] = *reinterpret_cast<const uint32_t*>(base);
-            bf[t * 8 + q][1] = *reinterpret_cast<const uint32_t*>(base + 16);
-          }
-      }
+      block_sum<4 * NB>(vs, s_sm);   // ends with __syncthreads: staging complete
       prev_li = it.li;
       prev_p = it.p;
       prev_sl = it.sl;
     }
-    for (int i = tid; i < B * kVRowChunk * 16; i += kVWarps * 32) acc[i] = 0;
-    __syncthreads();
 
-    // ---- this warp's tiles for every 16-row block of the chunk
-    if (nt > 0) {
-      for (int rb = rb_lo; rb < rb_hi; ++rb) {
-        const int slot = consumed % kVStages;
+    // ---- this warp's row blocks over the slice
+#pragma unroll 1
+    for (int grp = 0; grp * RPW < 2; ++grp) {
+      const int rbA = it.rc * kVRowChunk + 2 * warp + grp * RPW;
+      if (rbA >= n_rb) break;
+      const bool hasB = RPW == 2 && rbA + 1 < n_rb;
+      int d[RPW][8][NB][4];
+#pragma unroll 1
+      for (int kc = 0; kc * kChunkTiles < nkt; ++kc) {
         if (!dead && !mbar_wait(&my_bar[slot], (consumed / kVStages) & 1)) {
           dead = true;
           atomicOr(a.status, 1u << LB_ERR_TIMEOUT);
         }
-        const unsigned char* stage = my_ring + slot * kChunkBytes;
-        int d[8][NB][4];
-        // tile t of this warp's slice part, products q = 0..7 into d[q]
-        auto tile = [&](int t, bool first) {
-          const uint4 cur = *reinterpret_cast<const uint4*>(stage + t * kTileBytes + lane * 16);
+        const unsigned char* stage = my_ring + slot * kStageBytes;
+        const int ntile = min(kChunkTiles, nkt - kc * kChunkTiles);
+        // one K-tile of the chunk for both row blocks
+        auto ktile = [&](int t, bool first) {
+          uint4 cur[RPW];
+#pragma unroll
+          for (int r = 0; r < RPW; ++r)
+            cur[r] = (r == 0 || hasB) ? *reinterpret_cast<const uint4*>(stage + r * kChunkBytes + t * kTileBytes + lane * 16)
+                                      : make_uint4(0, 0, 0, 0);
+          const int kb0 = (kc * kChunkTiles + t) * 8;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const uint32_t m = 0x01010101u << q;
-            const uint32_t a0 = cur.x & m, a1 = cur.y & m, a2 = cur.z & m, a3 = cur.w & m;
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) {
-              uint32_t b0, b1;
-              if constexpr (NB == 1) {
-                b0 = bf[t * 8 + q][0];
-                b1 = bf[t * 8 + q][1];
-              } else {
-                const int kb = (kVTilesPerWarp * warp + t) * 8 + q;
-                const int8_t* base = bpl + ((size_t)kb * NCOL + nb * 8 + g) * 32 + 4 * c;
-                b0 = *reinterpret_cast<const uint32_t*>(base);
-                b1 = *reinterpret_cast<const uint32_t*>(base + 16);
+              const uint2 bb = bst[((size_t)(kb0 + q) * NCOL + nb * 8 + g) * 4 + c];
+#pragma unroll
+              for (int r = 0; r < RPW; ++r) {
+                if (r == 0 || hasB) {
+                  const uint32_t a0 = cur[r].x & m, a1 = cur[r].y & m, a2 = cur[r].z & m, a3 = cur[r].w & m;
+                  if (first) mma_u8s8_zc(d[r][q][nb], a0, a1, a2, a3, bb.x, bb.y);
+                  else mma_u8s8(d[r][q][nb], a0, a1, a2, a3, bb.x, bb.y);
+                }
               }
-              if (first) mma_u8s8_zc(d[q][nb], a0, a1, a2, a3, b0, b1);
-              else mma_u8s8(d[q][nb], a0, a1, a2, a3, b0, b1);
             }
           }
         };
-        if (nt == kVTilesPerWarp) {
-          tile(0, true);
+        if (kc == 0) ktile(0, true); else ktile(0, false);
+        if (ntile == kChunkTiles) {
 #pragma unroll
-          for (int t = 1; t < kVTilesPerWarp; ++t) tile(t, false);
+          for (int t = 1; t < kChunkTiles; ++t) ktile(t, false);
         } else {
-          tile(0, true);   // nt >= 1 here
-#pragma unroll
-          for (int t = 1; t < kVTilesPerWarp; ++t)
-            if (t < nt) tile(t, false);
+#pragma unroll 1
+          for (int t = 1; t < ntile; ++t) ktile(t, false);
         }
-        // the stage has been read (its words fed the products): refill it
+        // the stage has been read: refill it
         __syncwarp();
         if (feed.item < i_end) {
-          if (lane == 0) {
-            mbar_expect_tx(&my_bar[slot], feed.bytes);
-            bulk_g2s(my_ring + slot * kChunkBytes, feed.src(), feed.bytes, &my_bar[slot]);
-          }
+          if (lane == 0) feed.issue(my_ring + slot * kStageBytes, &my_bar[slot]);
           feed.advance(a, warp, i_end);
         }
         ++consumed;
-        // fold: sum_q D_q / 2^q per plane, as 2^-7 * sum_q D_q * 2^(7-q) (Horner
-        // from q = 0; every term is a multiple of 2^7 because D_q is a multiple
-        // of 2^q), then 256 * hi + lo
+        if (++slot == kVStages) slot = 0;
+      }
+      // fold: sum_q D_q / 2^q per plane = 2^-7 * sum_q D_q * 2^(7-q) (each term a
+      // multiple of 2^7), then 256*hi + lo; slice partial = step*(sum v - 2*that)
+      float* part = P.ws.partial + (size_t)it.sl * B * S16;
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-          int h0 = d[0][nb][0], l0 = d[0][nb][1], h1 = d[0][nb][2], l1 = d[0][nb][3];
+      for (int r = 0; r < RPW; ++r) {
+        if (r == 0 || hasB) {
+          const int row = 16 * (rbA + r) + g;
 #pragma unroll
-          for (int q = 1; q < 8; ++q) {
-            h0 = 2 * h0 + d[q][nb][0];
-            l0 = 2 * l0 + d[q][nb][1];
-            h1 = 2 * h1 + d[q][nb][2];
-            l1 = 2 * l1 + d[q][nb][3];
-          }
-          const int r0 = 2 * h0 + (l0 >> 7);
-          const int r1 = 2 * h1 + (l1 >> 7);
-          const int b = 4 * nb + c;
-          if (b < B) {
-            const int row = 16 * (rb - rb_lo) + g;
-            atomicAdd(&acc[b * (kVRowChunk * 16) + row], r0);
-            atomicAdd(&acc[b * (kVRowChunk * 16) + row + 8], r1);
+          for (int nb = 0; nb < NB; ++nb) {
+            int h0 = d[r][0][nb][0], l0 = d[r][0][nb][1], h1 = d[r][0][nb][2], l1 = d[r][0][nb][3];
+#pragma unroll
+            for (int q = 1; q < 8; ++q) {
+              h0 = 2 * h0 + d[r][q][nb][0];
+              l0 = 2 * l0 + d[r][q][nb][1];
+              h1 = 2 * h1 + d[r][q][nb][2];
+              l1 = 2 * l1 + d[r][q][nb][3];
+            }
+            const int b = 4 * nb + c;
+            if (b < B) {
+              float st = 0.f;
+              int vsum = 0;
+#pragma unroll
+              for (int bb = 0; bb < 4 * NB; ++bb)
+                if (bb == b) { st = step[bb]; vsum = vs[bb]; }
+              part[(size_t)b * S16 + row] = st * (float)(vsum - 2 * (2 * h0 + (l0 >> 7)));
+              part[(size_t)b * S16 + row + 8] = st * (float)(vsum - 2 * (2 * h1 + (l1 >> 7)));
+            }
           }
         }
       }
     }
-    __syncthreads();
+  }
+}
 
-    // ---- partial of this slice for the chunk's rows: step * (sum v - 2 * sum bit*v)
-    float* part = P.ws.partial + (size_t)it.sl * B * S16 + 16 * rb_lo;
-    for (int i = tid; i < B * nrow; i += kVWarps * 32) {
-      const int b = i / nrow, r = i - b * nrow;
-      float st = 0.f;
-      int vsum = 0;
+// ---------------------------------------------------------------------------
+// finalize:  t'_j = l_j * sum over slices of the partials, quantised to the
+// int8 hi/lo planes and the per-row step the output pass reads.  One CTA per
+// (layer, path), in a launch between the two passes.
+// ---------------------------------------------------------------------------
+template <int NB>
+__global__ void __launch_bounds__(kVWarps * 32) finalize_kernel(const DecodeArgs a) {
+  __shared__ float s_mx[kVWarps][16];
+  __shared__ int s_sm[kVWarps][16];
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* tp = reinterpret_cast<float*>(smem);   // [B][S16]
+  const int tid = threadIdx.x;
+  const int B = a.batch;
+  // (layer, path) of this CTA
+  int lo = 0, hi = a.n_layers - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.layers[mid].p_begin <= (int)blockIdx.x) lo = mid; else hi = mid - 1;
+  }
+  const LayerDesc& L = a.layers[lo];
+  const int p = blockIdx.x - L.p_begin;
+  const PathDesc& P = L.p[p];
+  const int s = L.s, S16 = (s + 15) & ~15, S32 = (s + 31) & ~31;
+  float mt[4 * NB];
+  int ts[4 * NB];
+#pragma unroll
+  for (int b = 0; b < 4 * NB; ++b) { mt[b] = 0.f; ts[b] = 0; }
+  for (int i = tid; i < B * S16; i += kVWarps * 32) {
+    const int b = i / S16, j = i - b * S16;
+    float t = 0.f;
+    if (j < s) {
+      for (int q = 0; q < L.n_slices; ++q) t += P.ws.partial[((size_t)q * B) * S16 + i];
+      t *= h2f(P.l[j]);
+    }
+    tp[i] = t;
+#pragma unroll
+    for (int bb = 0; bb < 4 * NB; ++bb)
+      if (bb == b) mt[bb] = fmaxf(mt[bb], fabsf(t));
+  }
+  block_max<4 * NB>(mt, s_mx);
+  for (int i = tid; i < B * S32; i += kVWarps * 32) {
+    const int b = i / S32, j = i - b * S32;
+    float tinv = 0.f;
+#pragma unroll
+    for (int bb = 0; bb < 4 * NB; ++bb)
+      if (bb == b) tinv = mt[bb] > 0.f ? kQMax / mt[bb] : 0.f;
+    int8_t hi8 = 0, lo8 = 0;
+    if (j < s) {
+      const int v = quantise(tp[b * S16 + j], tinv, hi8, lo8);
 #pragma unroll
       for (int bb = 0; bb < 4 * NB; ++bb)
-        if (bb == b) { st = step[bb]; vsum = vs[bb]; }
-      part[(size_t)b * S16 + r] = st * (float)(vsum - 2 * acc[b * (kVRowChunk * 16) + r]);
+        if (bb == b) ts[bb] += v;
     }
-    __syncthreads();
-    if (tid == 0) {
-      // the barrier orders every thread's partial before this release; the
-      // last arriver's acquire then sees all slices of the path
-      __threadfence();
-      s_last = (atomicAdd(P.ws.counter, 1u) == (unsigned)(L.n_slices * L.n_rchunks - 1));
-      __threadfence();
-    }
-    __syncthreads();
-
-    if (s_last) {
-      // ---- last item of this path: t' = l * (sum of slice partials), quantised
-      float mt[4 * NB];
-      int ts[4 * NB];
+    int8_t* pl = P.ws.planes + ((size_t)((j >> 5) * B + b) * 2) * 32 + (j & 31);
+    pl[0] = hi8;
+    pl[32] = lo8;
+  }
+  block_sum<4 * NB>(ts, s_sm);
+  if (tid < B) {
+    float m = 0.f;
+    int sum = 0;
 #pragma unroll
-      for (int b = 0; b < 4 * NB; ++b) { mt[b] = 0.f; ts[b] = 0; }
-      for (int i = tid; i < B * S16; i += kVWarps * 32) {
-        const int b = i / S16, j = i - b * S16;
-        float t = 0.f;
-        if (j < s) {
-          for (int q = 0; q < L.n_slices; ++q) t += __ldcg(P.ws.partial + ((size_t)q * B) * S16 + i);
-          t *= h2f(P.l[j]);
-        }
-        tp[i] = t;
-#pragma unroll
-        for (int bb = 0; bb < 4 * NB; ++bb)
-          if (bb == b) mt[bb] = fmaxf(mt[bb], fabsf(t));
-      }
-      block_max<4 * NB>(mt, s_mx);
-      const int S32 = (s + 31) & ~31;
-      for (int i = tid; i < B * S32; i += kVWarps * 32) {
-        const int b = i / S32, j = i - b * S32;
-        float tinv = 0.f;
-#pragma unroll
-        for (int bb = 0; bb < 4 * NB; ++bb)
-          if (bb == b) tinv = mt[bb] > 0.f ? kQMax / mt[bb] : 0.f;
-        int8_t hi = 0, lo = 0;
-        if (j < s) {
-          const int v = quantise(tp[b * S16 + j], tinv, hi, lo);
-#pragma unroll
-          for (int bb = 0; bb < 4 * NB; ++bb)
-            if (bb == b) ts[bb] += v;
-        }
-        int8_t* pl = P.ws.planes + ((size_t)((j >> 5) * B + b) * 2) * 32 + (j & 31);
-        pl[0] = hi;
-        pl[32] = lo;
-      }
-      block_sum<4 * NB>(ts, s_sm);
-      if (tid < B) {
-        float m = 0.f;
-        int sum = 0;
-#pragma unroll
-        for (int bb = 0; bb < 4 * NB; ++bb)
-          if (bb == tid) { m = mt[bb]; sum = ts[bb]; }
-        TStat st;
-        st.step = m > 0.f ? m / kQMax : 0.f;
-        st.sum = sum;
-        st.pad[0] = st.pad[1] = 0;
-        P.ws.tstat[tid] = st;
-      }
-      if (tid == 0) *P.ws.counter = 0u;
-      prev_li = -1;   // tp overwrote the staged B operand
-    }
-    __syncthreads();
+    for (int bb = 0; bb < 4 * NB; ++bb)
+      if (bb == tid) { m = mt[bb]; sum = ts[bb]; }
+    TStat st;
+    st.step = m > 0.f ? m / kQMax : 0.f;
+    st.sum = sum;
+    st.pad[0] = st.pad[1] = 0;
+    P.ws.tstat[tid] = st;
   }
 }
 
@@ -770,8 +800,22 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
 // ------------------------------------------------------------------ launchers
 
 size_t latent_smem(int nb) {
-  return (size_t)kVWarps * kVStages * kChunkBytes + (size_t)kVSlice * 8 * nb +
-         (size_t)kMaxBatchDecode * kVRowChunk * 16 * 4 + (size_t)kVWarps * kVStages * 8;
+  const int rpw = nb == 1 ? 2 : 1;
+  return (size_t)kVWarps * kVStages * rpw * kChunkBytes + (size_t)kVSlice * 8 * nb + (size_t)kVWarps * kVStages * 8;
+}
+
+template <int NB>
+cudaError_t launch_finalize(const DecodeArgs& a, int max_s16, cudaStream_t st) {
+  const size_t smem = (size_t)a.batch * max_s16 * 4;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(finalize_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)((size_t)4 * NB * kMaxRank * 4));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  finalize_kernel<NB><<<a.p_items, kVWarps * 32, smem, st>>>(a);
+  return cudaGetLastError();
 }
 
 template <int NB>
@@ -782,7 +826,6 @@ size_t output_smem(int batch) {
 template <int NB>
 cudaError_t launch_latent(const DecodeArgs& a, int max_s16, int num_sms, cudaStream_t st) {
   const size_t smem = latent_smem(NB);
-  if ((size_t)a.batch * max_s16 * 4 > (size_t)kVSlice * 8 * NB) return cudaErrorInvalidValue;   // t' fits bpl
   static bool attr_set = false;
   cudaError_t e;
   if (!attr_set) {
@@ -829,6 +872,16 @@ cudaError_t launch_latent_pass(const DecodeArgs& a, int max_s16, int num_sms, cu
     case 2: return launch_latent<2>(a, max_s16, num_sms, st);
     case 3: return launch_latent<3>(a, max_s16, num_sms, st);
     case 4: return launch_latent<4>(a, max_s16, num_sms, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_finalize_pass(const DecodeArgs& a, int max_s16, cudaStream_t st) {
+  switch ((a.batch + 3) / 4) {
+    case 1: return launch_finalize<1>(a, max_s16, st);
+    case 2: return launch_finalize<2>(a, max_s16, st);
+    case 3: return launch_finalize<3>(a, max_s16, st);
+    case 4: return launch_finalize<4>(a, max_s16, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -16,17 +16,15 @@ constexpr int kUTileRows = 128, kUTileK = 32;   // role-U tile
 constexpr int kTileBytes = 512;
 
 // Latent pass (V^T) work item: (layer, path, input slice, row chunk).  One CTA
-// of kVWarps warps covers kVSlice inputs; warp w owns the kVTilesPerWarp
-// K-tiles 4w..4w+3 of the slice and walks the kVRowChunk 16-row latent blocks
-// of the chunk.  Per 16-row block a warp's tiles are contiguous (2 KB), one
-// bulk copy.
+// of kVWarps warps covers kVSlice inputs (kVSliceTiles K-tiles) for kVRowChunk
+// 16-row latent blocks; warp w owns row blocks 2w and 2w+1 of the chunk over
+// the whole slice and streams their tiles in chunks of kChunkTiles K-tiles.
 constexpr int kVWarps = 4;
-constexpr int kVTilesPerWarp = 4;
-constexpr int kVSliceTiles = kVWarps * kVTilesPerWarp;   // 16 tiles
-constexpr int kVSlice = kVSliceTiles * kVTileK;          // 4096 inputs
-constexpr int kVRowChunk = 8;                            // 16-row blocks per item
-constexpr int kVStages = 4;                              // bulk-copy ring per warp
-constexpr int kChunkTiles = 4;                           // tiles per bulk copy
+constexpr int kVSliceTiles = 8;
+constexpr int kVSlice = kVSliceTiles * kVTileK;          // 2048 inputs
+constexpr int kVRowChunk = 2 * kVWarps;                  // 16-row blocks per item
+constexpr int kVStages = 3;                              // bulk-copy ring per warp
+constexpr int kChunkTiles = 4;                           // K-tiles per bulk copy
 constexpr int kChunkBytes = kChunkTiles * kTileBytes;    // 2048
 
 // Output pass (U) work item: (layer, 128 output rows), one warp.
@@ -55,7 +53,7 @@ struct TStat {
 //   partial : [n_slices][batch][s16] fp32  sums of one input slice
 //   planes  : [s32/32][batch][2][32] int8   hi and lo bytes of t', K-tile major
 //   tstat   : [batch] TStat
-//   counter : items of this path finished (reset to 0 by the last one)
+//   counter : unused (kept zero)
 struct PathScratch {
   float* partial;
   int8_t* planes;
@@ -81,6 +79,8 @@ struct LayerDesc {
   int n_rchunks;      // ceil(s16 / 16 / kVRowChunk)
   int v_begin;        // first latent-pass work item of this layer
   int u_begin;        // first output-pass work item of this layer
+  int p_begin;        // first (layer, path) index of this layer
+  int pad;
 };
 
 struct DecodeArgs {
@@ -90,10 +90,12 @@ struct DecodeArgs {
   int batch;
   int v_items;              // total latent-pass items
   int u_items;              // total output-pass items (layer, 128-row block)
+  int p_items;              // total (layer, path) pairs
 };
 
 // Launchers (decode.cu).  The batch selects the template (4 rows per n-block).
 cudaError_t launch_latent_pass(const DecodeArgs& a, int max_s16, int num_sms, cudaStream_t st);
+cudaError_t launch_finalize_pass(const DecodeArgs& a, int max_s16, cudaStream_t st);
 cudaError_t launch_output_pass(const DecodeArgs& a, int num_sms, cudaStream_t st);
 
 // prefill.cu: layers of M rows (multiple of 128), x fp16 or bf16 (y the same)

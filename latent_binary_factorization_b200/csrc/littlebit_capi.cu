@@ -113,7 +113,7 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   unsigned int* counters = reinterpret_cast<unsigned int*>(base + kStatusBytes + table_bytes);
   size_t off = kStatusBytes + table_bytes + counter_bytes;
   std::vector<lb::LayerDesc> tab(n);
-  int v_items = 0, u_items = 0;
+  int v_items = 0, u_items = 0, p_items = 0;
   for (int i = 0; i < n; ++i) {
     const lb_layer& L = layers[i];
     lb::LayerDesc& D = tab[i];
@@ -128,6 +128,8 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
     D.n_rchunks = lb::ceil_div(lb::s16(L.s) / 16, lb::kVRowChunk);
     D.v_begin = v_items;
     D.u_begin = u_items;
+    D.p_begin = p_items;
+    p_items += D.npaths;
     v_items += D.npaths * D.n_slices * D.n_rchunks;
     u_items += L.d_out / lb::kUTileRows;
     for (int p = 0; p < D.npaths; ++p) {
@@ -167,8 +169,11 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   a.batch = batch;
   a.v_items = v_items;
   a.u_items = u_items;
+  a.p_items = p_items;
   const int sms = num_sms(dev);
   e = lb::launch_latent_pass(a, max_s16, sms, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = lb::launch_finalize_pass(a, max_s16, st);
   if (e != cudaSuccess) return cuda_fail(e);
   if (between) {
     e = cudaEventRecord(between, st);

@@ -99,6 +99,7 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
   D.n_rchunks = lb::ceil_div(S16 / 16, lb::kVRowChunk);
   D.v_begin = 0;
   D.u_begin = 0;
+  D.p_begin = 0;
   size_t off = kPathOff;
   unsigned int* counters = reinterpret_cast<unsigned int*>(base + kCounterOff);
   for (int p = 0; p < npaths; ++p) {
@@ -130,10 +131,13 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
   a.batch = batch;
   a.v_items = npaths * D.n_slices * D.n_rchunks;
   a.u_items = L.d_out / lb::kUTileRows;
+  a.p_items = npaths;
   int sms = 0;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess || sms <= 0) return LB_ERR_CUDA;
   e = lb::launch_latent_pass(a, S16, sms, st);
+  if (e != cudaSuccess) return LB_ERR_CUDA;
+  e = lb::launch_finalize_pass(a, S16, st);
   if (e != cudaSuccess) return LB_ERR_CUDA;
   e = lb::launch_output_pass(a, sms, st);
   if (e != cudaSuccess) return LB_ERR_CUDA;
