@@ -515,7 +515,7 @@ template <int NB>
 __global__ void __launch_bounds__(kVWarps * 32) finalize_kernel(const DecodeArgs a) {
   __shared__ float s_mx[kVWarps][16];
   __shared__ int s_sm[kVWarps][16];
-  extern __shared__ __align__(16) unsigned char smem[];
+  extern __shared__ __align__(1024) unsigned char smem[];
   float* tp = reinterpret_cast<float*>(smem);   // [B][S16]
   const int tid = threadIdx.x;
   const int B = a.batch;
@@ -546,25 +546,27 @@ __global__ void __launch_bounds__(kVWarps * 32) finalize_kernel(const DecodeArgs
       if (bb == b) mt[bb] = fmaxf(mt[bb], fabsf(t));
   }
   block_max<4 * NB>(mt, s_mx);
-  for (int i = tid; i < B * S32; i += kVWarps * 32) {
+  // planes hold 4*NB batch rows (rows >= B are zero) so that the output pass
+  // loads every thread's B fragment without a predicate
+  for (int i = tid; i < 4 * NB * S32; i += kVWarps * 32) {
     const int b = i / S32, j = i - b * S32;
     float tinv = 0.f;
 #pragma unroll
     for (int bb = 0; bb < 4 * NB; ++bb)
       if (bb == b) tinv = mt[bb] > 0.f ? kQMax / mt[bb] : 0.f;
     int8_t hi8 = 0, lo8 = 0;
-    if (j < s) {
+    if (j < s && b < B) {
       const int v = quantise(tp[b * S16 + j], tinv, hi8, lo8);
 #pragma unroll
       for (int bb = 0; bb < 4 * NB; ++bb)
         if (bb == b) ts[bb] += v;
     }
-    int8_t* pl = P.ws.planes + ((size_t)((j >> 5) * B + b) * 2) * 32 + (j & 31);
+    int8_t* pl = P.ws.planes + ((size_t)((j >> 5) * 4 * NB + b) * 2) * 32 + (j & 31);
     pl[0] = hi8;
     pl[32] = lo8;
   }
   block_sum<4 * NB>(ts, s_sm);
-  if (tid < B) {
+  if (tid < 4 * NB) {
     float m = 0.f;
     int sum = 0;
 #pragma unroll
@@ -587,10 +589,11 @@ constexpr int kUChunkBytes = kUChunkTiles * kTileBytes;   // 4 KB
 
 template <int NB>
 struct OutCfg {
-  static constexpr int kStages = NB == 1 ? 3 : 2;
+  static constexpr int kStages = 2;
 };
 
-// stage: [8 tiles: 4 KB][t' bytes: 8 K-tiles x B x 64][h: 256][tstat: 16 B per row]
+// stage: [8 tiles: 4 KB][t' bytes: 8 K-tiles x 4NB x 64][h: 256][tstat: 16 B x 4NB]
+// (B below is the padded row count 4*NB)
 __host__ __device__ __forceinline__ int out_planes_off() { return kUChunkBytes; }
 __host__ __device__ __forceinline__ int out_h_off(int B) { return kUChunkBytes + kUChunkTiles * B * 64; }
 __host__ __device__ __forceinline__ int out_tstat_off(int B) { return out_h_off(B) + kUTileRows * 2; }
@@ -658,13 +661,13 @@ __device__ __forceinline__ void out_issue(const OutCursor& cu, unsigned char* st
 // `pl_step` = B * 64 bytes from one tile's t' bytes to the next.
 template <int NB>
 __device__ __forceinline__ void out_tile(int (&d)[8][NB][4], const unsigned char* stage, int t, int lane,
-                                         const unsigned char* pl, bool (&bval)[NB]) {
+                                         const unsigned char* pl) {
   const uint4 cur = *reinterpret_cast<const uint4*>(stage + t * kTileBytes + lane * 16);
   uint32_t b0[NB], b1[NB];
 #pragma unroll
   for (int nb = 0; nb < NB; ++nb) {
-    b0[nb] = bval[nb] ? *reinterpret_cast<const uint32_t*>(pl + nb * 256) : 0u;
-    b1[nb] = bval[nb] ? *reinterpret_cast<const uint32_t*>(pl + nb * 256 + 16) : 0u;
+    b0[nb] = *reinterpret_cast<const uint32_t*>(pl + t * (256 * NB) + nb * 256);
+    b1[nb] = *reinterpret_cast<const uint32_t*>(pl + t * (256 * NB) + nb * 256 + 16);
   }
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
@@ -680,8 +683,9 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
   constexpr int S = OutCfg<NB>::kStages;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-  const int B = a.batch;
-  const int sb = out_stage_bytes(B);
+  const int B = a.batch;            // rows stored
+  constexpr int BP = 4 * NB;        // rows in the t' planes and stats (padded)
+  const int sb = out_stage_bytes(BP);
   unsigned char* my_ring = smem + (size_t)warp * S * sb;
   uint64_t* my_bar = reinterpret_cast<uint64_t*>(smem + (size_t)kUWarps * S * sb) + warp * S;
 
@@ -705,7 +709,7 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
 #pragma unroll 1
   for (int st = 0; st < S; ++st) {
     if (fd.item < i_end) {
-      if (lane == 0) out_issue(fd, my_ring + st * sb, &my_bar[st], B);
+      if (lane == 0) out_issue(fd, my_ring + st * sb, &my_bar[st], BP);
       fd.advance(a);
     }
   }
@@ -723,11 +727,7 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
   int slot = 0;
   bool dead = false;
   // this thread's B-operand column: batch row 4nb + g/2, plane g%2
-  const int pl_off = out_planes_off() + ((g >> 1) * 2 + (g & 1)) * 32 + 4 * c;
-  const int pl_step = B * 64;
-  bool bval[NB];
-#pragma unroll
-  for (int nb = 0; nb < NB; ++nb) bval[nb] = 4 * nb + (g >> 1) < B;
+  const int pl_off = out_planes_off() + g * 32 + 4 * c;
 
   while (cs.item < i_end) {
     if (!dead && !mbar_wait(&my_bar[slot], (consumed / S) & 1)) {
@@ -739,15 +739,15 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
     const unsigned char* pl = stage + pl_off;
     if (nt == kUChunkTiles) {
 #pragma unroll
-      for (int t = 0; t < kUChunkTiles; ++t) out_tile<NB>(d, stage, t, lane, pl + t * pl_step, bval);
+      for (int t = 0; t < kUChunkTiles; ++t) out_tile<NB>(d, stage, t, lane, pl);
     } else {
 #pragma unroll 1
-      for (int t = 0; t < nt; ++t) out_tile<NB>(d, stage, t, lane, pl + t * pl_step, bval);
+      for (int t = 0; t < nt; ++t) out_tile<NB>(d, stage, t, lane, pl);
     }
     if (cs.path_end()) {
       // path finished: rows 128*ob + 16q + g (+8), batch row 4nb + c
-      const uint16_t* hs = reinterpret_cast<const uint16_t*>(stage + out_h_off(B));
-      const TStat* tst = reinterpret_cast<const TStat*>(stage + out_tstat_off(B));
+      const uint16_t* hs = reinterpret_cast<const uint16_t*>(stage + out_h_off(BP));
+      const TStat* tst = reinterpret_cast<const TStat*>(stage + out_tstat_off(BP));
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb) {
         const int b = 4 * nb + c;
@@ -788,7 +788,7 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
     // the stage has been read: refill it with the chunk `S` ahead
     __syncwarp();
     if (fd.item < i_end) {
-      if (lane == 0) out_issue(fd, my_ring + slot * sb, &my_bar[slot], B);
+      if (lane == 0) out_issue(fd, my_ring + slot * sb, &my_bar[slot], BP);
       fd.advance(a);
     }
     ++consumed;
@@ -819,8 +819,8 @@ cudaError_t launch_finalize(const DecodeArgs& a, int max_s16, cudaStream_t st) {
 }
 
 template <int NB>
-size_t output_smem(int batch) {
-  return (size_t)kUWarps * OutCfg<NB>::kStages * out_stage_bytes(batch) + (size_t)kUWarps * OutCfg<NB>::kStages * 8;
+size_t output_smem(int) {
+  return (size_t)kUWarps * OutCfg<NB>::kStages * out_stage_bytes(4 * NB) + (size_t)kUWarps * OutCfg<NB>::kStages * 8;
 }
 
 template <int NB>

@@ -51,8 +51,9 @@ struct TStat {
 
 // Per-path scratch written by the latent pass and read by the output pass.
 //   partial : [n_slices][batch][s16] fp32  sums of one input slice
-//   planes  : [s32/32][batch][2][32] int8   hi and lo bytes of t', K-tile major
-//   tstat   : [batch] TStat
+//   planes  : [s32/32][4*nb][2][32] int8    hi and lo bytes of t', K-tile major
+//                                            (nb = ceil(batch/4); rows >= batch are zero)
+//   tstat   : [4*nb] TStat
 //   counter : unused (kept zero)
 struct PathScratch {
   float* partial;

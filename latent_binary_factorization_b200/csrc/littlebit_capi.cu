@@ -64,8 +64,11 @@ lb_status check_layer(const lb_layer& L) {
 size_t partial_bytes(const lb_layer& L, int batch) {
   return align_up((size_t)lb::ceil_div(L.d_in, lb::kVSlice) * batch * lb::s16(L.s) * sizeof(float), 256);
 }
-size_t planes_bytes(const lb_layer& L, int batch) { return align_up((size_t)batch * 2 * lb::s32(L.s), 256); }
-size_t tstat_bytes(int batch) { return align_up((size_t)batch * sizeof(lb::TStat), 256); }
+// t' planes and stats are padded to whole groups of four batch rows
+size_t planes_bytes(const lb_layer& L, int batch) {
+  return align_up((size_t)lb::ceil_div(batch, 4) * 4 * 2 * lb::s32(L.s), 256);
+}
+size_t tstat_bytes(int batch) { return align_up((size_t)lb::ceil_div(batch, 4) * 4 * sizeof(lb::TStat), 256); }
 size_t path_scratch_bytes(const lb_layer& L, int batch) {
   return partial_bytes(L, batch) + planes_bytes(L, batch) + tstat_bytes(batch);
 }

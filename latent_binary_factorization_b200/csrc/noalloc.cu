@@ -69,8 +69,9 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
   const int n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
   const int S16 = lb::s16(L.s), S32 = lb::s32(L.s);
   const size_t part_b = round256((size_t)n_slices * batch * S16 * sizeof(float));
-  const size_t planes_b = round256((size_t)batch * 2 * S32);
-  const size_t tstat_b = round256((size_t)batch * sizeof(lb::TStat));
+  const int bpad = lb::ceil_div(batch, 4) * 4;   // t' planes and stats padded to groups of 4 rows
+  const size_t planes_b = round256((size_t)bpad * 2 * S32);
+  const size_t tstat_b = round256((size_t)bpad * sizeof(lb::TStat));
   const int npaths = L.residual + 1;
   if (kPathOff + (size_t)npaths * (part_b + planes_b + tstat_b) > kNoAllocScratchBytes) return LB_ERR_SHAPE;
 

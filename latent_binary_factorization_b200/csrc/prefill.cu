@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(256) prep_b1_kernel(const LayerDesc L, int Sp,
 // thread per 16-byte lane of a packed role-U tile: for each q its word gives
 // four consecutive j of one row.  Columns from the tiles' end up to Sp are zero.
 __global__ void __launch_bounds__(256) prep_b2_kernel(const LayerDesc L, int Sp, unsigned char* __restrict__ out) {
-  const int R = L.d_out, K = L.npaths * Sp;
+  const int R = L.d_out;
   const int n_kt = (L.s + 31) >> 5, n_ob = R / kUTileRows;
   const long long lanes = (long long)L.npaths * n_ob * n_kt * 32;
   const int zcols = Sp - 32 * n_kt;                       // zero columns per path
