@@ -398,7 +398,7 @@ def run_ours(args):
                           "output_pass_gbs": round(main["output_pass_gbs"], 1)},
         "e2e": {"value": round(1e3 * e2e_ms / max(3, args.steps // 4) / (n_layers * world), 5), "unit": "us/layer",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 4 * args.steps,   # quantise, latent, finalize, output per step
         "clocks": clocks,
         "extras": extras,
         "prefill": prefill,

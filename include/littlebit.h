@@ -160,9 +160,11 @@ lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, con
  * such interface; it has no counterpart in them.
  *   - Allocates nothing.  Its scratch is one fixed 1 MiB device array inside
  *     the library, held by every GPU that loads the library until the process
- *     exits.  A layer whose latent-pass scratch (ceil(d_in/4096) * batch *
- *     16*ceil(s/16) fp32 partials, plus t' bytes, per path) does not fit
- *     returns LB_ERR_SHAPE.
+ *     exits.  A layer whose scratch does not fit returns LB_ERR_SHAPE; per
+ *     path it needs, for n = ceil(d_in/2048) input slices and r = 1 at batch 1,
+ *     else 4*ceil(batch/4): n quantised input slices of 64*ceil(batch/4) +
+ *     4096*r bytes, 4*ceil(n/4) * batch * 16*ceil(s/16) fp32 partial sums,
+ *     and the t' bytes (about 2*r*s).
  *   - The first call on a device, with that device current, looks up the
  *     array's device address (cudaGetSymbolAddress); make that first call
  *     before any stream capture.

@@ -25,17 +25,20 @@
 // registers.  Every wait is bounded: after kSpinLimit polls the kernel sets
 // LB_ERR_TIMEOUT in the status word and stops waiting.
 //
-// Latent pass: CTA item = (layer, path, 4096-input slice, 128-row chunk); warp
-// w owns tiles 4w..4w+3 of the slice and walks the chunk's 16-row latent
-// blocks; exact integer sums are combined in shared memory and written as one
-// fp32 partial per latent row.  The CTA that finishes a path's last item
-// (atomic ticket, no waiting) sums the partials in slice order, multiplies by
-// l and quantises t'.
-// Output pass: warp item = (layer, 128 output rows); each warp owns a
-// contiguous item range and streams it as chunks of up to 8 K-tiles, across
-// path, item and layer boundaries; the bulk copies also bring the chunk's t'
-// bytes and, for the last chunk of a path, the 128 h values and the
-// quantisation step.  Paths are added in fp32 and y is written in fp16.
+// Four launches, in stream order:
+// quantise: CTA per (layer, path, 2048-input slice) quantises u = g*x per batch
+//   row and stores it as int8 B fragments with the step and sum per row.
+// latent:   CTA item = (layer, path, slice, 8 latent 16-row blocks); the
+//   slice's B fragments arrive by one bulk copy into a double buffer, warp w
+//   streams row blocks 2w, 2w+1 over the slice and writes one fp32 partial sum
+//   per latent row and slice.
+// finalize: CTA per (layer, path) sums the partials in slice order, multiplies
+//   by l and quantises t' to int8 hi/lo planes with a step per batch row.
+// output:   warp item = (layer, 128 output rows); each warp owns a contiguous
+//   item range and streams it as chunks of up to 8 K-tiles, across path, item
+//   and layer boundaries; the bulk copies also bring the chunk's t' bytes and,
+//   for the last chunk of a path, the 128 h values and the quantisation step.
+//   Paths are added in fp32 and y is written in fp16.
 #include <cuda_fp16.h>
 
 #include "lb_internal.h"
@@ -175,26 +178,122 @@ __device__ __forceinline__ void block_sum(int (&v)[N], int (*s_buf)[16]) {
   __syncthreads();
 }
 
-// Index of the layer whose item range holds `item` (binary search, once per
-// warp or CTA; later items are reached by walking forward).
-__device__ __forceinline__ int find_layer(const DecodeArgs& a, int item, bool latent) {
-  int lo = 0, hi = a.n_layers - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    const int begin = latent ? a.layers[mid].v_begin : a.layers[mid].u_begin;
-    if (begin <= item) lo = mid; else hi = mid - 1;
+// Layer of a work item: one load from the item's map (no map with one layer).
+__device__ __forceinline__ int layer_of(const int* map, int n_layers, int item) {
+  return n_layers == 1 ? 0 : __ldg(map + item);
+}
+
+// ---------------------------------------------------------------------------
+// quantise pass:  u = g (.) x on one 2048-input slice of one (layer, path),
+// quantised per batch row to 16 bits, v = step * (256*hi + lo), and stored as
+// the latent pass's int8 B fragments (slice block layout in lb_internal.h).
+// One warp per (layer, path, slice): lane i holds the 8-input chunks i + 32j
+// (j < 8) of g and of one batch row of x at a time; max and sum are warp
+// reductions, so the kernel has no CTA barrier.
+// ---------------------------------------------------------------------------
+constexpr int kQWarps = 4;                          // warps (slices) per CTA
+constexpr int kQChunks = kVSlice / 8 / 32;          // 8-input chunks per lane
+
+__global__ void __launch_bounds__(kQWarps * 32) quantise_input_kernel(const DecodeArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int item = blockIdx.x * kQWarps + (threadIdx.x >> 5);
+  if (item >= a.x_items) return;
+  const int B = a.batch, RB = xq_rows(B), NC = 2 * RB;
+  const LayerDesc& L = a.layers[layer_of(a.item_layer.x, a.n_layers, item)];
+  const int rel = item - L.x_begin;
+  const int p = rel / L.n_slices, sl = rel - p * L.n_slices;
+  const PathDesc& P = L.p[p];
+  const int d_in = L.d_in, k0 = sl * kVSlice;
+  const int nchunk = min(kVSlice, d_in - k0) / 8;
+  unsigned char* blk = P.ws.xq + (size_t)sl * xq_slice_bytes(B);
+  uint32_t* frag = reinterpret_cast<uint32_t*>(blk + xq_stats_bytes(B));
+
+  uint4 gq[kQChunks];
+#pragma unroll
+  for (int j = 0; j < kQChunks; ++j) {
+    const int ch = lane + 32 * j;
+    gq[j] = ch < nchunk ? ld_nc(P.g + k0 + 8 * ch) : make_uint4(0, 0, 0, 0);
   }
-  return lo;
+  const int nrow = 4 * xq_nb(B);   // stats rows (>= RB >= B)
+#pragma unroll 1
+  for (int row = 0; row < nrow; ++row) {
+    uint4 xq[kQChunks];
+#pragma unroll
+    for (int j = 0; j < kQChunks; ++j) {
+      const int ch = lane + 32 * j;
+      xq[j] = (row < B && ch < nchunk) ? ld_nc(L.x + (size_t)row * d_in + k0 + 8 * ch) : make_uint4(0, 0, 0, 0);
+    }
+    float mx = 0.f;
+#pragma unroll
+    for (int j = 0; j < kQChunks; ++j) {
+      const uint32_t* xw = &xq[j].x;
+      const uint32_t* gw = &gq[j].x;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 xf = h2x2(xw[e]), gf = h2x2(gw[e]);
+        mx = fmaxf(mx, fmaxf(fabsf(xf.x * gf.x), fabsf(xf.y * gf.y)));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float inv = mx > 0.f ? kQMax / mx : 0.f;
+    int vsum = 0;
+#pragma unroll
+    for (int j = 0; j < kQChunks; ++j) {
+      const int ch = lane + 32 * j;
+      const uint32_t* xw = &xq[j].x;
+      const uint32_t* gw = &gq[j].x;
+      uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 xf = h2x2(xw[e]), gf = h2x2(gw[e]);
+        int8_t h0, l0, h1, l1;
+        vsum += quantise(xf.x * gf.x, inv, h0, l0) + quantise(xf.y * gf.y, inv, h1, l1);
+        const int sh = 16 * (e & 1);
+        hw[e >> 1] |= ((uint32_t)(uint8_t)h0 | ((uint32_t)(uint8_t)h1 << 8)) << sh;
+        lw[e >> 1] |= ((uint32_t)(uint8_t)l0 | ((uint32_t)(uint8_t)l1 << 8)) << sh;
+      }
+      if (row < RB && ch < nchunk) {
+        // inputs 8ch..8ch+7: K-block kb, offset kk0 (0, 8, 16, 24) inside it;
+        // kk < 16 -> b0 words of threads c = kk/4, else b1 words of c = (kk-16)/4
+        const int kb = ch >> 2, kk0 = (ch & 3) * 8;
+        const int cc = (kk0 & 15) >> 2, half = kk0 >> 4;
+        uint32_t* fh = frag + ((size_t)kb * NC + 2 * row) * 8;   // column 2*row: 4 threads x (b0, b1)
+        uint32_t* fl = fh + 8;                                   // column 2*row + 1
+        fh[2 * cc + half] = hw[0];
+        fh[2 * (cc + 1) + half] = hw[1];
+        fl[2 * cc + half] = lw[0];
+        fl[2 * (cc + 1) + half] = lw[1];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) vsum += __shfl_xor_sync(0xffffffffu, vsum, o);
+    if (lane == 0) {
+      TStat st;
+      st.step = mx > 0.f ? mx / kQMax : 0.f;
+      st.sum = vsum;
+      st.pad[0] = st.pad[1] = 0;
+      reinterpret_cast<TStat*>(blk)[row] = st;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
 // latent pass:  t_j (partial over one slice) = sum_i V[i][j] g_i x_i
 // ---------------------------------------------------------------------------
-// CTA item = (layer, path, 2048-input slice, 8 latent row blocks).  The CTA
-// quantises g*x of the slice once into shared memory as B fragments; warp w
-// takes row blocks 2w, 2w+1 and accumulates their eight products per K-block
-// over the whole slice (one B fragment load feeds both blocks), then folds the
-// 2^q factors once and writes one fp32 partial per latent row.
+// CTA item = (layer, path, 2048-input slice, 8 latent row blocks).  The slice's
+// quantised input (B fragments and per-row step) arrives by one bulk copy into
+// one of two shared buffers; warp w takes row blocks 2w, 2w+1 and accumulates
+// their eight products per K-block over the whole slice (one B fragment load
+// feeds both blocks), then folds the 2^q factors once and writes one fp32
+// partial per latent row.
+//
+// Buffer hand-over without CTA barriers: the CTA's items are walked by every
+// warp in the same order, so each warp sees the same sequence of distinct
+// slices.  Slice n uses buffer n % 2.  A warp that moves on from slice n - 1
+// counts itself done on that buffer (shared atomic); the warp that completes
+// the count issues the copy of slice n + 1 into it.  Every warp then waits for
+// slice n's copy (bounded).
 
 struct VItem {
   int li, p, sl, rc;
@@ -221,6 +320,21 @@ template <int NB>
 struct VCfg {
   static constexpr int kRPW = NB == 1 ? 2 : 1;
 };
+
+// Bytes of one quantised input slice buffer (shared memory and global stride).
+__host__ __device__ constexpr int xq_buf_bytes(int nb, int rb) { return (64 * nb + kVSlice * 2 * rb + 127) & ~127; }
+
+// Copy the quantised slice of `item` (from its first byte to the end of its
+// last K-block) into `dst`, completion on `bar`.
+template <int NB, int RB>
+__device__ __forceinline__ void x_issue(const DecodeArgs& a, int item, int li, unsigned char* dst, uint64_t* bar) {
+  const VItem it = decode_v(a, item, li);
+  const LayerDesc& L = a.layers[it.li];
+  const int klen = min(kVSlice, L.d_in - it.sl * kVSlice);
+  const uint32_t bytes = 64 * NB + klen * 2 * RB;
+  mbar_expect_tx(bar, bytes);
+  bulk_g2s(dst, L.p[it.p].ws.xq + (size_t)it.sl * xq_buf_bytes(NB, RB), bytes, bar);
+}
 
 // One warp's sequence of bulk-copy chunks: per item, per group of kRPW row
 // blocks, per 4 K-tiles of the slice.
@@ -277,17 +391,18 @@ struct VFeed {
   }
 };
 
-template <int NB>
-__global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_kernel(const DecodeArgs a) {
-  constexpr int NCOL = 8 * NB;
+template <int NB, int RB>
+__global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 4 : 1) latent_pass_kernel(const DecodeArgs a) {
+  constexpr int NC = 2 * RB;                      // B-fragment columns stored per K-block
   constexpr int RPW = VCfg<NB>::kRPW;
   constexpr int kStageBytes = RPW * kChunkBytes;
+  constexpr int kXBuf = xq_buf_bytes(NB, RB);
   extern __shared__ __align__(1024) unsigned char smem[];
-  unsigned char* ring = smem;                                                          // [warps][stages][RPW x 2 KB]
-  uint2* bst = reinterpret_cast<uint2*>(smem + kVWarps * kVStages * kStageBytes);    // [64][NCOL][4] (b0, b1)
-  uint64_t* mbar = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(bst) + (size_t)kVSlice * NCOL);
-  __shared__ float s_mx[kVWarps][16];
-  __shared__ int s_sm[kVWarps][16];
+  unsigned char* ring = smem;                                        // [warps][stages][RPW x 2 KB]
+  unsigned char* xbuf = smem + kVWarps * kVStages * kStageBytes;     // [2][kXBuf]
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(xbuf + 2 * kXBuf);    // [warps][stages]
+  uint64_t* xfull = mbar + kVWarps * kVStages;                       // [2]
+  __shared__ int s_done[2];   // warps done with each buffer, accumulated over its uses
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
   const int B = a.batch;
@@ -299,11 +414,25 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_ker
   uint64_t* my_bar = mbar + warp * kVStages;
   if (lane == 0) {
     for (int st = 0; st < kVStages; ++st) mbar_init(&my_bar[st], 1);
-    fence_mbar_init();
   }
-  __syncwarp();
+  if (tid == 0) {
+    mbar_init(&xfull[0], 1);
+    mbar_init(&xfull[1], 1);
+    s_done[0] = s_done[1] = 0;
+  }
+  if (lane == 0) fence_mbar_init();
+  __syncthreads();   // the only CTA barrier: barriers and counters initialised
 
-  const int li0 = find_layer(a, i_begin, true);
+  const int li0 = layer_of(a.item_layer.v, a.n_layers, i_begin);
+  if (tid == 0) {
+    // slices 0 and 1 of this CTA's sequence
+    int lj = li0;
+    const VItem it = decode_v(a, i_begin, lj);
+    x_issue<NB, RB>(a, i_begin, li0, xbuf, &xfull[0]);
+    const int nxt = i_begin - it.rc + a.layers[it.li].n_rchunks;
+    if (nxt < i_end) x_issue<NB, RB>(a, nxt, it.li, xbuf + kXBuf, &xfull[1]);
+  }
+
   VFeed<NB> feed;
   feed.item = i_begin;
   feed.li = li0;
@@ -320,100 +449,50 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_ker
   int slot = 0;
   bool dead = false;
 
+  // this thread's B column in K-block 0 (uint2 units): column (8nb + g) mod NC
+  int boff[NB];
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) boff[nb] = ((8 * nb + g) % NC) * 4 + c;
+
   int li = li0;
-  int prev_li = -1, prev_p = -1, prev_sl = -1;   // slice whose B operand is staged
-  float step[4 * NB];
-  int vs[4 * NB];
+  int prev_li = -1, prev_p = -1, prev_sl = -1;
+  int seq = -1;   // index of the current slice in this CTA's sequence
 
   for (int item = i_begin; item < i_end; ++item) {
     const VItem it = decode_v(a, item, li);
     const LayerDesc& L = a.layers[li];
     const PathDesc& P = L.p[it.p];
-    const int d_in = L.d_in, s = L.s;
+    const int s = L.s;
     const int S16 = (s + 15) & ~15, n_rb = S16 >> 4;
-    const int k0 = it.sl * kVSlice;
-    const int klen = min(kVSlice, d_in - k0);   // multiple of 256
-    const int nkt = klen / kVTileK;
+    const int nkt = min(kVSlice, L.d_in - it.sl * kVSlice) / kVTileK;
 
     if (it.li != prev_li || it.p != prev_p || it.sl != prev_sl) {
-      // ---- u = g * x on the slice, quantised per batch row to 16 bits, staged
-      //      as (b0, b1) B-fragment pairs: column n = 2*(row%4) (+1 for lo) of
-      //      n-block row/4, K-block kb = k/32, thread column c
-      constexpr int kChunks = kVSlice / 8 / (kVWarps * 32);   // 8-input chunks per thread
-      const int nchunk = klen / 8;
-      __syncthreads();   // previous users of the staging area are done
-      uint4 gq[kChunks];
-#pragma unroll
-      for (int i = 0; i < kChunks; ++i) {
-        const int ch = tid + i * kVWarps * 32;
-        gq[i] = ch < nchunk ? ld_nc(P.g + k0 + 8 * ch) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int bg = 0; bg < NB; ++bg) {
-        uint4 xq[4][kChunks];
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-          for (int i = 0; i < kChunks; ++i) {
-            const int ch = tid + i * kVWarps * 32, b = 4 * bg + r;
-            xq[r][i] = (b < B && ch < nchunk) ? ld_nc(L.x + (size_t)b * d_in + k0 + 8 * ch)
-                                               : make_uint4(0, 0, 0, 0);
+      ++seq;
+      if (seq > 0) {
+        // done with slice seq - 1: the last warp out refills its buffer with slice seq + 1
+        __syncwarp();
+        if (lane == 0) {
+          const int b = (seq - 1) & 1;
+          __threadfence_block();
+          const int old = atomicAdd(&s_done[b], 1);
+          if (old == kVWarps * (((seq - 1) >> 1) + 1) - 1) {
+            __threadfence_block();
+            const int nxt = item - it.rc + L.n_rchunks;   // first item of the following slice
+            if (nxt < i_end) x_issue<NB, RB>(a, nxt, li, xbuf + b * kXBuf, &xfull[b]);
           }
-        float mx[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-          for (int i = 0; i < kChunks; ++i) {
-            const uint32_t* xw = &xq[r][i].x;
-            const uint32_t* gw = &gq[i].x;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 xf = h2x2(xw[e]), gf = h2x2(gw[e]);
-              mx[r] = fmaxf(mx[r], fmaxf(fabsf(xf.x * gf.x), fabsf(xf.y * gf.y)));
-            }
-          }
-        block_max<4>(mx, s_mx);
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const float inv = mx[r] > 0.f ? kQMax / mx[r] : 0.f;
-          step[4 * bg + r] = mx[r] > 0.f ? mx[r] / kQMax : 0.f;
-          int vsum = 0;
-#pragma unroll
-          for (int i = 0; i < kChunks; ++i) {
-            const int ch = tid + i * kVWarps * 32;
-            const uint32_t* xw = &xq[r][i].x;
-            const uint32_t* gw = &gq[i].x;
-            uint32_t hi[2] = {0u, 0u}, lo[2] = {0u, 0u};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 xf = h2x2(xw[e]), gf = h2x2(gw[e]);
-              int8_t h0, l0, h1, l1;
-              vsum += quantise(xf.x * gf.x, inv, h0, l0) + quantise(xf.y * gf.y, inv, h1, l1);
-              const int sh = 16 * (e & 1);
-              hi[e >> 1] |= ((uint32_t)(uint8_t)h0 | ((uint32_t)(uint8_t)h1 << 8)) << sh;
-              lo[e >> 1] |= ((uint32_t)(uint8_t)l0 | ((uint32_t)(uint8_t)l1 << 8)) << sh;
-            }
-            if (ch < nchunk) {
-              // inputs 8ch..8ch+7: K-block kb, within-block offset kk0 (0, 8, 16, 24);
-              // kk < 16 -> b0 bytes of columns c = kk/4, else b1 bytes of c = (kk-16)/4
-              const int kb = ch >> 2, kk0 = (ch & 3) * 8;
-              const int cc = (kk0 & 15) >> 2, half = kk0 >> 4;
-              uint32_t* base_hi = reinterpret_cast<uint32_t*>(bst + ((size_t)kb * NCOL + bg * 8 + 2 * r) * 4);
-              uint32_t* base_lo = reinterpret_cast<uint32_t*>(bst + ((size_t)kb * NCOL + bg * 8 + 2 * r + 1) * 4);
-              base_hi[2 * cc + half] = hi[0];
-              base_hi[2 * (cc + 1) + half] = hi[1];
-              base_lo[2 * cc + half] = lo[0];
-              base_lo[2 * (cc + 1) + half] = lo[1];
-            }
-          }
-          vs[4 * bg + r] = vsum;
         }
       }
-      block_sum<4 * NB>(vs, s_sm);   // ends with __syncthreads: staging complete
+      if (!dead && !mbar_wait(&xfull[seq & 1], (seq >> 1) & 1)) {
+        dead = true;
+        atomicOr(a.status, 1u << LB_ERR_TIMEOUT);
+      }
       prev_li = it.li;
       prev_p = it.p;
       prev_sl = it.sl;
     }
+    const unsigned char* xb = xbuf + (seq & 1) * kXBuf;
+    const uint2* frag = reinterpret_cast<const uint2*>(xb + 64 * NB);
+    const TStat* xst = reinterpret_cast<const TStat*>(xb);
 
     // ---- this warp's row blocks over the slice
 #pragma unroll 1
@@ -437,13 +516,13 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_ker
           for (int r = 0; r < RPW; ++r)
             cur[r] = (r == 0 || hasB) ? *reinterpret_cast<const uint4*>(stage + r * kChunkBytes + t * kTileBytes + lane * 16)
                                       : make_uint4(0, 0, 0, 0);
-          const int kb0 = (kc * kChunkTiles + t) * 8;
+          const uint2* fk = frag + (size_t)(kc * kChunkTiles + t) * 8 * NC * 4;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const uint32_t m = 0x01010101u << q;
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) {
-              const uint2 bb = bst[((size_t)(kb0 + q) * NCOL + nb * 8 + g) * 4 + c];
+              const uint2 bb = fk[q * NC * 4 + boff[nb]];
 #pragma unroll
               for (int r = 0; r < RPW; ++r) {
                 if (r == 0 || hasB) {
@@ -474,7 +553,8 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_ker
       }
       // fold: sum_q D_q / 2^q per plane = 2^-7 * sum_q D_q * 2^(7-q) (each term a
       // multiple of 2^7), then 256*hi + lo; slice partial = step*(sum v - 2*that)
-      float* part = P.ws.partial + (size_t)it.sl * B * S16;
+      const int ns4 = (L.n_slices + 3) & ~3;
+      float* part = P.ws.partial + it.sl;
 #pragma unroll
       for (int r = 0; r < RPW; ++r) {
         if (r == 0 || hasB) {
@@ -491,13 +571,10 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 3 : 1) latent_pass_ker
             }
             const int b = 4 * nb + c;
             if (b < B) {
-              float st = 0.f;
-              int vsum = 0;
-#pragma unroll
-              for (int bb = 0; bb < 4 * NB; ++bb)
-                if (bb == b) { st = step[bb]; vsum = vs[bb]; }
-              part[(size_t)b * S16 + row] = st * (float)(vsum - 2 * (2 * h0 + (l0 >> 7)));
-              part[(size_t)b * S16 + row + 8] = st * (float)(vsum - 2 * (2 * h1 + (l1 >> 7)));
+              const float st = xst[b].step;
+              const int vsum = xst[b].sum;
+              part[((size_t)b * S16 + row) * ns4] = st * (float)(vsum - 2 * (2 * h0 + (l0 >> 7)));
+              part[((size_t)b * S16 + row + 8) * ns4] = st * (float)(vsum - 2 * (2 * h1 + (l1 >> 7)));
             }
           }
         }
@@ -519,13 +596,7 @@ __global__ void __launch_bounds__(kVWarps * 32) finalize_kernel(const DecodeArgs
   float* tp = reinterpret_cast<float*>(smem);   // [B][S16]
   const int tid = threadIdx.x;
   const int B = a.batch;
-  // (layer, path) of this CTA
-  int lo = 0, hi = a.n_layers - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.layers[mid].p_begin <= (int)blockIdx.x) lo = mid; else hi = mid - 1;
-  }
-  const LayerDesc& L = a.layers[lo];
+  const LayerDesc& L = a.layers[layer_of(a.item_layer.p, a.n_layers, blockIdx.x)];
   const int p = blockIdx.x - L.p_begin;
   const PathDesc& P = L.p[p];
   const int s = L.s, S16 = (s + 15) & ~15, S32 = (s + 31) & ~31;
@@ -533,11 +604,23 @@ __global__ void __launch_bounds__(kVWarps * 32) finalize_kernel(const DecodeArgs
   int ts[4 * NB];
 #pragma unroll
   for (int b = 0; b < 4 * NB; ++b) { mt[b] = 0.f; ts[b] = 0; }
+  // a latent row's slice partials are contiguous: float4 loads, summed in slice order
+  const int ns = L.n_slices, ng = (ns + 3) >> 2;
+#pragma unroll 2
   for (int i = tid; i < B * S16; i += kVWarps * 32) {
     const int b = i / S16, j = i - b * S16;
     float t = 0.f;
     if (j < s) {
-      for (int q = 0; q < L.n_slices; ++q) t += P.ws.partial[((size_t)q * B) * S16 + i];
+      const float4* pp = reinterpret_cast<const float4*>(P.ws.partial) + (size_t)i * ng;
+#pragma unroll 4
+      for (int q4 = 0; q4 < ng; ++q4) {
+        const float4 v = pp[q4];
+        const int q = 4 * q4;
+        t += v.x;
+        if (q + 1 < ns) t += v.y;
+        if (q + 2 < ns) t += v.z;
+        if (q + 3 < ns) t += v.w;
+      }
       t *= h2f(P.l[j]);
     }
     tp[i] = t;
@@ -700,7 +783,7 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
   __syncwarp();
 
   OutCursor fd;
-  fd.enter(a, find_layer(a, i_begin, false));
+  fd.enter(a, layer_of(a.item_layer.u, a.n_layers, i_begin));
   fd.item = i_begin;
   fd.p = 0;
   fd.kt0 = 0;
@@ -799,10 +882,12 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
 
 // ------------------------------------------------------------------ launchers
 
-size_t latent_smem(int nb) {
-  const int rpw = nb == 1 ? 2 : 1;
-  return (size_t)kVWarps * kVStages * rpw * kChunkBytes + (size_t)kVSlice * 8 * nb + (size_t)kVWarps * kVStages * 8;
+template <int NB, int RB>
+constexpr size_t latent_smem() {
+  return (size_t)kVWarps * kVStages * VCfg<NB>::kRPW * kChunkBytes + 2 * (size_t)xq_buf_bytes(NB, RB) +
+         ((size_t)kVWarps * kVStages + 2) * 8;
 }
+
 
 template <int NB>
 cudaError_t launch_finalize(const DecodeArgs& a, int max_s16, cudaStream_t st) {
@@ -823,24 +908,26 @@ size_t output_smem(int) {
   return (size_t)kUWarps * OutCfg<NB>::kStages * out_stage_bytes(4 * NB) + (size_t)kUWarps * OutCfg<NB>::kStages * 8;
 }
 
-template <int NB>
-cudaError_t launch_latent(const DecodeArgs& a, int max_s16, int num_sms, cudaStream_t st) {
-  const size_t smem = latent_smem(NB);
+template <int NB, int RB>
+cudaError_t launch_latent(const DecodeArgs& a, int num_sms, cudaStream_t st) {
+  static_assert(RB == 4 * NB || (NB == 1 && RB == 1), "stored rows: 1 at batch 1, else 4 per n-block");
+  constexpr size_t smem = latent_smem<NB, RB>();
+  static_assert(smem <= 227 * 1024, "latent pass shared memory");
   static bool attr_set = false;
   cudaError_t e;
   if (!attr_set) {
-    e = cudaFuncSetAttribute(latent_pass_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(latent_pass_kernel<NB, RB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   static int per_sm = 0;
   if (per_sm == 0) {
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, latent_pass_kernel<NB>, kVWarps * 32, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, latent_pass_kernel<NB, RB>, kVWarps * 32, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
   }
   const int grid = max(1, min(a.v_items, per_sm * num_sms));
-  latent_pass_kernel<NB><<<grid, kVWarps * 32, smem, st>>>(a);
+  latent_pass_kernel<NB, RB><<<grid, kVWarps * 32, smem, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -866,12 +953,19 @@ cudaError_t launch_output(const DecodeArgs& a, int num_sms, cudaStream_t st) {
 
 }  // namespace
 
-cudaError_t launch_latent_pass(const DecodeArgs& a, int max_s16, int num_sms, cudaStream_t st) {
+cudaError_t launch_quantise_pass(const DecodeArgs& a, cudaStream_t st) {
+  if (a.x_items < 1) return cudaErrorInvalidValue;
+  quantise_input_kernel<<<(a.x_items + kQWarps - 1) / kQWarps, kQWarps * 32, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_latent_pass(const DecodeArgs& a, int, int num_sms, cudaStream_t st) {
+  if (a.batch == 1) return launch_latent<1, 1>(a, num_sms, st);
   switch ((a.batch + 3) / 4) {
-    case 1: return launch_latent<1>(a, max_s16, num_sms, st);
-    case 2: return launch_latent<2>(a, max_s16, num_sms, st);
-    case 3: return launch_latent<3>(a, max_s16, num_sms, st);
-    case 4: return launch_latent<4>(a, max_s16, num_sms, st);
+    case 1: return launch_latent<1, 4>(a, num_sms, st);
+    case 2: return launch_latent<2, 8>(a, num_sms, st);
+    case 3: return launch_latent<3, 12>(a, num_sms, st);
+    case 4: return launch_latent<4, 16>(a, num_sms, st);
   }
   return cudaErrorInvalidValue;
 }

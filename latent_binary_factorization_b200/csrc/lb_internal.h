@@ -23,9 +23,24 @@ constexpr int kVWarps = 4;
 constexpr int kVSliceTiles = 8;
 constexpr int kVSlice = kVSliceTiles * kVTileK;          // 2048 inputs
 constexpr int kVRowChunk = 2 * kVWarps;                  // 16-row blocks per item
-constexpr int kVStages = 3;                              // bulk-copy ring per warp
+constexpr int kVStages = 2;                              // bulk-copy ring per warp
 constexpr int kChunkTiles = 4;                           // K-tiles per bulk copy
 constexpr int kChunkBytes = kChunkTiles * kTileBytes;    // 2048
+
+// Quantised input slice (u = g * x on kVSlice inputs, per batch row), written by
+// the quantise pass and copied whole into the latent pass's shared memory:
+//   [TStat x 4*nb]  step and sum of v per batch row (rows >= batch are zero)
+//   [K-block kb][column n][thread c] (b0, b1) B-fragment pairs of the int8
+//       mma: b0 = inputs 32kb + 4c .. +3, b1 = inputs 32kb + 16 + 4c .. +3;
+//       column 2r holds batch row r's hi bytes, 2r + 1 its lo bytes.
+// xq_rows(batch) rows are stored: one at batch 1 (the product's other columns
+// then repeat row 0 and their sums are ignored), else 4*nb.
+__host__ __device__ inline int xq_nb(int batch) { return (batch + 3) / 4; }
+__host__ __device__ inline int xq_rows(int batch) { return batch == 1 ? 1 : 4 * xq_nb(batch); }
+__host__ __device__ inline int xq_stats_bytes(int batch) { return 64 * xq_nb(batch); }
+__host__ __device__ inline int xq_slice_bytes(int batch) {
+  return (xq_stats_bytes(batch) + kVSlice * 2 * xq_rows(batch) + 127) & ~127;
+}
 
 // Output pass (U) work item: (layer, 128 output rows), one warp.
 constexpr int kUWarps = 4;
@@ -49,17 +64,18 @@ struct TStat {
   int pad[2];
 };
 
-// Per-path scratch written by the latent pass and read by the output pass.
-//   partial : [n_slices][batch][s16] fp32  sums of one input slice
-//   planes  : [s32/32][4*nb][2][32] int8    hi and lo bytes of t', K-tile major
-//                                            (nb = ceil(batch/4); rows >= batch are zero)
-//   tstat   : [4*nb] TStat
-//   counter : unused (kept zero)
+// Per-path scratch of the decode passes.
+//   xq      : [n_slices][xq_slice_bytes]        quantised input slices (quantise pass)
+//   partial : [batch][s16][ns4] fp32             latent sums per input slice (latent pass;
+//                                                ns4 = n_slices rounded up to 4, pad unused)
+//   planes  : [s32/32][4*nb][2][32] int8         hi and lo bytes of t', K-tile major
+//                                                (nb = ceil(batch/4); rows >= batch are zero)
+//   tstat   : [4*nb] TStat                        (planes and tstat: finalize pass)
 struct PathScratch {
+  unsigned char* xq;
   float* partial;
   int8_t* planes;
   TStat* tstat;
-  unsigned int* counter;
 };
 
 struct PathDesc {
@@ -81,20 +97,33 @@ struct LayerDesc {
   int v_begin;        // first latent-pass work item of this layer
   int u_begin;        // first output-pass work item of this layer
   int p_begin;        // first (layer, path) index of this layer
-  int pad;
+  int x_begin;        // first quantise-pass item (layer, path, slice) of this layer
+};
+
+// Layer index of every work item of each pass (device arrays built with the
+// table; null when the call has one layer, whose index is 0).
+struct ItemLayers {
+  const int* x;   // quantise items
+  const int* v;   // latent items
+  const int* p;   // (layer, path) items
+  const int* u;   // output items
 };
 
 struct DecodeArgs {
   const LayerDesc* layers;  // device table
+  ItemLayers item_layer;
   unsigned int* status;     // device error word (LB_ERR_TIMEOUT bit on a wait timeout)
   int n_layers;
   int batch;
   int v_items;              // total latent-pass items
   int u_items;              // total output-pass items (layer, 128-row block)
   int p_items;              // total (layer, path) pairs
+  int x_items;              // total quantise-pass items (layer, path, input slice)
 };
 
-// Launchers (decode.cu).  The batch selects the template (4 rows per n-block).
+// Launchers (decode.cu), in stream order quantise -> latent -> finalize ->
+// output.  The batch selects the template (4 rows per n-block).
+cudaError_t launch_quantise_pass(const DecodeArgs& a, cudaStream_t st);
 cudaError_t launch_latent_pass(const DecodeArgs& a, int max_s16, int num_sms, cudaStream_t st);
 cudaError_t launch_finalize_pass(const DecodeArgs& a, int max_s16, cudaStream_t st);
 cudaError_t launch_output_pass(const DecodeArgs& a, int num_sms, cudaStream_t st);

@@ -61,8 +61,12 @@ lb_status check_layer(const lb_layer& L) {
 }
 
 // Bytes of per-path scratch for one layer at this batch.
+size_t xq_bytes(const lb_layer& L, int batch) {
+  return align_up((size_t)lb::ceil_div(L.d_in, lb::kVSlice) * lb::xq_slice_bytes(batch), 256);
+}
 size_t partial_bytes(const lb_layer& L, int batch) {
-  return align_up((size_t)lb::ceil_div(L.d_in, lb::kVSlice) * batch * lb::s16(L.s) * sizeof(float), 256);
+  const size_t ns4 = (size_t)lb::ceil_div(lb::ceil_div(L.d_in, lb::kVSlice), 4) * 4;
+  return align_up(ns4 * batch * lb::s16(L.s) * sizeof(float), 256);
 }
 // t' planes and stats are padded to whole groups of four batch rows
 size_t planes_bytes(const lb_layer& L, int batch) {
@@ -70,7 +74,7 @@ size_t planes_bytes(const lb_layer& L, int batch) {
 }
 size_t tstat_bytes(int batch) { return align_up((size_t)lb::ceil_div(batch, 4) * 4 * sizeof(lb::TStat), 256); }
 size_t path_scratch_bytes(const lb_layer& L, int batch) {
-  return partial_bytes(L, batch) + planes_bytes(L, batch) + tstat_bytes(batch);
+  return xq_bytes(L, batch) + partial_bytes(L, batch) + planes_bytes(L, batch) + tstat_bytes(batch);
 }
 
 constexpr size_t kStatusBytes = 256;   // device status word at the start of a workspace
@@ -81,15 +85,26 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
 
-  // ---- sizes: [status][table][counters][per-path scratch...]
-  const size_t table_bytes = align_up((size_t)n * sizeof(lb::LayerDesc), 256);
-  const size_t counter_bytes = align_up((size_t)n * 2 * sizeof(unsigned int), 256);
-  size_t total = kStatusBytes + table_bytes + counter_bytes;
+  // ---- work items of each pass, per layer
+  int x_items = 0, v_items = 0, p_items = 0, u_items = 0;
   int max_s16 = 16;
+  size_t scratch = 0;
   for (int i = 0; i < n; ++i) {
-    total += (size_t)(layers[i].residual + 1) * path_scratch_bytes(layers[i], batch);
-    max_s16 = std::max(max_s16, lb::s16(layers[i].s));
+    const lb_layer& L = layers[i];
+    const int npaths = L.residual + 1, n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
+    x_items += npaths * n_slices;
+    v_items += npaths * n_slices * lb::ceil_div(lb::s16(L.s) / 16, lb::kVRowChunk);
+    p_items += npaths;
+    u_items += L.d_out / lb::kUTileRows;
+    scratch += (size_t)npaths * path_scratch_bytes(L, batch);
+    max_s16 = std::max(max_s16, lb::s16(L.s));
   }
+  const int n_items = x_items + v_items + p_items + u_items;
+
+  // ---- sizes: [status][table][item -> layer maps][per-path scratch...]
+  const size_t table_bytes = align_up((size_t)n * sizeof(lb::LayerDesc), 256);
+  const size_t map_bytes = align_up((size_t)n_items * sizeof(int), 256);
+  const size_t total = kStatusBytes + table_bytes + map_bytes + scratch;
 
   std::lock_guard<std::mutex> lock(g_mu);
   Workspace& ws = g_ws[{dev, st}];
@@ -106,17 +121,24 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
     if (e != cudaSuccess) return cuda_fail(e);
     ws.cap = cap;
     ws.table.clear();
-    e = cudaMemsetAsync(ws.buf, 0, cap, st);   // counters start at zero
+    e = cudaMemsetAsync(ws.buf, 0, cap, st);   // the status word starts at zero
     if (e != cudaSuccess) return cuda_fail(e);
   }
 
-  // ---- descriptor table
+  // ---- descriptor table and item maps
   unsigned char* base = static_cast<unsigned char*>(ws.buf);
   lb::LayerDesc* table = reinterpret_cast<lb::LayerDesc*>(base + kStatusBytes);
-  unsigned int* counters = reinterpret_cast<unsigned int*>(base + kStatusBytes + table_bytes);
-  size_t off = kStatusBytes + table_bytes + counter_bytes;
-  std::vector<lb::LayerDesc> tab(n);
-  int v_items = 0, u_items = 0, p_items = 0;
+  int* maps = reinterpret_cast<int*>(base + kStatusBytes + table_bytes);
+  size_t off = kStatusBytes + table_bytes + map_bytes;
+  // the table and the maps are one host block, compared and uploaded together
+  const size_t tb = (size_t)n * sizeof(lb::LayerDesc);
+  std::vector<unsigned char> host(tb + (size_t)n_items * sizeof(int));
+  lb::LayerDesc* tab = reinterpret_cast<lb::LayerDesc*>(host.data());
+  int* xm = reinterpret_cast<int*>(host.data() + tb);
+  int* vm = xm + x_items;
+  int* pm = vm + v_items;
+  int* um = pm + p_items;
+  int xi = 0, vi = 0, pi = 0, ui = 0;
   for (int i = 0; i < n; ++i) {
     const lb_layer& L = layers[i];
     lb::LayerDesc& D = tab[i];
@@ -129,12 +151,14 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
     D.npaths = L.residual + 1;
     D.n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
     D.n_rchunks = lb::ceil_div(lb::s16(L.s) / 16, lb::kVRowChunk);
-    D.v_begin = v_items;
-    D.u_begin = u_items;
-    D.p_begin = p_items;
-    p_items += D.npaths;
-    v_items += D.npaths * D.n_slices * D.n_rchunks;
-    u_items += L.d_out / lb::kUTileRows;
+    D.x_begin = xi;
+    D.v_begin = vi;
+    D.p_begin = pi;
+    D.u_begin = ui;
+    for (int k = 0; k < D.npaths * D.n_slices; ++k) xm[xi++] = i;
+    for (int k = 0; k < D.npaths * D.n_slices * D.n_rchunks; ++k) vm[vi++] = i;
+    for (int k = 0; k < D.npaths; ++k) pm[pi++] = i;
+    for (int k = 0; k < L.d_out / lb::kUTileRows; ++k) um[ui++] = i;
     for (int p = 0; p < D.npaths; ++p) {
       lb::PathDesc& P = D.p[p];
       P.V = static_cast<const uint4*>(L.path[p].V_bits);
@@ -142,38 +166,44 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
       P.h = L.path[p].h;
       P.g = L.path[p].g;
       P.l = L.path[p].l;
+      P.ws.xq = base + off;
+      off += xq_bytes(L, batch);
       P.ws.partial = reinterpret_cast<float*>(base + off);
       off += partial_bytes(L, batch);
       P.ws.planes = reinterpret_cast<int8_t*>(base + off);
       off += planes_bytes(L, batch);
       P.ws.tstat = reinterpret_cast<lb::TStat*>(base + off);
       off += tstat_bytes(batch);
-      P.ws.counter = counters + 2 * i + p;
     }
   }
-  const size_t tb = (size_t)n * sizeof(lb::LayerDesc);
-  if (ws.table.size() != tb || std::memcmp(ws.table.data(), tab.data(), tb) != 0) {
-    // pageable source: the call returns once the bytes are staged, so `tab`
-    // may go out of scope; stream order protects kernels still reading the table
-    e = cudaMemcpyAsync(table, tab.data(), tb, cudaMemcpyHostToDevice, st);
+  if (ws.table.size() != host.size() || std::memcmp(ws.table.data(), host.data(), host.size()) != 0) {
+    // pageable source: the calls return once the bytes are staged, so `host`
+    // may go out of scope; stream order protects kernels still reading them
+    e = cudaMemcpyAsync(table, host.data(), tb, cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return cuda_fail(e);
-    // the counters' offset depends on the table size, so bytes that earlier
-    // calls used as scratch may now hold counters: start them at zero
-    e = cudaMemsetAsync(counters, 0, counter_bytes, st);
-    if (e != cudaSuccess) return cuda_fail(e);
-    ws.table.assign(reinterpret_cast<unsigned char*>(tab.data()),
-                    reinterpret_cast<unsigned char*>(tab.data()) + tb);
+    if (n_items > 0) {
+      e = cudaMemcpyAsync(maps, host.data() + tb, (size_t)n_items * sizeof(int), cudaMemcpyHostToDevice, st);
+      if (e != cudaSuccess) return cuda_fail(e);
+    }
+    ws.table.swap(host);
   }
 
   lb::DecodeArgs a;
   a.layers = table;
+  a.item_layer.x = maps;
+  a.item_layer.v = maps + x_items;
+  a.item_layer.p = maps + x_items + v_items;
+  a.item_layer.u = maps + x_items + v_items + p_items;
   a.status = reinterpret_cast<unsigned int*>(base);
   a.n_layers = n;
   a.batch = batch;
   a.v_items = v_items;
   a.u_items = u_items;
   a.p_items = p_items;
+  a.x_items = x_items;
   const int sms = num_sms(dev);
+  e = lb::launch_quantise_pass(a, st);
+  if (e != cudaSuccess) return cuda_fail(e);
   e = lb::launch_latent_pass(a, max_s16, sms, st);
   if (e != cudaSuccess) return cuda_fail(e);
   e = lb::launch_finalize_pass(a, max_s16, st);

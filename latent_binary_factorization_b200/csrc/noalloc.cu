@@ -22,13 +22,12 @@ constexpr size_t kNoAllocScratchBytes = 1u << 20;   // 1 MiB per device
 // device symbol: its device address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Layout inside the array: [status word][one LayerDesc][2 counters][per path:
-// partial | planes | tstat], each region 256-byte aligned.
+// Layout inside the array: [status word][one LayerDesc][per path: xq | partial
+// | planes | tstat], each region 256-byte aligned.
 constexpr size_t kStatusOff = 0;
 constexpr size_t kTableOff = 256;
-constexpr size_t kCounterOff = 512;
-constexpr size_t kPathOff = 768;
-static_assert(sizeof(lb::LayerDesc) <= kCounterOff - kTableOff, "layer descriptor must fit its slot");
+constexpr size_t kPathOff = 512;
+static_assert(sizeof(lb::LayerDesc) <= kPathOff - kTableOff, "layer descriptor must fit its slot");
 
 constexpr int kMaxDevices = 64;
 unsigned char* g_scratch_dev[kMaxDevices] = {nullptr};   // device address per device, set once
@@ -68,12 +67,13 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
   // scratch needed by this layer at this batch
   const int n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
   const int S16 = lb::s16(L.s), S32 = lb::s32(L.s);
-  const size_t part_b = round256((size_t)n_slices * batch * S16 * sizeof(float));
+  const size_t xq_b = round256((size_t)n_slices * lb::xq_slice_bytes(batch));
+  const size_t part_b = round256((size_t)lb::ceil_div(n_slices, 4) * 4 * batch * S16 * sizeof(float));
   const int bpad = lb::ceil_div(batch, 4) * 4;   // t' planes and stats padded to groups of 4 rows
   const size_t planes_b = round256((size_t)bpad * 2 * S32);
   const size_t tstat_b = round256((size_t)bpad * sizeof(lb::TStat));
   const int npaths = L.residual + 1;
-  if (kPathOff + (size_t)npaths * (part_b + planes_b + tstat_b) > kNoAllocScratchBytes) return LB_ERR_SHAPE;
+  if (kPathOff + (size_t)npaths * (xq_b + part_b + planes_b + tstat_b) > kNoAllocScratchBytes) return LB_ERR_SHAPE;
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -101,8 +101,8 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
   D.v_begin = 0;
   D.u_begin = 0;
   D.p_begin = 0;
+  D.x_begin = 0;
   size_t off = kPathOff;
-  unsigned int* counters = reinterpret_cast<unsigned int*>(base + kCounterOff);
   for (int p = 0; p < npaths; ++p) {
     lb::PathDesc& P = D.p[p];
     P.V = static_cast<const uint4*>(L.path[p].V_bits);
@@ -110,32 +110,37 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
     P.h = L.path[p].h;
     P.g = L.path[p].g;
     P.l = L.path[p].l;
+    P.ws.xq = base + off;
+    off += xq_b;
     P.ws.partial = reinterpret_cast<float*>(base + off);
     off += part_b;
     P.ws.planes = reinterpret_cast<int8_t*>(base + off);
     off += planes_b;
     P.ws.tstat = reinterpret_cast<lb::TStat*>(base + off);
     off += tstat_b;
-    P.ws.counter = counters + p;
   }
-  // every call shares the array: the counters and the status word must start
-  // at zero, whatever the previous call left there
-  e = cudaMemsetAsync(base, 0, kPathOff, st);
+  // every call shares the array: the status word must start at zero, whatever
+  // the previous call left there (every other region is written before it is read)
+  e = cudaMemsetAsync(base + kStatusOff, 0, kTableOff - kStatusOff, st);
   if (e != cudaSuccess) return LB_ERR_CUDA;
   e = cudaMemcpyAsync(base + kTableOff, &D, sizeof(D), cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return LB_ERR_CUDA;
 
   lb::DecodeArgs a;
   a.layers = reinterpret_cast<const lb::LayerDesc*>(base + kTableOff);
+  a.item_layer = lb::ItemLayers{nullptr, nullptr, nullptr, nullptr};   // one layer: index 0
   a.status = reinterpret_cast<unsigned int*>(base + kStatusOff);
   a.n_layers = 1;
   a.batch = batch;
   a.v_items = npaths * D.n_slices * D.n_rchunks;
   a.u_items = L.d_out / lb::kUTileRows;
   a.p_items = npaths;
+  a.x_items = npaths * D.n_slices;
   int sms = 0;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess || sms <= 0) return LB_ERR_CUDA;
+  e = lb::launch_quantise_pass(a, st);
+  if (e != cudaSuccess) return LB_ERR_CUDA;
   e = lb::launch_latent_pass(a, S16, sms, st);
   if (e != cudaSuccess) return LB_ERR_CUDA;
   e = lb::launch_finalize_pass(a, S16, st);

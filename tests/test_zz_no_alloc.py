@@ -78,7 +78,7 @@ def test_noalloc_matches_regular_forward_twice_in_a_row(env):
 
 def test_noalloc_rejects_scratch_beyond_its_array(env):
     lb, layers, f = env
-    # 32768 inputs (8 slices) x 16 rows x 1024 latent rows x 4 B x 2 paths = 1 MiB of partials alone
+    # 32768 inputs (16 slices) x 16 rows x 1024 latent rows x 4 B x 2 paths = 2 MiB of partials alone
     L = lb.LbLayer()
     L.d_in, L.d_out, L.s, L.residual = 32768, 128, 1024, 1
     for p in range(2):
