@@ -494,29 +494,35 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 4 : 1) latent_pass_ker
     const uint2* frag = reinterpret_cast<const uint2*>(xb + 64 * NB);
     const TStat* xst = reinterpret_cast<const TStat*>(xb);
 
-    // ---- this warp's row blocks over the slice
+    // ---- this warp's row blocks over the slice, RPW at once.  A block past the
+    //      last one (odd count) still runs its products on whatever its stage
+    //      half holds, so that the product loop has no branches; its sums are
+    //      not written.
+    const int ns4 = (L.n_slices + 3) & ~3;
+    float* part = P.ws.partial + it.sl;
 #pragma unroll 1
     for (int grp = 0; grp * RPW < 2; ++grp) {
       const int rbA = it.rc * kVRowChunk + 2 * warp + grp * RPW;
       if (rbA >= n_rb) break;
-      const bool hasB = RPW == 2 && rbA + 1 < n_rb;
-      int d[RPW][8][NB][4];
+      const int nvalid = min(RPW, n_rb - rbA);
+      constexpr int R = RPW;
+      int d[R][8][NB][4];
 #pragma unroll 1
       for (int kc = 0; kc * kChunkTiles < nkt; ++kc) {
         if (!dead && !mbar_wait(&my_bar[slot], (consumed / kVStages) & 1)) {
           dead = true;
           atomicOr(a.status, 1u << LB_ERR_TIMEOUT);
         }
-        const unsigned char* stage = my_ring + slot * kStageBytes;
+        const unsigned char* stage = my_ring + slot * kStageBytes + lane * 16;
+        const uint2* fc = frag + (size_t)kc * kChunkTiles * 8 * NC * 4;
         const int ntile = min(kChunkTiles, nkt - kc * kChunkTiles);
-        // one K-tile of the chunk for both row blocks
+        // one K-tile of the chunk for the R row blocks
         auto ktile = [&](int t, bool first) {
-          uint4 cur[RPW];
+          uint4 cur[R];
 #pragma unroll
-          for (int r = 0; r < RPW; ++r)
-            cur[r] = (r == 0 || hasB) ? *reinterpret_cast<const uint4*>(stage + r * kChunkBytes + t * kTileBytes + lane * 16)
-                                      : make_uint4(0, 0, 0, 0);
-          const uint2* fk = frag + (size_t)(kc * kChunkTiles + t) * 8 * NC * 4;
+          for (int r = 0; r < R; ++r)
+            cur[r] = *reinterpret_cast<const uint4*>(stage + r * kChunkBytes + t * kTileBytes);
+          const uint2* fk = fc + t * 8 * NC * 4;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const uint32_t m = 0x01010101u << q;
@@ -524,12 +530,10 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 4 : 1) latent_pass_ker
             for (int nb = 0; nb < NB; ++nb) {
               const uint2 bb = fk[q * NC * 4 + boff[nb]];
 #pragma unroll
-              for (int r = 0; r < RPW; ++r) {
-                if (r == 0 || hasB) {
-                  const uint32_t a0 = cur[r].x & m, a1 = cur[r].y & m, a2 = cur[r].z & m, a3 = cur[r].w & m;
-                  if (first) mma_u8s8_zc(d[r][q][nb], a0, a1, a2, a3, bb.x, bb.y);
-                  else mma_u8s8(d[r][q][nb], a0, a1, a2, a3, bb.x, bb.y);
-                }
+              for (int r = 0; r < R; ++r) {
+                const uint32_t a0 = cur[r].x & m, a1 = cur[r].y & m, a2 = cur[r].z & m, a3 = cur[r].w & m;
+                if (first) mma_u8s8_zc(d[r][q][nb], a0, a1, a2, a3, bb.x, bb.y);
+                else mma_u8s8(d[r][q][nb], a0, a1, a2, a3, bb.x, bb.y);
               }
             }
           }
@@ -553,29 +557,26 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 4 : 1) latent_pass_ker
       }
       // fold: sum_q D_q / 2^q per plane = 2^-7 * sum_q D_q * 2^(7-q) (each term a
       // multiple of 2^7), then 256*hi + lo; slice partial = step*(sum v - 2*that)
-      const int ns4 = (L.n_slices + 3) & ~3;
-      float* part = P.ws.partial + it.sl;
 #pragma unroll
-      for (int r = 0; r < RPW; ++r) {
-        if (r == 0 || hasB) {
-          const int row = 16 * (rbA + r) + g;
+      for (int r = 0; r < R; ++r) {
+        if (r >= nvalid) break;
+        const int row = 16 * (rbA + r) + g;
 #pragma unroll
-          for (int nb = 0; nb < NB; ++nb) {
-            int h0 = d[r][0][nb][0], l0 = d[r][0][nb][1], h1 = d[r][0][nb][2], l1 = d[r][0][nb][3];
+        for (int nb = 0; nb < NB; ++nb) {
+          int h0 = d[r][0][nb][0], l0 = d[r][0][nb][1], h1 = d[r][0][nb][2], l1 = d[r][0][nb][3];
 #pragma unroll
-            for (int q = 1; q < 8; ++q) {
-              h0 = 2 * h0 + d[r][q][nb][0];
-              l0 = 2 * l0 + d[r][q][nb][1];
-              h1 = 2 * h1 + d[r][q][nb][2];
-              l1 = 2 * l1 + d[r][q][nb][3];
-            }
-            const int b = 4 * nb + c;
-            if (b < B) {
-              const float st = xst[b].step;
-              const int vsum = xst[b].sum;
-              part[((size_t)b * S16 + row) * ns4] = st * (float)(vsum - 2 * (2 * h0 + (l0 >> 7)));
-              part[((size_t)b * S16 + row + 8) * ns4] = st * (float)(vsum - 2 * (2 * h1 + (l1 >> 7)));
-            }
+          for (int q = 1; q < 8; ++q) {
+            h0 = 2 * h0 + d[r][q][nb][0];
+            l0 = 2 * l0 + d[r][q][nb][1];
+            h1 = 2 * h1 + d[r][q][nb][2];
+            l1 = 2 * l1 + d[r][q][nb][3];
+          }
+          const int b = 4 * nb + c;
+          if (b < B) {
+            const float st = xst[b].step;
+            const int vsum = xst[b].sum;
+            part[((size_t)b * S16 + row) * ns4] = st * (float)(vsum - 2 * (2 * h0 + (l0 >> 7)));
+            part[((size_t)b * S16 + row + 8) * ns4] = st * (float)(vsum - 2 * (2 * h1 + (l1 >> 7)));
           }
         }
       }
@@ -742,7 +743,7 @@ __device__ __forceinline__ void out_issue(const OutCursor& cu, unsigned char* st
 // One K-tile of one path: eight m16n8k32 products (row block q = 0..7).
 // `pl` points at this thread's t' bytes of tile t (batch row g/2, plane g%2);
 // `pl_step` = B * 64 bytes from one tile's t' bytes to the next.
-template <int NB>
+template <int NB, bool kFirst = false>
 __device__ __forceinline__ void out_tile(int (&d)[8][NB][4], const unsigned char* stage, int t, int lane,
                                          const unsigned char* pl) {
   const uint4 cur = *reinterpret_cast<const uint4*>(stage + t * kTileBytes + lane * 16);
@@ -757,7 +758,10 @@ __device__ __forceinline__ void out_tile(int (&d)[8][NB][4], const unsigned char
     const uint32_t m = 0x01010101u << q;
     const uint32_t a0 = cur.x & m, a1 = cur.y & m, a2 = cur.z & m, a3 = cur.w & m;
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) mma_u8s8(d[q][nb], a0, a1, a2, a3, b0[nb], b1[nb]);
+    for (int nb = 0; nb < NB; ++nb) {
+      if (kFirst) mma_u8s8_zc(d[q][nb], a0, a1, a2, a3, b0[nb], b1[nb]);   // a path's first K-tile
+      else mma_u8s8(d[q][nb], a0, a1, a2, a3, b0[nb], b1[nb]);
+    }
   }
 }
 
@@ -797,15 +801,10 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
     }
   }
 
+  // d starts at a path's first K-tile (zero-accumulator product); yacc at its
+  // first path (assigned, not added)
   float yacc[8][2][NB];
   int d[8][NB][4];
-#pragma unroll
-  for (int q = 0; q < 8; ++q)
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      yacc[q][0][nb] = yacc[q][1][nb] = 0.f;
-      d[q][nb][0] = d[q][nb][1] = d[q][nb][2] = d[q][nb][3] = 0;
-    }
   uint32_t consumed = 0;
   int slot = 0;
   bool dead = false;
@@ -820,17 +819,20 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
     const unsigned char* stage = my_ring + slot * sb;
     const int nt = cs.ntile();
     const unsigned char* pl = stage + pl_off;
+    if (cs.kt0 == 0) out_tile<NB, true>(d, stage, 0, lane, pl);
+    else out_tile<NB>(d, stage, 0, lane, pl);
     if (nt == kUChunkTiles) {
 #pragma unroll
-      for (int t = 0; t < kUChunkTiles; ++t) out_tile<NB>(d, stage, t, lane, pl);
+      for (int t = 1; t < kUChunkTiles; ++t) out_tile<NB>(d, stage, t, lane, pl);
     } else {
 #pragma unroll 1
-      for (int t = 0; t < nt; ++t) out_tile<NB>(d, stage, t, lane, pl);
+      for (int t = 1; t < nt; ++t) out_tile<NB>(d, stage, t, lane, pl);
     }
     if (cs.path_end()) {
       // path finished: rows 128*ob + 16q + g (+8), batch row 4nb + c
       const uint16_t* hs = reinterpret_cast<const uint16_t*>(stage + out_h_off(BP));
       const TStat* tst = reinterpret_cast<const TStat*>(stage + out_tstat_off(BP));
+      const bool first_path = cs.p == 0;
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb) {
         const int b = 4 * nb + c;
@@ -842,12 +844,11 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
           for (int q = 0; q < 8; ++q) {
             const int c0 = ((d[q][nb][0] >> q) << 8) + (d[q][nb][1] >> q);
             const int c1 = ((d[q][nb][2] >> q) << 8) + (d[q][nb][3] >> q);
-            yacc[q][0][nb] = fmaf(h2f(hs[16 * q + g]), fmaf(m2, (float)c0, base), yacc[q][0][nb]);
-            yacc[q][1][nb] = fmaf(h2f(hs[16 * q + g + 8]), fmaf(m2, (float)c1, base), yacc[q][1][nb]);
+            const float y0 = first_path ? 0.f : yacc[q][0][nb], y1 = first_path ? 0.f : yacc[q][1][nb];
+            yacc[q][0][nb] = fmaf(h2f(hs[16 * q + g]), fmaf(m2, (float)c0, base), y0);
+            yacc[q][1][nb] = fmaf(h2f(hs[16 * q + g + 8]), fmaf(m2, (float)c1, base), y1);
           }
         }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) d[q][nb][0] = d[q][nb][1] = d[q][nb][2] = d[q][nb][3] = 0;
       }
       if (cs.p == cs.npaths - 1) {
         const LayerDesc& L = a.layers[cs.li];
@@ -863,8 +864,6 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
               yr[16 * q + 8] = f2h(yacc[q][1][nb]);
             }
           }
-#pragma unroll
-          for (int q = 0; q < 8; ++q) yacc[q][0][nb] = yacc[q][1][nb] = 0.f;
         }
       }
     }
