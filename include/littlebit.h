@@ -121,13 +121,15 @@ typedef struct lb_layer {
 /*
  * y = forward(x) for one layer (formula at the top of this file).
  *   x_dev : batch x d_in row-major activations, y_dev : batch x d_out.
- *   Decode (1 <= batch <= 16): x and y are fp16 (xdt = LB_F16); two kernel
- *   launches (latent pass, output pass) with fp32/int32 accumulation.
- *   Prefill (batch >= 256, multiple of 128): xdt = LB_BF16, y bf16 --
- *   tensor-core path, see littlebit_linear_forward_many.
+ *   Decode (1 <= batch <= 16): x and y are fp16 (xdt = LB_F16); four kernel
+ *   launches (input quantisation, latent pass, finalize, output pass), int8
+ *   tensor-core products with int32 accumulation, fp32 scaling.
+ *   Prefill (batch a multiple of 128, batch * d_in <= 2^30): xdt = LB_F16 or
+ *   LB_BF16, y of the same type -- fp16 tcgen05 tensor-core path, see
+ *   littlebit_linear_forward_many.
  *   x_dev and y_dev must be 16-byte aligned; every other pointer as in lb_path.
  * Errors: LB_ERR_ARG, LB_ERR_ALIGN, LB_ERR_SHAPE, LB_ERR_UNSUPPORTED (batch
- * 17..255 or an unsupported dtype), LB_ERR_CUDA.
+ * 17..127 or not a multiple of 128, or an unsupported dtype), LB_ERR_CUDA.
  */
 lb_status littlebit_linear_forward(const lb_layer* layer, const void* x_dev, void* y_dev,
                                    int batch, lb_dtype xdt, void* stream);
@@ -135,17 +137,20 @@ lb_status littlebit_linear_forward(const lb_layer* layer, const void* x_dev, voi
 /*
  * The same forward for n independent layers (each with its own input and
  * output buffer, e.g. every linear layer of a model stack), done by the same
- * two launches for the whole list, so that the weights of all layers stream
- * from HBM back to back.  layers, xs, ys are host arrays of length n.
+ * launches for the whole list (decode: the four passes; prefill: operand
+ * preparation per layer and two grouped GEMM launches per group of layers),
+ * so that the weights of all layers stream from HBM back to back.  layers, xs,
+ * ys are host arrays of length n.
  */
 lb_status littlebit_linear_forward_many(const lb_layer* layers, int n, const void* const* xs,
                                         void* const* ys, int batch, lb_dtype xdt, void* stream);
 
 /*
- * littlebit_linear_forward_many, and in addition records `event_between`
- * (a cudaEvent_t passed as void*, or NULL) on `stream` between the latent-pass
- * launch and the output-pass launch, so that a caller can time the two
- * kernels separately with CUDA events.
+ * littlebit_linear_forward_many, and in addition, on the decode path, records
+ * `event_between` (a cudaEvent_t passed as void*, or NULL) on `stream` after
+ * the finalize launch and before the output-pass launch, so that a caller can
+ * time the two halves (V side: quantise, latent, finalize; U side: output)
+ * separately with CUDA events.
  */
 lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, const void* const* xs,
                                               void* const* ys, int batch, lb_dtype xdt, void* stream,

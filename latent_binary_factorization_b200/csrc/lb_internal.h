@@ -132,8 +132,12 @@ cudaError_t launch_output_pass(const DecodeArgs& a, int num_sms, cudaStream_t st
 int prefill_sp(int s, int npaths);
 size_t prefill_layer_bytes(int M, int d_in, int d_out, int s, int npaths);
 size_t prefill_table_bytes(int n_layers);
-cudaError_t launch_prefill_group(const LayerDesc* Ls, const void* const* xs, void* const* ys, int n, int M,
-                                 int x_bf16, unsigned char* ws, unsigned int* status, int num_sms, cudaStream_t st);
+constexpr int kPrefillMaxGroup = 4096;   // layers per group
+// A group's operand preparation, then its two grouped GEMM launches (same ws).
+cudaError_t launch_prefill_prep(const LayerDesc* Ls, const void* const* xs, int n, int M, int x_bf16,
+                                unsigned char* ws, cudaStream_t st);
+cudaError_t launch_prefill_gemms(const LayerDesc* Ls, void* const* ys, int n, int M, int x_bf16,
+                                 unsigned char* ws, unsigned int* status, int num_sms, cudaStream_t st);
 
 // pack.cu
 cudaError_t launch_pack(const void* src, lb_dtype dt, int n_long, int s, int64_t stride_long,

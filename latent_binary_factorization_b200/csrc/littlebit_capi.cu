@@ -30,7 +30,20 @@ struct Workspace {
   void* buf = nullptr;
   size_t cap = 0;
   std::vector<unsigned char> table;   // last descriptor table uploaded
+  // prefill: side stream for operand preparation and the events that order it
+  // against the caller's stream (created on first use)
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr, prep_done[2] = {nullptr, nullptr}, gemm_done[2] = {nullptr, nullptr};
 };
+
+void release_workspace(Workspace& w) {
+  if (w.buf) cudaFree(w.buf);
+  cudaEvent_t* evs[] = {&w.fork, &w.join, &w.prep_done[0], &w.prep_done[1], &w.gemm_done[0], &w.gemm_done[1]};
+  for (cudaEvent_t* ev : evs)
+    if (*ev) cudaEventDestroy(*ev);
+  if (w.side) cudaStreamDestroy(w.side);
+  w = Workspace{};
+}
 
 std::mutex g_mu;
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
@@ -217,25 +230,43 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   return LB_OK;
 }
 
-// Prefill (batch >= 128, multiple of 128): the tensor-core path.  Layers are
-// taken in groups whose operand buffers fit kPrefillGroupBytes; each group is
-// one set of operand preparations plus two grouped GEMM launches.
-constexpr size_t kPrefillGroupBytes = (size_t)4 << 30;
+// Prefill (batch a multiple of 128): the tensor-core path.  Layers are taken
+// in chunks whose operand buffers fit kPrefillChunkBytes; each chunk is one set
+// of operand preparations plus two grouped GEMM launches.  Chunks alternate
+// between two halves of the workspace, and the preparation of chunk c + 1 runs
+// on a side stream while the GEMMs of chunk c run on the caller's stream:
+// preparation is memory-bound and needs no shared memory, so its CTAs run
+// beside the GEMM's.  Events fork the side stream from the caller's stream and
+// join it back before the call returns, so stream order (and graph capture)
+// hold as for a single stream.
+constexpr size_t kPrefillChunkBytes = (size_t)512 << 20;
+
+cudaError_t ensure_side(Workspace& ws) {
+  if (ws.side) return cudaSuccess;
+  cudaError_t e = cudaStreamCreateWithFlags(&ws.side, cudaStreamNonBlocking);
+  if (e != cudaSuccess) return e;
+  cudaEvent_t* evs[] = {&ws.fork, &ws.join, &ws.prep_done[0], &ws.prep_done[1], &ws.gemm_done[0], &ws.gemm_done[1]};
+  for (cudaEvent_t* ev : evs) {
+    e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
 
 lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
                           int x_bf16, cudaStream_t st) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
-  // plan the groups
+  // plan the chunks
   std::vector<int> starts;
-  size_t need = 0, cur = 0;
+  size_t half = 0, cur = 0;
   int cnt = 0;
   for (int i = 0; i < n; ++i) {
     const size_t b = lb::prefill_layer_bytes(batch, layers[i].d_in, layers[i].d_out, layers[i].s,
                                              layers[i].residual + 1);
-    if (cnt == 0 || cur + b > kPrefillGroupBytes || cnt == 4096) {
-      if (cnt) need = std::max(need, cur + lb::prefill_table_bytes(cnt));
+    if (cnt == 0 || cur + b > kPrefillChunkBytes || cnt == lb::kPrefillMaxGroup) {
+      if (cnt) half = std::max(half, cur + lb::prefill_table_bytes(cnt));
       starts.push_back(i);
       cur = 0;
       cnt = 0;
@@ -243,14 +274,16 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
     cur += b;
     ++cnt;
   }
-  need = std::max(need, cur + lb::prefill_table_bytes(cnt)) + kStatusBytes;
+  half = align_up(std::max(half, cur + lb::prefill_table_bytes(cnt)), 1024);
   starts.push_back(n);
+  const int n_chunks = (int)starts.size() - 1;
+  const size_t need = kStatusBytes + (n_chunks > 1 ? 2 : 1) * half;
 
   std::lock_guard<std::mutex> lock(g_mu);
   Workspace& ws = g_ws[{dev, st}];
   if (ws.cap < need) {
     if (ws.buf) {
-      e = cudaStreamSynchronize(st);
+      e = cudaStreamSynchronize(st);   // the side stream always joins `st`
       if (e != cudaSuccess) return cuda_fail(e);
       cudaFree(ws.buf);
       ws.buf = nullptr;
@@ -284,13 +317,35 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
     }
   }
   const int sms = num_sms(dev);
-  for (size_t gi = 0; gi + 1 < starts.size(); ++gi) {
-    const int i0 = starts[gi], cnt_g = starts[gi + 1] - starts[gi];
-    e = lb::launch_prefill_group(descs.data() + i0, xs + i0, ys + i0, cnt_g, batch, x_bf16, base + kStatusBytes,
-                                 status, sms, st);
+  auto chunk_ws = [&](int c) { return base + kStatusBytes + (size_t)(c & 1) * half; };
+  if (n_chunks == 1) {
+    e = lb::launch_prefill_prep(descs.data(), xs, n, batch, x_bf16, chunk_ws(0), st);
     if (e != cudaSuccess) return cuda_fail(e);
+    e = lb::launch_prefill_gemms(descs.data(), ys, n, batch, x_bf16, chunk_ws(0), status, sms, st);
+    return e == cudaSuccess ? LB_OK : cuda_fail(e);
   }
-  return LB_OK;
+  e = ensure_side(ws);
+  if (e != cudaSuccess) return cuda_fail(e);
+  // fork: the side stream starts after everything already enqueued on `st`
+  e = cudaEventRecord(ws.fork, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(ws.side, ws.fork, 0);
+  if (e != cudaSuccess) return cuda_fail(e);
+  for (int c = 0; c < n_chunks && e == cudaSuccess; ++c) {
+    const int i0 = starts[c], cn = starts[c + 1] - starts[c], h = c & 1;
+    // the half was last used by chunk c - 2's GEMMs
+    if (c >= 2) e = cudaStreamWaitEvent(ws.side, ws.gemm_done[h], 0);
+    if (e == cudaSuccess) e = lb::launch_prefill_prep(descs.data() + i0, xs + i0, cn, batch, x_bf16, chunk_ws(c), ws.side);
+    if (e == cudaSuccess) e = cudaEventRecord(ws.prep_done[h], ws.side);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ws.prep_done[h], 0);
+    if (e == cudaSuccess)
+      e = lb::launch_prefill_gemms(descs.data() + i0, ys + i0, cn, batch, x_bf16, chunk_ws(c), status, sms, st);
+    if (e == cudaSuccess) e = cudaEventRecord(ws.gemm_done[h], st);
+  }
+  // join, also after an error, so that no side-stream work outlives the call's stream order
+  cudaError_t j = cudaEventRecord(ws.join, ws.side);
+  if (j == cudaSuccess) j = cudaStreamWaitEvent(st, ws.join, 0);
+  if (e == cudaSuccess) e = j;
+  return e == cudaSuccess ? LB_OK : cuda_fail(e);
 }
 
 }  // namespace
@@ -340,6 +395,9 @@ lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, con
   }
   if (batch % 128 == 0) {
     if (xdt != LB_F16 && xdt != LB_BF16) return LB_ERR_UNSUPPORTED;
+    // operand preparation indexes one layer's fp16 copy of x with 32-bit offsets
+    for (int i = 0; i < n; ++i)
+      if ((size_t)batch * layers[i].d_in > ((size_t)1 << 30)) return LB_ERR_SHAPE;
     return prefill_forward(layers, n, xs, ys, batch, xdt == LB_BF16 ? 1 : 0, static_cast<cudaStream_t>(stream));
   }
   return LB_ERR_UNSUPPORTED;
@@ -376,9 +434,7 @@ lb_status littlebit_device_status(void* stream, unsigned int* status) {
 
 void littlebit_release(void) {
   std::lock_guard<std::mutex> lock(g_mu);
-  for (auto& kv : g_ws) {
-    if (kv.second.buf) cudaFree(kv.second.buf);
-  }
+  for (auto& kv : g_ws) release_workspace(kv.second);
   g_ws.clear();
 }
 

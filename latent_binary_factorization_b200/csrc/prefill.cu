@@ -131,121 +131,136 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 
 // ------------------------------------------------------------------ operand preparation
 
-// x (M x K, fp16 or bf16, row-major) -> fp16 core-matrix tiles.  Thread t
-// writes the 16-byte chunk t of the output; eight consecutive threads read
-// one 128-byte run of a row.
+// x (M x K, fp16 or bf16, row-major) -> fp16 core-matrix tiles.  Work unit =
+// one 16-byte chunk of the output; eight consecutive units read one 128-byte
+// run of a row.  Each thread takes kXUnroll units spaced a grid apart and
+// issues all their loads before converting, so several loads are in flight.
+constexpr int kXUnroll = 4;
+
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
+  uint32_t* w = &v.x;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
+    const __half2 h = __floats2half2_rn(__bfloat162float(b.x), __bfloat162float(b.y));
+    w[e] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return v;
+}
+
 __global__ void __launch_bounds__(256) prep_x_kernel(const uint16_t* __restrict__ x, int is_bf16, int M, int K,
                                                      unsigned char* __restrict__ out) {
-  const long long n16 = (long long)M * K / 8;
-  const int rgs = M >> 3;
-  for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < n16;
-       t += (long long)gridDim.x * blockDim.x) {
-    const int kc = (int)(t & 7), rr = (int)((t >> 3) & 7);
-    const long long blk = t >> 6;               // (K-block, row-group) block of 1 KB
-    const int rg = (int)(blk % rgs), kb = (int)(blk / rgs);
-    const int r = 8 * rg + rr, k = 64 * kb + 8 * kc;
-    uint4 v = *reinterpret_cast<const uint4*>(x + (size_t)r * K + k);
-    if (is_bf16) {
-      uint32_t* w = &v.x;
+  const unsigned n16 = (unsigned)((size_t)M * K / 8);   // < 2^32 for the shapes accepted
+  const unsigned rgs = (unsigned)M >> 3;
+  const unsigned stride = gridDim.x * blockDim.x;
+  for (unsigned t0 = blockIdx.x * blockDim.x + threadIdx.x; t0 < n16; t0 += stride * kXUnroll) {
+    uint4 v[kXUnroll];
+    unsigned dst[kXUnroll];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
-        const __half2 h = __floats2half2_rn(__bfloat162float(b.x), __bfloat162float(b.y));
-        w[e] = *reinterpret_cast<const uint32_t*>(&h);
+    for (int u = 0; u < kXUnroll; ++u) {
+      const unsigned t = t0 + u * stride;
+      if (t < n16) {
+        const unsigned kc = t & 7, rr = (t >> 3) & 7, blk = t >> 6;   // blk: (K-block, row-group) KB
+        const unsigned kb = blk / rgs, rg = blk - kb * rgs;
+        v[u] = *reinterpret_cast<const uint4*>(x + (size_t)(8 * rg + rr) * K + 64 * kb + 8 * kc);
+        dst[u] = blk * 1024 + kc * 128 + rr * 16;
       }
     }
-    *reinterpret_cast<uint4*>(out + blk * 1024 + kc * 128 + rr * 16) = v;
+#pragma unroll
+    for (int u = 0; u < kXUnroll; ++u) {
+      if (t0 + u * stride < n16)
+        *reinterpret_cast<uint4*>(out + dst[u]) = is_bf16 ? bf16x8_to_f16x8(v[u]) : v[u];
+    }
   }
 }
 
-// B1 (P*Sp rows x d_in): row p*Sp + j holds V_p[i][j] * g_p[i].  One thread per
-// 16-byte lane of a packed role-V tile: its four words hold, for each q, four
-// consecutive i of one row, i.e. one 8-byte piece of B1.  Rows j >= s inside
-// the packed tiles get +-g (finite; GEMM1's epilogue zeroes them through l);
-// rows from the tiles' end up to Sp are zero.
+// B1 (P*Sp rows x d_in): row p*Sp + j holds V_p[i][j] * g_p[i].  Work unit =
+// (16-byte lane of a packed role-V tile, word r, half qh of the eight
+// products): for each of its four q the word gives four consecutive i of one
+// row, i.e. one 8-byte piece of B1.  Units with the same tile, r and qh are 32
+// consecutive threads (one per lane), so a warp's stores cover whole 128-byte
+// core-matrix rows.  Rows j >= s inside the packed tiles get +-g (finite;
+// GEMM1's epilogue zeroes them through l); rows from the tiles' end up to Sp
+// are zero.
 __global__ void __launch_bounds__(256) prep_b1_kernel(const LayerDesc L, int Sp, unsigned char* __restrict__ out) {
   const int R = L.npaths * Sp, K = L.d_in;
   const int n_kt = K / kVTileK, n_rb = (L.s + 15) >> 4;
-  const long long lanes = (long long)L.npaths * n_rb * n_kt * 32;
-  const long long zero_rows = (long long)L.npaths * (Sp - 16 * n_rb);
-  const long long zeros = zero_rows * (K / 8);
-  for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < lanes + zeros;
-       t += (long long)gridDim.x * blockDim.x) {
-    if (t < lanes) {
-      const int lane = (int)(t & 31);
-      const long long tile = t >> 5;
-      const int p = (int)(tile / ((long long)n_rb * n_kt));
-      const int tt = (int)(tile - (long long)p * n_rb * n_kt);
+  const unsigned tiles_p = (unsigned)(n_rb * n_kt);
+  const unsigned units = (unsigned)L.npaths * tiles_p * 256;
+  const unsigned zrow16 = (unsigned)(K / 8);                    // 16-byte pieces per zero row
+  const unsigned zeros = (unsigned)(L.npaths * (Sp - 16 * n_rb)) * zrow16;
+  for (unsigned t = blockIdx.x * blockDim.x + threadIdx.x; t < units + zeros; t += gridDim.x * blockDim.x) {
+    if (t < units) {
+      const int lane = t & 31, r = (t >> 5) & 3, qh = (t >> 7) & 1;
+      const unsigned tile = t >> 8;
+      const int p = tile >= tiles_p ? 1 : 0;
+      const int tt = (int)(tile - p * tiles_p);
       const int rb = tt / n_kt, kt = tt - rb * n_kt;
-      const uint4 w4 = *reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned char*>(L.p[p].V) +
-                                                        (size_t)tt * kTileBytes + 16 * lane);
-      const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+      const uint32_t w = reinterpret_cast<const uint32_t*>(reinterpret_cast<const unsigned char*>(L.p[p].V) +
+                                                           (size_t)tt * kTileBytes + 16 * lane)[r];
       const uint16_t* g = L.p[p].g;
       const int gg = lane >> 2, c = lane & 3;
+      const int jr = p * Sp + 16 * rb + gg + 8 * (r & 1);
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int jr = p * Sp + 16 * rb + gg + 8 * (r & 1);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int i0 = 256 * kt + 32 * q + 16 * (r >> 1) + 4 * c;
-          const uint2 gv = *reinterpret_cast<const uint2*>(g + i0);
-          const uint32_t bits = (wv[r] >> q) & 0x01010101u;   // byte m: bit of i0 + m
-          const uint32_t s0 = (bits & 1u) << 15, s1 = ((bits >> 8) & 1u) << 31;
-          const uint32_t s2 = ((bits >> 16) & 1u) << 15, s3 = ((bits >> 24) & 1u) << 31;
-          *reinterpret_cast<uint2*>(out + tiled_off(jr, i0, R)) = make_uint2(gv.x ^ (s0 | s1), gv.y ^ (s2 | s3));
-        }
+      for (int qq = 0; qq < 4; ++qq) {
+        const int q = 4 * qh + qq;
+        const int i0 = 256 * kt + 32 * q + 16 * (r >> 1) + 4 * c;
+        const uint2 gv = *reinterpret_cast<const uint2*>(g + i0);
+        const uint32_t bits = (w >> q) & 0x01010101u;   // byte m: bit of i0 + m
+        const uint32_t s0 = (bits & 1u) << 15, s1 = ((bits >> 8) & 1u) << 31;
+        const uint32_t s2 = ((bits >> 16) & 1u) << 15, s3 = ((bits >> 24) & 1u) << 31;
+        *reinterpret_cast<uint2*>(out + tiled_off(jr, i0, R)) = make_uint2(gv.x ^ (s0 | s1), gv.y ^ (s2 | s3));
       }
     } else {
-      const long long z = t - lanes;
-      const int row_i = (int)(z / (K / 8)), k = (int)(z % (K / 8)) * 8;
+      const unsigned z = t - units;
+      const unsigned row_i = z / zrow16;
+      const int k = (int)(z - row_i * zrow16) * 8;
       const int per = Sp - 16 * n_rb;
-      const int p = row_i / per, jr = p * Sp + 16 * n_rb + (row_i - p * per);
+      const int p = (int)row_i / per, jr = p * Sp + 16 * n_rb + ((int)row_i - p * per);
       *reinterpret_cast<uint4*>(out + tiled_off(jr, k, R)) = make_uint4(0u, 0u, 0u, 0u);
     }
   }
 }
 
-// B2 (d_out rows x P*Sp): row o, column p*Sp + j holds U_p[o][j] * h_p[o].  One
-// thread per 16-byte lane of a packed role-U tile: for each q its word gives
-// four consecutive j of one row.  Columns from the tiles' end up to Sp are zero.
+// B2 (d_out rows x P*Sp): row o, column p*Sp + j holds U_p[o][j] * h_p[o].  Work
+// unit = (16-byte lane of a packed role-U tile, word r, half qh of the eight
+// products): for each of its four q the word gives four consecutive j of one
+// row.  Columns from the tiles' end up to Sp are zero.
 __global__ void __launch_bounds__(256) prep_b2_kernel(const LayerDesc L, int Sp, unsigned char* __restrict__ out) {
   const int R = L.d_out;
   const int n_kt = (L.s + 31) >> 5, n_ob = R / kUTileRows;
-  const long long lanes = (long long)L.npaths * n_ob * n_kt * 32;
-  const int zcols = Sp - 32 * n_kt;                       // zero columns per path
-  const long long zeros = (long long)L.npaths * R * (zcols / 8);
-  for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < lanes + zeros;
-       t += (long long)gridDim.x * blockDim.x) {
-    if (t < lanes) {
-      const int lane = (int)(t & 31);
-      const long long tile = t >> 5;
-      const int p = (int)(tile / ((long long)n_ob * n_kt));
-      const int tt = (int)(tile - (long long)p * n_ob * n_kt);
+  const unsigned tiles_p = (unsigned)(n_ob * n_kt);
+  const unsigned units = (unsigned)L.npaths * tiles_p * 256;
+  const int zc8 = (Sp - 32 * n_kt) / 8;                    // zero 16-byte pieces per row and path
+  const unsigned per = (unsigned)(R * zc8);
+  const unsigned zeros = (unsigned)L.npaths * per;
+  for (unsigned t = blockIdx.x * blockDim.x + threadIdx.x; t < units + zeros; t += gridDim.x * blockDim.x) {
+    if (t < units) {
+      const int lane = t & 31, r = (t >> 5) & 3, qh = (t >> 7) & 1;
+      const unsigned tile = t >> 8;
+      const int p = tile >= tiles_p ? 1 : 0;
+      const int tt = (int)(tile - p * tiles_p);
       const int ob = tt / n_kt, kt = tt - ob * n_kt;
-      const uint4 w4 = *reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned char*>(L.p[p].U) +
-                                                        (size_t)tt * kTileBytes + 16 * lane);
-      const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+      const uint32_t w = reinterpret_cast<const uint32_t*>(reinterpret_cast<const unsigned char*>(L.p[p].U) +
+                                                           (size_t)tt * kTileBytes + 16 * lane)[r];
       const uint16_t* h = L.p[p].h;
       const int gg = lane >> 2, c = lane & 3;
+      const int j0 = p * Sp + 32 * kt + 16 * (r >> 1) + 4 * c;
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int j0 = p * Sp + 32 * kt + 16 * (r >> 1) + 4 * c;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int o = kUTileRows * ob + 16 * q + gg + 8 * (r & 1);
-          const uint32_t hv = (uint32_t)h[o] * 0x00010001u;
-          const uint32_t bits = (wv[r] >> q) & 0x01010101u;
-          const uint32_t s0 = (bits & 1u) << 15, s1 = ((bits >> 8) & 1u) << 31;
-          const uint32_t s2 = ((bits >> 16) & 1u) << 15, s3 = ((bits >> 24) & 1u) << 31;
-          *reinterpret_cast<uint2*>(out + tiled_off(o, j0, R)) = make_uint2(hv ^ (s0 | s1), hv ^ (s2 | s3));
-        }
+      for (int qq = 0; qq < 4; ++qq) {
+        const int q = 4 * qh + qq;
+        const int o = kUTileRows * ob + 16 * q + gg + 8 * (r & 1);
+        const uint32_t hv = (uint32_t)h[o] * 0x00010001u;
+        const uint32_t bits = (w >> q) & 0x01010101u;
+        const uint32_t s0 = (bits & 1u) << 15, s1 = ((bits >> 8) & 1u) << 31;
+        const uint32_t s2 = ((bits >> 16) & 1u) << 15, s3 = ((bits >> 24) & 1u) << 31;
+        *reinterpret_cast<uint2*>(out + tiled_off(o, j0, R)) = make_uint2(hv ^ (s0 | s1), hv ^ (s2 | s3));
       }
     } else {
-      const long long z = t - lanes;
-      const int per = R * (zcols / 8);
+      const unsigned z = t - units;
       const int p = (int)(z / per);
-      const int zz = (int)(z - (long long)p * per);
-      const int o = zz / (zcols / 8), j = p * Sp + 32 * n_kt + (zz % (zcols / 8)) * 8;
+      const int zz = (int)(z - (unsigned)p * per);
+      const int o = zz / zc8, j = p * Sp + 32 * n_kt + (zz - o * zc8) * 8;
       *reinterpret_cast<uint4*>(out + tiled_off(o, j, R)) = make_uint4(0u, 0u, 0u, 0u);
     }
   }
@@ -464,11 +479,49 @@ size_t prefill_layer_bytes(int M, int d_in, int d_out, int s, int npaths) {
 
 size_t prefill_table_bytes(int n_layers) { return ((size_t)2 * n_layers * sizeof(GemmProblem) + 1023) & ~(size_t)1023; }
 
-// Prepare the operands of a group of layers and run GEMM1 and GEMM2 for all of
-// them, one grouped launch each.  `ws` holds, first, a table of 2n problems
-// (prefill_table_bytes(n)), then each layer's buffers (prefill_layer_bytes).
-cudaError_t launch_prefill_group(const LayerDesc* Ls, const void* const* xs, void* const* ys, int n, int M,
-                                 int x_bf16, unsigned char* ws, unsigned int* status, int num_sms, cudaStream_t st) {
+// Buffers of one group of layers inside `ws`: first a table of 2n problems
+// (prefill_table_bytes(n)), then each layer's X16 | B1 | B2 | T
+// (prefill_layer_bytes).
+struct LayerBufs {
+  unsigned char *X16, *B1, *B2, *T;
+};
+
+static LayerBufs layer_bufs(unsigned char*& buf, const LayerDesc& L, int M) {
+  const int P = L.npaths, NK = P * prefill_sp(L.s, P);
+  auto a1k = [](size_t v) { return (v + 1023) & ~(size_t)1023; };
+  LayerBufs b;
+  b.X16 = buf;
+  b.B1 = b.X16 + a1k((size_t)M * L.d_in * 2);
+  b.B2 = b.B1 + a1k((size_t)NK * L.d_in * 2);
+  b.T = b.B2 + a1k((size_t)L.d_out * NK * 2);
+  buf = b.T + a1k((size_t)M * NK * 2);
+  return b;
+}
+
+// Operand preparation of a group of layers (three launches per layer).
+cudaError_t launch_prefill_prep(const LayerDesc* Ls, const void* const* xs, int n, int M, int x_bf16,
+                                unsigned char* ws, cudaStream_t st) {
+  unsigned char* buf = ws + prefill_table_bytes(n);
+  for (int i = 0; i < n; ++i) {
+    const LayerDesc& L = Ls[i];
+    const int P = L.npaths, Sp = prefill_sp(L.s, P);
+    const LayerBufs b = layer_bufs(buf, L, M);
+    prep_x_kernel<<<grid_for((long long)M * L.d_in / 8 / kXUnroll, 256), 256, 0, st>>>(
+        static_cast<const uint16_t*>(xs[i]), x_bf16, M, L.d_in, b.X16);
+    const long long l1 = (long long)P * ((L.s + 15) >> 4) * (L.d_in / kVTileK) * 256 +
+                         (long long)P * (Sp - 16 * ((L.s + 15) >> 4)) * (L.d_in / 8);
+    prep_b1_kernel<<<grid_for(l1, 256), 256, 0, st>>>(L, Sp, b.B1);
+    const long long l2 = (long long)P * (L.d_out / kUTileRows) * ((L.s + 31) >> 5) * 256 +
+                         (long long)P * L.d_out * ((Sp - 32 * ((L.s + 31) >> 5)) / 8);
+    prep_b2_kernel<<<grid_for(l2, 256), 256, 0, st>>>(L, Sp, b.B2);
+  }
+  return cudaGetLastError();
+}
+
+// GEMM1 and GEMM2 of a group of layers whose operands launch_prefill_prep
+// prepared in the same `ws`: one grouped launch each.
+cudaError_t launch_prefill_gemms(const LayerDesc* Ls, void* const* ys, int n, int M, int x_bf16,
+                                 unsigned char* ws, unsigned int* status, int num_sms, cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(umma_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -479,43 +532,28 @@ cudaError_t launch_prefill_group(const LayerDesc* Ls, const void* const* xs, voi
   GemmProblem* table_dev = reinterpret_cast<GemmProblem*>(ws);
   unsigned char* buf = ws + prefill_table_bytes(n);
   // host copies of the two problem lists
-  static thread_local GemmProblem host[2 * 4096];
-  if (n > 4096) return cudaErrorInvalidValue;
+  static thread_local GemmProblem host[2 * kPrefillMaxGroup];
+  if (n > kPrefillMaxGroup) return cudaErrorInvalidValue;
   int tiles1 = 0, tiles2 = 0;
   for (int i = 0; i < n; ++i) {
     const LayerDesc& L = Ls[i];
     const int P = L.npaths, Sp = prefill_sp(L.s, P), NK = P * Sp;
-    auto a1k = [](size_t v) { return (v + 1023) & ~(size_t)1023; };
-    unsigned char* X16 = buf;
-    unsigned char* B1 = X16 + a1k((size_t)M * L.d_in * 2);
-    unsigned char* B2 = B1 + a1k((size_t)NK * L.d_in * 2);
-    unsigned char* T = B2 + a1k((size_t)L.d_out * NK * 2);
-    buf = T + a1k((size_t)M * NK * 2);
-
-    prep_x_kernel<<<grid_for((long long)M * L.d_in / 8, 256), 256, 0, st>>>(static_cast<const uint16_t*>(xs[i]),
-                                                                            x_bf16, M, L.d_in, X16);
-    const long long l1 = (long long)P * ((L.s + 15) >> 4) * (L.d_in / kVTileK) * 32 +
-                         (long long)P * (Sp - 16 * ((L.s + 15) >> 4)) * (L.d_in / 8);
-    prep_b1_kernel<<<grid_for(l1, 256), 256, 0, st>>>(L, Sp, B1);
-    const long long l2 = (long long)P * (L.d_out / kUTileRows) * ((L.s + 31) >> 5) * 32 +
-                         (long long)P * L.d_out * ((Sp - 32 * ((L.s + 31) >> 5)) / 8);
-    prep_b2_kernel<<<grid_for(l2, 256), 256, 0, st>>>(L, Sp, B2);
-
+    const LayerBufs b = layer_bufs(buf, L, M);
     GemmProblem& g1 = host[i];
     g1 = GemmProblem{};
-    g1.A = X16; g1.B = B1; g1.M = M; g1.N = NK; g1.K = L.d_in; g1.mode = 0;
-    g1.l0 = L.p[0].l; g1.l1 = P == 2 ? L.p[1].l : L.p[0].l; g1.s = L.s; g1.Sp = Sp; g1.T = T;
+    g1.A = b.X16; g1.B = b.B1; g1.M = M; g1.N = NK; g1.K = L.d_in; g1.mode = 0;
+    g1.l0 = L.p[0].l; g1.l1 = P == 2 ? L.p[1].l : L.p[0].l; g1.s = L.s; g1.Sp = Sp; g1.T = b.T;
     g1.tiles_n = ceil_div(NK, kBN); g1.tile_begin = tiles1;
     tiles1 += (M / kBM) * g1.tiles_n;
     GemmProblem& g2 = host[n + i];
     g2 = GemmProblem{};
-    g2.A = T; g2.B = B2; g2.M = M; g2.N = L.d_out; g2.K = NK; g2.mode = 1; g2.Y = ys[i]; g2.y_bf16 = x_bf16;
+    g2.A = b.T; g2.B = b.B2; g2.M = M; g2.N = L.d_out; g2.K = NK; g2.mode = 1; g2.Y = ys[i]; g2.y_bf16 = x_bf16;
     g2.tiles_n = ceil_div(L.d_out, kBN); g2.tile_begin = tiles2;
     tiles2 += (M / kBM) * g2.tiles_n;
   }
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  e = cudaMemcpyAsync(table_dev, host, sizeof(GemmProblem) * 2 * n, cudaMemcpyHostToDevice, st);
+  // pageable source: the copy is staged before the call returns, so `host`
+  // may be refilled by the next group
+  cudaError_t e = cudaMemcpyAsync(table_dev, host, sizeof(GemmProblem) * 2 * n, cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return e;
   GroupArgs g1a{table_dev, n, tiles1, status};
   umma_group_kernel<<<min(tiles1, num_sms), kGroupThreads, group_smem(), st>>>(g1a);

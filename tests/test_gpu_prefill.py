@@ -98,3 +98,30 @@ def test_prefill_forward_many(lbm):
     torch.cuda.synchronize()
     for i, (y, ref) in enumerate(zip(Y, refs)):
         _check(y, ref, f"layer {i}")
+
+
+def test_prefill_chunked_stack_matches_single_layer_calls(lbm):
+    """A stack whose operand buffers span several chunks (preparation of one
+    chunk overlapped with the GEMMs of the previous one, two workspace halves
+    reused in turn) gives, layer by layer, exactly what one-layer calls give;
+    a second call in a row, after the halves hold the last call's operands,
+    gives it again."""
+    lb, layers = lbm
+    gen = torch.Generator(device="cuda").manual_seed(11)
+    M, n = 2048, 40   # ~29 MB of operands per layer: three chunks
+    L, X, Y = [], [], []
+    for i in range(n):
+        L.append(layers.random_layer(4096, 4096, 290, True, gen)[0])
+        X.append(torch.randn(M, 4096, generator=gen, device="cuda").to(torch.bfloat16))
+        Y.append(torch.full((M, 4096), float("nan"), dtype=torch.bfloat16, device="cuda"))
+    st = lb.Stack(L, X, Y)
+    st()
+    for rep in range(2):
+        torch.cuda.synchronize()
+        for i in range(n):
+            y1 = lb.forward(L[i], X[i])
+            assert torch.equal(Y[i], y1), f"layer {i} differs from its single-layer call (pass {rep})"
+        for y in Y:
+            y.fill_(float("nan"))
+        st()
+    assert lb.device_status() == 0
