@@ -131,7 +131,8 @@ cudaError_t launch_output_pass(const DecodeArgs& a, int num_sms, cudaStream_t st
 // prefill.cu: layers of M rows (multiple of 128), x fp16 or bf16 (y the same)
 int prefill_sp(int s, int npaths);
 size_t prefill_layer_bytes(int M, int d_in, int d_out, int s, int npaths);
-size_t prefill_table_bytes(int n_layers);
+long long prefill_layer_tiles(int M, int d_out, int s, int npaths);   // GEMM1 + GEMM2 tiles
+size_t prefill_table_bytes(int n_layers, long long tiles);
 constexpr int kPrefillMaxGroup = 4096;   // layers per group
 // A group's operand preparation, then its two grouped GEMM launches (same ws).
 cudaError_t launch_prefill_prep(const LayerDesc* Ls, const void* const* xs, int n, int M, int x_bf16,

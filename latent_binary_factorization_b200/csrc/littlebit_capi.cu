@@ -261,20 +261,23 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
   // plan the chunks
   std::vector<int> starts;
   size_t half = 0, cur = 0;
+  long long tiles = 0;
   int cnt = 0;
   for (int i = 0; i < n; ++i) {
-    const size_t b = lb::prefill_layer_bytes(batch, layers[i].d_in, layers[i].d_out, layers[i].s,
-                                             layers[i].residual + 1);
+    const lb_layer& L = layers[i];
+    const size_t b = lb::prefill_layer_bytes(batch, L.d_in, L.d_out, L.s, L.residual + 1);
     if (cnt == 0 || cur + b > kPrefillChunkBytes || cnt == lb::kPrefillMaxGroup) {
-      if (cnt) half = std::max(half, cur + lb::prefill_table_bytes(cnt));
+      if (cnt) half = std::max(half, cur + lb::prefill_table_bytes(cnt, tiles));
       starts.push_back(i);
       cur = 0;
       cnt = 0;
+      tiles = 0;
     }
     cur += b;
+    tiles += lb::prefill_layer_tiles(batch, L.d_out, L.s, L.residual + 1);
     ++cnt;
   }
-  half = align_up(std::max(half, cur + lb::prefill_table_bytes(cnt)), 1024);
+  half = align_up(std::max(half, cur + lb::prefill_table_bytes(cnt, tiles)), 1024);
   starts.push_back(n);
   const int n_chunks = (int)starts.size() - 1;
   const size_t need = kStatusBytes + (n_chunks > 1 ? 2 : 1) * half;

@@ -25,6 +25,12 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <algorithm>
+#include <functional>
+#include <queue>
+#include <utility>
+#include <vector>
+
 #include "lb_internal.h"
 
 namespace lb {
@@ -36,6 +42,7 @@ constexpr int kBK = 64;           // K per stage
 constexpr int kStages = 4;
 constexpr int kABytes = kBM * kBK * 2;   // 16 KB
 constexpr int kBBytes = kBN * kBK * 2;   // 32 KB
+constexpr int kYPitch = 144;             // y staging row: 64 outputs (128 B) + 16 B against bank conflicts
 
 __host__ __device__ __forceinline__ size_t tiled_off(int r, int k, int R) {
   return ((size_t)(k >> 6) * (R >> 3) + (r >> 3)) * 1024 + ((k & 63) >> 3) * 128 + (r & 7) * 16 + (k & 7) * 2;
@@ -287,8 +294,12 @@ struct GemmProblem {
   int tiles_n, tile_begin;
 };
 
+// Tiles of CTA b: sched[begin[b] .. begin[b+1]), built on the host (longest
+// first, each to the least-loaded CTA).
 struct GroupArgs {
   const GemmProblem* probs;
+  const int* sched;
+  const int* begin;
   int n_probs, total_tiles;
   unsigned int* status;
 };
@@ -330,6 +341,8 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
   uint64_t* accf = empty + kStages;
   uint64_t* acce = accf + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+  // y staging of the epilogue warps: [4 warps][32 rows][kYPitch bytes]
+  unsigned char* ystage = smem + kStages * (kABytes + kBBytes) + 1024;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0) {
@@ -358,8 +371,8 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
   if (threadIdx.x == 0) {
     // ---- producer
     uint32_t it = 0;
-    for (int tile = blockIdx.x; tile < ga.total_tiles; tile += gridDim.x) {
-      const TileInfo ti = tile_info(ga, tile);
+    for (int k = ga.begin[blockIdx.x]; k < ga.begin[blockIdx.x + 1]; ++k) {
+      const TileInfo ti = tile_info(ga, ga.sched[k]);
       const uint32_t bbytes = (uint32_t)ti.n_len * kBK * 2;
       const int Mg = ti.P->M >> 3, Ng = ti.P->N >> 3;
       for (int kb = 0; kb < ti.nk; ++kb, ++it) {
@@ -373,8 +386,8 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
   } else if (threadIdx.x == 32) {
     // ---- MMA issuer
     uint32_t it = 0, nt = 0;
-    for (int tile = blockIdx.x; tile < ga.total_tiles; tile += gridDim.x, ++nt) {
-      const TileInfo ti = tile_info(ga, tile);
+    for (int k = ga.begin[blockIdx.x]; k < ga.begin[blockIdx.x + 1]; ++k, ++nt) {
+      const TileInfo ti = tile_info(ga, ga.sched[k]);
       const int ab = nt & 1;
       if (nt >= 2 && !dead && !mbar_wait(&acce[ab], ((nt >> 1) - 1) & 1)) dead = true;
       tc_fence_after();
@@ -397,8 +410,8 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
     // ---- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
     const int quarter = warp & 3;
     uint32_t nt = 0;
-    for (int tile = blockIdx.x; tile < ga.total_tiles; tile += gridDim.x, ++nt) {
-      const TileInfo ti = tile_info(ga, tile);
+    for (int k = ga.begin[blockIdx.x]; k < ga.begin[blockIdx.x + 1]; ++k, ++nt) {
+      const TileInfo ti = tile_info(ga, ga.sched[k]);
       const int ab = nt & 1;
       if (!dead && !mbar_wait(&accf[ab], (nt >> 1) & 1)) dead = true;
       dead = __any_sync(0xffffffffu, dead);
@@ -406,11 +419,46 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
       const GemmProblem& P = *ti.P;
       const int row = ti.m0 + 32 * quarter + lane;
       const uint32_t taddr = tmem + (uint32_t)(ab * kBN) + ((uint32_t)(32 * quarter) << 16);
-      for (int c0 = 0; c0 < ti.n_len; c0 += 16) {
+      if (P.mode == 1) {
+        // y: 64 columns at a time through shared memory, so that eight lanes
+        // write one row's 128 contiguous bytes
+        unsigned char* sy = ystage + (size_t)quarter * 32 * kYPitch;
+        for (int c0 = 0; c0 < ti.n_len; c0 += 64) {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            float v[16];
+            tmem_ld16(taddr + (uint32_t)(c0 + 16 * h), v);
+            uint32_t w[8];
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              if (P.y_bf16) {
+                const __nv_bfloat162 bb = __floats2bfloat162_rn(v[e], v[e + 1]);
+                w[e >> 1] = *reinterpret_cast<const uint32_t*>(&bb);
+              } else {
+                const __half2 hh = __floats2half2_rn(v[e], v[e + 1]);
+                w[e >> 1] = *reinterpret_cast<const uint32_t*>(&hh);
+              }
+            }
+            *reinterpret_cast<uint4*>(sy + lane * kYPitch + 32 * h) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(sy + lane * kYPitch + 32 * h + 16) = make_uint4(w[4], w[5], w[6], w[7]);
+          }
+          __syncwarp();
+          const int cb = lane & 7;
+#pragma unroll
+          for (int r4 = 0; r4 < 32; r4 += 4) {
+            const int r = r4 + (lane >> 3);
+            const uint4 val = *reinterpret_cast<const uint4*>(sy + r * kYPitch + cb * 16);
+            uint16_t* yr = static_cast<uint16_t*>(P.Y) + (size_t)(ti.m0 + 32 * quarter + r) * P.N + ti.n0 + c0;
+            *reinterpret_cast<uint4*>(yr + 8 * cb) = val;
+          }
+          __syncwarp();
+        }
+      }
+      for (int c0 = 0; P.mode == 0 && c0 < ti.n_len; c0 += 16) {
         float v[16];
         tmem_ld16(taddr + (uint32_t)c0, v);
         uint32_t w[8];
-        if (P.mode == 0) {
+        {
 #pragma unroll
           for (int e = 0; e < 16; e += 2) {
             float lv[2];
@@ -427,20 +475,6 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
           *reinterpret_cast<uint4*>(P.T + tiled_off(row, ti.n0 + c0, P.M)) = make_uint4(w[0], w[1], w[2], w[3]);
           *reinterpret_cast<uint4*>(P.T + tiled_off(row, ti.n0 + c0 + 8, P.M)) =
               make_uint4(w[4], w[5], w[6], w[7]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            if (P.y_bf16) {
-              const __nv_bfloat162 bb = __floats2bfloat162_rn(v[e], v[e + 1]);
-              w[e >> 1] = *reinterpret_cast<const uint32_t*>(&bb);
-            } else {
-              const __half2 hh = __floats2half2_rn(v[e], v[e + 1]);
-              w[e >> 1] = *reinterpret_cast<const uint32_t*>(&hh);
-            }
-          }
-          uint16_t* yr = static_cast<uint16_t*>(P.Y) + (size_t)row * P.N + ti.n0 + c0;
-          *reinterpret_cast<uint4*>(yr) = make_uint4(w[0], w[1], w[2], w[3]);
-          *reinterpret_cast<uint4*>(yr + 8) = make_uint4(w[4], w[5], w[6], w[7]);
         }
       }
       tc_fence_before();
@@ -459,7 +493,7 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
   }
 }
 
-size_t group_smem() { return (size_t)kStages * (kABytes + kBBytes) + (2 * kStages + 4) * 8 + 16; }
+size_t group_smem() { return (size_t)kStages * (kABytes + kBBytes) + 1024 + (size_t)4 * 32 * kYPitch; }
 
 int grid_for(long long work, int per_block) {
   long long b = (work + per_block - 1) / per_block;
@@ -477,11 +511,28 @@ size_t prefill_layer_bytes(int M, int d_in, int d_out, int s, int npaths) {
   return a1k((size_t)M * d_in * 2) + a1k(NK * d_in * 2) + a1k((size_t)d_out * NK * 2) + a1k((size_t)M * NK * 2);
 }
 
-size_t prefill_table_bytes(int n_layers) { return ((size_t)2 * n_layers * sizeof(GemmProblem) + 1023) & ~(size_t)1023; }
+constexpr int kMaxGemmGrid = 1024;
 
-// Buffers of one group of layers inside `ws`: first a table of 2n problems
-// (prefill_table_bytes(n)), then each layer's X16 | B1 | B2 | T
-// (prefill_layer_bytes).
+long long prefill_layer_tiles(int M, int d_out, int s, int npaths) {
+  const int NK = npaths * prefill_sp(s, npaths);
+  return (long long)(M / kBM) * (ceil_div(NK, kBN) + ceil_div(d_out, kBN));
+}
+
+size_t prefill_table_bytes(int n_layers, long long tiles) {
+  const size_t b = (size_t)2 * n_layers * sizeof(GemmProblem) + (size_t)2 * (kMaxGemmGrid + 1) * sizeof(int) +
+                   (size_t)tiles * sizeof(int);
+  return (b + 1023) & ~(size_t)1023;
+}
+
+static long long group_tiles(const LayerDesc* Ls, int n, int M) {
+  long long t = 0;
+  for (int i = 0; i < n; ++i) t += prefill_layer_tiles(M, Ls[i].d_out, Ls[i].s, Ls[i].npaths);
+  return t;
+}
+
+// Buffers of one group of layers inside `ws`: first the table (2n problems,
+// then the two GEMMs' CTA list offsets and tile lists; prefill_table_bytes),
+// then each layer's X16 | B1 | B2 | T (prefill_layer_bytes).
 struct LayerBufs {
   unsigned char *X16, *B1, *B2, *T;
 };
@@ -501,7 +552,7 @@ static LayerBufs layer_bufs(unsigned char*& buf, const LayerDesc& L, int M) {
 // Operand preparation of a group of layers (three launches per layer).
 cudaError_t launch_prefill_prep(const LayerDesc* Ls, const void* const* xs, int n, int M, int x_bf16,
                                 unsigned char* ws, cudaStream_t st) {
-  unsigned char* buf = ws + prefill_table_bytes(n);
+  unsigned char* buf = ws + prefill_table_bytes(n, group_tiles(Ls, n, M));
   for (int i = 0; i < n; ++i) {
     const LayerDesc& L = Ls[i];
     const int P = L.npaths, Sp = prefill_sp(L.s, P);
@@ -518,6 +569,36 @@ cudaError_t launch_prefill_prep(const LayerDesc* Ls, const void* const* xs, int 
   return cudaGetLastError();
 }
 
+// Longest-first schedule of `cost` over `grid` CTAs: every tile, in order of
+// decreasing cost, goes to the CTA with the least work so far.  Writes the
+// CTA lists to sched (tile indices) and their offsets to begin[0..grid].
+static void lpt_schedule(const std::vector<double>& cost, int grid, int* sched, int* begin) {
+  const int T = (int)cost.size();
+  std::vector<int> order(T);
+  for (int i = 0; i < T; ++i) order[i] = i;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+  using Slot = std::pair<double, int>;   // (load, cta)
+  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
+  for (int b = 0; b < grid; ++b) heap.push({0.0, b});
+  std::vector<std::vector<int>> lists(grid);
+  for (int t : order) {
+    Slot sl = heap.top();
+    heap.pop();
+    lists[sl.second].push_back(t);
+    heap.push({sl.first + cost[t], sl.second});
+  }
+  int k = 0;
+  for (int b = 0; b < grid; ++b) {
+    begin[b] = k;
+    for (int t : lists[b]) sched[k++] = t;
+  }
+  begin[grid] = k;
+}
+
+// Tile cost for the schedule: K-blocks times the tile's share of a full-width
+// product, plus about one K-block of fixed per-tile work.
+static double tile_cost(int K, int n_len) { return (double)(K / kBK) * (double)max(n_len, 64) / kBN + 1.0; }
+
 // GEMM1 and GEMM2 of a group of layers whose operands launch_prefill_prep
 // prepared in the same `ws`: one grouped launch each.
 cudaError_t launch_prefill_gemms(const LayerDesc* Ls, void* const* ys, int n, int M, int x_bf16,
@@ -529,36 +610,54 @@ cudaError_t launch_prefill_gemms(const LayerDesc* Ls, void* const* ys, int n, in
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  GemmProblem* table_dev = reinterpret_cast<GemmProblem*>(ws);
-  unsigned char* buf = ws + prefill_table_bytes(n);
-  // host copies of the two problem lists
-  static thread_local GemmProblem host[2 * kPrefillMaxGroup];
   if (n > kPrefillMaxGroup) return cudaErrorInvalidValue;
+  const long long tiles_all = group_tiles(Ls, n, M);
+  unsigned char* buf = ws + prefill_table_bytes(n, tiles_all);
+  // host image of the table: 2n problems | begin1 | begin2 | sched1 | sched2
+  const size_t prob_b = (size_t)2 * n * sizeof(GemmProblem);
+  static thread_local std::vector<unsigned char> host;
+  host.assign(prob_b + (size_t)2 * (kMaxGemmGrid + 1) * sizeof(int) + (size_t)tiles_all * sizeof(int), 0);
+  GemmProblem* probs = reinterpret_cast<GemmProblem*>(host.data());
+  int* begin1 = reinterpret_cast<int*>(host.data() + prob_b);
+  int* begin2 = begin1 + kMaxGemmGrid + 1;
+  int* sched1 = begin2 + kMaxGemmGrid + 1;
+  std::vector<double> cost1, cost2;
   int tiles1 = 0, tiles2 = 0;
   for (int i = 0; i < n; ++i) {
     const LayerDesc& L = Ls[i];
     const int P = L.npaths, Sp = prefill_sp(L.s, P), NK = P * Sp;
     const LayerBufs b = layer_bufs(buf, L, M);
-    GemmProblem& g1 = host[i];
+    GemmProblem& g1 = probs[i];
     g1 = GemmProblem{};
     g1.A = b.X16; g1.B = b.B1; g1.M = M; g1.N = NK; g1.K = L.d_in; g1.mode = 0;
     g1.l0 = L.p[0].l; g1.l1 = P == 2 ? L.p[1].l : L.p[0].l; g1.s = L.s; g1.Sp = Sp; g1.T = b.T;
     g1.tiles_n = ceil_div(NK, kBN); g1.tile_begin = tiles1;
     tiles1 += (M / kBM) * g1.tiles_n;
-    GemmProblem& g2 = host[n + i];
+    for (int mt = 0; mt < M / kBM; ++mt)
+      for (int nt = 0; nt < g1.tiles_n; ++nt) cost1.push_back(tile_cost(g1.K, min(kBN, NK - nt * kBN)));
+    GemmProblem& g2 = probs[n + i];
     g2 = GemmProblem{};
     g2.A = b.T; g2.B = b.B2; g2.M = M; g2.N = L.d_out; g2.K = NK; g2.mode = 1; g2.Y = ys[i]; g2.y_bf16 = x_bf16;
     g2.tiles_n = ceil_div(L.d_out, kBN); g2.tile_begin = tiles2;
     tiles2 += (M / kBM) * g2.tiles_n;
+    for (int mt = 0; mt < M / kBM; ++mt)
+      for (int nt = 0; nt < g2.tiles_n; ++nt) cost2.push_back(tile_cost(g2.K, min(kBN, L.d_out - nt * kBN)));
   }
+  int* sched2 = sched1 + tiles1;
+  const int grid1 = min(min(tiles1, num_sms), kMaxGemmGrid), grid2 = min(min(tiles2, num_sms), kMaxGemmGrid);
+  lpt_schedule(cost1, grid1, sched1, begin1);
+  lpt_schedule(cost2, grid2, sched2, begin2);
   // pageable source: the copy is staged before the call returns, so `host`
   // may be refilled by the next group
-  cudaError_t e = cudaMemcpyAsync(table_dev, host, sizeof(GemmProblem) * 2 * n, cudaMemcpyHostToDevice, st);
+  cudaError_t e = cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return e;
-  GroupArgs g1a{table_dev, n, tiles1, status};
-  umma_group_kernel<<<min(tiles1, num_sms), kGroupThreads, group_smem(), st>>>(g1a);
-  GroupArgs g2a{table_dev + n, n, tiles2, status};
-  umma_group_kernel<<<min(tiles2, num_sms), kGroupThreads, group_smem(), st>>>(g2a);
+  const GemmProblem* table_dev = reinterpret_cast<const GemmProblem*>(ws);
+  const int* begin_dev = reinterpret_cast<const int*>(ws + prob_b);
+  const int* sched_dev = begin_dev + 2 * (kMaxGemmGrid + 1);
+  GroupArgs g1a{table_dev, sched_dev, begin_dev, n, tiles1, status};
+  umma_group_kernel<<<grid1, kGroupThreads, group_smem(), st>>>(g1a);
+  GroupArgs g2a{table_dev + n, sched_dev + tiles1, begin_dev + kMaxGemmGrid + 1, n, tiles2, status};
+  umma_group_kernel<<<grid2, kGroupThreads, group_smem(), st>>>(g2a);
   return cudaGetLastError();
 }
 
