@@ -62,13 +62,18 @@ def algorithmic_bytes(d_in, d_out, s, residual, batch):
     return paths * per_path + 2 * batch * (d_in + d_out)
 
 
+KERNELS = ("quantise", "latent_pass", "finalize", "output_pass")
+
+
 def kernel_bytes(d_in, d_out, s, residual, batch):
-    """Algorithmic bytes split by kernel: latent pass (V bits, g, l, x) and
-    output pass (U bits, h, y)."""
+    """Algorithmic bytes split by decode kernel (they sum to algorithmic_bytes):
+    quantise (g per path, x), latent pass (V bits), finalize (l), output pass
+    (U bits, h, y)."""
     paths = 2 if residual else 1
-    lat = paths * (s * d_in / 8 + 2 * (d_in + s)) + 2 * batch * d_in
-    out = paths * (s * d_out / 8 + 2 * d_out) + 2 * batch * d_out
-    return lat, out
+    return {"quantise": paths * 2 * d_in + 2 * batch * d_in,
+            "latent_pass": paths * s * d_in / 8,
+            "finalize": paths * 2 * s,
+            "output_pass": paths * (s * d_out / 8 + 2 * d_out) + 2 * batch * d_out}
 
 
 def load_peaks():
@@ -181,36 +186,41 @@ def stack_reps_for_l2(mats, batch, l2_bytes, factor=4.0):
 
 
 def time_device(stack, steps, warmup, dist):
-    """K device-timed steps (CUDA events on the launching stream), and the
-    per-kernel split from an event recorded between the two launches."""
+    """K device-timed steps (CUDA events on the launching stream, nothing else
+    recorded in between), then K more steps for each decode kernel's share,
+    from events the library records after the first three of its four
+    launches."""
     import torch
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
         stack()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     if dist:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     t0.record(stream)
-    for k in range(steps):
-        ev[k][0].record(stream)
-        # torch only times events it recorded itself; an event keeps its latest
-        # record, so record it here and let the library re-record it between
-        # its latent-pass and output-pass launches
-        ev[k][1].record(stream)
-        stack(event_between=ev[k][1])
-        ev[k][2].record(stream)
+    for _ in range(steps):
+        stack()
     t1.record(stream)
     torch.cuda.synchronize()
     if dist:
         torch.distributed.barrier()
     total_ms = t0.elapsed_time(t1)
-    lat = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
-    out = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
-    return total_ms, lat, out
+    # per-kernel split (separate pass: the extra event records add small gaps)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    for k in range(steps):
+        ev[k][0].record(stream)
+        # torch only times events it recorded itself; an event keeps its latest
+        # record, so record the three inner ones here and let the library
+        # re-record them after its quantise, latent and finalize launches
+        for e in ev[k][1:4]:
+            e.record(stream)
+        stack(events=ev[k][1:4])
+        ev[k][4].record(stream)
+    torch.cuda.synchronize()
+    per = {name: sum(e[i].elapsed_time(e[i + 1]) for e in ev) / steps for i, name in enumerate(KERNELS)}
+    return total_ms, per
 
 
 def time_e2e(stack, x_all, y_all, steps, warmup):
@@ -244,24 +254,22 @@ def measure_workload(name, batch, steps, warmup, device, dist, world, l2, seed=1
     reps = stack_reps_for_l2(mats, batch, l2, l2_factor)
     stack, Ls, x_all, y_all = build_stack(mats, reps, batch, seed, device)
     n_layers = len(Ls)
-    total_ms, lat_ms, out_ms = time_device(stack, steps, warmup, dist)
+    total_ms, per_ms = time_device(stack, steps, warmup, dist)
     if dist:
         import torch
-        t = torch.tensor([total_ms, lat_ms, out_ms], device=device, dtype=torch.float64)
+        t = torch.tensor([total_ms] + [per_ms[k] for k in KERNELS], device=device, dtype=torch.float64)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms, lat_ms, out_ms = t.tolist()
+        total_ms, per_ms = t[0].item(), dict(zip(KERNELS, t[1:].tolist()))
     alg = sum(algorithmic_bytes(*m, batch) for m in mats) * reps
-    lat_b = sum(kernel_bytes(*m, batch)[0] for m in mats) * reps
-    out_b = sum(kernel_bytes(*m, batch)[1] for m in mats) * reps
+    kb = {k: sum(kernel_bytes(*m, batch)[k] for m in mats) * reps for k in KERNELS}
     ms_step = total_ms / steps
     res = {
         "workload": name, "desc": WORKLOADS[name]["desc"], "batch": batch, "layers_per_step": n_layers,
         "model_layers_per_step": reps, "stack_bytes": int(alg), "ms_per_step": ms_step,
         "us_per_matrix": 1e3 * ms_step / n_layers, "us_per_model_layer": 1e3 * ms_step / reps,
         "step_gbs": alg / (ms_step * 1e-3) / 1e9,
-        "latent_pass_ms": lat_ms, "output_pass_ms": out_ms,
-        "latent_pass_gbs": lat_b / (lat_ms * 1e-3) / 1e9, "output_pass_gbs": out_b / (out_ms * 1e-3) / 1e9,
-        "latent_bytes": lat_b, "output_bytes": out_b,
+        "kernels": {k: {"ms": per_ms[k], "algorithmic_bytes": kb[k],
+                        "gbs": kb[k] / (per_ms[k] * 1e-3) / 1e9 if per_ms[k] > 0 else None} for k in KERNELS},
         "world": world,
     }
     return res, (stack, x_all, y_all)
@@ -363,10 +371,9 @@ def run_ours(args):
     clocks = sampler.stop()
 
     n_layers = main["layers_per_step"]
-    lat, out = main["latent_pass_ms"], main["output_pass_ms"]
-    dom = "output_pass" if out >= lat else "latent_pass"
-    dom_bytes = main["output_bytes"] if dom == "output_pass" else main["latent_bytes"]
-    dom_ms = max(lat, out)
+    dom = max(KERNELS, key=lambda k: main["kernels"][k]["ms"])
+    dom_bytes = main["kernels"][dom]["algorithmic_bytes"]
+    dom_ms = main["kernels"][dom]["ms"]
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     traffic = traffic_record(dom, args.workload, main["model_layers_per_step"])
     value = 1e3 * main["ms_per_step"] / (n_layers * world)   # us per layer over all ranks' layers
@@ -394,8 +401,9 @@ def run_ours(args):
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                      else "fallback", "algorithmic_bytes_per_launch": int(dom_bytes)},
         "step_roofline": {"achieved": round(main["step_gbs"], 1), "frac": round(main["step_gbs"] / peak, 4),
-                          "latent_pass_gbs": round(main["latent_pass_gbs"], 1),
-                          "output_pass_gbs": round(main["output_pass_gbs"], 1)},
+                          "kernels": {k: {"ms_per_step": round(main["kernels"][k]["ms"], 5),
+                                          "gbs": round(main["kernels"][k]["gbs"], 1)
+                                          if main["kernels"][k]["gbs"] else None} for k in KERNELS}},
         "e2e": {"value": round(1e3 * e2e_ms / max(3, args.steps // 4) / (n_layers * world), 5), "unit": "us/layer",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": 4 * args.steps,   # quantise, latent, finalize, output per step

@@ -147,14 +147,15 @@ lb_status littlebit_linear_forward_many(const lb_layer* layers, int n, const voi
 
 /*
  * littlebit_linear_forward_many, and in addition, on the decode path, records
- * `event_between` (a cudaEvent_t passed as void*, or NULL) on `stream` after
- * the finalize launch and before the output-pass launch, so that a caller can
- * time the two halves (V side: quantise, latent, finalize; U side: output)
- * separately with CUDA events.
+ * events[i] (cudaEvent_t values passed as void*; a NULL entry is skipped) on
+ * `stream` right after kernel launch i, for i < n_events <= 3: 0 = input
+ * quantisation, 1 = latent pass, 2 = finalize (the output pass is last), so
+ * that a caller can time each kernel with CUDA events.  The prefill path
+ * records none.  events may be NULL when n_events is 0.
  */
 lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, const void* const* xs,
                                               void* const* ys, int batch, lb_dtype xdt, void* stream,
-                                              void* event_between);
+                                              void* const* events, int n_events);
 
 /*
  * The decode forward of littlebit_linear_forward (one layer, 1 <= batch <= 16,

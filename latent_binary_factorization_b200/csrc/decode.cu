@@ -127,153 +127,114 @@ __device__ __forceinline__ float2 h2x2(uint32_t v) {
 __device__ __forceinline__ float h2f(uint16_t v) { return __half2float(__ushort_as_half(v)); }
 __device__ __forceinline__ uint16_t f2h(float v) { return __half_as_ushort(__float2half_rn(v)); }
 
-// quantise to v = 256*hi + lo; returns v and writes the two int8 bytes
-__device__ __forceinline__ int quantise(float u, float inv, int8_t& hi, int8_t& lo) {
-  int v = __float2int_rn(u * inv);
-  v = max(-32639, min(32639, v));
-  const int h = (v + 128) >> 8;   // floor((v + 128) / 256) in [-127, 127]
-  hi = (int8_t)h;
-  lo = (int8_t)(v - 256 * h);     // in [-128, 127]
-  return v;
-}
-
-// Block-wide max / sum of N values per thread (all threads get the result).
-template <int N>
-__device__ __forceinline__ void block_max(float (&v)[N], float (*s_buf)[16]) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-#pragma unroll
-  for (int i = 0; i < N; ++i) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v[i] = fmaxf(v[i], __shfl_xor_sync(0xffffffffu, v[i], o));
-    if (lane == 0) s_buf[warp][i] = v[i];
-  }
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < N; ++i) {
-    float m = s_buf[0][i];
-#pragma unroll
-    for (int w = 1; w < kVWarps; ++w) m = fmaxf(m, s_buf[w][i]);
-    v[i] = m;
-  }
-  __syncthreads();
-}
-
-template <int N>
-__device__ __forceinline__ void block_sum(int (&v)[N], int (*s_buf)[16]) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-#pragma unroll
-  for (int i = 0; i < N; ++i) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
-    if (lane == 0) s_buf[warp][i] = v[i];
-  }
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < N; ++i) {
-    int m = s_buf[0][i];
-#pragma unroll
-    for (int w = 1; w < kVWarps; ++w) m += s_buf[w][i];
-    v[i] = m;
-  }
-  __syncthreads();
-}
-
 // Layer of a work item: one load from the item's map (no map with one layer).
 __device__ __forceinline__ int layer_of(const int* map, int n_layers, int item) {
   return n_layers == 1 ? 0 : __ldg(map + item);
 }
 
 // ---------------------------------------------------------------------------
-// quantise pass:  u = g (.) x on one 2048-input slice of one (layer, path),
-// quantised per batch row to 16 bits, v = step * (256*hi + lo), and stored as
-// the latent pass's int8 B fragments (slice block layout in lb_internal.h).
-// One warp per (layer, path, slice): lane i holds the 8-input chunks i + 32j
-// (j < 8) of g and of one batch row of x at a time; max and sum are warp
-// reductions, so the kernel has no CTA barrier.
+// quantise pass:  u = g_p (.) x on one 2048-input slice of one layer, for each
+// path p, quantised per batch row to 16 bits, v = step * (256*hi + lo), and
+// stored as the latent pass's int8 B fragments (slice block layout in
+// lb_internal.h).  One warp per (layer, slice): lane i holds the 8-input
+// chunks i + 32j (j < 8) of one batch row; max and sum are warp reductions, so
+// the kernel has no CTA barrier.
+//
+// Arithmetic per value: u = g*x in fp32 (exact for fp16 operands); v =
+// round(u * 32639 / max|u|) by adding 1.5*2^23 in fp32, which leaves v in the
+// low bits of the float's encoding: its low byte is the int8 lo byte of
+// v = 256*hi + lo, and byte 1 of (encoding + 128) is hi.  |v| <= 32639 holds
+// because max|u| is taken over the same fp32 values.
 // ---------------------------------------------------------------------------
 constexpr int kQWarps = 4;                          // warps (slices) per CTA
 constexpr int kQChunks = kVSlice / 8 / 32;          // 8-input chunks per lane
+constexpr float kRoundMagic = 12582912.f;           // 1.5 * 2^23
+
+// byte b (0 or 1) of a, c, d, e packed low to high
+__device__ __forceinline__ uint32_t pack_byte(uint32_t a, uint32_t c, uint32_t d, uint32_t e, int b) {
+  const uint32_t sel = b == 0 ? 0x0040u : 0x0051u;   // {a.b, c.b} into the low half
+  const uint32_t lo = __byte_perm(a, c, sel), hi = __byte_perm(d, e, sel);
+  return __byte_perm(lo, hi, 0x5410);
+}
 
 __global__ void __launch_bounds__(kQWarps * 32) quantise_input_kernel(const DecodeArgs a) {
   const int lane = threadIdx.x & 31;
   const int item = blockIdx.x * kQWarps + (threadIdx.x >> 5);
   if (item >= a.x_items) return;
-  const int B = a.batch, RB = xq_rows(B), NC = 2 * RB;
+  const int B = a.batch, NC = 2 * xq_rows(B);
   const LayerDesc& L = a.layers[layer_of(a.item_layer.x, a.n_layers, item)];
-  const int rel = item - L.x_begin;
-  const int p = rel / L.n_slices, sl = rel - p * L.n_slices;
-  const PathDesc& P = L.p[p];
+  const int sl = item - L.x_begin;
   const int d_in = L.d_in, k0 = sl * kVSlice;
   const int nchunk = min(kVSlice, d_in - k0) / 8;
-  unsigned char* blk = P.ws.xq + (size_t)sl * xq_slice_bytes(B);
-  uint32_t* frag = reinterpret_cast<uint32_t*>(blk + xq_stats_bytes(B));
+  const size_t blk_off = (size_t)sl * xq_slice_bytes(B);
 
-  uint4 gq[kQChunks];
-#pragma unroll
-  for (int j = 0; j < kQChunks; ++j) {
-    const int ch = lane + 32 * j;
-    gq[j] = ch < nchunk ? ld_nc(P.g + k0 + 8 * ch) : make_uint4(0, 0, 0, 0);
-  }
-  const int nrow = 4 * xq_nb(B);   // stats rows (>= RB >= B)
 #pragma unroll 1
-  for (int row = 0; row < nrow; ++row) {
-    uint4 xq[kQChunks];
+  for (int p = 0; p < L.npaths; ++p) {
+    const PathDesc& P = L.p[p];
+    unsigned char* blk = P.ws.xq + blk_off;
+    uint32_t* frag = reinterpret_cast<uint32_t*>(blk + xq_stats_bytes(B));
+    // rows B .. 4*nb-1 of the block are never read: their product columns are
+    // independent of the batch rows' and their sums are discarded
+#pragma unroll 1
+    for (int row = 0; row < B; ++row) {
+      float u[kQChunks][8];
+      float mx = 0.f;
 #pragma unroll
-    for (int j = 0; j < kQChunks; ++j) {
-      const int ch = lane + 32 * j;
-      xq[j] = (row < B && ch < nchunk) ? ld_nc(L.x + (size_t)row * d_in + k0 + 8 * ch) : make_uint4(0, 0, 0, 0);
-    }
-    float mx = 0.f;
+      for (int j = 0; j < kQChunks; ++j) {
+        const int ch = lane + 32 * j;
+        const bool live = ch < nchunk;
+        const uint4 xq = live ? ld_nc(L.x + (size_t)row * d_in + k0 + 8 * ch) : make_uint4(0, 0, 0, 0);
+        const uint4 gq = live ? ld_nc(P.g + k0 + 8 * ch) : make_uint4(0, 0, 0, 0);
+        const uint32_t* xw = &xq.x;
+        const uint32_t* gw = &gq.x;
 #pragma unroll
-    for (int j = 0; j < kQChunks; ++j) {
-      const uint32_t* xw = &xq[j].x;
-      const uint32_t* gw = &gq[j].x;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 xf = h2x2(xw[e]), gf = h2x2(gw[e]);
-        mx = fmaxf(mx, fmaxf(fabsf(xf.x * gf.x), fabsf(xf.y * gf.y)));
+        for (int e = 0; e < 4; ++e) {
+          const float2 xf = h2x2(xw[e]), gf = h2x2(gw[e]);
+          u[j][2 * e] = xf.x * gf.x;
+          u[j][2 * e + 1] = xf.y * gf.y;
+          mx = fmaxf(mx, fmaxf(fabsf(u[j][2 * e]), fabsf(u[j][2 * e + 1])));
+        }
       }
-    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const float inv = mx > 0.f ? kQMax / mx : 0.f;
-    int vsum = 0;
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float inv = mx > 0.f ? kQMax / mx : 0.f;
+      int sum_hi = 0, sum_lo = 0;
 #pragma unroll
-    for (int j = 0; j < kQChunks; ++j) {
-      const int ch = lane + 32 * j;
-      const uint32_t* xw = &xq[j].x;
-      const uint32_t* gw = &gq[j].x;
-      uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
+      for (int j = 0; j < kQChunks; ++j) {
+        const int ch = lane + 32 * j;
+        uint32_t fb[8], fh[8];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 xf = h2x2(xw[e]), gf = h2x2(gw[e]);
-        int8_t h0, l0, h1, l1;
-        vsum += quantise(xf.x * gf.x, inv, h0, l0) + quantise(xf.y * gf.y, inv, h1, l1);
-        const int sh = 16 * (e & 1);
-        hw[e >> 1] |= ((uint32_t)(uint8_t)h0 | ((uint32_t)(uint8_t)h1 << 8)) << sh;
-        lw[e >> 1] |= ((uint32_t)(uint8_t)l0 | ((uint32_t)(uint8_t)l1 << 8)) << sh;
+        for (int e = 0; e < 8; ++e) {
+          fb[e] = __float_as_uint(fmaf(u[j][e], inv, kRoundMagic));
+          fh[e] = fb[e] + 128u;
+        }
+        const uint32_t lw0 = pack_byte(fb[0], fb[1], fb[2], fb[3], 0), lw1 = pack_byte(fb[4], fb[5], fb[6], fb[7], 0);
+        const uint32_t hw0 = pack_byte(fh[0], fh[1], fh[2], fh[3], 1), hw1 = pack_byte(fh[4], fh[5], fh[6], fh[7], 1);
+        sum_hi = __dp4a((int)hw0, 0x01010101, __dp4a((int)hw1, 0x01010101, sum_hi));
+        sum_lo = __dp4a((int)lw0, 0x01010101, __dp4a((int)lw1, 0x01010101, sum_lo));
+        if (ch < nchunk) {
+          // inputs 8ch..8ch+7: K-block kb, offset kk0 (0, 8, 16, 24) inside it;
+          // kk < 16 -> b0 words of threads c = kk/4, else b1 words of c = (kk-16)/4
+          const int kb = ch >> 2, kk0 = (ch & 3) * 8;
+          const int cc = (kk0 & 15) >> 2, half = kk0 >> 4;
+          uint32_t* fhp = frag + ((size_t)kb * NC + 2 * row) * 8;   // column 2*row: 4 threads x (b0, b1)
+          uint32_t* flp = fhp + 8;                                  // column 2*row + 1
+          fhp[2 * cc + half] = hw0;
+          fhp[2 * (cc + 1) + half] = hw1;
+          flp[2 * cc + half] = lw0;
+          flp[2 * (cc + 1) + half] = lw1;
+        }
       }
-      if (row < RB && ch < nchunk) {
-        // inputs 8ch..8ch+7: K-block kb, offset kk0 (0, 8, 16, 24) inside it;
-        // kk < 16 -> b0 words of threads c = kk/4, else b1 words of c = (kk-16)/4
-        const int kb = ch >> 2, kk0 = (ch & 3) * 8;
-        const int cc = (kk0 & 15) >> 2, half = kk0 >> 4;
-        uint32_t* fh = frag + ((size_t)kb * NC + 2 * row) * 8;   // column 2*row: 4 threads x (b0, b1)
-        uint32_t* fl = fh + 8;                                   // column 2*row + 1
-        fh[2 * cc + half] = hw[0];
-        fh[2 * (cc + 1) + half] = hw[1];
-        fl[2 * cc + half] = lw[0];
-        fl[2 * (cc + 1) + half] = lw[1];
-      }
-    }
+      int vsum = 256 * sum_hi + sum_lo;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) vsum += __shfl_xor_sync(0xffffffffu, vsum, o);
-    if (lane == 0) {
-      TStat st;
-      st.step = mx > 0.f ? mx / kQMax : 0.f;
-      st.sum = vsum;
-      st.pad[0] = st.pad[1] = 0;
-      reinterpret_cast<TStat*>(blk)[row] = st;
+      for (int o = 16; o > 0; o >>= 1) vsum += __shfl_xor_sync(0xffffffffu, vsum, o);
+      if (lane == 0) {
+        TStat st;
+        st.step = mx > 0.f ? mx / kQMax : 0.f;
+        st.sum = vsum;
+        st.pad[0] = st.pad[1] = 0;
+        reinterpret_cast<TStat*>(blk)[row] = st;
+      }
     }
   }
 }
@@ -585,82 +546,91 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 4 : 1) latent_pass_ker
 }
 
 // ---------------------------------------------------------------------------
-// finalize:  t'_j = l_j * sum over slices of the partials, quantised to the
-// int8 hi/lo planes and the per-row step the output pass reads.  One CTA per
-// (layer, path), in a launch between the two passes.
+// finalize:  t'_j = l_j * sum over slices of the partials, quantised per batch
+// row to the int8 hi/lo planes and the step the output pass reads.  One warp
+// per (layer, path), in a launch between the two passes; lane i owns latent
+// rows j = i + 32k (k < ceil(s/32)), max and sum are warp reductions.  Plane
+// bytes of rows >= batch are not written: the output pass's product columns
+// for them are independent of the batch rows' and their sums are discarded.
 // ---------------------------------------------------------------------------
 template <int NB>
-__global__ void __launch_bounds__(kVWarps * 32) finalize_kernel(const DecodeArgs a) {
-  __shared__ float s_mx[kVWarps][16];
-  __shared__ int s_sm[kVWarps][16];
-  extern __shared__ __align__(1024) unsigned char smem[];
-  float* tp = reinterpret_cast<float*>(smem);   // [B][S16]
-  const int tid = threadIdx.x;
+__global__ void __launch_bounds__(kQWarps * 32) finalize_kernel(const DecodeArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int item = blockIdx.x * kQWarps + (threadIdx.x >> 5);
+  if (item >= a.p_items) return;
   const int B = a.batch;
-  const LayerDesc& L = a.layers[layer_of(a.item_layer.p, a.n_layers, blockIdx.x)];
-  const int p = blockIdx.x - L.p_begin;
-  const PathDesc& P = L.p[p];
-  const int s = L.s, S16 = (s + 15) & ~15, S32 = (s + 31) & ~31;
-  float mt[4 * NB];
-  int ts[4 * NB];
-#pragma unroll
-  for (int b = 0; b < 4 * NB; ++b) { mt[b] = 0.f; ts[b] = 0; }
-  // a latent row's slice partials are contiguous: float4 loads, summed in slice order
+  const LayerDesc& L = a.layers[layer_of(a.item_layer.p, a.n_layers, item)];
+  const PathDesc& P = L.p[item - L.p_begin];
+  const int s = L.s, S16 = (s + 15) & ~15, nkt = (s + 31) >> 5;
   const int ns = L.n_slices, ng = (ns + 3) >> 2;
-#pragma unroll 2
-  for (int i = tid; i < B * S16; i += kVWarps * 32) {
-    const int b = i / S16, j = i - b * S16;
-    float t = 0.f;
-    if (j < s) {
-      const float4* pp = reinterpret_cast<const float4*>(P.ws.partial) + (size_t)i * ng;
-#pragma unroll 4
-      for (int q4 = 0; q4 < ng; ++q4) {
-        const float4 v = pp[q4];
-        const int q = 4 * q4;
-        t += v.x;
-        if (q + 1 < ns) t += v.y;
-        if (q + 2 < ns) t += v.z;
-        if (q + 3 < ns) t += v.w;
+  // loads depend only on the warp-uniform k < nkt (no divergent branch around
+  // them); lanes past the last latent row read row s-1 (l) or S16-1 (partials,
+  // finite: the latent pass writes every row below S16) and are zeroed by select
+  float lv[kMaxRank / 32];
+#pragma unroll
+  for (int k = 0; k < kMaxRank / 32; ++k) {
+    const int j = lane + 32 * k;
+    lv[k] = 0.f;
+    if (k < nkt) {
+      const float l = h2f(P.l[min(j, s - 1)]);
+      lv[k] = j < s ? l : 0.f;
+    }
+  }
+#pragma unroll 1
+  for (int b = 0; b < B; ++b) {
+    // a latent row's slice partials are contiguous float4s, summed in slice
+    // order; the four-slice groups are the outer loop so that the loads of
+    // all of a lane's rows are in flight together
+    float t[kMaxRank / 32];
+#pragma unroll
+    for (int k = 0; k < kMaxRank / 32; ++k) t[k] = 0.f;
+    const float4* pb = reinterpret_cast<const float4*>(P.ws.partial) + ((size_t)b * S16 + lane) * ng;
+#pragma unroll 1
+    for (int q4 = 0; q4 < ng; ++q4) {
+      const int q = 4 * q4;
+#pragma unroll
+      for (int k = 0; k < kMaxRank / 32; ++k) {
+        if (k < nkt) {
+          const int jr = min(lane + 32 * k, S16 - 1) - lane;   // row offset from this lane's first row
+          const float4 f = pb[(size_t)jr * ng + q4];
+          t[k] += f.x;
+          if (q + 1 < ns) t[k] += f.y;
+          if (q + 2 < ns) t[k] += f.z;
+          if (q + 3 < ns) t[k] += f.w;
+        }
       }
-      t *= h2f(P.l[j]);
     }
-    tp[i] = t;
+    float mx = 0.f;
 #pragma unroll
-    for (int bb = 0; bb < 4 * NB; ++bb)
-      if (bb == b) mt[bb] = fmaxf(mt[bb], fabsf(t));
-  }
-  block_max<4 * NB>(mt, s_mx);
-  // planes hold 4*NB batch rows (rows >= B are zero) so that the output pass
-  // loads every thread's B fragment without a predicate
-  for (int i = tid; i < 4 * NB * S32; i += kVWarps * 32) {
-    const int b = i / S32, j = i - b * S32;
-    float tinv = 0.f;
-#pragma unroll
-    for (int bb = 0; bb < 4 * NB; ++bb)
-      if (bb == b) tinv = mt[bb] > 0.f ? kQMax / mt[bb] : 0.f;
-    int8_t hi8 = 0, lo8 = 0;
-    if (j < s && b < B) {
-      const int v = quantise(tp[b * S16 + j], tinv, hi8, lo8);
-#pragma unroll
-      for (int bb = 0; bb < 4 * NB; ++bb)
-        if (bb == b) ts[bb] += v;
+    for (int k = 0; k < kMaxRank / 32; ++k) {
+      t[k] = lv[k] != 0.f ? t[k] * lv[k] : 0.f;   // rows >= s: 0 whatever the clamped loads gave
+      mx = fmaxf(mx, fabsf(t[k]));
     }
-    int8_t* pl = P.ws.planes + ((size_t)((j >> 5) * 4 * NB + b) * 2) * 32 + (j & 31);
-    pl[0] = hi8;
-    pl[32] = lo8;
-  }
-  block_sum<4 * NB>(ts, s_sm);
-  if (tid < 4 * NB) {
-    float m = 0.f;
-    int sum = 0;
 #pragma unroll
-    for (int bb = 0; bb < 4 * NB; ++bb)
-      if (bb == tid) { m = mt[bb]; sum = ts[bb]; }
-    TStat st;
-    st.step = m > 0.f ? m / kQMax : 0.f;
-    st.sum = sum;
-    st.pad[0] = st.pad[1] = 0;
-    P.ws.tstat[tid] = st;
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float inv = mx > 0.f ? kQMax / mx : 0.f;
+    int vsum = 0;
+#pragma unroll
+    for (int k = 0; k < kMaxRank / 32; ++k) {
+      if (k < nkt) {
+        // v = round(t * inv) in the low bits of the float's encoding (see the
+        // quantise pass); lo = its low byte, hi = byte 1 of v + 128
+        const uint32_t fb = __float_as_uint(fmaf(t[k], inv, kRoundMagic));
+        vsum += (int)(fb - 0x4B400000u);
+        int8_t* pl = P.ws.planes + ((size_t)(k * 4 * NB + b) * 2) * 32 + lane;
+        pl[0] = (int8_t)((fb + 128u) >> 8);
+        pl[32] = (int8_t)fb;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) vsum += __shfl_xor_sync(0xffffffffu, vsum, o);
+    if (lane == 0) {
+      TStat st;
+      st.step = mx > 0.f ? mx / kQMax : 0.f;
+      st.sum = vsum;
+      st.pad[0] = st.pad[1] = 0;
+      P.ws.tstat[b] = st;
+    }
   }
 }
 
@@ -889,16 +859,8 @@ constexpr size_t latent_smem() {
 
 
 template <int NB>
-cudaError_t launch_finalize(const DecodeArgs& a, int max_s16, cudaStream_t st) {
-  const size_t smem = (size_t)a.batch * max_s16 * 4;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(finalize_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)((size_t)4 * NB * kMaxRank * 4));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  finalize_kernel<NB><<<a.p_items, kVWarps * 32, smem, st>>>(a);
+cudaError_t launch_finalize(const DecodeArgs& a, int, cudaStream_t st) {
+  finalize_kernel<NB><<<(a.p_items + kQWarps - 1) / kQWarps, kQWarps * 32, 0, st>>>(a);
   return cudaGetLastError();
 }
 

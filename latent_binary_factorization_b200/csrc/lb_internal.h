@@ -97,7 +97,7 @@ struct LayerDesc {
   int v_begin;        // first latent-pass work item of this layer
   int u_begin;        // first output-pass work item of this layer
   int p_begin;        // first (layer, path) index of this layer
-  int x_begin;        // first quantise-pass item (layer, path, slice) of this layer
+  int x_begin;        // first quantise-pass item (layer, input slice) of this layer
 };
 
 // Layer index of every work item of each pass (device arrays built with the
@@ -118,7 +118,7 @@ struct DecodeArgs {
   int v_items;              // total latent-pass items
   int u_items;              // total output-pass items (layer, 128-row block)
   int p_items;              // total (layer, path) pairs
-  int x_items;              // total quantise-pass items (layer, path, input slice)
+  int x_items;              // total quantise-pass items (layer, input slice)
 };
 
 // Launchers (decode.cu), in stream order quantise -> latent -> finalize ->

@@ -93,7 +93,7 @@ size_t path_scratch_bytes(const lb_layer& L, int batch) {
 constexpr size_t kStatusBytes = 256;   // device status word at the start of a workspace
 
 lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
-                         cudaStream_t st, cudaEvent_t between) {
+                         cudaStream_t st, const cudaEvent_t* events, int n_events) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -105,7 +105,7 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   for (int i = 0; i < n; ++i) {
     const lb_layer& L = layers[i];
     const int npaths = L.residual + 1, n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
-    x_items += npaths * n_slices;
+    x_items += n_slices;
     v_items += npaths * n_slices * lb::ceil_div(lb::s16(L.s) / 16, lb::kVRowChunk);
     p_items += npaths;
     u_items += L.d_out / lb::kUTileRows;
@@ -168,7 +168,7 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
     D.v_begin = vi;
     D.p_begin = pi;
     D.u_begin = ui;
-    for (int k = 0; k < D.npaths * D.n_slices; ++k) xm[xi++] = i;
+    for (int k = 0; k < D.n_slices; ++k) xm[xi++] = i;
     for (int k = 0; k < D.npaths * D.n_slices * D.n_rchunks; ++k) vm[vi++] = i;
     for (int k = 0; k < D.npaths; ++k) pm[pi++] = i;
     for (int k = 0; k < L.d_out / lb::kUTileRows; ++k) um[ui++] = i;
@@ -215,16 +215,15 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   a.p_items = p_items;
   a.x_items = x_items;
   const int sms = num_sms(dev);
+  // events[i] (if given) is recorded right after launch i
+  auto mark = [&](int i) { return i < n_events && events[i] ? cudaEventRecord(events[i], st) : cudaSuccess; };
   e = lb::launch_quantise_pass(a, st);
+  if (e == cudaSuccess) e = mark(0);
+  if (e == cudaSuccess) e = lb::launch_latent_pass(a, max_s16, sms, st);
+  if (e == cudaSuccess) e = mark(1);
+  if (e == cudaSuccess) e = lb::launch_finalize_pass(a, max_s16, st);
+  if (e == cudaSuccess) e = mark(2);
   if (e != cudaSuccess) return cuda_fail(e);
-  e = lb::launch_latent_pass(a, max_s16, sms, st);
-  if (e != cudaSuccess) return cuda_fail(e);
-  e = lb::launch_finalize_pass(a, max_s16, st);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (between) {
-    e = cudaEventRecord(between, st);
-    if (e != cudaSuccess) return cuda_fail(e);
-  }
   e = lb::launch_output_pass(a, sms, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return LB_OK;
@@ -382,7 +381,7 @@ lb_status littlebit_pack_signs(const void* src_dev, lb_dtype dt, int n_long, int
 
 lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, const void* const* xs,
                                               void* const* ys, int batch, lb_dtype xdt, void* stream,
-                                              void* event_between) {
+                                              void* const* events, int n_events) {
   if (!layers || !xs || !ys || n < 1) return LB_ERR_ARG;
   if (batch < 1) return LB_ERR_SHAPE;
   for (int i = 0; i < n; ++i) {
@@ -394,7 +393,7 @@ lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, con
   if (batch <= lb::kMaxBatchDecode) {
     if (xdt != LB_F16) return LB_ERR_UNSUPPORTED;
     return decode_forward(layers, n, xs, ys, batch, static_cast<cudaStream_t>(stream),
-                          static_cast<cudaEvent_t>(event_between));
+                          reinterpret_cast<const cudaEvent_t*>(events), n_events);
   }
   if (batch % 128 == 0) {
     if (xdt != LB_F16 && xdt != LB_BF16) return LB_ERR_UNSUPPORTED;
@@ -408,7 +407,7 @@ lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, con
 
 lb_status littlebit_linear_forward_many(const lb_layer* layers, int n, const void* const* xs, void* const* ys,
                                         int batch, lb_dtype xdt, void* stream) {
-  return littlebit_linear_forward_many_timed(layers, n, xs, ys, batch, xdt, stream, nullptr);
+  return littlebit_linear_forward_many_timed(layers, n, xs, ys, batch, xdt, stream, nullptr, 0);
 }
 
 lb_status littlebit_linear_forward(const lb_layer* layer, const void* x_dev, void* y_dev, int batch,

@@ -62,7 +62,7 @@ _lib.littlebit_linear_forward_many_timed.restype = ctypes.c_int
 _lib.littlebit_linear_forward_many_timed.argtypes = [ctypes.POINTER(LbLayer), ctypes.c_int,
                                                      ctypes.POINTER(ctypes.c_void_p),
                                                      ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_int,
-                                                     ctypes.c_void_p, ctypes.c_void_p]
+                                                     ctypes.c_void_p, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]
 _lib.littlebit_device_status.restype = ctypes.c_int
 _lib.littlebit_device_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint)]
 _lib.littlebit_release.restype = None
@@ -183,15 +183,18 @@ class Stack:
         self._xp = (ctypes.c_void_p * n)(*[x.data_ptr() for x in xs])
         self._yp = (ctypes.c_void_p * n)(*[y.data_ptr() for y in ys])
 
-    def __call__(self, stream=None, event_between: torch.cuda.Event | None = None) -> None:
-        if event_between is None:
+    def __call__(self, stream=None, events: list | None = None) -> None:
+        """One forward of every layer.  ``events`` (decode only): up to three
+        torch.cuda.Event recorded after the quantise, latent and finalize
+        launches (the output pass follows the last)."""
+        if not events:
             _check(_lib.littlebit_linear_forward_many(self._arr, self._n, self._xp, self._yp, self.batch,
                                                       self.dtype, _stream(stream)),
                    "littlebit_linear_forward_many")
         else:
+            evs = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
             _check(_lib.littlebit_linear_forward_many_timed(self._arr, self._n, self._xp, self._yp, self.batch,
-                                                            self.dtype, _stream(stream),
-                                                            ctypes.c_void_p(event_between.cuda_event)),
+                                                            self.dtype, _stream(stream), evs, len(events)),
                    "littlebit_linear_forward_many_timed")
 
 
