@@ -547,90 +547,86 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 4 : 1) latent_pass_ker
 
 // ---------------------------------------------------------------------------
 // finalize:  t'_j = l_j * sum over slices of the partials, quantised per batch
-// row to the int8 hi/lo planes and the step the output pass reads.  One warp
-// per (layer, path), in a launch between the two passes; lane i owns latent
-// rows j = i + 32k (k < ceil(s/32)), max and sum are warp reductions.  Plane
-// bytes of rows >= batch are not written: the output pass's product columns
-// for them are independent of the batch rows' and their sums are discarded.
+// row to the int8 hi/lo planes and the step the output pass reads.  One CTA
+// per (layer, path), in a launch between the two passes: warp w takes the
+// 32-row groups k = w, w+4, ...; the max and the sum over the path are combined
+// with integer atomics in shared memory (order-independent, so deterministic).
+// Plane bytes of rows >= batch are not written: the output pass's product
+// columns for them are independent of the batch rows' and their sums are
+// discarded.
 // ---------------------------------------------------------------------------
+constexpr int kFWarps = 4;
+
 template <int NB>
-__global__ void __launch_bounds__(kQWarps * 32) finalize_kernel(const DecodeArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int item = blockIdx.x * kQWarps + (threadIdx.x >> 5);
-  if (item >= a.p_items) return;
+__global__ void __launch_bounds__(kFWarps * 32) finalize_kernel(const DecodeArgs a) {
+  __shared__ float s_t[kMaxRank];   // t' of this path, one batch row at a time
+  __shared__ unsigned s_mx;         // max |t'| (non-negative float bits order as unsigned)
+  __shared__ int s_sum;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int item = blockIdx.x;
   const int B = a.batch;
   const LayerDesc& L = a.layers[layer_of(a.item_layer.p, a.n_layers, item)];
   const PathDesc& P = L.p[item - L.p_begin];
   const int s = L.s, S16 = (s + 15) & ~15, nkt = (s + 31) >> 5;
   const int ns = L.n_slices, ng = (ns + 3) >> 2;
-  // loads depend only on the warp-uniform k < nkt (no divergent branch around
-  // them); lanes past the last latent row read row s-1 (l) or S16-1 (partials,
-  // finite: the latent pass writes every row below S16) and are zeroed by select
-  float lv[kMaxRank / 32];
-#pragma unroll
-  for (int k = 0; k < kMaxRank / 32; ++k) {
-    const int j = lane + 32 * k;
-    lv[k] = 0.f;
-    if (k < nkt) {
-      const float l = h2f(P.l[min(j, s - 1)]);
-      lv[k] = j < s ? l : 0.f;
-    }
-  }
 #pragma unroll 1
   for (int b = 0; b < B; ++b) {
-    // a latent row's slice partials are contiguous float4s, summed in slice
-    // order; the four-slice groups are the outer loop so that the loads of
-    // all of a lane's rows are in flight together
-    float t[kMaxRank / 32];
-#pragma unroll
-    for (int k = 0; k < kMaxRank / 32; ++k) t[k] = 0.f;
-    const float4* pb = reinterpret_cast<const float4*>(P.ws.partial) + ((size_t)b * S16 + lane) * ng;
-#pragma unroll 1
-    for (int q4 = 0; q4 < ng; ++q4) {
-      const int q = 4 * q4;
-#pragma unroll
-      for (int k = 0; k < kMaxRank / 32; ++k) {
-        if (k < nkt) {
-          const int jr = min(lane + 32 * k, S16 - 1) - lane;   // row offset from this lane's first row
-          const float4 f = pb[(size_t)jr * ng + q4];
-          t[k] += f.x;
-          if (q + 1 < ns) t[k] += f.y;
-          if (q + 2 < ns) t[k] += f.z;
-          if (q + 3 < ns) t[k] += f.w;
-        }
-      }
+    if (tid == 0) {
+      s_mx = 0u;
+      s_sum = 0;
     }
+    __syncthreads();
+    // a latent row's slice partials are contiguous float4s, summed in slice order
     float mx = 0.f;
-#pragma unroll
-    for (int k = 0; k < kMaxRank / 32; ++k) {
-      t[k] = lv[k] != 0.f ? t[k] * lv[k] : 0.f;   // rows >= s: 0 whatever the clamped loads gave
-      mx = fmaxf(mx, fabsf(t[k]));
+#pragma unroll 2
+    for (int k = warp; k < nkt; k += kFWarps) {
+      const int j = lane + 32 * k;
+      const int jc = min(j, S16 - 1);   // rows past S16 clamp (finite; zeroed below)
+      const float4* pp = reinterpret_cast<const float4*>(P.ws.partial) + ((size_t)b * S16 + jc) * ng;
+      float t = 0.f;
+#pragma unroll 4
+      for (int q4 = 0; q4 < ng; ++q4) {
+        const float4 f = pp[q4];
+        const int q = 4 * q4;
+        t += f.x;
+        if (q + 1 < ns) t += f.y;
+        if (q + 2 < ns) t += f.z;
+        if (q + 3 < ns) t += f.w;
+      }
+      const float l = h2f(P.l[min(j, s - 1)]);
+      const float v = j < s ? t * l : 0.f;
+      s_t[j] = v;
+      mx = fmaxf(mx, fabsf(v));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) atomicMax(&s_mx, __float_as_uint(mx));
+    __syncthreads();
+    mx = __uint_as_float(s_mx);
     const float inv = mx > 0.f ? kQMax / mx : 0.f;
     int vsum = 0;
-#pragma unroll
-    for (int k = 0; k < kMaxRank / 32; ++k) {
-      if (k < nkt) {
-        // v = round(t * inv) in the low bits of the float's encoding (see the
-        // quantise pass); lo = its low byte, hi = byte 1 of v + 128
-        const uint32_t fb = __float_as_uint(fmaf(t[k], inv, kRoundMagic));
-        vsum += (int)(fb - 0x4B400000u);
-        int8_t* pl = P.ws.planes + ((size_t)(k * 4 * NB + b) * 2) * 32 + lane;
-        pl[0] = (int8_t)((fb + 128u) >> 8);
-        pl[32] = (int8_t)fb;
-      }
+#pragma unroll 2
+    for (int k = warp; k < nkt; k += kFWarps) {
+      // v = round(t' * inv) in the low bits of the float's encoding (see the
+      // quantise pass); lo = its low byte, hi = byte 1 of v + 128
+      const uint32_t fb = __float_as_uint(fmaf(s_t[lane + 32 * k], inv, kRoundMagic));
+      vsum += (int)(fb - 0x4B400000u);
+      int8_t* pl = P.ws.planes + ((size_t)(k * 4 * NB + b) * 2) * 32 + lane;
+      pl[0] = (int8_t)((fb + 128u) >> 8);
+      pl[32] = (int8_t)fb;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) vsum += __shfl_xor_sync(0xffffffffu, vsum, o);
-    if (lane == 0) {
+    if (lane == 0) atomicAdd(&s_sum, vsum);
+    __syncthreads();
+    if (tid == 0) {
       TStat st;
       st.step = mx > 0.f ? mx / kQMax : 0.f;
-      st.sum = vsum;
+      st.sum = s_sum;
       st.pad[0] = st.pad[1] = 0;
       P.ws.tstat[b] = st;
     }
+    __syncthreads();   // s_mx, s_sum and s_t are reset for the next batch row
   }
 }
 
@@ -860,7 +856,7 @@ constexpr size_t latent_smem() {
 
 template <int NB>
 cudaError_t launch_finalize(const DecodeArgs& a, int, cudaStream_t st) {
-  finalize_kernel<NB><<<(a.p_items + kQWarps - 1) / kQWarps, kQWarps * 32, 0, st>>>(a);
+  finalize_kernel<NB><<<a.p_items, kFWarps * 32, 0, st>>>(a);
   return cudaGetLastError();
 }
 
