@@ -547,7 +547,10 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 4 : 1) latent_pass_ker
 
 // ---------------------------------------------------------------------------
 // finalize:  t'_j = l_j * sum over slices of the partials, quantised per batch
-// row to the int8 hi/lo planes and the step the output pass reads.  One CTA
+// row to the int8 hi/lo planes and the step the output pass reads.  At batch 1
+// the planes of a layer's paths form one K range (packed output pass): path
+// p's K-tiles come after path p-1's, with its t' in row p of each tile and
+// zeros in the other path's row.  One CTA
 // per (layer, path), in a launch between the two passes: warp w takes the
 // 32-row groups k = w, w+4, ...; the max and the sum over the path are combined
 // with integer atomics in shared memory (order-independent, so deterministic).
@@ -566,9 +569,11 @@ __global__ void __launch_bounds__(kFWarps * 32) finalize_kernel(const DecodeArgs
   const int item = blockIdx.x;
   const int B = a.batch;
   const LayerDesc& L = a.layers[layer_of(a.item_layer.p, a.n_layers, item)];
-  const PathDesc& P = L.p[item - L.p_begin];
+  const int pi = item - L.p_begin;
+  const PathDesc& P = L.p[pi];
   const int s = L.s, S16 = (s + 15) & ~15, nkt = (s + 31) >> 5;
   const int ns = L.n_slices, ng = (ns + 3) >> 2;
+  const bool packed = B == 1;   // batch 1: the output pass takes both paths as one K range
 #pragma unroll 1
   for (int b = 0; b < B; ++b) {
     if (tid == 0) {
@@ -611,9 +616,21 @@ __global__ void __launch_bounds__(kFWarps * 32) finalize_kernel(const DecodeArgs
       // quantise pass); lo = its low byte, hi = byte 1 of v + 128
       const uint32_t fb = __float_as_uint(fmaf(s_t[lane + 32 * k], inv, kRoundMagic));
       vsum += (int)(fb - 0x4B400000u);
-      int8_t* pl = P.ws.planes + ((size_t)(k * 4 * NB + b) * 2) * 32 + lane;
-      pl[0] = (int8_t)((fb + 128u) >> 8);
-      pl[32] = (int8_t)fb;
+      if (packed) {
+        // K-tile pi*nkt + k of the layer's combined planes: row pi holds this
+        // path's t', the other path's row is zero
+        int8_t* pl = L.p[0].ws.planes + ((size_t)(pi * nkt + k) * 4 * 2) * 32 + lane;
+        pl[pi * 64] = (int8_t)((fb + 128u) >> 8);
+        pl[pi * 64 + 32] = (int8_t)fb;
+        if (L.npaths == 2) {
+          pl[(1 - pi) * 64] = 0;
+          pl[(1 - pi) * 64 + 32] = 0;
+        }
+      } else {
+        int8_t* pl = P.ws.planes + ((size_t)(k * 4 * NB + b) * 2) * 32 + lane;
+        pl[0] = (int8_t)((fb + 128u) >> 8);
+        pl[32] = (int8_t)fb;
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) vsum += __shfl_xor_sync(0xffffffffu, vsum, o);
@@ -845,6 +862,173 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
   }
 }
 
+// ---------------------------------------------------------------------------
+// output pass, batch 1 ("packed"): the product's 8 columns hold 4 batch rows,
+// of which batch 1 uses one, so the paths take the spare ones instead.  Both
+// paths' K-tiles form one K range (path 1's after path 0's); the t' operand
+// of path p's tiles sits in column pair p with zeros in the other path's pair,
+// so one accumulator holds both paths' sums, in different columns.  Lanes with
+// c = 0 and c = 1 scale their path's rows (h_p, step_p) and one shuffle adds
+// the paths.  One chunk carries up to 8 K-tiles of the range, so a small-rank
+// residual layer's 128-row item is one chunk and one epilogue.
+// ---------------------------------------------------------------------------
+// stage: [8 tiles: 4 KB][t' bytes: 8 x 256][h of path 0, 1: 2 x 256][TStat of path 0, 1]
+constexpr int kPkPlanesOff = kUChunkBytes;
+constexpr int kPkHOff = kPkPlanesOff + kUChunkTiles * 256;
+constexpr int kPkTsOff = kPkHOff + 2 * kUTileRows * 2;
+constexpr int kPkStageBytes = (kPkTsOff + 2 * 16 + 127) & ~127;
+constexpr int kPkStages = 2;
+
+struct PkCursor {
+  int li, item, kv0;                 // item, first K-tile of the chunk in the packed range
+  int n_kt, npaths, u_begin, u_end;
+  const unsigned char *U0, *U1;      // path 1 = path 0 for a single-path layer
+  const int8_t* planes;              // the layer's combined t' bytes
+  const uint16_t *h0, *h1;
+  const TStat *ts0, *ts1;
+
+  __device__ __forceinline__ void enter(const DecodeArgs& a, int l) {
+    li = l;
+    const LayerDesc& L = a.layers[l];
+    n_kt = (L.s + 31) >> 5;
+    npaths = L.npaths;
+    u_begin = L.u_begin;
+    u_end = (l + 1 < a.n_layers) ? a.layers[l + 1].u_begin : a.u_items;
+    const PathDesc& P0 = L.p[0];
+    const PathDesc& P1 = L.p[npaths - 1];
+    U0 = reinterpret_cast<const unsigned char*>(P0.U);
+    U1 = reinterpret_cast<const unsigned char*>(P1.U);
+    h0 = P0.h;
+    h1 = P1.h;
+    ts0 = P0.ws.tstat;
+    ts1 = P1.ws.tstat;
+    planes = P0.ws.planes;
+  }
+  __device__ __forceinline__ int n_kv() const { return npaths * n_kt; }
+  __device__ __forceinline__ int ntile() const { return min(kUChunkTiles, n_kv() - kv0); }
+  __device__ __forceinline__ bool item_end() const { return kv0 + kUChunkTiles >= n_kv(); }
+  __device__ __forceinline__ void advance(const DecodeArgs& a) {
+    kv0 += kUChunkTiles;
+    if (kv0 >= n_kv()) {
+      kv0 = 0;
+      if (++item == u_end && item < a.u_items) enter(a, li + 1);
+    }
+  }
+};
+
+__device__ __forceinline__ void pk_issue(const PkCursor& cu, unsigned char* stage, uint64_t* bar) {
+  const int ob = cu.item - cu.u_begin;
+  const int nt = cu.ntile();
+  const int t0 = max(0, min(nt, cu.n_kt - cu.kv0));   // tiles of path 0 in this chunk
+  const int t1 = nt - t0;                              // tiles of path 1
+  const bool last = cu.item_end();
+  mbar_expect_tx(bar, (uint32_t)nt * (kTileBytes + 256) + (last ? cu.npaths * (kUTileRows * 2 + 16) : 0));
+  if (t0 > 0)
+    bulk_g2s(stage, cu.U0 + ((size_t)ob * cu.n_kt + cu.kv0) * kTileBytes, (uint32_t)t0 * kTileBytes, bar);
+  if (t1 > 0)
+    bulk_g2s(stage + t0 * kTileBytes, cu.U1 + ((size_t)ob * cu.n_kt + (cu.kv0 + t0 - cu.n_kt)) * kTileBytes,
+             (uint32_t)t1 * kTileBytes, bar);
+  bulk_g2s(stage + kPkPlanesOff, cu.planes + (size_t)cu.kv0 * 256, (uint32_t)nt * 256, bar);
+  if (last) {
+    bulk_g2s(stage + kPkHOff, cu.h0 + (size_t)ob * kUTileRows, kUTileRows * 2, bar);
+    bulk_g2s(stage + kPkTsOff, cu.ts0, 16, bar);
+    if (cu.npaths == 2) {
+      bulk_g2s(stage + kPkHOff + kUTileRows * 2, cu.h1 + (size_t)ob * kUTileRows, kUTileRows * 2, bar);
+      bulk_g2s(stage + kPkTsOff + 16, cu.ts1, 16, bar);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kUWarps * 32) output_packed_kernel(const DecodeArgs a) {
+  constexpr int S = kPkStages;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  unsigned char* my_ring = smem + (size_t)warp * S * kPkStageBytes;
+  uint64_t* my_bar = reinterpret_cast<uint64_t*>(smem + (size_t)kUWarps * S * kPkStageBytes) + warp * S;
+
+  const long long W = (long long)gridDim.x * kUWarps, gw = (long long)blockIdx.x * kUWarps + warp;
+  const int i_begin = (int)(a.u_items * gw / W), i_end = (int)(a.u_items * (gw + 1) / W);
+  if (i_begin >= i_end) return;   // no CTA-wide barriers in this kernel
+
+  if (lane == 0) {
+    for (int st = 0; st < S; ++st) mbar_init(&my_bar[st], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  PkCursor fd;
+  fd.enter(a, layer_of(a.item_layer.u, a.n_layers, i_begin));
+  fd.item = i_begin;
+  fd.kv0 = 0;
+  PkCursor cs = fd;
+#pragma unroll 1
+  for (int st = 0; st < S; ++st) {
+    if (fd.item < i_end) {
+      if (lane == 0) pk_issue(fd, my_ring + st * kPkStageBytes, &my_bar[st]);
+      fd.advance(a);
+    }
+  }
+
+  int d[8][1][4];   // starts at an item's first K-tile (zero-accumulator product)
+  uint32_t consumed = 0;
+  int slot = 0;
+  bool dead = false;
+  // this thread's B-operand column: row g/2 (path g/2 for g < 4), plane g%2
+  const int pl_off = kPkPlanesOff + g * 32 + 4 * c;
+  const int pc = min(c, 1);   // path whose sums this lane's columns 2c, 2c+1 hold (c < 2)
+
+  while (cs.item < i_end) {
+    if (!dead && !mbar_wait(&my_bar[slot], (consumed / S) & 1)) {
+      dead = true;
+      atomicOr(a.status, 1u << LB_ERR_TIMEOUT);
+    }
+    const unsigned char* stage = my_ring + slot * kPkStageBytes;
+    const int nt = cs.ntile();
+    const unsigned char* pl = stage + pl_off;
+    if (cs.kv0 == 0) out_tile<1, true>(d, stage, 0, lane, pl);
+    else out_tile<1>(d, stage, 0, lane, pl);
+    if (nt == kUChunkTiles) {
+#pragma unroll
+      for (int t = 1; t < kUChunkTiles; ++t) out_tile<1>(d, stage, t, lane, pl);
+    } else {
+#pragma unroll 1
+      for (int t = 1; t < nt; ++t) out_tile<1>(d, stage, t, lane, pl);
+    }
+    if (cs.item_end()) {
+      // rows 128*ob + 16q + g (+8); lane c < npaths scales path c, then c = 0
+      // adds c = 1's value and stores
+      const bool live = c < cs.npaths;
+      const uint16_t* hs = reinterpret_cast<const uint16_t*>(stage + kPkHOff + pc * kUTileRows * 2);
+      const TStat tsp = reinterpret_cast<const TStat*>(stage + kPkTsOff)[pc];
+      const float base = tsp.step * (float)tsp.sum, m2 = -2.f * tsp.step;
+      const LayerDesc& L = a.layers[cs.li];
+      uint16_t* yr = L.y + (cs.item - cs.u_begin) * kUTileRows + g;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int c0 = ((d[q][0][0] >> q) << 8) + (d[q][0][1] >> q);
+        const int c1 = ((d[q][0][2] >> q) << 8) + (d[q][0][3] >> q);
+        float v0 = live ? h2f(hs[16 * q + g]) * fmaf(m2, (float)c0, base) : 0.f;
+        float v1 = live ? h2f(hs[16 * q + g + 8]) * fmaf(m2, (float)c1, base) : 0.f;
+        v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
+        v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+        if (c == 0) {
+          yr[16 * q] = f2h(v0);
+          yr[16 * q + 8] = f2h(v1);
+        }
+      }
+    }
+    // the stage has been read: refill it with the chunk `S` ahead
+    __syncwarp();
+    if (fd.item < i_end) {
+      if (lane == 0) pk_issue(fd, my_ring + slot * kPkStageBytes, &my_bar[slot]);
+      fd.advance(a);
+    }
+    ++consumed;
+    if (++slot == S) slot = 0;
+    cs.advance(a);
+  }
+}
+
 // ------------------------------------------------------------------ launchers
 
 template <int NB, int RB>
@@ -937,7 +1121,28 @@ cudaError_t launch_finalize_pass(const DecodeArgs& a, int max_s16, cudaStream_t 
   return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_output_packed(const DecodeArgs& a, int num_sms, cudaStream_t st) {
+  const size_t smem = (size_t)kUWarps * kPkStages * kPkStageBytes + (size_t)kUWarps * kPkStages * 8;
+  static bool attr_set = false;
+  cudaError_t e;
+  if (!attr_set) {
+    e = cudaFuncSetAttribute(output_packed_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, output_packed_kernel, kUWarps * 32, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  }
+  const int grid = max(1, min((a.u_items + kUWarps - 1) / kUWarps, per_sm * num_sms));
+  output_packed_kernel<<<grid, kUWarps * 32, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_output_pass(const DecodeArgs& a, int num_sms, cudaStream_t st) {
+  if (a.batch == 1) return launch_output_packed(a, num_sms, st);
   switch ((a.batch + 3) / 4) {
     case 1: return launch_output<1>(a, num_sms, st);
     case 2: return launch_output<2>(a, num_sms, st);

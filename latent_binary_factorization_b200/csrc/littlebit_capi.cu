@@ -81,9 +81,10 @@ size_t partial_bytes(const lb_layer& L, int batch) {
   const size_t ns4 = (size_t)lb::ceil_div(lb::ceil_div(L.d_in, lb::kVSlice), 4) * 4;
   return align_up(ns4 * batch * lb::s16(L.s) * sizeof(float), 256);
 }
-// t' planes and stats are padded to whole groups of four batch rows
+// t' planes and stats are padded to whole groups of four batch rows; at batch
+// 1 path 0's planes hold the combined K range of both paths (packed output pass)
 size_t planes_bytes(const lb_layer& L, int batch) {
-  return align_up((size_t)lb::ceil_div(batch, 4) * 4 * 2 * lb::s32(L.s), 256);
+  return align_up((size_t)lb::ceil_div(batch, 4) * 4 * 2 * lb::s32(L.s) * (batch == 1 ? 2 : 1), 256);
 }
 size_t tstat_bytes(int batch) { return align_up((size_t)lb::ceil_div(batch, 4) * 4 * sizeof(lb::TStat), 256); }
 size_t path_scratch_bytes(const lb_layer& L, int batch) {

@@ -70,7 +70,8 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
   const size_t xq_b = round256((size_t)n_slices * lb::xq_slice_bytes(batch));
   const size_t part_b = round256((size_t)lb::ceil_div(n_slices, 4) * 4 * batch * S16 * sizeof(float));
   const int bpad = lb::ceil_div(batch, 4) * 4;   // t' planes and stats padded to groups of 4 rows
-  const size_t planes_b = round256((size_t)bpad * 2 * S32);
+  // at batch 1 path 0's planes hold the combined K range of both paths
+  const size_t planes_b = round256((size_t)bpad * 2 * S32 * (batch == 1 ? 2 : 1));
   const size_t tstat_b = round256((size_t)bpad * sizeof(lb::TStat));
   const int npaths = L.residual + 1;
   if (kPathOff + (size_t)npaths * (xq_b + part_b + planes_b + tstat_b) > kNoAllocScratchBytes) return LB_ERR_SHAPE;
