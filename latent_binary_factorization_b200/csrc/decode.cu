@@ -299,7 +299,7 @@ __device__ __forceinline__ void x_issue(const DecodeArgs& a, int item, int li, u
 
 // One warp's sequence of bulk-copy chunks: per item, per group of kRPW row
 // blocks, per 4 K-tiles of the slice.
-template <int NB>
+template <int NB, int W>
 struct VFeed {
   static constexpr int RPW = VCfg<NB>::kRPW;
   int item, li, grp, kc;
@@ -307,6 +307,7 @@ struct VFeed {
   const unsigned char* V;
 
   __device__ __forceinline__ void set(const DecodeArgs& a, int warp) {
+    static_assert(W == 3 || W == 4, "latent-pass CTA width");
     const VItem it = decode_v(a, item, li);
     const LayerDesc& L = a.layers[li];
     const int k0 = it.sl * kVSlice;
@@ -314,7 +315,7 @@ struct VFeed {
     n_kt_all = L.d_in / kVTileK;
     kt0 = k0 / kVTileK;
     n_rb = (L.s + 15) >> 4;
-    rb0 = it.rc * kVRowChunk + 2 * warp;
+    rb0 = it.rc * (2 * W) + 2 * warp;
     V = reinterpret_cast<const unsigned char*>(L.p[it.p].V);
     grp = 0;
     kc = 0;
@@ -352,17 +353,17 @@ struct VFeed {
   }
 };
 
-template <int NB, int RB>
-__global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 4 : 1) latent_pass_kernel(const DecodeArgs a) {
+template <int NB, int RB, int W>
+__global__ void __launch_bounds__(W * 32, NB == 1 ? 4 : 1) latent_pass_kernel(const DecodeArgs a) {
   constexpr int NC = 2 * RB;                      // B-fragment columns stored per K-block
   constexpr int RPW = VCfg<NB>::kRPW;
   constexpr int kStageBytes = RPW * kChunkBytes;
   constexpr int kXBuf = xq_buf_bytes(NB, RB);
   extern __shared__ __align__(1024) unsigned char smem[];
   unsigned char* ring = smem;                                        // [warps][stages][RPW x 2 KB]
-  unsigned char* xbuf = smem + kVWarps * kVStages * kStageBytes;     // [2][kXBuf]
+  unsigned char* xbuf = smem + W * kVStages * kStageBytes;           // [2][kXBuf]
   uint64_t* mbar = reinterpret_cast<uint64_t*>(xbuf + 2 * kXBuf);    // [warps][stages]
-  uint64_t* xfull = mbar + kVWarps * kVStages;                       // [2]
+  uint64_t* xfull = mbar + W * kVStages;                             // [2]
   __shared__ int s_done[2];   // warps done with each buffer, accumulated over its uses
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
@@ -394,7 +395,7 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 4 : 1) latent_pass_ker
     if (nxt < i_end) x_issue<NB, RB>(a, nxt, it.li, xbuf + kXBuf, &xfull[1]);
   }
 
-  VFeed<NB> feed;
+  VFeed<NB, W> feed;
   feed.item = i_begin;
   feed.li = li0;
   feed.set(a, warp);
@@ -436,7 +437,7 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 4 : 1) latent_pass_ker
           const int b = (seq - 1) & 1;
           __threadfence_block();
           const int old = atomicAdd(&s_done[b], 1);
-          if (old == kVWarps * (((seq - 1) >> 1) + 1) - 1) {
+          if (old == W * (((seq - 1) >> 1) + 1) - 1) {
             __threadfence_block();
             const int nxt = item - it.rc + L.n_rchunks;   // first item of the following slice
             if (nxt < i_end) x_issue<NB, RB>(a, nxt, li, xbuf + b * kXBuf, &xfull[b]);
@@ -463,7 +464,7 @@ __global__ void __launch_bounds__(kVWarps * 32, NB == 1 ? 4 : 1) latent_pass_ker
     float* part = P.ws.partial + it.sl;
 #pragma unroll 1
     for (int grp = 0; grp * RPW < 2; ++grp) {
-      const int rbA = it.rc * kVRowChunk + 2 * warp + grp * RPW;
+      const int rbA = it.rc * (2 * W) + 2 * warp + grp * RPW;
       if (rbA >= n_rb) break;
       const int nvalid = min(RPW, n_rb - rbA);
       constexpr int R = RPW;
@@ -1031,10 +1032,10 @@ __global__ void __launch_bounds__(kUWarps * 32) output_packed_kernel(const Decod
 
 // ------------------------------------------------------------------ launchers
 
-template <int NB, int RB>
+template <int NB, int RB, int W>
 constexpr size_t latent_smem() {
-  return (size_t)kVWarps * kVStages * VCfg<NB>::kRPW * kChunkBytes + 2 * (size_t)xq_buf_bytes(NB, RB) +
-         ((size_t)kVWarps * kVStages + 2) * 8;
+  return (size_t)W * kVStages * VCfg<NB>::kRPW * kChunkBytes + 2 * (size_t)xq_buf_bytes(NB, RB) +
+         ((size_t)W * kVStages + 2) * 8;
 }
 
 
@@ -1049,26 +1050,27 @@ size_t output_smem(int) {
   return (size_t)kUWarps * OutCfg<NB>::kStages * out_stage_bytes(4 * NB) + (size_t)kUWarps * OutCfg<NB>::kStages * 8;
 }
 
-template <int NB, int RB>
+template <int NB, int RB, int W>
 cudaError_t launch_latent(const DecodeArgs& a, int num_sms, cudaStream_t st) {
   static_assert(RB == 4 * NB || (NB == 1 && RB == 1), "stored rows: 1 at batch 1, else 4 per n-block");
-  constexpr size_t smem = latent_smem<NB, RB>();
+  constexpr size_t smem = latent_smem<NB, RB, W>();
   static_assert(smem <= 227 * 1024, "latent pass shared memory");
+  auto kern = latent_pass_kernel<NB, RB, W>;
   static bool attr_set = false;
   cudaError_t e;
   if (!attr_set) {
-    e = cudaFuncSetAttribute(latent_pass_kernel<NB, RB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   static int per_sm = 0;
   if (per_sm == 0) {
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, latent_pass_kernel<NB, RB>, kVWarps * 32, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, W * 32, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
   }
   const int grid = max(1, min(a.v_items, per_sm * num_sms));
-  latent_pass_kernel<NB, RB><<<grid, kVWarps * 32, smem, st>>>(a);
+  kern<<<grid, W * 32, smem, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -1101,12 +1103,17 @@ cudaError_t launch_quantise_pass(const DecodeArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_latent_pass(const DecodeArgs& a, int, int num_sms, cudaStream_t st) {
-  if (a.batch == 1) return launch_latent<1, 1>(a, num_sms, st);
+  if (a.batch == 1) {
+    if (a.v_warps == 3) return launch_latent<1, 1, 3>(a, num_sms, st);
+    if (a.v_warps == 4) return launch_latent<1, 1, 4>(a, num_sms, st);
+    return cudaErrorInvalidValue;
+  }
+  if (a.v_warps != 4) return cudaErrorInvalidValue;
   switch ((a.batch + 3) / 4) {
-    case 1: return launch_latent<1, 4>(a, num_sms, st);
-    case 2: return launch_latent<2, 8>(a, num_sms, st);
-    case 3: return launch_latent<3, 12>(a, num_sms, st);
-    case 4: return launch_latent<4, 16>(a, num_sms, st);
+    case 1: return launch_latent<1, 4, 4>(a, num_sms, st);
+    case 2: return launch_latent<2, 8, 4>(a, num_sms, st);
+    case 3: return launch_latent<3, 12, 4>(a, num_sms, st);
+    case 4: return launch_latent<4, 16, 4>(a, num_sms, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -16,14 +16,32 @@ constexpr int kUTileRows = 128, kUTileK = 32;   // role-U tile
 constexpr int kTileBytes = 512;
 
 // Latent pass (V^T) work item: (layer, path, input slice, row chunk).  One CTA
-// of kVWarps warps covers kVSlice inputs (kVSliceTiles K-tiles) for kVRowChunk
-// 16-row latent blocks; warp w owns row blocks 2w and 2w+1 of the chunk over
-// the whole slice and streams their tiles in chunks of kChunkTiles K-tiles.
-constexpr int kVWarps = 4;
+// of W warps (latent_warps: 3 or 4) covers kVSlice inputs (kVSliceTiles
+// K-tiles) for 2*W 16-row latent blocks; warp w owns row blocks 2w and 2w+1 of
+// the chunk over the whole slice and streams their tiles in chunks of
+// kChunkTiles K-tiles.
 constexpr int kVSliceTiles = 8;
 constexpr int kVSlice = kVSliceTiles * kVTileK;          // 2048 inputs
-constexpr int kVRowChunk = 2 * kVWarps;                  // 16-row blocks per item
 constexpr int kVStages = 2;                              // bulk-copy ring per warp
+
+// Latent-pass CTA width for a call: at batch 1, 3 or 4 warps, whichever leaves
+// fewer row-block slots of the items idle (a chunk is 2*W row blocks), weighted
+// by each layer's V bits and with 3-warp CTAs discounted for their occupancy
+// (15 against 16 resident warps per SM); else 4.  rb_work(i, n_rb, w) gives
+// layer i's 16-row block count and weight.
+template <class F>
+inline int latent_warps(int n, int batch, F rb_work) {
+  if (batch != 1) return 4;
+  double sc3 = 0.0, sc4 = 0.0;
+  for (int i = 0; i < n; ++i) {
+    int n_rb = 1;
+    double w = 0.0;
+    rb_work(i, n_rb, w);
+    sc3 += w * n_rb / (double)(((n_rb + 5) / 6) * 6) * (15.0 / 16.0);
+    sc4 += w * n_rb / (double)(((n_rb + 7) / 8) * 8);
+  }
+  return sc3 > sc4 ? 3 : 4;
+}
 constexpr int kChunkTiles = 4;                           // K-tiles per bulk copy
 constexpr int kChunkBytes = kChunkTiles * kTileBytes;    // 2048
 
@@ -93,7 +111,7 @@ struct LayerDesc {
   uint16_t* y;        // [batch][d_out] fp16
   int d_in, d_out, s, npaths;
   int n_slices;       // ceil(d_in / kVSlice)
-  int n_rchunks;      // ceil(s16 / 16 / kVRowChunk)
+  int n_rchunks;      // ceil(s16 / 16 / (2 * latent-pass warps))
   int v_begin;        // first latent-pass work item of this layer
   int u_begin;        // first output-pass work item of this layer
   int p_begin;        // first (layer, path) index of this layer
@@ -119,6 +137,7 @@ struct DecodeArgs {
   int u_items;              // total output-pass items (layer, 128-row block)
   int p_items;              // total (layer, path) pairs
   int x_items;              // total quantise-pass items (layer, input slice)
+  int v_warps;              // latent-pass CTA width (3 or 4; latent_warps)
 };
 
 // Launchers (decode.cu), in stream order quantise -> latent -> finalize ->

@@ -100,6 +100,10 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   if (e != cudaSuccess) return cuda_fail(e);
 
   // ---- work items of each pass, per layer
+  const int vw = lb::latent_warps(n, batch, [&](int i, int& n_rb, double& w) {
+    n_rb = lb::s16(layers[i].s) / 16;
+    w = (double)(layers[i].residual + 1) * n_rb * layers[i].d_in;
+  });
   int x_items = 0, v_items = 0, p_items = 0, u_items = 0;
   int max_s16 = 16;
   size_t scratch = 0;
@@ -107,7 +111,7 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
     const lb_layer& L = layers[i];
     const int npaths = L.residual + 1, n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
     x_items += n_slices;
-    v_items += npaths * n_slices * lb::ceil_div(lb::s16(L.s) / 16, lb::kVRowChunk);
+    v_items += npaths * n_slices * lb::ceil_div(lb::s16(L.s) / 16, 2 * vw);
     p_items += npaths;
     u_items += L.d_out / lb::kUTileRows;
     scratch += (size_t)npaths * path_scratch_bytes(L, batch);
@@ -164,7 +168,7 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
     D.s = L.s;
     D.npaths = L.residual + 1;
     D.n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
-    D.n_rchunks = lb::ceil_div(lb::s16(L.s) / 16, lb::kVRowChunk);
+    D.n_rchunks = lb::ceil_div(lb::s16(L.s) / 16, 2 * vw);
     D.x_begin = xi;
     D.v_begin = vi;
     D.p_begin = pi;
@@ -215,6 +219,7 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   a.u_items = u_items;
   a.p_items = p_items;
   a.x_items = x_items;
+  a.v_warps = vw;
   const int sms = num_sms(dev);
   // events[i] (if given) is recorded right after launch i
   auto mark = [&](int i) { return i < n_events && events[i] ? cudaEventRecord(events[i], st) : cudaSuccess; };

@@ -98,7 +98,11 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
   D.s = L.s;
   D.npaths = npaths;
   D.n_slices = n_slices;
-  D.n_rchunks = lb::ceil_div(S16 / 16, lb::kVRowChunk);
+  const int vw = lb::latent_warps(1, batch, [&](int, int& n_rb, double& w) {
+    n_rb = S16 / 16;
+    w = 1.0;
+  });
+  D.n_rchunks = lb::ceil_div(S16 / 16, 2 * vw);
   D.v_begin = 0;
   D.u_begin = 0;
   D.p_begin = 0;
@@ -137,6 +141,7 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
   a.u_items = L.d_out / lb::kUTileRows;
   a.p_items = npaths;
   a.x_items = D.n_slices;
+  a.v_warps = vw;
   int sms = 0;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess || sms <= 0) return LB_ERR_CUDA;
