@@ -136,7 +136,7 @@ __device__ __forceinline__ int layer_of(const int* map, int n_layers, int item) 
 // quantise pass:  u = g_p (.) x on one 2048-input slice of one layer, for each
 // path p, quantised per batch row to 16 bits, v = step * (256*hi + lo), and
 // stored as the latent pass's int8 B fragments (slice block layout in
-// lb_internal.h).  One warp per (layer, slice): lane i holds the 8-input
+// lb_internal.h).  One warp per (layer, path, slice): lane i holds the 8-input
 // chunks i + 32j (j < 8) of one batch row; max and sum are warp reductions, so
 // the kernel has no CTA barrier.
 //
@@ -163,13 +163,12 @@ __global__ void __launch_bounds__(kQWarps * 32) quantise_input_kernel(const Deco
   if (item >= a.x_items) return;
   const int B = a.batch, NC = 2 * xq_rows(B);
   const LayerDesc& L = a.layers[layer_of(a.item_layer.x, a.n_layers, item)];
-  const int sl = item - L.x_begin;
+  const int p = (item - L.x_begin) / L.n_slices, sl = item - L.x_begin - p * L.n_slices;
   const int d_in = L.d_in, k0 = sl * kVSlice;
   const int nchunk = min(kVSlice, d_in - k0) / 8;
   const size_t blk_off = (size_t)sl * xq_slice_bytes(B);
 
-#pragma unroll 1
-  for (int p = 0; p < L.npaths; ++p) {
+  {
     const PathDesc& P = L.p[p];
     unsigned char* blk = P.ws.xq + blk_off;
     uint32_t* frag = reinterpret_cast<uint32_t*>(blk + xq_stats_bytes(B));
@@ -548,8 +547,9 @@ __global__ void __launch_bounds__(W * 32, NB == 1 ? 4 : 1) latent_pass_kernel(co
 
 // ---------------------------------------------------------------------------
 // finalize:  t'_j = l_j * sum over slices of the partials, quantised per batch
-// row to the int8 hi/lo planes and the step the output pass reads.  At batch 1
-// the planes of a layer's paths form one K range (packed output pass): path
+// row to the int8 hi/lo planes and the step the output pass reads.  In a
+// packed call (batch 1 with a residual layer) the planes of a layer's paths
+// form one K range (packed output pass): path
 // p's K-tiles come after path p-1's, with its t' in row p of each tile and
 // zeros in the other path's row.  One CTA
 // per (layer, path), in a launch between the two passes: warp w takes the
@@ -574,7 +574,7 @@ __global__ void __launch_bounds__(kFWarps * 32) finalize_kernel(const DecodeArgs
   const PathDesc& P = L.p[pi];
   const int s = L.s, S16 = (s + 15) & ~15, nkt = (s + 31) >> 5;
   const int ns = L.n_slices, ng = (ns + 3) >> 2;
-  const bool packed = B == 1;   // batch 1: the output pass takes both paths as one K range
+  const bool packed = a.packed != 0;   // the output pass takes both paths as one K range
 #pragma unroll 1
   for (int b = 0; b < B; ++b) {
     if (tid == 0) {
@@ -864,8 +864,9 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
 }
 
 // ---------------------------------------------------------------------------
-// output pass, batch 1 ("packed"): the product's 8 columns hold 4 batch rows,
-// of which batch 1 uses one, so the paths take the spare ones instead.  Both
+// output pass, batch 1 with residual layers ("packed"): the product's 8
+// columns hold 4 batch rows, of which batch 1 uses one, so the paths take the
+// spare ones instead.  Both
 // paths' K-tiles form one K range (path 1's after path 0's); the t' operand
 // of path p's tiles sits in column pair p with zeros in the other path's pair,
 // so one accumulator holds both paths' sums, in different columns.  Lanes with
@@ -1149,7 +1150,7 @@ cudaError_t launch_output_packed(const DecodeArgs& a, int num_sms, cudaStream_t 
 }
 
 cudaError_t launch_output_pass(const DecodeArgs& a, int num_sms, cudaStream_t st) {
-  if (a.batch == 1) return launch_output_packed(a, num_sms, st);
+  if (a.packed) return launch_output_packed(a, num_sms, st);
   switch ((a.batch + 3) / 4) {
     case 1: return launch_output<1>(a, num_sms, st);
     case 2: return launch_output<2>(a, num_sms, st);

@@ -115,7 +115,7 @@ struct LayerDesc {
   int v_begin;        // first latent-pass work item of this layer
   int u_begin;        // first output-pass work item of this layer
   int p_begin;        // first (layer, path) index of this layer
-  int x_begin;        // first quantise-pass item (layer, input slice) of this layer
+  int x_begin;        // first quantise-pass item (layer, path, input slice) of this layer
 };
 
 // Layer index of every work item of each pass (device arrays built with the
@@ -136,8 +136,9 @@ struct DecodeArgs {
   int v_items;              // total latent-pass items
   int u_items;              // total output-pass items (layer, 128-row block)
   int p_items;              // total (layer, path) pairs
-  int x_items;              // total quantise-pass items (layer, input slice)
+  int x_items;              // total quantise-pass items (layer, path, input slice)
   int v_warps;              // latent-pass CTA width (3 or 4; latent_warps)
+  int packed;               // batch 1 with a residual layer: paths share the output pass's product
 };
 
 // Launchers (decode.cu), in stream order quantise -> latent -> finalize ->

@@ -110,7 +110,7 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   for (int i = 0; i < n; ++i) {
     const lb_layer& L = layers[i];
     const int npaths = L.residual + 1, n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
-    x_items += n_slices;
+    x_items += npaths * n_slices;
     v_items += npaths * n_slices * lb::ceil_div(lb::s16(L.s) / 16, 2 * vw);
     p_items += npaths;
     u_items += L.d_out / lb::kUTileRows;
@@ -173,7 +173,7 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
     D.v_begin = vi;
     D.p_begin = pi;
     D.u_begin = ui;
-    for (int k = 0; k < D.n_slices; ++k) xm[xi++] = i;
+    for (int k = 0; k < D.npaths * D.n_slices; ++k) xm[xi++] = i;
     for (int k = 0; k < D.npaths * D.n_slices * D.n_rchunks; ++k) vm[vi++] = i;
     for (int k = 0; k < D.npaths; ++k) pm[pi++] = i;
     for (int k = 0; k < L.d_out / lb::kUTileRows; ++k) um[ui++] = i;
@@ -220,6 +220,9 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   a.p_items = p_items;
   a.x_items = x_items;
   a.v_warps = vw;
+  a.packed = 0;
+  if (batch == 1)
+    for (int i = 0; i < n; ++i) a.packed |= layers[i].residual;
   const int sms = num_sms(dev);
   // events[i] (if given) is recorded right after launch i
   auto mark = [&](int i) { return i < n_events && events[i] ? cudaEventRecord(events[i], st) : cudaSuccess; };

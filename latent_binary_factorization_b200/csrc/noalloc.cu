@@ -140,8 +140,9 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
   a.v_items = npaths * D.n_slices * D.n_rchunks;
   a.u_items = L.d_out / lb::kUTileRows;
   a.p_items = npaths;
-  a.x_items = D.n_slices;
+  a.x_items = npaths * D.n_slices;
   a.v_warps = vw;
+  a.packed = batch == 1 && L.residual ? 1 : 0;
   int sms = 0;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess || sms <= 0) return LB_ERR_CUDA;
