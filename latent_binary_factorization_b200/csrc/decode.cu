@@ -96,6 +96,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return false;
 }
 
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream serialization attribute may start before the previous kernel in the
+// stream has finished; grid_dep_wait() returns once that kernel has completed
+// and its writes are visible.  grid_dep_launch() lets the next such kernel
+// start launching.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint4 ld_nc(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -158,6 +166,7 @@ __device__ __forceinline__ uint32_t pack_byte(uint32_t a, uint32_t c, uint32_t d
 }
 
 __global__ void __launch_bounds__(kQWarps * 32) quantise_input_kernel(const DecodeArgs a) {
+  grid_dep_launch();
   const int lane = threadIdx.x & 31;
   const int item = blockIdx.x * kQWarps + (threadIdx.x >> 5);
   if (item >= a.x_items) return;
@@ -384,16 +393,8 @@ __global__ void __launch_bounds__(W * 32, NB == 1 ? 4 : 1) latent_pass_kernel(co
   if (lane == 0) fence_mbar_init();
   __syncthreads();   // the only CTA barrier: barriers and counters initialised
 
+  grid_dep_launch();
   const int li0 = layer_of(a.item_layer.v, a.n_layers, i_begin);
-  if (tid == 0) {
-    // slices 0 and 1 of this CTA's sequence
-    int lj = li0;
-    const VItem it = decode_v(a, i_begin, lj);
-    x_issue<NB, RB>(a, i_begin, li0, xbuf, &xfull[0]);
-    const int nxt = i_begin - it.rc + a.layers[it.li].n_rchunks;
-    if (nxt < i_end) x_issue<NB, RB>(a, nxt, it.li, xbuf + kXBuf, &xfull[1]);
-  }
-
   VFeed<NB, W> feed;
   feed.item = i_begin;
   feed.li = li0;
@@ -405,6 +406,17 @@ __global__ void __launch_bounds__(W * 32, NB == 1 ? 4 : 1) latent_pass_kernel(co
       if (lane == 0) feed.issue(my_ring + st * kStageBytes, &my_bar[st]);
       feed.advance(a, warp, i_end);
     }
+  }
+  // the sign tiles above are weights; the quantised slices are the quantise
+  // pass's output
+  grid_dep_wait();
+  if (tid == 0) {
+    // slices 0 and 1 of this CTA's sequence
+    int lj = li0;
+    const VItem it = decode_v(a, i_begin, lj);
+    x_issue<NB, RB>(a, i_begin, li0, xbuf, &xfull[0]);
+    const int nxt = i_begin - it.rc + a.layers[it.li].n_rchunks;
+    if (nxt < i_end) x_issue<NB, RB>(a, nxt, it.li, xbuf + kXBuf, &xfull[1]);
   }
   uint32_t consumed = 0;
   int slot = 0;
@@ -566,6 +578,8 @@ __global__ void __launch_bounds__(kFWarps * 32) finalize_kernel(const DecodeArgs
   __shared__ float s_t[kMaxRank];   // t' of this path, one batch row at a time
   __shared__ unsigned s_mx;         // max |t'| (non-negative float bits order as unsigned)
   __shared__ int s_sum;
+  grid_dep_launch();
+  grid_dep_wait();   // the latent pass's partials
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int item = blockIdx.x;
   const int B = a.batch;
@@ -769,6 +783,7 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
     fence_mbar_init();
   }
   __syncwarp();
+  grid_dep_wait();   // finalize's t' planes and steps
 
   OutCursor fd;
   fd.enter(a, layer_of(a.item_layer.u, a.n_layers, i_begin));
@@ -957,6 +972,7 @@ __global__ void __launch_bounds__(kUWarps * 32) output_packed_kernel(const Decod
     fence_mbar_init();
   }
   __syncwarp();
+  grid_dep_wait();   // finalize's t' planes and steps
 
   PkCursor fd;
   fd.enter(a, layer_of(a.item_layer.u, a.n_layers, i_begin));
@@ -1033,6 +1049,24 @@ __global__ void __launch_bounds__(kUWarps * 32) output_packed_kernel(const Decod
 
 // ------------------------------------------------------------------ launchers
 
+// Launch `kern` on `st` with programmatic stream serialization: it may start
+// while the previous kernel of the stream finishes, and waits for it with
+// grid_dep_wait() before reading its output.
+template <class K>
+cudaError_t launch_dependent(K kern, int grid, int block, size_t smem, cudaStream_t st, const DecodeArgs& a) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
 template <int NB, int RB, int W>
 constexpr size_t latent_smem() {
   return (size_t)W * kVStages * VCfg<NB>::kRPW * kChunkBytes + 2 * (size_t)xq_buf_bytes(NB, RB) +
@@ -1042,8 +1076,7 @@ constexpr size_t latent_smem() {
 
 template <int NB>
 cudaError_t launch_finalize(const DecodeArgs& a, int, cudaStream_t st) {
-  finalize_kernel<NB><<<a.p_items, kFWarps * 32, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_dependent(finalize_kernel<NB>, a.p_items, kFWarps * 32, 0, st, a);
 }
 
 template <int NB>
@@ -1071,8 +1104,7 @@ cudaError_t launch_latent(const DecodeArgs& a, int num_sms, cudaStream_t st) {
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
   }
   const int grid = max(1, min(a.v_items, per_sm * num_sms));
-  kern<<<grid, W * 32, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_dependent(kern, grid, W * 32, smem, st, a);
 }
 
 template <int NB>
@@ -1091,8 +1123,7 @@ cudaError_t launch_output(const DecodeArgs& a, int num_sms, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
   const int grid = max(1, min((a.u_items + kUWarps - 1) / kUWarps, per_sm * num_sms));
-  output_pass_kernel<NB><<<grid, kUWarps * 32, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_dependent(output_pass_kernel<NB>, grid, kUWarps * 32, smem, st, a);
 }
 
 }  // namespace
@@ -1145,8 +1176,7 @@ cudaError_t launch_output_packed(const DecodeArgs& a, int num_sms, cudaStream_t 
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
   }
   const int grid = max(1, min((a.u_items + kUWarps - 1) / kUWarps, per_sm * num_sms));
-  output_packed_kernel<<<grid, kUWarps * 32, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_dependent(output_packed_kernel, grid, kUWarps * 32, smem, st, a);
 }
 
 cudaError_t launch_output_pass(const DecodeArgs& a, int num_sms, cudaStream_t st) {
