@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <vector>
+
 #include "littlebit.h"
 
 namespace lb {
@@ -153,12 +155,24 @@ int prefill_sp(int s, int npaths);
 size_t prefill_layer_bytes(int M, int d_in, int d_out, int s, int npaths);
 long long prefill_layer_tiles(int M, int d_out, int s, int npaths);   // GEMM1 + GEMM2 tiles
 size_t prefill_table_bytes(int n_layers, long long tiles);
-constexpr int kPrefillMaxGroup = 4096;   // layers per group
-// A group's operand preparation, then its two grouped GEMM launches (same ws).
+constexpr int kPrefillMaxGroup = 4096;   // layers per chunk
+// A chunk of layers: its table's place in the call's table image and the two
+// GEMMs' tile counts and grids.
+struct PrefillPlan {
+  int n;
+  int tiles1, tiles2, grid1, grid2;
+  size_t table_off, table_bytes;
+};
+// Append the chunk's table image (problems and tile schedules) to img; its
+// device pointers refer to the chunk's operand buffers at `bufs`.
+void plan_prefill_chunk(const LayerDesc* Ls, void* const* ys, int n, int M, int x_bf16, unsigned char* bufs,
+                        int num_sms, std::vector<unsigned char>& img, PrefillPlan& plan);
+// A chunk's operand preparation (buffers at `bufs`), then its two grouped
+// GEMM launches (table image uploaded at table_dev).
 cudaError_t launch_prefill_prep(const LayerDesc* Ls, const void* const* xs, int n, int M, int x_bf16,
-                                unsigned char* ws, cudaStream_t st);
-cudaError_t launch_prefill_gemms(const LayerDesc* Ls, void* const* ys, int n, int M, int x_bf16,
-                                 unsigned char* ws, unsigned int* status, int num_sms, cudaStream_t st);
+                                unsigned char* bufs, cudaStream_t st);
+cudaError_t launch_prefill_gemms(const PrefillPlan& plan, const unsigned char* table_dev, unsigned int* status,
+                                 cudaStream_t st);
 
 // pack.cu
 cudaError_t launch_pack(const void* src, lb_dtype dt, int n_long, int s, int64_t stride_long,

@@ -266,16 +266,19 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
-  // plan the chunks
+  // plan the chunks: operand bytes per chunk (a workspace half) and table bytes
   std::vector<int> starts;
-  size_t half = 0, cur = 0;
+  size_t half = 0, cur = 0, tables = 0;
   long long tiles = 0;
   int cnt = 0;
   for (int i = 0; i < n; ++i) {
     const lb_layer& L = layers[i];
     const size_t b = lb::prefill_layer_bytes(batch, L.d_in, L.d_out, L.s, L.residual + 1);
     if (cnt == 0 || cur + b > kPrefillChunkBytes || cnt == lb::kPrefillMaxGroup) {
-      if (cnt) half = std::max(half, cur + lb::prefill_table_bytes(cnt, tiles));
+      if (cnt) {
+        half = std::max(half, cur);
+        tables += align_up(lb::prefill_table_bytes(cnt, tiles), 1024);
+      }
       starts.push_back(i);
       cur = 0;
       cnt = 0;
@@ -285,10 +288,12 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
     tiles += lb::prefill_layer_tiles(batch, L.d_out, L.s, L.residual + 1);
     ++cnt;
   }
-  half = align_up(std::max(half, cur + lb::prefill_table_bytes(cnt, tiles)), 1024);
+  half = align_up(std::max(half, cur), 1024);
+  tables = align_up(tables + align_up(lb::prefill_table_bytes(cnt, tiles), 1024), 1024);
   starts.push_back(n);
   const int n_chunks = (int)starts.size() - 1;
-  const size_t need = kStatusBytes + (n_chunks > 1 ? 2 : 1) * half;
+  // workspace: [status][tables of all chunks][half 0][half 1]
+  const size_t need = kStatusBytes + tables + (n_chunks > 1 ? 2 : 1) * half;
 
   std::lock_guard<std::mutex> lock(g_mu);
   Workspace& ws = g_ws[{dev, st}];
@@ -304,12 +309,14 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
     e = cudaMalloc(&ws.buf, cap);
     if (e != cudaSuccess) return cuda_fail(e);
     ws.cap = cap;
+    ws.table.clear();
     e = cudaMemsetAsync(ws.buf, 0, cap, st);
     if (e != cudaSuccess) return cuda_fail(e);
   }
-  ws.table.clear();   // the decode table region is overwritten below
   unsigned char* base = static_cast<unsigned char*>(ws.buf);
   unsigned int* status = reinterpret_cast<unsigned int*>(base);
+  unsigned char* table_dev = base + kStatusBytes;
+  auto chunk_bufs = [&](int c) { return base + kStatusBytes + tables + (size_t)(c & 1) * half; };
   std::vector<lb::LayerDesc> descs(n);
   for (int i = 0; i < n; ++i) {
     const lb_layer& L = layers[i];
@@ -327,12 +334,26 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
       D.p[p].l = L.path[p].l;
     }
   }
+  // the tables of every chunk, uploaded only when they change (as the decode
+  // table), so that a repeated call enqueues kernels and events only and can
+  // be captured into a CUDA graph
   const int sms = num_sms(dev);
-  auto chunk_ws = [&](int c) { return base + kStatusBytes + (size_t)(c & 1) * half; };
-  if (n_chunks == 1) {
-    e = lb::launch_prefill_prep(descs.data(), xs, n, batch, x_bf16, chunk_ws(0), st);
+  std::vector<unsigned char> img;
+  std::vector<lb::PrefillPlan> plans(n_chunks);
+  for (int c = 0; c < n_chunks; ++c)
+    lb::plan_prefill_chunk(descs.data() + starts[c], ys + starts[c], starts[c + 1] - starts[c], batch, x_bf16,
+                           chunk_bufs(c), sms, img, plans[c]);
+  if (img.size() > tables) return LB_ERR_SHAPE;   // the plan above sized the tables
+  if (ws.table.size() != img.size() || std::memcmp(ws.table.data(), img.data(), img.size()) != 0) {
+    // pageable source: the copy is staged before the call returns
+    e = cudaMemcpyAsync(table_dev, img.data(), img.size(), cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return cuda_fail(e);
-    e = lb::launch_prefill_gemms(descs.data(), ys, n, batch, x_bf16, chunk_ws(0), status, sms, st);
+    ws.table.swap(img);
+  }
+  if (n_chunks == 1) {
+    e = lb::launch_prefill_prep(descs.data(), xs, n, batch, x_bf16, chunk_bufs(0), st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = lb::launch_prefill_gemms(plans[0], table_dev, status, st);
     return e == cudaSuccess ? LB_OK : cuda_fail(e);
   }
   e = ensure_side(ws);
@@ -345,11 +366,10 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
     const int i0 = starts[c], cn = starts[c + 1] - starts[c], h = c & 1;
     // the half was last used by chunk c - 2's GEMMs
     if (c >= 2) e = cudaStreamWaitEvent(ws.side, ws.gemm_done[h], 0);
-    if (e == cudaSuccess) e = lb::launch_prefill_prep(descs.data() + i0, xs + i0, cn, batch, x_bf16, chunk_ws(c), ws.side);
+    if (e == cudaSuccess) e = lb::launch_prefill_prep(descs.data() + i0, xs + i0, cn, batch, x_bf16, chunk_bufs(c), ws.side);
     if (e == cudaSuccess) e = cudaEventRecord(ws.prep_done[h], ws.side);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ws.prep_done[h], 0);
-    if (e == cudaSuccess)
-      e = lb::launch_prefill_gemms(descs.data() + i0, ys + i0, cn, batch, x_bf16, chunk_ws(c), status, sms, st);
+    if (e == cudaSuccess) e = lb::launch_prefill_gemms(plans[c], table_dev, status, st);
     if (e == cudaSuccess) e = cudaEventRecord(ws.gemm_done[h], st);
   }
   // join, also after an error, so that no side-stream work outlives the call's stream order

@@ -530,9 +530,8 @@ static long long group_tiles(const LayerDesc* Ls, int n, int M) {
   return t;
 }
 
-// Buffers of one group of layers inside `ws`: first the table (2n problems,
-// then the two GEMMs' CTA list offsets and tile lists; prefill_table_bytes),
-// then each layer's X16 | B1 | B2 | T (prefill_layer_bytes).
+// Buffers of one chunk of layers: each layer's X16 | B1 | B2 | T
+// (prefill_layer_bytes), from `bufs` on.
 struct LayerBufs {
   unsigned char *X16, *B1, *B2, *T;
 };
@@ -549,10 +548,10 @@ static LayerBufs layer_bufs(unsigned char*& buf, const LayerDesc& L, int M) {
   return b;
 }
 
-// Operand preparation of a group of layers (three launches per layer).
+// Operand preparation of a chunk of layers (three launches per layer).
 cudaError_t launch_prefill_prep(const LayerDesc* Ls, const void* const* xs, int n, int M, int x_bf16,
-                                unsigned char* ws, cudaStream_t st) {
-  unsigned char* buf = ws + prefill_table_bytes(n, group_tiles(Ls, n, M));
+                                unsigned char* bufs, cudaStream_t st) {
+  unsigned char* buf = bufs;
   for (int i = 0; i < n; ++i) {
     const LayerDesc& L = Ls[i];
     const int P = L.npaths, Sp = prefill_sp(L.s, P);
@@ -599,30 +598,26 @@ static void lpt_schedule(const std::vector<double>& cost, int grid, int* sched, 
 // product, plus about one K-block of fixed per-tile work.
 static double tile_cost(int K, int n_len) { return (double)(K / kBK) * (double)max(n_len, 64) / kBN + 1.0; }
 
-// GEMM1 and GEMM2 of a group of layers whose operands launch_prefill_prep
-// prepared in the same `ws`: one grouped launch each.
-cudaError_t launch_prefill_gemms(const LayerDesc* Ls, void* const* ys, int n, int M, int x_bf16,
-                                 unsigned char* ws, unsigned int* status, int num_sms, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(umma_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)group_smem());
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
-  if (n > kPrefillMaxGroup) return cudaErrorInvalidValue;
+// Host image of a chunk's table, appended to `img` at a 1 KB boundary:
+// 2n problems | begin1 | begin2 | sched1 | sched2.  Device pointers in it refer
+// to the chunk's buffers at `bufs` and to the image's own place at
+// table_dev + plan.table_off.
+void plan_prefill_chunk(const LayerDesc* Ls, void* const* ys, int n, int M, int x_bf16, unsigned char* bufs,
+                        int num_sms, std::vector<unsigned char>& img, PrefillPlan& plan) {
   const long long tiles_all = group_tiles(Ls, n, M);
-  unsigned char* buf = ws + prefill_table_bytes(n, tiles_all);
-  // host image of the table: 2n problems | begin1 | begin2 | sched1 | sched2
+  plan.n = n;
+  plan.table_off = (img.size() + 1023) & ~(size_t)1023;
+  plan.table_bytes = prefill_table_bytes(n, tiles_all);
+  img.resize(plan.table_off + plan.table_bytes, 0);
+  unsigned char* base = img.data() + plan.table_off;
   const size_t prob_b = (size_t)2 * n * sizeof(GemmProblem);
-  static thread_local std::vector<unsigned char> host;
-  host.assign(prob_b + (size_t)2 * (kMaxGemmGrid + 1) * sizeof(int) + (size_t)tiles_all * sizeof(int), 0);
-  GemmProblem* probs = reinterpret_cast<GemmProblem*>(host.data());
-  int* begin1 = reinterpret_cast<int*>(host.data() + prob_b);
+  GemmProblem* probs = reinterpret_cast<GemmProblem*>(base);
+  int* begin1 = reinterpret_cast<int*>(base + prob_b);
   int* begin2 = begin1 + kMaxGemmGrid + 1;
   int* sched1 = begin2 + kMaxGemmGrid + 1;
   std::vector<double> cost1, cost2;
   int tiles1 = 0, tiles2 = 0;
+  unsigned char* buf = bufs;
   for (int i = 0; i < n; ++i) {
     const LayerDesc& L = Ls[i];
     const int P = L.npaths, Sp = prefill_sp(L.s, P), NK = P * Sp;
@@ -644,20 +639,35 @@ cudaError_t launch_prefill_gemms(const LayerDesc* Ls, void* const* ys, int n, in
       for (int nt = 0; nt < g2.tiles_n; ++nt) cost2.push_back(tile_cost(g2.K, min(kBN, L.d_out - nt * kBN)));
   }
   int* sched2 = sched1 + tiles1;
-  const int grid1 = min(min(tiles1, num_sms), kMaxGemmGrid), grid2 = min(min(tiles2, num_sms), kMaxGemmGrid);
-  lpt_schedule(cost1, grid1, sched1, begin1);
-  lpt_schedule(cost2, grid2, sched2, begin2);
-  // pageable source: the copy is staged before the call returns, so `host`
-  // may be refilled by the next group
-  cudaError_t e = cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, st);
-  if (e != cudaSuccess) return e;
-  const GemmProblem* table_dev = reinterpret_cast<const GemmProblem*>(ws);
-  const int* begin_dev = reinterpret_cast<const int*>(ws + prob_b);
+  plan.tiles1 = tiles1;
+  plan.tiles2 = tiles2;
+  plan.grid1 = min(min(tiles1, num_sms), kMaxGemmGrid);
+  plan.grid2 = min(min(tiles2, num_sms), kMaxGemmGrid);
+  lpt_schedule(cost1, plan.grid1, sched1, begin1);
+  lpt_schedule(cost2, plan.grid2, sched2, begin2);
+}
+
+// GEMM1 and GEMM2 of a planned chunk (table uploaded at table_dev +
+// plan.table_off, operands prepared by launch_prefill_prep): one grouped
+// launch each.
+cudaError_t launch_prefill_gemms(const PrefillPlan& plan, const unsigned char* table_dev, unsigned int* status,
+                                 cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(umma_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)group_smem());
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const unsigned char* base = table_dev + plan.table_off;
+  const size_t prob_b = (size_t)2 * plan.n * sizeof(GemmProblem);
+  const GemmProblem* probs = reinterpret_cast<const GemmProblem*>(base);
+  const int* begin_dev = reinterpret_cast<const int*>(base + prob_b);
   const int* sched_dev = begin_dev + 2 * (kMaxGemmGrid + 1);
-  GroupArgs g1a{table_dev, sched_dev, begin_dev, n, tiles1, status};
-  umma_group_kernel<<<grid1, kGroupThreads, group_smem(), st>>>(g1a);
-  GroupArgs g2a{table_dev + n, sched_dev + tiles1, begin_dev + kMaxGemmGrid + 1, n, tiles2, status};
-  umma_group_kernel<<<grid2, kGroupThreads, group_smem(), st>>>(g2a);
+  GroupArgs g1a{probs, sched_dev, begin_dev, plan.n, plan.tiles1, status};
+  umma_group_kernel<<<plan.grid1, kGroupThreads, group_smem(), st>>>(g1a);
+  GroupArgs g2a{probs + plan.n, sched_dev + plan.tiles1, begin_dev + kMaxGemmGrid + 1, plan.n, plan.tiles2, status};
+  umma_group_kernel<<<plan.grid2, kGroupThreads, group_smem(), st>>>(g2a);
   return cudaGetLastError();
 }
 

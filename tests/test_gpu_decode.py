@@ -141,12 +141,15 @@ def test_basis_vector_input_gives_weight_column(lbm):
     _check(y, W[:, cols].T, "basis")
 
 
-def test_forward_many_mixed_stack(lbm):
-    """One forward_many call over layers of different shapes, ranks and path counts."""
+@pytest.mark.parametrize("B", [1, 2])
+def test_forward_many_mixed_stack(lbm, B):
+    """One forward_many call over layers of different shapes, ranks and path
+    counts.  At batch 1 with residual layers the output pass takes both paths
+    as one K range (single-path layers, and chunks that span the two paths'
+    K-tiles, included)."""
     lb, layers = lbm
     specs = [(4096, 4096, 86, True), (4096, 11008, 133, True), (11008, 4096, 133, True),
              (512, 512, 32, False), (8192, 1024, 620, False)]
-    B = 2
     L, X, Y, refs = [], [], [], []
     for i, (a, b, s, r) in enumerate(specs):
         paths = synth.layer(a, b, s, r, seed=100 + i, index=i)
@@ -198,3 +201,36 @@ def test_full_size_70b_mlp_sampled_rows(lbm):
     rows = np.sort(np.random.default_rng(0).choice(28672, 512, replace=False))
     y_ref = orc.factored_forward(x.cpu().numpy(), host, rows=rows)
     _check(y[:, rows], y_ref, "70B sampled")
+
+
+@pytest.mark.parametrize("B", [1, 3])
+def test_forward_many_in_cuda_graph(lbm, B):
+    """The decode stack captured into a CUDA graph (on the stream of an earlier
+    eager call, whose workspace and tables it reuses) and replayed gives
+    exactly what the eager call gave, twice in a row."""
+    lb, layers = lbm
+    specs = [(4096, 4096, 86, True), (8192, 2048, 620, False), (1024, 4096, 45, True)]
+    L, X, Y = [], [], []
+    for i, (a, b, s, r) in enumerate(specs):
+        paths = synth.layer(a, b, s, r, seed=300 + i, index=i)
+        L.append(layers.upload(paths, a, b, s))
+        X.append(torch.from_numpy(synth.activations(B, a, seed=300 + i, index=i)).cuda())
+        Y.append(torch.empty(B, b, dtype=torch.float16, device="cuda"))
+    stack = lb.Stack(L, X, Y)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        stack()
+    torch.cuda.synchronize()
+    ref = [y.clone() for y in Y]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        stack()
+    for _ in range(2):
+        for y in Y:
+            y.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        for i, (y, r) in enumerate(zip(Y, ref)):
+            assert torch.equal(y, r), f"layer {i}"
+    del g

@@ -125,3 +125,34 @@ def test_prefill_chunked_stack_matches_single_layer_calls(lbm):
             y.fill_(float("nan"))
         st()
     assert lb.device_status() == 0
+
+
+def test_prefill_stack_in_cuda_graph(lbm):
+    """A two-chunk prefill stack (side-stream preparation forked from and
+    joined to the caller's stream) captured into a CUDA graph on the stream of
+    an earlier eager call and replayed gives exactly the eager result."""
+    lb, layers = lbm
+    gen = torch.Generator(device="cuda").manual_seed(12)
+    M, n = 2048, 20   # ~29 MB of operands per layer: two chunks
+    L, X, Y = [], [], []
+    for i in range(n):
+        L.append(layers.random_layer(4096, 4096, 290, True, gen)[0])
+        X.append(torch.randn(M, 4096, generator=gen, device="cuda").to(torch.bfloat16))
+        Y.append(torch.empty(M, 4096, dtype=torch.bfloat16, device="cuda"))
+    st = lb.Stack(L, X, Y)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        st()
+    torch.cuda.synchronize()
+    ref = [y.clone() for y in Y]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        st()
+    for y in Y:
+        y.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    for i, (y, r) in enumerate(zip(Y, ref)):
+        assert torch.equal(y, r), f"layer {i}"
+    del g
