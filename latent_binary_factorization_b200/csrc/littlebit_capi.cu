@@ -34,7 +34,33 @@ struct Workspace {
   // against the caller's stream (created on first use)
   cudaStream_t side = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr, prep_done[2] = {nullptr, nullptr}, gemm_done[2] = {nullptr, nullptr};
+  // the last call's arguments and what was derived from them: a call with the
+  // same arguments (a serving loop's every step) reuses them and enqueues
+  // kernels and events only
+  std::vector<unsigned char> key;
+  lb::DecodeArgs dargs{};
+  int d_max_s16 = 16;
+  std::vector<lb::LayerDesc> p_descs;
+  std::vector<lb::PrefillPlan> p_plans;
+  std::vector<int> p_starts;
+  size_t p_tables = 0, p_half = 0;
 };
+
+// Call arguments that determine a forward's tables and plans.
+std::vector<unsigned char> call_key(char mode, const lb_layer* layers, int n, const void* const* xs,
+                                    void* const* ys, int batch, int x_bf16) {
+  std::vector<unsigned char> k;
+  const size_t lb = (size_t)n * sizeof(lb_layer), pb = (size_t)n * sizeof(void*);
+  k.resize(16 + lb + 2 * pb);
+  k[0] = (unsigned char)mode;
+  std::memcpy(k.data() + 4, &batch, 4);
+  std::memcpy(k.data() + 8, &x_bf16, 4);
+  std::memcpy(k.data() + 12, &n, 4);
+  std::memcpy(k.data() + 16, layers, lb);
+  std::memcpy(k.data() + 16 + lb, xs, pb);
+  std::memcpy(k.data() + 16 + lb + pb, ys, pb);
+  return k;
+}
 
 void release_workspace(Workspace& w) {
   if (w.buf) cudaFree(w.buf);
@@ -42,7 +68,7 @@ void release_workspace(Workspace& w) {
   for (cudaEvent_t* ev : evs)
     if (*ev) cudaEventDestroy(*ev);
   if (w.side) cudaStreamDestroy(w.side);
-  w = Workspace{};
+  w = Workspace();
 }
 
 std::mutex g_mu;
@@ -93,11 +119,31 @@ size_t path_scratch_bytes(const lb_layer& L, int batch) {
 
 constexpr size_t kStatusBytes = 256;   // device status word at the start of a workspace
 
+// The four decode launches of a prepared call; events[i] (if given) is
+// recorded right after launch i.
+lb_status decode_launch(const lb::DecodeArgs& a, int max_s16, int sms, cudaStream_t st, const cudaEvent_t* events,
+                        int n_events) {
+  auto mark = [&](int i) { return i < n_events && events[i] ? cudaEventRecord(events[i], st) : cudaSuccess; };
+  cudaError_t e = lb::launch_quantise_pass(a, st);
+  if (e == cudaSuccess) e = mark(0);
+  if (e == cudaSuccess) e = lb::launch_latent_pass(a, max_s16, sms, st);
+  if (e == cudaSuccess) e = mark(1);
+  if (e == cudaSuccess) e = lb::launch_finalize_pass(a, max_s16, st);
+  if (e == cudaSuccess) e = mark(2);
+  if (e == cudaSuccess) e = lb::launch_output_pass(a, sms, st);
+  return e == cudaSuccess ? LB_OK : cuda_fail(e);
+}
+
 lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
                          cudaStream_t st, const cudaEvent_t* events, int n_events) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
+  std::lock_guard<std::mutex> lock(g_mu);
+  Workspace& ws = g_ws[{dev, st}];
+  std::vector<unsigned char> key = call_key('D', layers, n, xs, ys, batch, 0);
+  if (ws.buf && ws.key == key) return decode_launch(ws.dargs, ws.d_max_s16, num_sms(dev), st, events, n_events);
+  ws.key.clear();
 
   // ---- work items of each pass, per layer
   const int vw = lb::latent_warps(n, batch, [&](int i, int& n_rb, double& w) {
@@ -124,8 +170,6 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   const size_t map_bytes = align_up((size_t)n_items * sizeof(int), 256);
   const size_t total = kStatusBytes + table_bytes + map_bytes + scratch;
 
-  std::lock_guard<std::mutex> lock(g_mu);
-  Workspace& ws = g_ws[{dev, st}];
   if (ws.cap < total) {
     if (ws.buf) {
       e = cudaStreamSynchronize(st);
@@ -223,19 +267,10 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   a.packed = 0;
   if (batch == 1)
     for (int i = 0; i < n; ++i) a.packed |= layers[i].residual;
-  const int sms = num_sms(dev);
-  // events[i] (if given) is recorded right after launch i
-  auto mark = [&](int i) { return i < n_events && events[i] ? cudaEventRecord(events[i], st) : cudaSuccess; };
-  e = lb::launch_quantise_pass(a, st);
-  if (e == cudaSuccess) e = mark(0);
-  if (e == cudaSuccess) e = lb::launch_latent_pass(a, max_s16, sms, st);
-  if (e == cudaSuccess) e = mark(1);
-  if (e == cudaSuccess) e = lb::launch_finalize_pass(a, max_s16, st);
-  if (e == cudaSuccess) e = mark(2);
-  if (e != cudaSuccess) return cuda_fail(e);
-  e = lb::launch_output_pass(a, sms, st);
-  if (e != cudaSuccess) return cuda_fail(e);
-  return LB_OK;
+  ws.key.swap(key);
+  ws.dargs = a;
+  ws.d_max_s16 = max_s16;
+  return decode_launch(a, max_s16, num_sms(dev), st, events, n_events);
 }
 
 // Prefill (batch a multiple of 128): the tensor-core path.  Layers are taken
@@ -261,11 +296,18 @@ cudaError_t ensure_side(Workspace& ws) {
   return cudaSuccess;
 }
 
+lb_status prefill_launch(Workspace& ws, const void* const* xs, int batch, int x_bf16, cudaStream_t st);
+
 lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
                           int x_bf16, cudaStream_t st) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
+  std::lock_guard<std::mutex> lock(g_mu);
+  Workspace& ws = g_ws[{dev, st}];
+  std::vector<unsigned char> key = call_key('P', layers, n, xs, ys, batch, x_bf16);
+  if (ws.buf && ws.key == key) return prefill_launch(ws, xs, batch, x_bf16, st);
+  ws.key.clear();
   // plan the chunks: operand bytes per chunk (a workspace half) and table bytes
   std::vector<int> starts;
   size_t half = 0, cur = 0, tables = 0;
@@ -295,8 +337,6 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
   // workspace: [status][tables of all chunks][half 0][half 1]
   const size_t need = kStatusBytes + tables + (n_chunks > 1 ? 2 : 1) * half;
 
-  std::lock_guard<std::mutex> lock(g_mu);
-  Workspace& ws = g_ws[{dev, st}];
   if (ws.cap < need) {
     if (ws.buf) {
       e = cudaStreamSynchronize(st);   // the side stream always joins `st`
@@ -314,7 +354,6 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
     if (e != cudaSuccess) return cuda_fail(e);
   }
   unsigned char* base = static_cast<unsigned char*>(ws.buf);
-  unsigned int* status = reinterpret_cast<unsigned int*>(base);
   unsigned char* table_dev = base + kStatusBytes;
   auto chunk_bufs = [&](int c) { return base + kStatusBytes + tables + (size_t)(c & 1) * half; };
   std::vector<lb::LayerDesc> descs(n);
@@ -350,10 +389,29 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
     if (e != cudaSuccess) return cuda_fail(e);
     ws.table.swap(img);
   }
+  ws.p_descs.swap(descs);
+  ws.p_plans.swap(plans);
+  ws.p_starts.swap(starts);
+  ws.p_tables = tables;
+  ws.p_half = half;
+  ws.key.swap(key);
+  return prefill_launch(ws, xs, batch, x_bf16, st);
+}
+
+// The launches of a planned prefill call (plans, descriptors and tables in ws).
+lb_status prefill_launch(Workspace& ws, const void* const* xs, int batch, int x_bf16, cudaStream_t st) {
+  unsigned char* base = static_cast<unsigned char*>(ws.buf);
+  unsigned int* status = reinterpret_cast<unsigned int*>(base);
+  unsigned char* table_dev = base + kStatusBytes;
+  auto chunk_bufs = [&](int c) { return base + kStatusBytes + ws.p_tables + (size_t)(c & 1) * ws.p_half; };
+  const int n_chunks = (int)ws.p_plans.size();
+  const lb::LayerDesc* descs = ws.p_descs.data();
+  const std::vector<int>& starts = ws.p_starts;
+  cudaError_t e;
   if (n_chunks == 1) {
-    e = lb::launch_prefill_prep(descs.data(), xs, n, batch, x_bf16, chunk_bufs(0), st);
+    e = lb::launch_prefill_prep(descs, xs, starts[1], batch, x_bf16, chunk_bufs(0), st);
     if (e != cudaSuccess) return cuda_fail(e);
-    e = lb::launch_prefill_gemms(plans[0], table_dev, status, st);
+    e = lb::launch_prefill_gemms(ws.p_plans[0], table_dev, status, st);
     return e == cudaSuccess ? LB_OK : cuda_fail(e);
   }
   e = ensure_side(ws);
@@ -366,10 +424,10 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
     const int i0 = starts[c], cn = starts[c + 1] - starts[c], h = c & 1;
     // the half was last used by chunk c - 2's GEMMs
     if (c >= 2) e = cudaStreamWaitEvent(ws.side, ws.gemm_done[h], 0);
-    if (e == cudaSuccess) e = lb::launch_prefill_prep(descs.data() + i0, xs + i0, cn, batch, x_bf16, chunk_bufs(c), ws.side);
+    if (e == cudaSuccess) e = lb::launch_prefill_prep(descs + i0, xs + i0, cn, batch, x_bf16, chunk_bufs(c), ws.side);
     if (e == cudaSuccess) e = cudaEventRecord(ws.prep_done[h], ws.side);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ws.prep_done[h], 0);
-    if (e == cudaSuccess) e = lb::launch_prefill_gemms(plans[c], table_dev, status, st);
+    if (e == cudaSuccess) e = lb::launch_prefill_gemms(ws.p_plans[c], table_dev, status, st);
     if (e == cudaSuccess) e = cudaEventRecord(ws.gemm_done[h], st);
   }
   // join, also after an error, so that no side-stream work outlives the call's stream order
@@ -378,6 +436,7 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
   if (e == cudaSuccess) e = j;
   return e == cudaSuccess ? LB_OK : cuda_fail(e);
 }
+
 
 }  // namespace
 
