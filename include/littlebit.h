@@ -141,6 +141,14 @@ lb_status littlebit_linear_forward(const lb_layer* layer, const void* x_dev, voi
  * preparation per layer and two grouped GEMM launches per group of layers),
  * so that the weights of all layers stream from HBM back to back.  layers, xs,
  * ys are host arrays of length n.
+ *
+ * The library keeps one workspace per (device, stream) and remembers the last
+ * call's arguments on it (the layer structs and the x and y pointers): a call
+ * that repeats them enqueues kernels and events only -- no allocation, no
+ * host-to-device copy -- and may therefore be captured into a CUDA graph, on
+ * the same stream as an earlier eager call with the same arguments.  Kernels
+ * read the pointed-to data when they run, so new contents at the same
+ * addresses are picked up.
  */
 lb_status littlebit_linear_forward_many(const lb_layer* layers, int n, const void* const* xs,
                                         void* const* ys, int batch, lb_dtype xdt, void* stream);
