@@ -185,6 +185,25 @@ def stack_reps_for_l2(mats, batch, l2_bytes, factor=4.0):
     return max(1, math.ceil(factor * l2_bytes / per))
 
 
+def max_over_ranks(values, device):
+    """Each value's maximum over all ranks of the default process group (a
+    no-op with one process): device times of a multi-rank step are the
+    slowest rank's."""
+    import torch
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_us_per_layer(ms_per_step, layers_per_rank, world):
+    """Whole-job figure: every rank runs its own stack of `layers_per_rank`
+    layers per step (weak scaling), so one step processes layers_per_rank *
+    world layers in the slowest rank's step time."""
+    return 1e3 * ms_per_step / (layers_per_rank * world)
+
+
 def time_device(stack, steps, warmup, dist):
     """K device-timed steps (CUDA events on the launching stream, nothing else
     recorded in between), then K more steps for each decode kernel's share,
@@ -255,11 +274,8 @@ def measure_workload(name, batch, steps, warmup, device, dist, world, l2, seed=1
     stack, Ls, x_all, y_all = build_stack(mats, reps, batch, seed, device)
     n_layers = len(Ls)
     total_ms, per_ms = time_device(stack, steps, warmup, dist)
-    if dist:
-        import torch
-        t = torch.tensor([total_ms] + [per_ms[k] for k in KERNELS], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms, per_ms = t[0].item(), dict(zip(KERNELS, t[1:].tolist()))
+    red = max_over_ranks([total_ms] + [per_ms[k] for k in KERNELS], device)
+    total_ms, per_ms = red[0], dict(zip(KERNELS, red[1:]))
     alg = sum(algorithmic_bytes(*m, batch) for m in mats) * reps
     kb = {k: sum(kernel_bytes(*m, batch)[k] for m in mats) * reps for k in KERNELS}
     ms_step = total_ms / steps
@@ -302,11 +318,7 @@ def measure_prefill(n_layers, M, steps, warmup, device, dist, seed=4321):
         stack()
     t1.record()
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / steps
-    if dist:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = t.item()
+    ms = max_over_ranks([t0.elapsed_time(t1) / steps], device)[0]
     flops = sum(2 * M * s * (a + b) * (2 if r else 1) for a, b, s, r in PREFILL_MATS) * n_layers
     del stack, Ls, X, Y
     torch.cuda.empty_cache()
@@ -335,10 +347,7 @@ def run_ours(args):
     main, (stack, x_all, y_all) = measure_workload(args.workload, args.batch, args.steps, args.warmup, device,
                                                    dist, world, l2, l2_factor=args.l2_factor)
     e2e_ms, h2d, d2h = time_e2e(stack, x_all, y_all, max(3, args.steps // 4), 2)
-    if dist:
-        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = t.item()
+    e2e_ms = max_over_ranks([e2e_ms], device)[0]
     del stack, x_all, y_all
     extras = {}
     if not args.no_extras:
@@ -376,7 +385,7 @@ def run_ours(args):
     dom_ms = main["kernels"][dom]["ms"]
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     traffic = traffic_record(dom, args.workload, main["model_layers_per_step"])
-    value = 1e3 * main["ms_per_step"] / (n_layers * world)   # us per layer over all ranks' layers
+    value = job_us_per_layer(main["ms_per_step"], n_layers, world)   # us per layer over all ranks' layers
     line = {
         "metric": METRIC,
         "value": round(value, 5),
@@ -404,7 +413,7 @@ def run_ours(args):
                           "kernels": {k: {"ms_per_step": round(main["kernels"][k]["ms"], 5),
                                           "gbs": round(main["kernels"][k]["gbs"], 1)
                                           if main["kernels"][k]["gbs"] else None} for k in KERNELS}},
-        "e2e": {"value": round(1e3 * e2e_ms / max(3, args.steps // 4) / (n_layers * world), 5), "unit": "us/layer",
+        "e2e": {"value": round(job_us_per_layer(e2e_ms / max(3, args.steps // 4), n_layers, world), 5), "unit": "us/layer",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": 4 * args.steps,   # quantise, latent, finalize, output per step
         "clocks": clocks,
