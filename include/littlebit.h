@@ -86,7 +86,9 @@ size_t littlebit_packed_bytes(lb_role role, int rows, int cols);
 double littlebit_eff_bits(int d_in, int d_out, int s, int residual);
 
 /*
- * Pack the signs of a real (or +-1) factor into the layout above.
+ * Pack the signs of a real (or +-1) factor into the layout above: the
+ * binarisation U = sign(U_real), V = sign(V_real) of the LittleBit-2 column
+ * (chapter 2, the Dual-SVID initialisation step), stored one bit per sign.
  *   src_dev : factor in its natural orientation, n_long x s elements of type
  *             dt (LB_F16, LB_BF16, LB_F32 or LB_I8); element (a, j) is read at
  *             src_dev[a * stride_long + j * stride_s] (strides in elements).
@@ -192,6 +194,7 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
                                            int batch, lb_dtype xdt, void* stream);
 
 /*
+ * (Host helpers below: no counterpart in the pages.)
  * Waits for `stream`, then returns in *status the device-side error bits that
  * the forward kernels enqueued on it have raised since the last call, and
  * clears them.  Bit (1 << LB_ERR_TIMEOUT) means a bounded wait for a bulk copy
@@ -200,7 +203,8 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
  */
 lb_status littlebit_device_status(void* stream, unsigned int* status);
 
-/* Free every workspace of every device (call with no work in flight). */
+/* Free every workspace of every device, with its side stream and events (call
+ * with no work in flight on any stream the library was given). */
 void littlebit_release(void);
 
 /* Human-readable name of a status code (static string). */
