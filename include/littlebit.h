@@ -87,8 +87,9 @@ double littlebit_eff_bits(int d_in, int d_out, int s, int residual);
 
 /*
  * Pack the signs of a real (or +-1) factor into the layout above: the
- * binarisation U = sign(U_real), V = sign(V_real) of the LittleBit-2 column
- * (chapter 2, the Dual-SVID initialisation step), stored one bit per sign.
+ * binarisation of the factors to +-1 (Samsung LittleBit article, section 2,
+ * the "latent factorisation" and "Dual-SVID initialisation" bullets;
+ * LittleBit-2 column, chapter 2: sign(U), sign(V)), stored one bit per sign.
  *   src_dev : factor in its natural orientation, n_long x s elements of type
  *             dt (LB_F16, LB_BF16, LB_F32 or LB_I8); element (a, j) is read at
  *             src_dev[a * stride_long + j * stride_s] (strides in elements).
