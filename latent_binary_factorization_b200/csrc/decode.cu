@@ -25,20 +25,22 @@
 // registers.  Every wait is bounded: after kSpinLimit polls the kernel sets
 // LB_ERR_TIMEOUT in the status word and stops waiting.
 //
-// Four launches, in stream order:
-// quantise: CTA per (layer, path, 2048-input slice) quantises u = g*x per batch
-//   row and stores it as int8 B fragments with the step and sum per row.
-// latent:   CTA item = (layer, path, slice, 8 latent 16-row blocks); the
-//   slice's B fragments arrive by one bulk copy into a double buffer, warp w
-//   streams row blocks 2w, 2w+1 over the slice and writes one fp32 partial sum
-//   per latent row and slice.
+// Four launches, in stream order, chained by programmatic dependent launch
+// (each later kernel starts early and waits for its predecessor's output):
+// quantise: warp per (layer, path, 2048-input slice) quantises u = g*x per
+//   batch row and stores it as int8 B fragments with the step and sum per row.
+// latent:   CTA item = (layer, path, slice, 2W latent 16-row blocks) for a
+//   CTA of W = 3 or 4 warps; the slice's B fragments arrive by one bulk copy
+//   into a double buffer, warp w streams row blocks 2w, 2w+1 over the slice
+//   and writes one fp32 partial sum per latent row and slice.
 // finalize: CTA per (layer, path) sums the partials in slice order, multiplies
 //   by l and quantises t' to int8 hi/lo planes with a step per batch row.
 // output:   warp item = (layer, 128 output rows); each warp owns a contiguous
 //   item range and streams it as chunks of up to 8 K-tiles, across path, item
 //   and layer boundaries; the bulk copies also bring the chunk's t' bytes and,
 //   for the last chunk of a path, the 128 h values and the quantisation step.
-//   Paths are added in fp32 and y is written in fp16.
+//   Paths are added in fp32 and y is written in fp16.  At batch 1 with
+//   residual layers the two paths share one accumulator (packed form).
 #include <cuda_fp16.h>
 
 #include "lb_internal.h"

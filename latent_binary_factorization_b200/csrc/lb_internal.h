@@ -21,7 +21,10 @@ constexpr int kTileBytes = 512;
 // of W warps (latent_warps: 3 or 4) covers kVSlice inputs (kVSliceTiles
 // K-tiles) for 2*W 16-row latent blocks; warp w owns row blocks 2w and 2w+1 of
 // the chunk over the whole slice and streams their tiles in chunks of
-// kChunkTiles K-tiles.
+// kChunkTiles K-tiles.  (Shorter slices for larger batches would shrink the
+// quantised-input buffers and raise occupancy, but each slice change costs a
+// buffer copy and wait, and finalize sums more partials: at batch 16 on a
+// 28672-input layer, 512-input slices ran 4x slower.)
 constexpr int kVSliceTiles = 8;
 constexpr int kVSlice = kVSliceTiles * kVTileK;          // 2048 inputs
 constexpr int kVStages = 2;                              // bulk-copy ring per warp
