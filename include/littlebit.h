@@ -130,9 +130,13 @@ typedef struct lb_layer {
  *   Prefill (batch a multiple of 128, batch * d_in <= 2^30): xdt = LB_F16 or
  *   LB_BF16, y of the same type -- fp16 tcgen05 tensor-core path, see
  *   littlebit_linear_forward_many.
+ *   Any other batch above 16 (fp16 only, batch * d_in <= 2^30): the leading
+ *   multiple of 128 rows take the prefill path and the remaining rows the
+ *   decode path in groups of at most 16 (the weights stream once per group).
  *   x_dev and y_dev must be 16-byte aligned; every other pointer as in lb_path.
- * Errors: LB_ERR_ARG, LB_ERR_ALIGN, LB_ERR_SHAPE, LB_ERR_UNSUPPORTED (batch
- * 17..127 or not a multiple of 128, or an unsupported dtype), LB_ERR_CUDA.
+ * Errors: LB_ERR_ARG, LB_ERR_ALIGN, LB_ERR_SHAPE, LB_ERR_UNSUPPORTED (a dtype
+ * the batch's path does not take: bf16 below 128 rows or off a multiple of
+ * 128, f32 or i8 activations), LB_ERR_CUDA.
  */
 lb_status littlebit_linear_forward(const lb_layer* layer, const void* x_dev, void* y_dev,
                                    int batch, lb_dtype xdt, void* stream);
@@ -162,7 +166,8 @@ lb_status littlebit_linear_forward_many(const lb_layer* layers, int n, const voi
  * `stream` right after kernel launch i, for i < n_events <= 3: 0 = input
  * quantisation, 1 = latent pass, 2 = finalize (the output pass is last), so
  * that a caller can time each kernel with CUDA events.  The prefill path
- * records none.  events may be NULL when n_events is 0.
+ * records none; a batch split into groups records them in its first decode
+ * group.  events may be NULL when n_events is 0.
  */
 lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, const void* const* xs,
                                               void* const* ys, int batch, lb_dtype xdt, void* stream,

@@ -478,19 +478,42 @@ lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, con
     if (!xs[i] || !ys[i]) return LB_ERR_ARG;
     if (!aligned(xs[i], 16) || !aligned(ys[i], 16)) return LB_ERR_ALIGN;
   }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaEvent_t* evs = reinterpret_cast<const cudaEvent_t*>(events);
   if (batch <= lb::kMaxBatchDecode) {
     if (xdt != LB_F16) return LB_ERR_UNSUPPORTED;
-    return decode_forward(layers, n, xs, ys, batch, static_cast<cudaStream_t>(stream),
-                          reinterpret_cast<const cudaEvent_t*>(events), n_events);
+    return decode_forward(layers, n, xs, ys, batch, st, evs, n_events);
   }
-  if (batch % 128 == 0) {
-    if (xdt != LB_F16 && xdt != LB_BF16) return LB_ERR_UNSUPPORTED;
-    // operand preparation indexes one layer's fp16 copy of x with 32-bit offsets
-    for (int i = 0; i < n; ++i)
-      if ((size_t)batch * layers[i].d_in > ((size_t)1 << 30)) return LB_ERR_SHAPE;
-    return prefill_forward(layers, n, xs, ys, batch, xdt == LB_BF16 ? 1 : 0, static_cast<cudaStream_t>(stream));
+  if (xdt != LB_F16 && xdt != LB_BF16) return LB_ERR_UNSUPPORTED;
+  // operand preparation indexes one layer's fp16 copy of x with 32-bit offsets
+  for (int i = 0; i < n; ++i)
+    if ((size_t)batch * layers[i].d_in > ((size_t)1 << 30)) return LB_ERR_SHAPE;
+  if (batch % 128 == 0) return prefill_forward(layers, n, xs, ys, batch, xdt == LB_BF16 ? 1 : 0, st);
+  // Any other batch (fp16): the leading multiple of 128 rows through the
+  // prefill path, the rest through the decode path in groups of at most 16
+  // rows (rows are contiguous in x and y, so a group is an offset view).
+  if (xdt != LB_F16) return LB_ERR_UNSUPPORTED;
+  std::vector<const void*> xv(n);
+  std::vector<void*> yv(n);
+  auto views = [&](int r0) {
+    for (int i = 0; i < n; ++i) {
+      xv[i] = static_cast<const unsigned char*>(xs[i]) + (size_t)r0 * layers[i].d_in * 2;
+      yv[i] = static_cast<unsigned char*>(ys[i]) + (size_t)r0 * layers[i].d_out * 2;
+    }
+  };
+  const int m128 = batch / 128 * 128;
+  if (m128 > 0) {
+    const lb_status r = prefill_forward(layers, n, xs, ys, m128, 0, st);
+    if (r != LB_OK) return r;
   }
-  return LB_ERR_UNSUPPORTED;
+  for (int r0 = m128; r0 < batch; r0 += lb::kMaxBatchDecode) {
+    views(r0);
+    const int rows = std::min(lb::kMaxBatchDecode, batch - r0);
+    const lb_status r = decode_forward(layers, n, xv.data(), yv.data(), rows, st, r0 == m128 ? evs : nullptr,
+                                       r0 == m128 ? n_events : 0);
+    if (r != LB_OK) return r;
+  }
+  return LB_OK;
 }
 
 lb_status littlebit_linear_forward_many(const lb_layer* layers, int n, const void* const* xs, void* const* ys,

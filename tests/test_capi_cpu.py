@@ -88,7 +88,8 @@ def test_forward_rejects_bad_arguments_without_device_work(lib):
     L.path[0] = lb.LbPath(16, 32, 64, 48, 6)
     assert f(ctypes.byref(L), ctypes.c_void_p(24), x, 1, 0, None) == 2   # x misaligned
     assert f(ctypes.byref(L), x, x, 0, 0, None) == 3           # batch 0
-    assert f(ctypes.byref(L), x, x, 100, 0, None) == 6         # batch 17..255 unsupported
+    assert f(ctypes.byref(L), x, x, 100, 1, None) == 6         # bf16 off a multiple of 128 rows
+    assert f(ctypes.byref(L), x, x, 100, 2, None) == 6         # f32 activations
     assert f(ctypes.byref(L), x, x, 1, 1, None) == 6           # decode wants fp16
     pack = lb.library().littlebit_pack_signs
     assert pack(None, 0, 4, 4, 4, 1, 0, ctypes.c_void_p(16), None) == 1

@@ -237,3 +237,18 @@ def test_forward_many_in_cuda_graph(lbm, B):
         for i, (y, r) in enumerate(zip(Y, ref)):
             assert torch.equal(y, r), f"layer {i}"
     del g
+
+
+@pytest.mark.parametrize("batch", [17, 40, 130])
+def test_batches_between_decode_and_prefill(lbm, batch):
+    """Batches above 16 that are not a multiple of 128: the leading multiple
+    of 128 rows take the prefill path, the rest the decode path in groups of
+    at most 16 rows."""
+    lb, layers = lbm
+    d_in, d_out, s = 1024, 768, 90
+    paths = synth.layer(d_in, d_out, s, True, seed=batch)
+    x = synth.activations(batch, d_in, seed=batch)
+    layer = layers.upload(paths, d_in, d_out, s)
+    y = lb.forward(layer, torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    _check(y, orc.factored_forward(x, paths), f"B={batch}")
