@@ -397,7 +397,9 @@ def run_ours(args):
         "higher_is_better": False,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f16",
+        "dtype": "i8",
+        "dtype_note": "int8 tensor-core products (u8 sign planes x s8 hi/lo bytes of the 16-bit quantised vector), "
+                      "int32 accumulation, fp32 scaling; fp16 x and y",
         "data": "synthetic: fair random signs, scales ~U[0.5,1.5]/sqrt(s), x ~ N(0,1) fp16",
         "config": {"workload": WORKLOADS[args.workload]["desc"] + f", decode batch {args.batch}, "
                    f"stack of {n_layers} distinct layers per GPU ({main['stack_bytes'] / 1e6:.0f} MB packed, "
