@@ -242,6 +242,50 @@ def time_device(stack, steps, warmup, dist):
     return total_ms, per
 
 
+def measure_latency(device, reps=200, seed=99):
+    """Latency view: one Llama-2-7B attention projection (4096x4096, 0.1 BPW
+    residual, s = 86 x 2) at batch 1 per call, its 0.1 MB of weights staying
+    in L2 between calls.  Eager: back-to-back forward calls (host work and four
+    launches each).  Graph: the same call captured once into a CUDA graph and
+    replayed.  CUDA events on the stream, microseconds per call."""
+    import torch
+    from latent_binary_factorization_b200 import layers as lbl, littlebit as lb
+    gen = torch.Generator(device=device).manual_seed(seed)
+    L = lbl.random_layer(4096, 4096, 86, True, gen, device=device)[0]
+    x = torch.randn(1, 4096, generator=gen, device=device).half()
+    y = torch.empty(1, 4096, dtype=torch.float16, device=device)
+    stack = lb.Stack([L], [x], [y])
+    side = torch.cuda.Stream(device)
+    side.wait_stream(torch.cuda.current_stream(device))
+    out = {}
+    with torch.cuda.stream(side):
+        for _ in range(10):
+            stack()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(side)
+        for _ in range(reps):
+            stack()
+        e1.record(side)
+        torch.cuda.synchronize(device)
+        out["eager_us"] = round(1e3 * e0.elapsed_time(e1) / reps, 3)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        stack()
+    with torch.cuda.stream(side):
+        for _ in range(10):
+            g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(side)
+        for _ in range(reps):
+            g.replay()
+        e1.record(side)
+        torch.cuda.synchronize(device)
+        out["graph_us"] = round(1e3 * e0.elapsed_time(e1) / reps, 3)
+    del g
+    out["workload"] = "one Llama-2-7B attention projection 4096x4096, 0.1 BPW residual (s=86 x 2), batch 1, per call"
+    return out
+
+
 def time_e2e(stack, x_all, y_all, steps, warmup):
     """Same forward through the public API with host buffers: H2D of every
     layer's input from pinned memory, forward, D2H of every output."""
@@ -361,6 +405,7 @@ def run_ours(args):
             torch.cuda.empty_cache()
             r["roofline_frac_step"] = r["step_gbs"] / peak
             extras[f"{name}_b{b}"] = r
+        extras["latency_single_layer"] = measure_latency(device)
     prefill = None
     if not args.no_prefill:
         pms, pflops = measure_prefill(args.prefill_layers, 2048, max(3, args.steps // 20), 3, device, dist)
@@ -435,6 +480,17 @@ def run_ours(args):
 # CPU oracle arm
 # ---------------------------------------------------------------------------
 
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def _blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -467,7 +523,7 @@ def cpu_baseline(workload, batch, budget_s=10.0, n_distinct=4):
     dt = time.perf_counter() - t0
     return {"value": round(1e6 * dt / n, 3), "unit": "us/layer", "cores": _blas_threads(), "kind": "oracle",
             "sample": f"{n} forwards of {n_distinct} distinct {WORKLOADS[workload]['desc']} layers, batch {batch}, "
-                      f"fp64 numpy, {dt:.1f} s"}
+                      f"fp64 numpy, {dt:.1f} s", "nproc": os.cpu_count(), "cpu_model": _cpu_model()}
 
 
 def run_reference(args):

@@ -104,6 +104,18 @@ lb_status littlebit_pack_signs(const void* src_dev, lb_dtype dt, int n_long, int
                                int64_t stride_long, int64_t stride_s, lb_role role,
                                void* dst_dev, void* stream);
 
+/*
+ * Inverse of littlebit_pack_signs (a test and inspection aid): the packed
+ * factor at src_dev (littlebit_packed_bytes(role, R, K) bytes, 16-byte
+ * aligned) back to +-1 values in its natural orientation, n_long x s int8,
+ * row-major (element (a, j) at dst_dev[a * s + j]; role V: n_long = d_in,
+ * role U: n_long = d_out).  Padding bits are not read.
+ * Errors: LB_ERR_ARG (null, bad role), LB_ERR_SHAPE (n_long or s < 1),
+ * LB_ERR_ALIGN (src not 16-byte aligned), LB_ERR_CUDA.
+ */
+lb_status littlebit_unpack_signs(const void* src_dev, lb_role role, int n_long, int s, int8_t* dst_dev,
+                                 void* stream);
+
 /* One path of a layer: device pointers, all owned by the caller. */
 typedef struct lb_path {
   const void* V_bits;    /* packed LB_ROLE_V factor, 16-byte aligned */

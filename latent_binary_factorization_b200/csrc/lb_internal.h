@@ -178,6 +178,7 @@ cudaError_t launch_prefill_gemms(const PrefillPlan& plan, const unsigned char* t
                                  cudaStream_t st);
 
 // pack.cu
+cudaError_t launch_unpack(const void* src, int n_long, int s, lb_role role, int8_t* dst, cudaStream_t st);
 cudaError_t launch_pack(const void* src, lb_dtype dt, int n_long, int s, int64_t stride_long,
                         int64_t stride_s, lb_role role, void* dst, cudaStream_t st);
 

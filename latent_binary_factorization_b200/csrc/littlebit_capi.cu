@@ -467,6 +467,16 @@ lb_status littlebit_pack_signs(const void* src_dev, lb_dtype dt, int n_long, int
   return e == cudaSuccess ? LB_OK : cuda_fail(e);
 }
 
+lb_status littlebit_unpack_signs(const void* src_dev, lb_role role, int n_long, int s, int8_t* dst_dev,
+                                 void* stream) {
+  if (!src_dev || !dst_dev) return LB_ERR_ARG;
+  if (role != LB_ROLE_V && role != LB_ROLE_U) return LB_ERR_ARG;
+  if (n_long < 1 || s < 1) return LB_ERR_SHAPE;
+  if (!aligned(src_dev, 16)) return LB_ERR_ALIGN;
+  cudaError_t e = lb::launch_unpack(src_dev, n_long, s, role, dst_dev, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LB_OK : cuda_fail(e);
+}
+
 lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, const void* const* xs,
                                               void* const* ys, int batch, lb_dtype xdt, void* stream,
                                               void* const* events, int n_events) {

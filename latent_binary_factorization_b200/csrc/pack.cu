@@ -89,7 +89,59 @@ cudaError_t launch_dt(const void* src, int n_long, int s, int64_t sl, int64_t ss
   return cudaGetLastError();
 }
 
+// Inverse of pack_kernel: one thread per element (a, j) of the natural
+// n_long x s factor, written row-major as +-1 int8.  The (row, k) of the
+// element in F gives its tile, lane, word and bit by inverting the layout.
+template <lb_role ROLE>
+__global__ void __launch_bounds__(256) unpack_kernel(const unsigned char* __restrict__ src, int n_long, int s,
+                                                     int n_kt, int8_t* __restrict__ dst) {
+  const long long total = (long long)n_long * s;
+  for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < total;
+       t += (long long)gridDim.x * blockDim.x) {
+    const int a = (int)(t / s), j = (int)(t - (long long)a * s);
+    const int row = (ROLE == LB_ROLE_V) ? j : a, k = (ROLE == LB_ROLE_V) ? a : j;
+    int rb, kt, g, c, m, q, rlo, rhi;
+    if (ROLE == LB_ROLE_V) {
+      // row = 16 rb + g + 8 (r % 2),  k = 256 kt + 32 q + 16 (r / 2) + 4 c + m
+      rb = row >> 4;
+      g = row & 7;
+      rlo = (row >> 3) & 1;
+      kt = k >> 8;
+      q = (k >> 5) & 7;
+      rhi = (k >> 4) & 1;
+      c = (k >> 2) & 3;
+      m = k & 3;
+    } else {
+      // row = 128 rb + 16 q + g + 8 (r % 2),  k = 32 kt + 16 (r / 2) + 4 c + m
+      rb = row >> 7;
+      q = (row >> 4) & 7;
+      g = row & 7;
+      rlo = (row >> 3) & 1;
+      kt = k >> 5;
+      rhi = (k >> 4) & 1;
+      c = (k >> 2) & 3;
+      m = k & 3;
+    }
+    const int r = 2 * rhi + rlo, lane = 4 * g + c;
+    const uint32_t word =
+        *reinterpret_cast<const uint32_t*>(src + 512 * ((size_t)rb * n_kt + kt) + 16 * lane + 4 * r);
+    dst[t] = ((word >> (8 * m + q)) & 1u) ? (int8_t)-1 : (int8_t)1;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_unpack(const void* src, int n_long, int s, lb_role role, int8_t* dst, cudaStream_t st) {
+  const int K = (role == LB_ROLE_V) ? n_long : s;
+  const int n_kt = ceil_div(K, (role == LB_ROLE_V) ? kVTileK : kUTileK);
+  const long long total = (long long)n_long * s;
+  long long blocks = (total + 255) / 256;
+  if (blocks > 148 * 32) blocks = 148 * 32;
+  const unsigned char* p = static_cast<const unsigned char*>(src);
+  if (role == LB_ROLE_V) unpack_kernel<LB_ROLE_V><<<(int)blocks, 256, 0, st>>>(p, n_long, s, n_kt, dst);
+  else unpack_kernel<LB_ROLE_U><<<(int)blocks, 256, 0, st>>>(p, n_long, s, n_kt, dst);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pack(const void* src, lb_dtype dt, int n_long, int s, int64_t stride_long,
                         int64_t stride_s, lb_role role, void* dst, cudaStream_t st) {

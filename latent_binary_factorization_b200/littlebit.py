@@ -50,6 +50,9 @@ _lib.littlebit_pack_signs.restype = ctypes.c_int
 _lib.littlebit_pack_signs.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p,
                                       ctypes.c_void_p]
+_lib.littlebit_unpack_signs.restype = ctypes.c_int
+_lib.littlebit_unpack_signs.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                        ctypes.c_void_p]
 _lib.littlebit_linear_forward.restype = ctypes.c_int
 _lib.littlebit_linear_forward.argtypes = [ctypes.POINTER(LbLayer), ctypes.c_void_p, ctypes.c_void_p,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
@@ -121,6 +124,15 @@ def pack_signs(factor: torch.Tensor, role: str, out: torch.Tensor | None = None,
                                      factor.stride(0), factor.stride(1), ROLE[role],
                                      ctypes.c_void_p(out.data_ptr()), _stream(stream)),
            "littlebit_pack_signs")
+    return out
+
+
+def unpack_signs(packed: torch.Tensor, role: str, n_long: int, s: int, stream=None) -> torch.Tensor:
+    """Packed factor bytes (CUDA) back to its +-1 values, n_long x s int8."""
+    out = torch.empty((n_long, s), dtype=torch.int8, device=packed.device)
+    _check(_lib.littlebit_unpack_signs(ctypes.c_void_p(packed.data_ptr()), ROLE[role], n_long, s,
+                                       ctypes.c_void_p(out.data_ptr()), _stream(stream)),
+           "littlebit_unpack_signs")
     return out
 
 

@@ -68,6 +68,22 @@ def test_pack_full_size_70b_factor(lbm):
         assert np.array_equal(got, orc.pack_signs(orc.factor_matrix(role, Sh), role)), role
 
 
+@pytest.mark.parametrize("role,n_long,s", [("V", 256, 1), ("V", 4096 + 256, 86), ("V", 512, 1024),
+                                           ("U", 128, 1), ("U", 4096, 188), ("U", 384, 45)])
+def test_unpack_inverts_pack(lbm, role, n_long, s):
+    """unpack(pack(F)) = sign(F) as +-1, and it equals the oracle's unpacking
+    of the same bytes."""
+    lb, _ = lbm
+    F = synth.real_factor(n_long, s, seed=n_long + s, zeros=0.05)
+    t = torch.from_numpy(F).cuda()
+    packed = lb.pack_signs(t, role)
+    got = lb.unpack_signs(packed, role, n_long, s).cpu().numpy()
+    assert np.array_equal(got, np.where(F < 0, -1, 1).astype(np.int8))
+    R, K = (s, n_long) if role == "V" else (n_long, s)
+    want = orc.unpack_signs(packed.cpu().numpy(), role, R, K)
+    assert np.array_equal(got, orc.factor_matrix(role, want) if role == "V" else want)
+
+
 # ----------------------------------------------------------------- forward
 
 def _run(lbm, d_in, d_out, s, residual, batch, seed=0):
