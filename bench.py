@@ -512,18 +512,31 @@ def cpu_baseline(workload, batch, budget_s=10.0, n_distinct=4):
         a, b, s, r = mats[i % len(mats)]
         samples.append((synth.layer(a, b, s, r, seed=77, index=i), synth.activations(batch, a, seed=77, index=i)))
     orc.factored_forward(samples[0][1], samples[0][0])   # warm
-    t0 = time.perf_counter()
-    n = 0
-    while True:
-        paths, x = samples[n % n_distinct]
-        orc.factored_forward(x, paths)
-        n += 1
-        if time.perf_counter() - t0 >= budget_s and n >= 3:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": round(1e6 * dt / n, 3), "unit": "us/layer", "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{n} forwards of {n_distinct} distinct {WORKLOADS[workload]['desc']} layers, batch {batch}, "
-                      f"fp64 numpy, {dt:.1f} s", "nproc": os.cpu_count(), "cpu_model": _cpu_model()}
+
+    def timed(seconds):
+        t0 = time.perf_counter()
+        n = 0
+        while True:
+            paths, x = samples[n % n_distinct]
+            orc.factored_forward(x, paths)
+            n += 1
+            if time.perf_counter() - t0 >= seconds and n >= 3:
+                break
+        return n, time.perf_counter() - t0
+
+    n, dt = timed(budget_s)
+    out = {"value": round(1e6 * dt / n, 3), "unit": "us/layer", "cores": _blas_threads(), "kind": "oracle",
+           "sample": f"{n} forwards of {n_distinct} distinct {WORKLOADS[workload]['desc']} layers, batch {batch}, "
+                     f"fp64 numpy, {dt:.1f} s", "nproc": os.cpu_count(), "cpu_model": _cpu_model()}
+    try:   # the same oracle with its BLAS held to one thread
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1, user_api="blas"):
+            n1, dt1 = timed(budget_s / 4)
+        out["single_thread"] = {"value": round(1e6 * dt1 / n1, 3), "unit": "us/layer", "cores": 1,
+                                "sample": f"{n1} forwards, {dt1:.1f} s"}
+    except ImportError:
+        pass
+    return out
 
 
 def run_reference(args):

@@ -96,3 +96,24 @@ def test_forward_rejects_bad_arguments_without_device_work(lib):
     assert pack(ctypes.c_void_p(16), 9, 4, 4, 4, 1, 0, ctypes.c_void_p(16), None) == 1
     assert pack(ctypes.c_void_p(16), 0, 0, 4, 4, 1, 0, ctypes.c_void_p(16), None) == 3
     assert pack(ctypes.c_void_p(16), 0, 4, 4, 4, 1, 0, ctypes.c_void_p(8), None) == 2
+
+
+def test_header_compiles_as_c_and_links(tmp_path):
+    """A C program (tests/c_abi_host_check.c) compiles against the header with
+    a C compiler, links with the library and runs its host entry points."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "c_abi_host_check"
+    libdir = os.path.dirname(LIB)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi_host_check.c"), "-o", str(exe),
+                    "-L", libdir, "-llittlebit", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    from oracle import littlebit_oracle as orc
+    assert abs(float(out[0].split()[1]) - float(orc.eff_bits_exact(4096, 4096, 86, True))) < 1e-8
+    assert int(out[1].split()[1]) == orc.packed_nbytes("V", 86, 4096)
+    assert out[2] == "forward 3"
+    assert out[3].startswith("status LB_ERR_SHAPE")
