@@ -221,6 +221,20 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
  */
 lb_status littlebit_device_status(void* stream, unsigned int* status);
 
+/*
+ * Exercises the error path that every bounded device wait of the library
+ * takes when it gives up, without any fault or hang: enqueues on `stream` one
+ * kernel of one warp that polls an mbarrier that nothing completes, `polls`
+ * times (each poll may suspend for up to about 1 us; 1000 polls last about a
+ * millisecond), and then raises bit (1 << LB_ERR_TIMEOUT) in the status word
+ * of the (device, stream) workspace.  It issues no copy, so nothing is left
+ * in flight.  The next littlebit_device_status on the stream reports the bit
+ * and clears it; the stream and its workspace remain usable.  Allocates the
+ * workspace's status word if no forward has run on the stream yet.
+ * Errors: LB_ERR_ARG (polls outside 1 .. 4194304), LB_ERR_CUDA.
+ */
+lb_status littlebit_check_wait_timeout(void* stream, int polls);
+
 /* Free every workspace of every device, with its side stream and events (call
  * with no work in flight on any stream the library was given). */
 void littlebit_release(void);

@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "liblittlebit.so")
-SOURCES = ["littlebit_capi.cu", "pack.cu", "decode.cu", "prefill.cu", "noalloc.cu"]
+SOURCES = ["littlebit_capi.cu", "pack.cu", "decode.cu", "prefill.cu", "noalloc.cu", "selfcheck.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -152,6 +152,10 @@ cudaError_t launch_quantise_pass(const DecodeArgs& a, cudaStream_t st);
 cudaError_t launch_latent_pass(const DecodeArgs& a, int max_s16, int num_sms, cudaStream_t st);
 cudaError_t launch_finalize_pass(const DecodeArgs& a, int max_s16, cudaStream_t st);
 cudaError_t launch_output_pass(const DecodeArgs& a, int num_sms, cudaStream_t st);
+// selfcheck.cu: one warp polls `polls` times (1..kSpinLimit) an mbarrier that
+// nothing completes and raises LB_ERR_TIMEOUT in *status, as every bounded
+// wait of the forward kernels does when it gives up.
+cudaError_t launch_wait_timeout_probe(unsigned int* status, int polls, cudaStream_t st);
 
 // prefill.cu: layers of M rows (multiple of 128), x fp16 or bf16 (y the same)
 int prefill_sp(int s, int npaths);

@@ -119,6 +119,31 @@ size_t path_scratch_bytes(const lb_layer& L, int batch) {
 
 constexpr size_t kStatusBytes = 256;   // device status word at the start of a workspace
 
+// Replaces the workspace buffer with a zeroed one of `cap` bytes.  The old
+// buffer is freed once `st` has drained; its status word is carried over, so
+// bits raised before the growth are still reported by littlebit_device_status.
+lb_status grow_workspace(Workspace& ws, size_t cap, cudaStream_t st) {
+  unsigned int status = 0;
+  cudaError_t e;
+  if (ws.buf) {
+    e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaMemcpy(&status, ws.buf, sizeof(status), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e);
+    cudaFree(ws.buf);
+    ws.buf = nullptr;
+    ws.cap = 0;
+  }
+  e = cudaMalloc(&ws.buf, cap);
+  if (e != cudaSuccess) return cuda_fail(e);
+  ws.cap = cap;
+  ws.table.clear();
+  e = cudaMemsetAsync(ws.buf, 0, cap, st);
+  // pageable source: staged before cudaMemcpyAsync returns
+  if (e == cudaSuccess && status) e = cudaMemcpyAsync(ws.buf, &status, sizeof(status), cudaMemcpyHostToDevice, st);
+  return e == cudaSuccess ? LB_OK : cuda_fail(e);
+}
+
 // The four decode launches of a prepared call; events[i] (if given) is
 // recorded right after launch i.
 lb_status decode_launch(const lb::DecodeArgs& a, int max_s16, int sms, cudaStream_t st, const cudaEvent_t* events,
@@ -171,20 +196,8 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   const size_t total = kStatusBytes + table_bytes + map_bytes + scratch;
 
   if (ws.cap < total) {
-    if (ws.buf) {
-      e = cudaStreamSynchronize(st);
-      if (e != cudaSuccess) return cuda_fail(e);
-      cudaFree(ws.buf);
-      ws.buf = nullptr;
-      ws.cap = 0;
-    }
-    const size_t cap = align_up(total + total / 4, 1 << 20);
-    e = cudaMalloc(&ws.buf, cap);
-    if (e != cudaSuccess) return cuda_fail(e);
-    ws.cap = cap;
-    ws.table.clear();
-    e = cudaMemsetAsync(ws.buf, 0, cap, st);   // the status word starts at zero
-    if (e != cudaSuccess) return cuda_fail(e);
+    const lb_status r = grow_workspace(ws, align_up(total + total / 4, 1 << 20), st);
+    if (r != LB_OK) return r;
   }
 
   // ---- descriptor table and item maps
@@ -338,20 +351,9 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
   const size_t need = kStatusBytes + tables + (n_chunks > 1 ? 2 : 1) * half;
 
   if (ws.cap < need) {
-    if (ws.buf) {
-      e = cudaStreamSynchronize(st);   // the side stream always joins `st`
-      if (e != cudaSuccess) return cuda_fail(e);
-      cudaFree(ws.buf);
-      ws.buf = nullptr;
-      ws.cap = 0;
-    }
-    const size_t cap = align_up(need + need / 8, 1 << 20);
-    e = cudaMalloc(&ws.buf, cap);
-    if (e != cudaSuccess) return cuda_fail(e);
-    ws.cap = cap;
-    ws.table.clear();
-    e = cudaMemsetAsync(ws.buf, 0, cap, st);
-    if (e != cudaSuccess) return cuda_fail(e);
+    // the side stream always joins `st`, so waiting for `st` covers it
+    const lb_status r = grow_workspace(ws, align_up(need + need / 8, 1 << 20), st);
+    if (r != LB_OK) return r;
   }
   unsigned char* base = static_cast<unsigned char*>(ws.buf);
   unsigned char* table_dev = base + kStatusBytes;
@@ -553,6 +555,23 @@ lb_status littlebit_device_status(void* stream, unsigned int* status) {
   e = cudaMemset(it->second.buf, 0, sizeof(unsigned int));
   if (e != cudaSuccess) return cuda_fail(e);
   return LB_OK;
+}
+
+lb_status littlebit_check_wait_timeout(void* stream, int polls) {
+  if (polls < 1 || polls > lb::kSpinLimit) return LB_ERR_ARG;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_mu);
+  Workspace& ws = g_ws[{dev, st}];
+  if (!ws.buf) {
+    // just the status word; a later forward grows the workspace
+    const lb_status r = grow_workspace(ws, kStatusBytes, st);
+    if (r != LB_OK) return r;
+  }
+  e = lb::launch_wait_timeout_probe(static_cast<unsigned int*>(ws.buf), polls, st);
+  return e == cudaSuccess ? LB_OK : cuda_fail(e);
 }
 
 void littlebit_release(void) {

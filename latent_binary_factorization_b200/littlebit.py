@@ -68,6 +68,8 @@ _lib.littlebit_linear_forward_many_timed.argtypes = [ctypes.POINTER(LbLayer), ct
                                                      ctypes.c_void_p, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]
 _lib.littlebit_device_status.restype = ctypes.c_int
 _lib.littlebit_device_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint)]
+_lib.littlebit_check_wait_timeout.restype = ctypes.c_int
+_lib.littlebit_check_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_int]
 _lib.littlebit_release.restype = None
 _lib.littlebit_release.argtypes = []
 _lib.littlebit_status_string.restype = ctypes.c_char_p
@@ -220,6 +222,13 @@ def device_status(stream=None) -> int:
     out = ctypes.c_uint(0)
     _check(_lib.littlebit_device_status(_stream(stream), ctypes.byref(out)), "littlebit_device_status")
     return int(out.value)
+
+
+def check_wait_timeout(stream=None, polls: int = 1000) -> None:
+    """Enqueue the self-check of the bounded-wait error path: a wait on a
+    barrier that nothing completes gives up after `polls` polls and raises
+    the LB_ERR_TIMEOUT bit, which the next device_status() returns."""
+    _check(_lib.littlebit_check_wait_timeout(_stream(stream), int(polls)), "littlebit_check_wait_timeout")
 
 
 def release() -> None:

@@ -96,6 +96,9 @@ def test_forward_rejects_bad_arguments_without_device_work(lib):
     assert pack(ctypes.c_void_p(16), 9, 4, 4, 4, 1, 0, ctypes.c_void_p(16), None) == 1
     assert pack(ctypes.c_void_p(16), 0, 0, 4, 4, 1, 0, ctypes.c_void_p(16), None) == 3
     assert pack(ctypes.c_void_p(16), 0, 4, 4, 4, 1, 0, ctypes.c_void_p(8), None) == 2
+    chk = lb.library().littlebit_check_wait_timeout
+    assert chk(None, 0) == 1                                     # polls < 1
+    assert chk(None, (1 << 22) + 1) == 1                         # polls above the kernels' own limit
 
 
 def test_header_compiles_as_c_and_links(tmp_path):

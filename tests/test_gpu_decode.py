@@ -196,6 +196,47 @@ def test_device_status_clean_after_forward(lbm):
     assert lb.device_status() == 0
 
 
+def test_bounded_wait_timeout_is_reported_and_recoverable(lbm):
+    """The error path of a bounded device wait, run for real: a wait on a
+    barrier that nothing completes gives up after 1000 polls (about 1 ms) and
+    raises LB_ERR_TIMEOUT; the status read returns the bit and clears it, a
+    workspace growth carries an unread bit over, and the stream keeps working."""
+    lb, layers = lbm
+    timeout_bit = 1 << 5                                         # LB_ERR_TIMEOUT
+    st = torch.cuda.Stream()
+    lb.check_wait_timeout(st, polls=1000)                        # no workspace yet on this stream
+    assert lb.device_status(st) == timeout_bit
+    assert lb.device_status(st) == 0
+
+    paths = synth.layer(2048, 1024, 200, True, seed=6)
+    layer = layers.upload(paths, 2048, 1024, 200)
+    xh = synth.activations(2, 2048, seed=6)
+    x = torch.from_numpy(xh).cuda()
+    ref = orc.factored_forward(xh, paths)
+    st.wait_stream(torch.cuda.current_stream())                  # packed factors and x are ready
+    with torch.cuda.stream(st):
+        y = lb.forward(layer, x, stream=st)
+    assert lb.device_status(st) == 0
+    _check(y, ref, "after the self-check")
+
+    lb.check_wait_timeout(st, polls=1000)
+    # 16384 inputs at batch 16: about 1.4 MB of scratch, more than the 1 MB
+    # workspace the first forward allocated, so this call regrows it
+    big = synth.layer(16384, 1024, 300, True, seed=7)
+    big_layer = layers.upload(big, 16384, 1024, 300)
+    xbh = synth.activations(16, 16384, seed=7)
+    xb = torch.from_numpy(xbh).cuda()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        yb = lb.forward(big_layer, xb, stream=st)
+    assert lb.device_status(st) == timeout_bit
+    _check(yb, orc.factored_forward(xbh, big), "after a workspace growth")
+    with torch.cuda.stream(st):
+        y2 = lb.forward(layer, x, stream=st)
+    assert lb.device_status(st) == 0
+    _check(y2, ref, "second forward")
+
+
 def test_repeatable_and_deterministic(lbm):
     lb, layers = lbm
     paths = synth.layer(4096, 4096, 86, True, seed=9)
