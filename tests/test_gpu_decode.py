@@ -119,9 +119,10 @@ def test_7b_attention_projection(lbm, batch, residual, s):
     (4096, 11008, 133, True, 1),        # 7B MLP gate/up at 0.1 BPW
     (11008, 4096, 135, True, 2),        # 7B MLP down, the quoted rank
     (1024, 1024, 1024, False, 1),       # maximum rank
+    (1024, 512, 1024, True, 16),        # maximum rank, both paths, full batch
     (512, 256, 511, True, 16),          # ragged rank, full batch
-    (768, 384, 40, True, 16),           # 512-input slices at batch 16: last slice one K-tile
-    (1280, 256, 70, False, 8),          # 1024-input slices at batch 8: last slice one K-tile
+    (768, 384, 40, True, 16),           # one partial slice (3 of 8 K-tiles) at batch 16
+    (1280, 256, 70, False, 8),          # one partial slice (5 of 8 K-tiles) at batch 8
     (4096, 4096, 86, True, 12),         # three groups of batch rows
 ])
 def test_shapes_and_ragged_edges(lbm, d_in, d_out, s, residual, batch):

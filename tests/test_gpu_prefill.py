@@ -43,6 +43,7 @@ def _check(y, y_ref, tag):
     (1024, 384, 100, True, 256),     # ragged N tile of GEMM2 (384 = 256 + 128), ragged rank
     (768, 640, 1, False, 128),       # rank 1
     (256, 128, 45, True, 384),       # smallest shapes
+    (1024, 512, 1024, True, 128),    # maximum rank, both paths: GEMM1 N = GEMM2 K = 2048
 ])
 def test_prefill_small_full_output(lbm, dtype, d_in, d_out, s, residual, M):
     lb, layers = lbm
