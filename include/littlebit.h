@@ -22,11 +22,12 @@
  *    stream).  Device work is enqueued on it and the call returns without
  *    waiting; the return value reports only what the host can check
  *    (arguments, alignment, shapes, launch errors).
- *  - The library keeps one workspace per (device, stream) -- a descriptor
- *    table and the latent-vector scratch of the forward -- allocated on first
- *    use with cudaMalloc, grown when needed and freed by littlebit_release().
- *    Calls enqueued on the same stream are ordered; calls on different streams
- *    use different workspaces.
+ *  - The library keeps workspaces per (device, stream) -- descriptor tables
+ *    and the latent-vector scratch of the forward; one each for the prefill
+ *    part and each 16-row decode group of a call, and for each chunk of a
+ *    host-buffer call -- allocated on first use with cudaMalloc, grown when
+ *    needed and freed by littlebit_release().  Calls enqueued on the same
+ *    stream are ordered; calls on different streams use different workspaces.
  *  - No entry point falls back to the CPU: without a usable CUDA device the
  *    call returns LB_ERR_CUDA.
  */
@@ -161,7 +162,7 @@ lb_status littlebit_linear_forward(const lb_layer* layer, const void* x_dev, voi
  * so that the weights of all layers stream from HBM back to back.  layers, xs,
  * ys are host arrays of length n.
  *
- * The library keeps one workspace per (device, stream) and remembers the last
+ * The library keeps a workspace per (device, stream) and remembers the last
  * call's arguments on it (the layer structs and the x and y pointers): a call
  * that repeats them enqueues kernels and events only -- no allocation, no
  * host-to-device copy -- and may therefore be captured into a CUDA graph, on
@@ -184,6 +185,31 @@ lb_status littlebit_linear_forward_many(const lb_layer* layers, int n, const voi
 lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, const void* const* xs,
                                               void* const* ys, int batch, lb_dtype xdt, void* stream,
                                               void* const* events, int n_events);
+
+/*
+ * littlebit_linear_forward_many with the activations in HOST memory (no
+ * counterpart in the pages; a transport wrapper around the same forward).
+ *   x_host: the n layers' inputs back to back -- layer i's batch x d_in[i]
+ *     row-major matrix starts at element sum_{j<i} batch * d_in[j] -- in xdt
+ *     (2-byte elements).  y_host: the outputs the same way with d_out (y has
+ *     x's dtype).  Both are caller-owned host memory.
+ *   n_chunks (>= 1; at most min(n, 64) are used): the stack is cut into that
+ *     many consecutive groups of layers of about equal bytes.  Group c's input
+ *     copy, its forward and its output copy are chained by events on two
+ *     library-owned copy streams and `stream`, so that copies of one group
+ *     overlap the kernels of its neighbours.  Page-locked host buffers
+ *     (cudaHostAlloc / cudaHostRegister) are needed for that overlap; with
+ *     pageable memory the result is the same but the copies serialise.
+ * Device copies of the whole stack's x and y are held per (device, stream)
+ * until littlebit_release().  Both copy streams start after the work already
+ * enqueued on `stream`, and `stream` continues only after the last output
+ * copy, so y_host is complete once `stream` has been synchronised (the host
+ * buffers must stay untouched until then).  Not for CUDA-graph capture.
+ * Batch, dtype and layer rules, and errors, as littlebit_linear_forward_many;
+ * LB_ERR_ARG also for NULL host pointers or n_chunks < 1.
+ */
+lb_status littlebit_linear_forward_many_host(const lb_layer* layers, int n, const void* x_host, void* y_host,
+                                             int batch, lb_dtype xdt, int n_chunks, void* stream);
 
 /*
  * The decode forward of littlebit_linear_forward (one layer, 1 <= batch <= 16,

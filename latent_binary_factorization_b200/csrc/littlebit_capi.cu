@@ -3,10 +3,12 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <climits>
 #include <cstdio>
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
 #include <vector>
 
@@ -71,8 +73,17 @@ void release_workspace(Workspace& w) {
   w = Workspace();
 }
 
+// Workspaces are keyed by (device, stream, tag).  The tag separates calls
+// that alternate on one stream, so that each keeps its cached tables: the
+// prefill part and each 16-row decode group of a mixed batch, and each chunk
+// of a host-buffer stack call (ws_tag below).
 std::mutex g_mu;
-std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+using WsKey = std::tuple<int, cudaStream_t, int>;
+std::map<WsKey, Workspace> g_ws;
+
+// tag = (base << 8) | part; base 0 is the device-pointer API, base c+1 chunk c
+// of littlebit_linear_forward_many_host; part 0 is prefill, 1 + g decode group g.
+int ws_tag(int base, int part) { return (base << 8) | part; }
 int g_num_sms[64] = {0};
 
 int num_sms(int dev) {
@@ -118,6 +129,7 @@ size_t path_scratch_bytes(const lb_layer& L, int batch) {
 }
 
 constexpr size_t kStatusBytes = 256;   // device status word at the start of a workspace
+constexpr int kMaxHostChunks = 64;     // chunks of one host-buffer stack call
 
 // Replaces the workspace buffer with a zeroed one of `cap` bytes.  The old
 // buffer is freed once `st` has drained; its status word is carried over, so
@@ -160,12 +172,12 @@ lb_status decode_launch(const lb::DecodeArgs& a, int max_s16, int sms, cudaStrea
 }
 
 lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
-                         cudaStream_t st, const cudaEvent_t* events, int n_events) {
+                         cudaStream_t st, const cudaEvent_t* events, int n_events, int tag) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
   std::lock_guard<std::mutex> lock(g_mu);
-  Workspace& ws = g_ws[{dev, st}];
+  Workspace& ws = g_ws[{dev, st, tag}];
   std::vector<unsigned char> key = call_key('D', layers, n, xs, ys, batch, 0);
   if (ws.buf && ws.key == key) return decode_launch(ws.dargs, ws.d_max_s16, num_sms(dev), st, events, n_events);
   ws.key.clear();
@@ -312,12 +324,12 @@ cudaError_t ensure_side(Workspace& ws) {
 lb_status prefill_launch(Workspace& ws, const void* const* xs, int batch, int x_bf16, cudaStream_t st);
 
 lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
-                          int x_bf16, cudaStream_t st) {
+                          int x_bf16, cudaStream_t st, int tag) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
   std::lock_guard<std::mutex> lock(g_mu);
-  Workspace& ws = g_ws[{dev, st}];
+  Workspace& ws = g_ws[{dev, st, tag}];
   std::vector<unsigned char> key = call_key('P', layers, n, xs, ys, batch, x_bf16);
   if (ws.buf && ws.key == key) return prefill_launch(ws, xs, batch, x_bf16, st);
   ws.key.clear();
@@ -440,6 +452,124 @@ lb_status prefill_launch(Workspace& ws, const void* const* xs, int batch, int x_
 }
 
 
+// State of littlebit_linear_forward_many_host per (device, stream): device
+// copies of the whole stack's x and y, the two copy streams and the events
+// that chain copy-in -> forward -> copy-out chunk by chunk.
+struct HostPipe {
+  unsigned char* x_dev = nullptr;
+  unsigned char* y_dev = nullptr;
+  size_t x_cap = 0, y_cap = 0;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t fork = nullptr, join_in = nullptr, join_out = nullptr;
+  std::vector<cudaEvent_t> in_done, fwd_done;   // per chunk
+  // the last call's plan (layers, batch, dtype, chunk count) and what follows
+  std::vector<unsigned char> key;
+  std::vector<int> starts;             // chunk c = layers starts[c] .. starts[c+1]-1
+  std::vector<size_t> xo, yo;          // byte offsets of each layer's x and y; [n] = totals
+  std::vector<const void*> xs;         // device views into x_dev / y_dev
+  std::vector<void*> ys;
+};
+
+std::mutex g_host_mu;   // taken before g_mu, never after it
+std::map<std::pair<int, cudaStream_t>, HostPipe> g_pipes;
+
+void release_pipe(HostPipe& hp) {
+  if (hp.x_dev) cudaFree(hp.x_dev);
+  if (hp.y_dev) cudaFree(hp.y_dev);
+  for (cudaEvent_t ev : {hp.fork, hp.join_in, hp.join_out})
+    if (ev) cudaEventDestroy(ev);
+  for (cudaEvent_t ev : hp.in_done) cudaEventDestroy(ev);
+  for (cudaEvent_t ev : hp.fwd_done) cudaEventDestroy(ev);
+  if (hp.h2d) cudaStreamDestroy(hp.h2d);
+  if (hp.d2h) cudaStreamDestroy(hp.d2h);
+  hp = HostPipe();
+}
+
+cudaError_t ensure_pipe_objects(HostPipe& hp, int n_chunks) {
+  cudaError_t e = cudaSuccess;
+  if (!hp.h2d) e = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking);
+  if (e == cudaSuccess && !hp.d2h) e = cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking);
+  for (cudaEvent_t* ev : {&hp.fork, &hp.join_in, &hp.join_out})
+    if (e == cudaSuccess && !*ev) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+  while (e == cudaSuccess && (int)hp.in_done.size() < n_chunks) {
+    cudaEvent_t a = nullptr, b = nullptr;
+    e = cudaEventCreateWithFlags(&a, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&b, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      if (a) cudaEventDestroy(a);
+      break;
+    }
+    hp.in_done.push_back(a);
+    hp.fwd_done.push_back(b);
+  }
+  return e;
+}
+
+// Cut layers 0..n-1 into `chunks` consecutive groups of about equal x + y bytes.
+std::vector<int> chunk_starts(const std::vector<size_t>& xo, const std::vector<size_t>& yo, int n, int chunks) {
+  std::vector<int> starts{0};
+  const double total = (double)(xo[n] + yo[n]);
+  for (int c = 1; c < chunks; ++c) {
+    const double target = total * c / chunks;
+    int i = starts.back() + 1;
+    while (i < n && (double)(xo[i] + yo[i]) < target) ++i;
+    if (i >= n) break;
+    starts.push_back(i);
+  }
+  starts.push_back(n);
+  return starts;
+}
+
+// Host-checkable conditions of a forward call, before any device work.
+lb_status check_call(const lb_layer* layers, int n, int batch, lb_dtype xdt) {
+  if (batch < 1) return LB_ERR_SHAPE;
+  for (int i = 0; i < n; ++i) {
+    const lb_status st = check_layer(layers[i]);
+    if (st != LB_OK) return st;
+  }
+  if (batch <= lb::kMaxBatchDecode) return xdt == LB_F16 ? LB_OK : LB_ERR_UNSUPPORTED;
+  if (xdt != LB_F16 && xdt != LB_BF16) return LB_ERR_UNSUPPORTED;
+  // operand preparation indexes one layer's fp16 copy of x with 32-bit offsets
+  for (int i = 0; i < n; ++i)
+    if ((size_t)batch * layers[i].d_in > ((size_t)1 << 30)) return LB_ERR_SHAPE;
+  if (batch % 128 != 0 && xdt != LB_F16) return LB_ERR_UNSUPPORTED;
+  return LB_OK;
+}
+
+// The forward of a checked call on `st`, with the workspaces of tag base
+// `base`: batch <= 16 on the decode path, a multiple of 128 on the prefill
+// path, any other batch (fp16) the leading multiple of 128 rows through the
+// prefill path and the rest through the decode path in groups of at most 16
+// rows (rows are contiguous in x and y, so a group is an offset view).
+lb_status forward_dispatch(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
+                           lb_dtype xdt, cudaStream_t st, const cudaEvent_t* evs, int n_events, int base) {
+  if (batch <= lb::kMaxBatchDecode)
+    return decode_forward(layers, n, xs, ys, batch, st, evs, n_events, ws_tag(base, 1));
+  if (batch % 128 == 0)
+    return prefill_forward(layers, n, xs, ys, batch, xdt == LB_BF16 ? 1 : 0, st, ws_tag(base, 0));
+  std::vector<const void*> xv(n);
+  std::vector<void*> yv(n);
+  auto views = [&](int r0) {
+    for (int i = 0; i < n; ++i) {
+      xv[i] = static_cast<const unsigned char*>(xs[i]) + (size_t)r0 * layers[i].d_in * 2;
+      yv[i] = static_cast<unsigned char*>(ys[i]) + (size_t)r0 * layers[i].d_out * 2;
+    }
+  };
+  const int m128 = batch / 128 * 128;
+  if (m128 > 0) {
+    const lb_status r = prefill_forward(layers, n, xs, ys, m128, 0, st, ws_tag(base, 0));
+    if (r != LB_OK) return r;
+  }
+  for (int r0 = m128, grp = 0; r0 < batch; r0 += lb::kMaxBatchDecode, ++grp) {
+    views(r0);
+    const int rows = std::min(lb::kMaxBatchDecode, batch - r0);
+    const lb_status r = decode_forward(layers, n, xv.data(), yv.data(), rows, st, r0 == m128 ? evs : nullptr,
+                                       r0 == m128 ? n_events : 0, ws_tag(base, 1 + grp));
+    if (r != LB_OK) return r;
+  }
+  return LB_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -483,49 +613,14 @@ lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, con
                                               void* const* ys, int batch, lb_dtype xdt, void* stream,
                                               void* const* events, int n_events) {
   if (!layers || !xs || !ys || n < 1) return LB_ERR_ARG;
-  if (batch < 1) return LB_ERR_SHAPE;
+  const lb_status chk = check_call(layers, n, batch, xdt);
+  if (chk != LB_OK) return chk;
   for (int i = 0; i < n; ++i) {
-    const lb_status st = check_layer(layers[i]);
-    if (st != LB_OK) return st;
     if (!xs[i] || !ys[i]) return LB_ERR_ARG;
     if (!aligned(xs[i], 16) || !aligned(ys[i], 16)) return LB_ERR_ALIGN;
   }
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const cudaEvent_t* evs = reinterpret_cast<const cudaEvent_t*>(events);
-  if (batch <= lb::kMaxBatchDecode) {
-    if (xdt != LB_F16) return LB_ERR_UNSUPPORTED;
-    return decode_forward(layers, n, xs, ys, batch, st, evs, n_events);
-  }
-  if (xdt != LB_F16 && xdt != LB_BF16) return LB_ERR_UNSUPPORTED;
-  // operand preparation indexes one layer's fp16 copy of x with 32-bit offsets
-  for (int i = 0; i < n; ++i)
-    if ((size_t)batch * layers[i].d_in > ((size_t)1 << 30)) return LB_ERR_SHAPE;
-  if (batch % 128 == 0) return prefill_forward(layers, n, xs, ys, batch, xdt == LB_BF16 ? 1 : 0, st);
-  // Any other batch (fp16): the leading multiple of 128 rows through the
-  // prefill path, the rest through the decode path in groups of at most 16
-  // rows (rows are contiguous in x and y, so a group is an offset view).
-  if (xdt != LB_F16) return LB_ERR_UNSUPPORTED;
-  std::vector<const void*> xv(n);
-  std::vector<void*> yv(n);
-  auto views = [&](int r0) {
-    for (int i = 0; i < n; ++i) {
-      xv[i] = static_cast<const unsigned char*>(xs[i]) + (size_t)r0 * layers[i].d_in * 2;
-      yv[i] = static_cast<unsigned char*>(ys[i]) + (size_t)r0 * layers[i].d_out * 2;
-    }
-  };
-  const int m128 = batch / 128 * 128;
-  if (m128 > 0) {
-    const lb_status r = prefill_forward(layers, n, xs, ys, m128, 0, st);
-    if (r != LB_OK) return r;
-  }
-  for (int r0 = m128; r0 < batch; r0 += lb::kMaxBatchDecode) {
-    views(r0);
-    const int rows = std::min(lb::kMaxBatchDecode, batch - r0);
-    const lb_status r = decode_forward(layers, n, xv.data(), yv.data(), rows, st, r0 == m128 ? evs : nullptr,
-                                       r0 == m128 ? n_events : 0);
-    if (r != LB_OK) return r;
-  }
-  return LB_OK;
+  return forward_dispatch(layers, n, xs, ys, batch, xdt, static_cast<cudaStream_t>(stream),
+                          reinterpret_cast<const cudaEvent_t*>(events), n_events, 0);
 }
 
 lb_status littlebit_linear_forward_many(const lb_layer* layers, int n, const void* const* xs, void* const* ys,
@@ -548,12 +643,19 @@ lb_status littlebit_device_status(void* stream, unsigned int* status) {
   e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e);
   std::lock_guard<std::mutex> lock(g_mu);
-  auto it = g_ws.find({dev, st});
-  if (it == g_ws.end() || !it->second.buf) return LB_OK;
-  e = cudaMemcpy(status, it->second.buf, sizeof(unsigned int), cudaMemcpyDeviceToHost);
-  if (e != cudaSuccess) return cuda_fail(e);
-  e = cudaMemset(it->second.buf, 0, sizeof(unsigned int));
-  if (e != cudaSuccess) return cuda_fail(e);
+  // every workspace of this stream (all tags): their status words, OR-ed
+  for (auto it = g_ws.lower_bound({dev, st, INT_MIN}); it != g_ws.end(); ++it) {
+    if (std::get<0>(it->first) != dev || std::get<1>(it->first) != st) break;
+    if (!it->second.buf) continue;
+    unsigned int bits = 0;
+    e = cudaMemcpy(&bits, it->second.buf, sizeof(bits), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (bits) {
+      e = cudaMemset(it->second.buf, 0, sizeof(unsigned int));
+      if (e != cudaSuccess) return cuda_fail(e);
+    }
+    *status |= bits;
+  }
   return LB_OK;
 }
 
@@ -564,7 +666,7 @@ lb_status littlebit_check_wait_timeout(void* stream, int polls) {
   if (e != cudaSuccess) return cuda_fail(e);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   std::lock_guard<std::mutex> lock(g_mu);
-  Workspace& ws = g_ws[{dev, st}];
+  Workspace& ws = g_ws[{dev, st, ws_tag(0, 1)}];   // the decode workspace of the device API
   if (!ws.buf) {
     // just the status word; a later forward grows the workspace
     const lb_status r = grow_workspace(ws, kStatusBytes, st);
@@ -574,7 +676,108 @@ lb_status littlebit_check_wait_timeout(void* stream, int polls) {
   return e == cudaSuccess ? LB_OK : cuda_fail(e);
 }
 
+lb_status littlebit_linear_forward_many_host(const lb_layer* layers, int n, const void* x_host, void* y_host,
+                                             int batch, lb_dtype xdt, int n_chunks, void* stream) {
+  if (!layers || n < 1 || !x_host || !y_host || n_chunks < 1) return LB_ERR_ARG;
+  const lb_status chk = check_call(layers, n, batch, xdt);
+  if (chk != LB_OK) return chk;
+  n_chunks = std::min(std::min(n_chunks, n), kMaxHostChunks);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_host_mu);
+  HostPipe& hp = g_pipes[{dev, st}];
+
+  // ---- plan: offsets, chunks, device views (reused while the call repeats)
+  std::vector<unsigned char> key((size_t)n * sizeof(lb_layer) + 12);
+  std::memcpy(key.data(), &batch, 4);
+  std::memcpy(key.data() + 4, &xdt, 4);
+  std::memcpy(key.data() + 8, &n_chunks, 4);
+  std::memcpy(key.data() + 12, layers, (size_t)n * sizeof(lb_layer));
+  if (hp.key != key) {
+    hp.key.clear();
+    hp.xo.assign(n + 1, 0);
+    hp.yo.assign(n + 1, 0);
+    for (int i = 0; i < n; ++i) {   // 2-byte elements; d_in % 256 == 0 and d_out % 128 == 0 keep 256-byte steps
+      hp.xo[i + 1] = hp.xo[i] + (size_t)batch * layers[i].d_in * 2;
+      hp.yo[i + 1] = hp.yo[i] + (size_t)batch * layers[i].d_out * 2;
+    }
+    if (hp.x_cap < hp.xo[n] || hp.y_cap < hp.yo[n]) {
+      e = cudaStreamSynchronize(st);   // every earlier call on `st` joined its copies into `st`
+      if (e != cudaSuccess) return cuda_fail(e);
+      if (hp.x_cap < hp.xo[n]) {
+        if (hp.x_dev) cudaFree(hp.x_dev);
+        hp.x_dev = nullptr;
+        hp.x_cap = 0;
+        e = cudaMalloc(&hp.x_dev, hp.xo[n]);
+        if (e != cudaSuccess) return cuda_fail(e);
+        hp.x_cap = hp.xo[n];
+      }
+      if (hp.y_cap < hp.yo[n]) {
+        if (hp.y_dev) cudaFree(hp.y_dev);
+        hp.y_dev = nullptr;
+        hp.y_cap = 0;
+        e = cudaMalloc(&hp.y_dev, hp.yo[n]);
+        if (e != cudaSuccess) return cuda_fail(e);
+        hp.y_cap = hp.yo[n];
+      }
+    }
+    hp.xs.resize(n);
+    hp.ys.resize(n);
+    for (int i = 0; i < n; ++i) {
+      hp.xs[i] = hp.x_dev + hp.xo[i];
+      hp.ys[i] = hp.y_dev + hp.yo[i];
+    }
+    hp.starts = chunk_starts(hp.xo, hp.yo, n, n_chunks);
+    hp.key = key;
+  }
+  const int chunks = (int)hp.starts.size() - 1;
+  e = ensure_pipe_objects(hp, chunks);
+  if (e != cudaSuccess) return cuda_fail(e);
+
+  // ---- enqueue: both copy streams start after everything already on `st`
+  // (so x_dev, y_dev and the host buffers are free), and `st` ends after both
+  e = cudaEventRecord(hp.fork, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(hp.h2d, hp.fork, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(hp.d2h, hp.fork, 0);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const unsigned char* xh = static_cast<const unsigned char*>(x_host);
+  unsigned char* yh = static_cast<unsigned char*>(y_host);
+  lb_status r = LB_OK;
+  for (int c = 0; c < chunks && r == LB_OK; ++c) {
+    const int i0 = hp.starts[c], i1 = hp.starts[c + 1];
+    e = cudaMemcpyAsync(hp.x_dev + hp.xo[i0], xh + hp.xo[i0], hp.xo[i1] - hp.xo[i0], cudaMemcpyHostToDevice,
+                        hp.h2d);
+    if (e == cudaSuccess) e = cudaEventRecord(hp.in_done[c], hp.h2d);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, hp.in_done[c], 0);
+    if (e != cudaSuccess) {
+      r = cuda_fail(e);
+      break;
+    }
+    r = forward_dispatch(layers + i0, i1 - i0, hp.xs.data() + i0, hp.ys.data() + i0, batch, xdt, st, nullptr, 0,
+                         c + 1);
+    if (r != LB_OK) break;
+    e = cudaEventRecord(hp.fwd_done[c], st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hp.d2h, hp.fwd_done[c], 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(yh + hp.yo[i0], hp.y_dev + hp.yo[i0], hp.yo[i1] - hp.yo[i0], cudaMemcpyDeviceToHost,
+                          hp.d2h);
+    if (e != cudaSuccess) r = cuda_fail(e);
+  }
+  // join on every path, so that `st` always covers the copies it started
+  e = cudaEventRecord(hp.join_in, hp.h2d);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, hp.join_in, 0);
+  if (e == cudaSuccess) e = cudaEventRecord(hp.join_out, hp.d2h);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, hp.join_out, 0);
+  if (e != cudaSuccess && r == LB_OK) r = cuda_fail(e);
+  return r;
+}
+
 void littlebit_release(void) {
+  std::lock_guard<std::mutex> host_lock(g_host_mu);
+  for (auto& kv : g_pipes) release_pipe(kv.second);
+  g_pipes.clear();
   std::lock_guard<std::mutex> lock(g_mu);
   for (auto& kv : g_ws) release_workspace(kv.second);
   g_ws.clear();

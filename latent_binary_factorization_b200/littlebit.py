@@ -66,6 +66,10 @@ _lib.littlebit_linear_forward_many_timed.argtypes = [ctypes.POINTER(LbLayer), ct
                                                      ctypes.POINTER(ctypes.c_void_p),
                                                      ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_int,
                                                      ctypes.c_void_p, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]
+_lib.littlebit_linear_forward_many_host.restype = ctypes.c_int
+_lib.littlebit_linear_forward_many_host.argtypes = [ctypes.POINTER(LbLayer), ctypes.c_int, ctypes.c_void_p,
+                                                    ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                    ctypes.c_void_p]
 _lib.littlebit_device_status.restype = ctypes.c_int
 _lib.littlebit_device_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint)]
 _lib.littlebit_check_wait_timeout.restype = ctypes.c_int
@@ -210,6 +214,34 @@ class Stack:
             _check(_lib.littlebit_linear_forward_many_timed(self._arr, self._n, self._xp, self._yp, self.batch,
                                                             self.dtype, _stream(stream), evs, len(events)),
                    "littlebit_linear_forward_many_timed")
+
+
+class HostStack:
+    """A list of independent layers whose activations live in host memory.
+
+    One call copies every layer's input in, runs the stack forward and copies
+    every output back, in ``n_chunks`` groups of layers whose copies overlap
+    the neighbouring groups' kernels.  ``x_host`` holds the layers' inputs
+    back to back (layer i: batch x d_in[i], row-major), ``y_host`` the outputs
+    the same way; both CPU tensors, page-locked (``pin_memory=True``) for the
+    overlap.  y_host is complete once the stream has been synchronised."""
+
+    def __init__(self, layers: list, batch: int, dtype=torch.float16):
+        assert layers and batch >= 1
+        self.layers, self.batch, self.dtype = layers, batch, dtype
+        self._n = len(layers)
+        self._arr = (LbLayer * self._n)(*[L.c_struct() for L in layers])
+        self.x_numel = batch * sum(L.d_in for L in layers)
+        self.y_numel = batch * sum(L.d_out for L in layers)
+
+    def __call__(self, x_host: torch.Tensor, y_host: torch.Tensor, n_chunks: int = 8, stream=None) -> None:
+        for t, numel in ((x_host, self.x_numel), (y_host, self.y_numel)):
+            if t.device.type != "cpu" or not t.is_contiguous() or t.numel() != numel or t.dtype != self.dtype:
+                raise ValueError(f"host buffer must be a contiguous CPU {self.dtype} tensor of {numel} elements")
+        _check(_lib.littlebit_linear_forward_many_host(self._arr, self._n, ctypes.c_void_p(x_host.data_ptr()),
+                                                       ctypes.c_void_p(y_host.data_ptr()), self.batch,
+                                                       _DTYPE[self.dtype], int(n_chunks), _stream(stream)),
+               "littlebit_linear_forward_many_host")
 
 
 def forward_many(layers: list, xs: list, ys: list, stream=None) -> None:

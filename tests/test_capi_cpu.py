@@ -96,6 +96,15 @@ def test_forward_rejects_bad_arguments_without_device_work(lib):
     assert pack(ctypes.c_void_p(16), 9, 4, 4, 4, 1, 0, ctypes.c_void_p(16), None) == 1
     assert pack(ctypes.c_void_p(16), 0, 0, 4, 4, 1, 0, ctypes.c_void_p(16), None) == 3
     assert pack(ctypes.c_void_p(16), 0, 4, 4, 4, 1, 0, ctypes.c_void_p(8), None) == 2
+    host = lb.library().littlebit_linear_forward_many_host
+    hx = ctypes.c_void_p(4096)                                   # never dereferenced: rejected first
+    assert host(ctypes.byref(L), 1, None, hx, 1, 0, 4, None) == 1            # null x_host
+    assert host(ctypes.byref(L), 1, hx, hx, 1, 0, 0, None) == 1              # n_chunks < 1
+    assert host(ctypes.byref(L), 0, hx, hx, 1, 0, 4, None) == 1              # no layers
+    assert host(ctypes.byref(L), 1, hx, hx, 1, 2, 4, None) == 6              # f32 activations
+    L.d_in = 100
+    assert host(ctypes.byref(L), 1, hx, hx, 1, 0, 4, None) == 3              # bad layer shape
+    L.d_in = 256
     chk = lb.library().littlebit_check_wait_timeout
     assert chk(None, 0) == 1                                     # polls < 1
     assert chk(None, (1 << 22) + 1) == 1                         # polls above the kernels' own limit

@@ -1,0 +1,135 @@
+"""GPU parity of the host-buffer stack call (littlebit_linear_forward_many_host):
+inputs copied in from host memory, the stack forward and outputs copied back,
+chunk by chunk, against the fp64 oracle and against the device-pointer call."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import littlebit_oracle as orc
+from latent_binary_factorization_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 2e-3
+MAX_ABS = 1e-2
+
+SPECS = [(4096, 4096, 86, True), (512, 512, 32, False), (4096, 1024, 133, True), (1024, 2048, 45, False),
+         (2048, 512, 200, True)]
+
+
+@pytest.fixture(scope="module")
+def lbm():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from latent_binary_factorization_b200 import layers, littlebit
+    return littlebit, layers
+
+
+def _check(y, y_ref, tag):
+    y = y.float().numpy()
+    e, m = orc.rel_l2(y, y_ref), orc.max_abs_ratio(y, y_ref)
+    assert e <= REL_L2 and m <= MAX_ABS, f"{tag} rel_l2={e:.3e} max_abs_ratio={m:.3e}"
+
+
+def _stack(lbm, specs, batch, seed):
+    _, layers = lbm
+    L, xs, paths_all = [], [], []
+    for i, (a, b, s, r) in enumerate(specs):
+        paths = synth.layer(a, b, s, r, seed=seed + i, index=i)
+        L.append(layers.upload(paths, a, b, s))
+        xs.append(synth.activations(batch, a, seed=seed + i, index=i))
+        paths_all.append(paths)
+    return L, xs, paths_all
+
+
+def _host(arrs, dtype, pinned):
+    flat = np.concatenate([a.reshape(-1) for a in arrs]).astype(np.float32)
+    t = torch.from_numpy(flat).to(dtype)
+    return t.pin_memory() if pinned else t
+
+
+def _split(y_host, specs, batch):
+    out, o = [], 0
+    for (_, b, _, _) in specs:
+        out.append(y_host[o:o + batch * b].view(batch, b))
+        o += batch * b
+    return out
+
+
+@pytest.mark.parametrize("batch", [1, 3])
+@pytest.mark.parametrize("n_chunks", [1, 3, 64])
+@pytest.mark.parametrize("pinned", [True, False])
+def test_host_stack_matches_oracle(lbm, batch, n_chunks, pinned):
+    lb, _ = lbm
+    L, xs, paths = _stack(lbm, SPECS, batch, seed=500)
+    refs = [orc.factored_forward(x, p) for x, p in zip(xs, paths)]
+    xh = _host(xs, torch.float16, pinned)
+    yh = torch.full((batch * sum(b for _, b, _, _ in SPECS),), float("nan"), dtype=torch.float16)
+    yh = yh.pin_memory() if pinned else yh
+    hs = lb.HostStack(L, batch)
+    for rep in range(2):            # the second call reuses the plan and the device copies
+        yh.fill_(float("nan"))
+        hs(xh, yh, n_chunks=n_chunks)
+        torch.cuda.synchronize()
+        for i, (y, ref) in enumerate(zip(_split(yh, SPECS, batch), refs)):
+            _check(y, ref, f"rep {rep} layer {i}")
+    assert lb.device_status() == 0
+
+
+def test_host_stack_equals_device_stack_and_follows_new_inputs(lbm):
+    """One chunk runs exactly the device-pointer call's kernels: identical
+    bits.  New host contents at the same addresses give the new outputs."""
+    lb, _ = lbm
+    batch = 2
+    L, xs, paths = _stack(lbm, SPECS, batch, seed=600)
+    X = [torch.from_numpy(x).cuda() for x in xs]
+    Y = [torch.empty(batch, b, dtype=torch.float16, device="cuda") for _, b, _, _ in SPECS]
+    lb.Stack(L, X, Y)()
+    torch.cuda.synchronize()
+    xh = _host(xs, torch.float16, True)
+    yh = torch.empty(batch * sum(b for _, b, _, _ in SPECS), dtype=torch.float16).pin_memory()
+    hs = lb.HostStack(L, batch)
+    hs(xh, yh, n_chunks=1)
+    torch.cuda.synchronize()
+    for i, (y, yd) in enumerate(zip(_split(yh, SPECS, batch), Y)):
+        assert torch.equal(y, yd.cpu()), f"layer {i}"
+    xs2 = [synth.activations(batch, a, seed=700 + i, index=i) for i, (a, _, _, _) in enumerate(SPECS)]
+    xh.copy_(_host(xs2, torch.float16, False))
+    hs(xh, yh, n_chunks=4)
+    torch.cuda.synchronize()
+    for i, (y, x2, p) in enumerate(zip(_split(yh, SPECS, batch), xs2, paths)):
+        _check(y, orc.factored_forward(x2, p), f"new inputs, layer {i}")
+
+
+def test_host_stack_prefill_bf16(lbm):
+    lb, _ = lbm
+    batch = 128
+    specs = [(1024, 512, 100, True), (512, 1024, 64, False), (768, 384, 40, True)]
+    L, xs, paths = _stack(lbm, specs, batch, seed=800)
+    xh = _host(xs, torch.bfloat16, True)
+    yh = torch.empty(batch * sum(b for _, b, _, _ in specs), dtype=torch.bfloat16).pin_memory()
+    lb.HostStack(L, batch, torch.bfloat16)(xh, yh, n_chunks=2)
+    torch.cuda.synchronize()
+    for i, (y, x, p) in enumerate(zip(_split(yh, specs, batch), _split_in(xh, specs, batch), paths)):
+        _check(y, orc.factored_forward(x, p), f"prefill layer {i}")
+    assert lb.device_status() == 0
+
+
+def _split_in(x_host, specs, batch):
+    """The inputs exactly as the GPU saw them (after rounding to bf16), fp64."""
+    out, o = [], 0
+    for (a, _, _, _) in specs:
+        out.append(x_host[o:o + batch * a].view(batch, a).double().numpy())
+        o += batch * a
+    return out
+
+
+def test_host_stack_rejects_bad_buffers(lbm):
+    lb, _ = lbm
+    L, xs, _ = _stack(lbm, SPECS[:2], 1, seed=900)
+    hs = lb.HostStack(L, 1)
+    xh = _host(xs, torch.float16, False)
+    with pytest.raises(ValueError):
+        hs(xh[:-1], torch.empty(1024, dtype=torch.float16))
+    with pytest.raises(lb.LittleBitError):
+        hs(xh, torch.empty(hs.y_numel, dtype=torch.float16), n_chunks=0)
