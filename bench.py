@@ -242,6 +242,43 @@ def time_device(stack, steps, warmup, dist):
     return total_ms, per
 
 
+def measure_mixed(name, batch, steps, warmup, device, dist, l2, seed=4321):
+    """A batch between the decode and prefill ranges (fp16): the leading
+    multiple of 128 rows run on the prefill path and the rest on the decode
+    path in groups of at most 16 rows, each group streaming the weights again.
+    Whole-step time only (the per-kernel event split is a decode-only view)."""
+    import torch
+    mats = WORKLOADS[name]["mats"]
+    reps = stack_reps_for_l2(mats, batch, l2)
+    stack, Ls, x_all, y_all = build_stack(mats, reps, batch, seed, device)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        stack()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if dist:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(steps):
+        stack()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        torch.distributed.barrier()
+    ms = max_over_ranks([t0.elapsed_time(t1) / steps], device)[0]
+    alg = sum(algorithmic_bytes(*m, batch) for m in mats) * reps
+    prefill_rows = batch // 128 * 128
+    res = {"workload": name, "desc": WORKLOADS[name]["desc"], "batch": batch, "layers_per_step": len(Ls),
+           "prefill_rows": prefill_rows, "decode_groups": -(-(batch - prefill_rows) // 16),
+           "ms_per_step": ms, "us_per_matrix": 1e3 * ms / len(Ls),
+           "us_per_matrix_row": 1e3 * ms / len(Ls) / batch,
+           "step_gbs_algorithmic": alg / (ms * 1e-3) / 1e9}
+    del stack, x_all, y_all
+    torch.cuda.empty_cache()
+    return res
+
+
 def measure_latency(device, reps=200, seed=99):
     """Latency view: one Llama-2-7B attention projection (4096x4096, 0.1 BPW
     residual, s = 86 x 2) at batch 1 per call, its 0.1 MB of weights staying
@@ -404,6 +441,9 @@ def run_ours(args):
             torch.cuda.empty_cache()
             r["roofline_frac_step"] = r["step_gbs"] / peak
             extras[f"{name}_b{b}"] = r
+        for b in (40, 130):
+            extras[f"7b_attn_0.1bpw_residual_b{b}_mixed"] = measure_mixed(
+                "7b_attn_0.1bpw_residual", b, max(5, args.steps // 4), args.warmup, device, dist, l2)
         extras["latency_single_layer"] = measure_latency(device)
     prefill = None
     if not args.no_prefill:
