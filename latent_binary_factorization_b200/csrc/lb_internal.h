@@ -168,16 +168,18 @@ constexpr int kPrefillMaxGroup = 4096;   // layers per chunk
 struct PrefillPlan {
   int n;
   int tiles1, tiles2, grid1, grid2;
+  int prep_grid[3];              // blocks of the grouped x, B1 and B2 preparation launches
   size_t table_off, table_bytes;
+  size_t jobs_off;               // preparation jobs, from table_off
 };
-// Append the chunk's table image (problems and tile schedules) to img; its
-// device pointers refer to the chunk's operand buffers at `bufs`.
-void plan_prefill_chunk(const LayerDesc* Ls, void* const* ys, int n, int M, int x_bf16, unsigned char* bufs,
-                        int num_sms, std::vector<unsigned char>& img, PrefillPlan& plan);
-// A chunk's operand preparation (buffers at `bufs`), then its two grouped
-// GEMM launches (table image uploaded at table_dev).
-cudaError_t launch_prefill_prep(const LayerDesc* Ls, const void* const* xs, int n, int M, int x_bf16,
-                                unsigned char* bufs, cudaStream_t st);
+// Append the chunk's table image (GEMM problems, tile schedules and the
+// per-layer preparation jobs) to img; its device pointers refer to the
+// chunk's operand buffers at `bufs`, the inputs xs and the outputs ys.
+void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const* ys, int n, int M, int x_bf16,
+                        unsigned char* bufs, int num_sms, std::vector<unsigned char>& img, PrefillPlan& plan);
+// A chunk's operand preparation (three grouped launches), then its two
+// grouped GEMM launches; both read the table image uploaded at table_dev.
+cudaError_t launch_prefill_prep(const PrefillPlan& plan, const unsigned char* table_dev, cudaStream_t st);
 cudaError_t launch_prefill_gemms(const PrefillPlan& plan, const unsigned char* table_dev, unsigned int* status,
                                  cudaStream_t st);
 

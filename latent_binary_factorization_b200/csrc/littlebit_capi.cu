@@ -42,10 +42,7 @@ struct Workspace {
   std::vector<unsigned char> key;
   lb::DecodeArgs dargs{};
   int d_max_s16 = 16;
-  std::vector<lb::LayerDesc> p_descs;
   std::vector<lb::PrefillPlan> p_plans;
-  std::vector<int> p_starts;
-  size_t p_tables = 0, p_half = 0;
 };
 
 // Call arguments that determine a forward's tables and plans.
@@ -321,7 +318,7 @@ cudaError_t ensure_side(Workspace& ws) {
   return cudaSuccess;
 }
 
-lb_status prefill_launch(Workspace& ws, const void* const* xs, int batch, int x_bf16, cudaStream_t st);
+lb_status prefill_launch(Workspace& ws, cudaStream_t st);
 
 lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
                           int x_bf16, cudaStream_t st, int tag) {
@@ -331,7 +328,7 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
   std::lock_guard<std::mutex> lock(g_mu);
   Workspace& ws = g_ws[{dev, st, tag}];
   std::vector<unsigned char> key = call_key('P', layers, n, xs, ys, batch, x_bf16);
-  if (ws.buf && ws.key == key) return prefill_launch(ws, xs, batch, x_bf16, st);
+  if (ws.buf && ws.key == key) return prefill_launch(ws, st);
   ws.key.clear();
   // plan the chunks: operand bytes per chunk (a workspace half) and table bytes
   std::vector<int> starts;
@@ -394,8 +391,8 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
   std::vector<unsigned char> img;
   std::vector<lb::PrefillPlan> plans(n_chunks);
   for (int c = 0; c < n_chunks; ++c)
-    lb::plan_prefill_chunk(descs.data() + starts[c], ys + starts[c], starts[c + 1] - starts[c], batch, x_bf16,
-                           chunk_bufs(c), sms, img, plans[c]);
+    lb::plan_prefill_chunk(descs.data() + starts[c], xs + starts[c], ys + starts[c], starts[c + 1] - starts[c],
+                           batch, x_bf16, chunk_bufs(c), sms, img, plans[c]);
   if (img.size() > tables) return LB_ERR_SHAPE;   // the plan above sized the tables
   if (ws.table.size() != img.size() || std::memcmp(ws.table.data(), img.data(), img.size()) != 0) {
     // pageable source: the copy is staged before the call returns
@@ -403,27 +400,20 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
     if (e != cudaSuccess) return cuda_fail(e);
     ws.table.swap(img);
   }
-  ws.p_descs.swap(descs);
   ws.p_plans.swap(plans);
-  ws.p_starts.swap(starts);
-  ws.p_tables = tables;
-  ws.p_half = half;
   ws.key.swap(key);
-  return prefill_launch(ws, xs, batch, x_bf16, st);
+  return prefill_launch(ws, st);
 }
 
-// The launches of a planned prefill call (plans, descriptors and tables in ws).
-lb_status prefill_launch(Workspace& ws, const void* const* xs, int batch, int x_bf16, cudaStream_t st) {
+// The launches of a planned prefill call (plans and tables in ws).
+lb_status prefill_launch(Workspace& ws, cudaStream_t st) {
   unsigned char* base = static_cast<unsigned char*>(ws.buf);
   unsigned int* status = reinterpret_cast<unsigned int*>(base);
   unsigned char* table_dev = base + kStatusBytes;
-  auto chunk_bufs = [&](int c) { return base + kStatusBytes + ws.p_tables + (size_t)(c & 1) * ws.p_half; };
   const int n_chunks = (int)ws.p_plans.size();
-  const lb::LayerDesc* descs = ws.p_descs.data();
-  const std::vector<int>& starts = ws.p_starts;
   cudaError_t e;
   if (n_chunks == 1) {
-    e = lb::launch_prefill_prep(descs, xs, starts[1], batch, x_bf16, chunk_bufs(0), st);
+    e = lb::launch_prefill_prep(ws.p_plans[0], table_dev, st);
     if (e != cudaSuccess) return cuda_fail(e);
     e = lb::launch_prefill_gemms(ws.p_plans[0], table_dev, status, st);
     return e == cudaSuccess ? LB_OK : cuda_fail(e);
@@ -435,10 +425,10 @@ lb_status prefill_launch(Workspace& ws, const void* const* xs, int batch, int x_
   if (e == cudaSuccess) e = cudaStreamWaitEvent(ws.side, ws.fork, 0);
   if (e != cudaSuccess) return cuda_fail(e);
   for (int c = 0; c < n_chunks && e == cudaSuccess; ++c) {
-    const int i0 = starts[c], cn = starts[c + 1] - starts[c], h = c & 1;
+    const int h = c & 1;
     // the half was last used by chunk c - 2's GEMMs
     if (c >= 2) e = cudaStreamWaitEvent(ws.side, ws.gemm_done[h], 0);
-    if (e == cudaSuccess) e = lb::launch_prefill_prep(descs + i0, xs + i0, cn, batch, x_bf16, chunk_bufs(c), ws.side);
+    if (e == cudaSuccess) e = lb::launch_prefill_prep(ws.p_plans[c], table_dev, ws.side);
     if (e == cudaSuccess) e = cudaEventRecord(ws.prep_done[h], ws.side);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ws.prep_done[h], 0);
     if (e == cudaSuccess) e = lb::launch_prefill_gemms(ws.p_plans[c], table_dev, status, st);

@@ -26,6 +26,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <cstring>
 #include <functional>
 #include <queue>
 #include <utility>
@@ -155,12 +156,15 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
   return v;
 }
 
-__global__ void __launch_bounds__(256) prep_x_kernel(const uint16_t* __restrict__ x, int is_bf16, int M, int K,
-                                                     unsigned char* __restrict__ out) {
+// The three preparation steps below each run as one grouped launch over all
+// layers of a chunk: a layer owns a contiguous range of blocks (PrepJob) and
+// its step runs with block `bid` of `nblk` in place of blockIdx/gridDim.
+__device__ __forceinline__ void prep_x(const uint16_t* __restrict__ x, int is_bf16, int M, int K,
+                                       unsigned char* __restrict__ out, unsigned bid, unsigned nblk) {
   const unsigned n16 = (unsigned)((size_t)M * K / 8);   // < 2^32 for the shapes accepted
   const unsigned rgs = (unsigned)M >> 3;
-  const unsigned stride = gridDim.x * blockDim.x;
-  for (unsigned t0 = blockIdx.x * blockDim.x + threadIdx.x; t0 < n16; t0 += stride * kXUnroll) {
+  const unsigned stride = nblk * blockDim.x;
+  for (unsigned t0 = bid * blockDim.x + threadIdx.x; t0 < n16; t0 += stride * kXUnroll) {
     uint4 v[kXUnroll];
     unsigned dst[kXUnroll];
 #pragma unroll
@@ -189,14 +193,15 @@ __global__ void __launch_bounds__(256) prep_x_kernel(const uint16_t* __restrict_
 // core-matrix rows.  Rows j >= s inside the packed tiles get +-g (finite;
 // GEMM1's epilogue zeroes them through l); rows from the tiles' end up to Sp
 // are zero.
-__global__ void __launch_bounds__(256) prep_b1_kernel(const LayerDesc L, int Sp, unsigned char* __restrict__ out) {
+__device__ __forceinline__ void prep_b1(const LayerDesc& L, int Sp, unsigned char* __restrict__ out, unsigned bid,
+                                        unsigned nblk) {
   const int R = L.npaths * Sp, K = L.d_in;
   const int n_kt = K / kVTileK, n_rb = (L.s + 15) >> 4;
   const unsigned tiles_p = (unsigned)(n_rb * n_kt);
   const unsigned units = (unsigned)L.npaths * tiles_p * 256;
   const unsigned zrow16 = (unsigned)(K / 8);                    // 16-byte pieces per zero row
   const unsigned zeros = (unsigned)(L.npaths * (Sp - 16 * n_rb)) * zrow16;
-  for (unsigned t = blockIdx.x * blockDim.x + threadIdx.x; t < units + zeros; t += gridDim.x * blockDim.x) {
+  for (unsigned t = bid * blockDim.x + threadIdx.x; t < units + zeros; t += nblk * blockDim.x) {
     if (t < units) {
       const int lane = t & 31, r = (t >> 5) & 3, qh = (t >> 7) & 1;
       const unsigned tile = t >> 8;
@@ -233,7 +238,8 @@ __global__ void __launch_bounds__(256) prep_b1_kernel(const LayerDesc L, int Sp,
 // unit = (16-byte lane of a packed role-U tile, word r, half qh of the eight
 // products): for each of its four q the word gives four consecutive j of one
 // row.  Columns from the tiles' end up to Sp are zero.
-__global__ void __launch_bounds__(256) prep_b2_kernel(const LayerDesc L, int Sp, unsigned char* __restrict__ out) {
+__device__ __forceinline__ void prep_b2(const LayerDesc& L, int Sp, unsigned char* __restrict__ out, unsigned bid,
+                                        unsigned nblk) {
   const int R = L.d_out;
   const int n_kt = (L.s + 31) >> 5, n_ob = R / kUTileRows;
   const unsigned tiles_p = (unsigned)(n_ob * n_kt);
@@ -241,7 +247,7 @@ __global__ void __launch_bounds__(256) prep_b2_kernel(const LayerDesc L, int Sp,
   const int zc8 = (Sp - 32 * n_kt) / 8;                    // zero 16-byte pieces per row and path
   const unsigned per = (unsigned)(R * zc8);
   const unsigned zeros = (unsigned)L.npaths * per;
-  for (unsigned t = blockIdx.x * blockDim.x + threadIdx.x; t < units + zeros; t += gridDim.x * blockDim.x) {
+  for (unsigned t = bid * blockDim.x + threadIdx.x; t < units + zeros; t += nblk * blockDim.x) {
     if (t < units) {
       const int lane = t & 31, r = (t >> 5) & 3, qh = (t >> 7) & 1;
       const unsigned tile = t >> 8;
@@ -271,6 +277,40 @@ __global__ void __launch_bounds__(256) prep_b2_kernel(const LayerDesc L, int Sp,
       *reinterpret_cast<uint4*>(out + tiled_off(o, j, R)) = make_uint4(0u, 0u, 0u, 0u);
     }
   }
+}
+
+// One layer of a chunk in the grouped preparation launches: its arguments and
+// the first block it owns in each of the three launches (blocks first[k] up to
+// the next layer's first[k], or the grid's end, belong to it).
+struct PrepJob {
+  LayerDesc L;
+  const uint16_t* x;
+  unsigned char *X16, *B1, *B2;
+  int M, x_bf16, Sp;
+  int first[3];   // 0: x, 1: B1, 2: B2
+};
+
+// The job that owns block b of launch k: the last one whose first[k] <= b.
+__device__ __forceinline__ int prep_job_of(const PrepJob* jobs, int n, int k, unsigned b) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((unsigned)jobs[mid].first[k] <= b) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(256) prep_group_kernel(const PrepJob* __restrict__ jobs, int n) {
+  const int j = prep_job_of(jobs, n, KIND, blockIdx.x);
+  const PrepJob& J = jobs[j];
+  const unsigned b0 = (unsigned)J.first[KIND];
+  const unsigned b1 = j + 1 < n ? (unsigned)jobs[j + 1].first[KIND] : gridDim.x;
+  const unsigned bid = blockIdx.x - b0, nblk = b1 - b0;
+  if (KIND == 0) prep_x(J.x, J.x_bf16, J.M, J.L.d_in, J.X16, bid, nblk);
+  else if (KIND == 1) prep_b1(J.L, J.Sp, J.B1, bid, nblk);
+  else prep_b2(J.L, J.Sp, J.B2, bid, nblk);
 }
 
 // ------------------------------------------------------------------ grouped persistent tcgen05 GEMM
@@ -518,9 +558,16 @@ long long prefill_layer_tiles(int M, int d_out, int s, int npaths) {
   return (long long)(M / kBM) * (ceil_div(NK, kBN) + ceil_div(d_out, kBN));
 }
 
-size_t prefill_table_bytes(int n_layers, long long tiles) {
+// Offset of the PrepJob array inside a chunk's table (after the problems,
+// the two CTA offset arrays and the tile lists), 16-byte aligned.
+static size_t prep_jobs_off(int n_layers, long long tiles) {
   const size_t b = (size_t)2 * n_layers * sizeof(GemmProblem) + (size_t)2 * (kMaxGemmGrid + 1) * sizeof(int) +
                    (size_t)tiles * sizeof(int);
+  return (b + 15) & ~(size_t)15;
+}
+
+size_t prefill_table_bytes(int n_layers, long long tiles) {
+  const size_t b = prep_jobs_off(n_layers, tiles) + (size_t)n_layers * sizeof(PrepJob);
   return (b + 1023) & ~(size_t)1023;
 }
 
@@ -548,23 +595,25 @@ static LayerBufs layer_bufs(unsigned char*& buf, const LayerDesc& L, int M) {
   return b;
 }
 
-// Operand preparation of a chunk of layers (three launches per layer).
-cudaError_t launch_prefill_prep(const LayerDesc* Ls, const void* const* xs, int n, int M, int x_bf16,
-                                unsigned char* bufs, cudaStream_t st) {
-  unsigned char* buf = bufs;
-  for (int i = 0; i < n; ++i) {
-    const LayerDesc& L = Ls[i];
-    const int P = L.npaths, Sp = prefill_sp(L.s, P);
-    const LayerBufs b = layer_bufs(buf, L, M);
-    prep_x_kernel<<<grid_for((long long)M * L.d_in / 8 / kXUnroll, 256), 256, 0, st>>>(
-        static_cast<const uint16_t*>(xs[i]), x_bf16, M, L.d_in, b.X16);
-    const long long l1 = (long long)P * ((L.s + 15) >> 4) * (L.d_in / kVTileK) * 256 +
-                         (long long)P * (Sp - 16 * ((L.s + 15) >> 4)) * (L.d_in / 8);
-    prep_b1_kernel<<<grid_for(l1, 256), 256, 0, st>>>(L, Sp, b.B1);
-    const long long l2 = (long long)P * (L.d_out / kUTileRows) * ((L.s + 31) >> 5) * 256 +
-                         (long long)P * L.d_out * ((Sp - 32 * ((L.s + 31) >> 5)) / 8);
-    prep_b2_kernel<<<grid_for(l2, 256), 256, 0, st>>>(L, Sp, b.B2);
-  }
+// Blocks of one layer's preparation steps (x, B1, B2), as for a launch of its own.
+static void prep_blocks(const LayerDesc& L, int M, int Sp, int (&blocks)[3]) {
+  const int P = L.npaths;
+  blocks[0] = grid_for((long long)M * L.d_in / 8 / kXUnroll, 256);
+  const long long l1 = (long long)P * ((L.s + 15) >> 4) * (L.d_in / kVTileK) * 256 +
+                       (long long)P * (Sp - 16 * ((L.s + 15) >> 4)) * (L.d_in / 8);
+  blocks[1] = grid_for(l1, 256);
+  const long long l2 = (long long)P * (L.d_out / kUTileRows) * ((L.s + 31) >> 5) * 256 +
+                       (long long)P * L.d_out * ((Sp - 32 * ((L.s + 31) >> 5)) / 8);
+  blocks[2] = grid_for(l2, 256);
+}
+
+// Operand preparation of a planned chunk: three grouped launches (x, B1, B2)
+// over all its layers, arguments in the chunk's table at table_dev.
+cudaError_t launch_prefill_prep(const PrefillPlan& plan, const unsigned char* table_dev, cudaStream_t st) {
+  const PrepJob* jobs = reinterpret_cast<const PrepJob*>(table_dev + plan.table_off + plan.jobs_off);
+  prep_group_kernel<0><<<plan.prep_grid[0], 256, 0, st>>>(jobs, plan.n);
+  prep_group_kernel<1><<<plan.prep_grid[1], 256, 0, st>>>(jobs, plan.n);
+  prep_group_kernel<2><<<plan.prep_grid[2], 256, 0, st>>>(jobs, plan.n);
   return cudaGetLastError();
 }
 
@@ -602,14 +651,17 @@ static double tile_cost(int K, int n_len) { return (double)(K / kBK) * (double)m
 // 2n problems | begin1 | begin2 | sched1 | sched2.  Device pointers in it refer
 // to the chunk's buffers at `bufs` and to the image's own place at
 // table_dev + plan.table_off.
-void plan_prefill_chunk(const LayerDesc* Ls, void* const* ys, int n, int M, int x_bf16, unsigned char* bufs,
-                        int num_sms, std::vector<unsigned char>& img, PrefillPlan& plan) {
+void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const* ys, int n, int M, int x_bf16,
+                        unsigned char* bufs, int num_sms, std::vector<unsigned char>& img, PrefillPlan& plan) {
   const long long tiles_all = group_tiles(Ls, n, M);
   plan.n = n;
   plan.table_off = (img.size() + 1023) & ~(size_t)1023;
   plan.table_bytes = prefill_table_bytes(n, tiles_all);
+  plan.jobs_off = prep_jobs_off(n, tiles_all);
   img.resize(plan.table_off + plan.table_bytes, 0);
   unsigned char* base = img.data() + plan.table_off;
+  PrepJob* jobs = reinterpret_cast<PrepJob*>(base + plan.jobs_off);
+  plan.prep_grid[0] = plan.prep_grid[1] = plan.prep_grid[2] = 0;
   const size_t prob_b = (size_t)2 * n * sizeof(GemmProblem);
   GemmProblem* probs = reinterpret_cast<GemmProblem*>(base);
   int* begin1 = reinterpret_cast<int*>(base + prob_b);
@@ -622,6 +674,18 @@ void plan_prefill_chunk(const LayerDesc* Ls, void* const* ys, int n, int M, int 
     const LayerDesc& L = Ls[i];
     const int P = L.npaths, Sp = prefill_sp(L.s, P), NK = P * Sp;
     const LayerBufs b = layer_bufs(buf, L, M);
+    PrepJob& J = jobs[i];
+    std::memset(&J, 0, sizeof(J));
+    J.L = L;
+    J.x = static_cast<const uint16_t*>(xs[i]);
+    J.X16 = b.X16; J.B1 = b.B1; J.B2 = b.B2;
+    J.M = M; J.x_bf16 = x_bf16; J.Sp = Sp;
+    int blocks[3];
+    prep_blocks(L, M, Sp, blocks);
+    for (int k = 0; k < 3; ++k) {
+      J.first[k] = plan.prep_grid[k];
+      plan.prep_grid[k] += blocks[k];
+    }
     GemmProblem& g1 = probs[i];
     g1 = GemmProblem{};
     g1.A = b.X16; g1.B = b.B1; g1.M = M; g1.N = NK; g1.K = L.d_in; g1.mode = 0;
