@@ -158,7 +158,7 @@ lb_status littlebit_linear_forward(const lb_layer* layer, const void* x_dev, voi
  * The same forward for n independent layers (each with its own input and
  * output buffer, e.g. every linear layer of a model stack), done by the same
  * launches for the whole list (decode: the four passes; prefill: operand
- * preparation per layer and two grouped GEMM launches per group of layers),
+ * preparation and two grouped GEMM launches per group of layers),
  * so that the weights of all layers stream from HBM back to back.  layers, xs,
  * ys are host arrays of length n.
  *
