@@ -261,8 +261,9 @@ lb_status littlebit_device_status(void* stream, unsigned int* status);
  */
 lb_status littlebit_check_wait_timeout(void* stream, int polls);
 
-/* Free every workspace of every device, with its side stream and events (call
- * with no work in flight on any stream the library was given). */
+/* Free every workspace of every device, with its side stream and events, and
+ * the device copies, copy streams and events of the host-buffer stack call
+ * (call with no work in flight on any stream the library was given). */
 void littlebit_release(void);
 
 /* Human-readable name of a status code (static string). */
