@@ -102,6 +102,19 @@ def _stream(stream=None) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _activation(t: torch.Tensor, rows: int | None, cols: int, name: str) -> None:
+    """A row-major (rows x cols) CUDA activation buffer: the library reads and
+    writes it through a raw pointer, so a CPU tensor or a strided view would
+    be misread."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != 2 or t.shape[1] != cols or (rows is not None and t.shape[0] != rows):
+        raise ValueError(f"{name} must have shape ({rows if rows is not None else 'batch'}, {cols}), "
+                         f"got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
 def library():
     """The loaded ctypes CDLL (for tests that call the C ABI directly)."""
     return _lib
@@ -164,6 +177,12 @@ class Layer:
         return len(self.paths) == 2
 
     def c_struct(self) -> LbLayer:
+        if len(self.paths) not in (1, 2):
+            raise ValueError("a layer has one path, or two with residual compensation")
+        for p in self.paths:
+            for name in ("V_bits", "U_bits", "h", "g", "l"):
+                if not getattr(p, name).is_cuda:
+                    raise ValueError(f"path tensor {name} must be a CUDA tensor")
         L = LbLayer()
         L.d_in, L.d_out, L.s, L.residual = self.d_in, self.d_out, self.s, int(self.residual)
         for i, p in enumerate(self.paths):
@@ -174,9 +193,13 @@ class Layer:
 
 def forward(layer: Layer, x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """y = layer(x); x is (batch, d_in) fp16 (decode) on the layer's device."""
+    _activation(x, None, layer.d_in, "x")
     batch = x.shape[0]
     if y is None:
         y = torch.empty((batch, layer.d_out), dtype=x.dtype, device=x.device)
+    _activation(y, batch, layer.d_out, "y")
+    if y.dtype != x.dtype:
+        raise ValueError("y must have x's dtype")
     L = layer.c_struct()
     _check(_lib.littlebit_linear_forward(ctypes.byref(L), ctypes.c_void_p(x.data_ptr()),
                                          ctypes.c_void_p(y.data_ptr()), batch, _DTYPE[x.dtype], _stream(stream)),
@@ -191,9 +214,15 @@ class Stack:
     do no Python-side allocation."""
 
     def __init__(self, layers: list, xs: list, ys: list):
-        assert len(layers) == len(xs) == len(ys) and layers
+        if not layers or not len(layers) == len(xs) == len(ys):
+            raise ValueError("layers, xs and ys must be non-empty lists of the same length")
         self.layers, self.xs, self.ys = layers, xs, ys
         self.batch = xs[0].shape[0]
+        for i, (L, x, y) in enumerate(zip(layers, xs, ys)):
+            _activation(x, self.batch, L.d_in, f"xs[{i}]")
+            _activation(y, self.batch, L.d_out, f"ys[{i}]")
+            if x.dtype != xs[0].dtype or y.dtype != x.dtype:
+                raise ValueError(f"xs[{i}] and ys[{i}] must share xs[0]'s dtype")
         self.dtype = _DTYPE[xs[0].dtype]
         n = len(layers)
         self._n = n

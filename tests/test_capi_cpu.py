@@ -129,3 +129,25 @@ def test_header_compiles_as_c_and_links(tmp_path):
     assert int(out[1].split()[1]) == orc.packed_nbytes("V", 86, 4096)
     assert out[2] == "forward 3"
     assert out[3].startswith("status LB_ERR_SHAPE")
+
+
+def test_binding_rejects_buffers_the_library_would_misread():
+    """CPU tensors, strided views and wrong shapes are refused in Python,
+    before a pointer reaches the library (a host pointer would fault a kernel)."""
+    import torch
+    from latent_binary_factorization_b200 import littlebit as lb
+    z = torch.zeros(16, dtype=torch.uint8)
+    s16 = torch.zeros(256, dtype=torch.float16)
+    layer = lb.Layer(256, 128, 4, [lb.Path(z, z, s16[:128], s16, s16[:4])])
+    with pytest.raises(ValueError):
+        layer.c_struct()                                       # path tensors on the CPU
+    with pytest.raises(ValueError):
+        lb.forward(layer, torch.zeros(1, 256, dtype=torch.float16))   # x on the CPU
+    with pytest.raises(ValueError):
+        lb.Stack([layer], [], [])                              # lengths differ
+    with pytest.raises(ValueError):
+        lb.Stack([layer], [torch.zeros(1, 256, dtype=torch.float16)], [torch.zeros(1, 128, dtype=torch.float16)])
+    with pytest.raises(ValueError):
+        lb.Layer(256, 128, 4, []).c_struct()                   # no path
+    with pytest.raises(ValueError):
+        lb.HostStack([layer], 1)                               # path tensors on the CPU
