@@ -14,5 +14,7 @@ int main(void) {
   printf("packed_bytes %zu\n", littlebit_packed_bytes(LB_ROLE_V, 86, 4096));
   printf("forward %d\n", (int)littlebit_linear_forward(&L, (const void*)16, (void*)16, 1, LB_F16, NULL));
   printf("status %s\n", littlebit_status_string(LB_ERR_SHAPE));
+  /* host-buffer stack call: NULL host buffers are refused before device work */
+  printf("host %d\n", (int)littlebit_linear_forward_many_host(&L, 1, NULL, NULL, 1, LB_F16, 4, NULL));
   return 0;
 }

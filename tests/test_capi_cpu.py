@@ -129,6 +129,7 @@ def test_header_compiles_as_c_and_links(tmp_path):
     assert int(out[1].split()[1]) == orc.packed_nbytes("V", 86, 4096)
     assert out[2] == "forward 3"
     assert out[3].startswith("status LB_ERR_SHAPE")
+    assert out[4] == "host 1"
 
 
 def test_binding_rejects_buffers_the_library_would_misread():
