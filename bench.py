@@ -2,11 +2,13 @@
 """Benchmark of the LittleBit layer forward on B200; prints ONE JSON line.
 
 Default workload (one "step" = one forward over a stack of layers, batch 1):
-Llama-2-7B attention projection 4096 -> 4096 at 0.1 BPW with residual
-compensation (s = 86, two paths), replicated as distinct layers (own signs,
-scales, input and output) until the packed bytes exceed 4x the L2 cache, so
-that every step streams its weights from HBM.  The metric is microseconds per
-layer; the roofline object reports the dominant kernel's achieved HBM GB/s.
+the Llama-2-70B MLP stack at 0.1 BPW, single path s = 620 (8192 -> 28672 gate
+and up, 28672 -> 8192 down per model layer), 80 distinct model layers (own
+signs, scales, input and output; 722 MB of packed weights, 5.7x the L2 cache),
+so that every step streams its weights from HBM.  The metric is microseconds
+per model layer; the roofline object reports the dominant kernel's achieved
+HBM GB/s.  The residual variant of the same stack, the Llama-2-7B full linear
+stack and the prefill stack are reported as secondary figures.
 
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload (the only other place that runs the oracle).
@@ -42,16 +44,20 @@ WORKLOADS = {
     "70b_mlp_0.1bpw_single": {
         "desc": "Llama-2-70B MLP layer (8192->28672 gate, up; 28672->8192 down), 0.1 BPW single path s=620",
         "mats": [(8192, 28672, 620, False), (8192, 28672, 620, False), (28672, 8192, 620, False)],
+        "model_layers": 80,
     },
     "70b_mlp_0.1bpw_residual": {
         "desc": "Llama-2-70B MLP layer, 0.1 BPW residual s=302 x 2 paths",
         "mats": [(8192, 28672, 302, True), (8192, 28672, 302, True), (28672, 8192, 302, True)],
+        "model_layers": 80,
     },
     "7b_layer_0.1bpw_residual": {
         "desc": "Llama-2-7B layer (4x 4096^2 s=86; 2x 4096->11008 and 11008->4096 s=133), 0.1 BPW residual",
         "mats": [(4096, 4096, 86, True)] * 4 + [(4096, 11008, 133, True)] * 2 + [(11008, 4096, 133, True)],
+        "model_layers": 32,
     },
 }
+DEFAULT_WORKLOAD = "70b_mlp_0.1bpw_single"
 
 
 def algorithmic_bytes(d_in, d_out, s, residual, batch):
@@ -180,9 +186,11 @@ def build_stack(mats, n_rep, batch, seed, device):
     return lb.Stack(Ls, xs, ys), Ls, x_all, y_all
 
 
-def stack_reps_for_l2(mats, batch, l2_bytes, factor=4.0):
+def stack_reps_for_l2(mats, batch, l2_bytes, factor=4.0, model_layers=1):
+    """Model layers per step: the model's own layer count, or more distinct
+    copies if needed for the packed bytes to reach `factor` x L2."""
     per = sum(algorithmic_bytes(*m, batch) for m in mats)
-    return max(1, math.ceil(factor * l2_bytes / per))
+    return max(1, model_layers, math.ceil(factor * l2_bytes / per))
 
 
 def max_over_ranks(values, device):
@@ -353,7 +361,8 @@ def time_e2e(stack, x_all, y_all, steps, warmup, n_chunks):
 
 def measure_workload(name, batch, steps, warmup, device, dist, world, l2, seed=1234, l2_factor=4.0):
     mats = WORKLOADS[name]["mats"]
-    reps = stack_reps_for_l2(mats, batch, l2, l2_factor)
+    model_layers = WORKLOADS[name].get("model_layers", 1) if l2_factor >= 4.0 else 1
+    reps = stack_reps_for_l2(mats, batch, l2, l2_factor, model_layers)
     stack, Ls, x_all, y_all = build_stack(mats, reps, batch, seed, device)
     n_layers = len(Ls)
     total_ms, per_ms = time_device(stack, steps, warmup, dist)
@@ -429,53 +438,65 @@ def run_ours(args):
     sampler.start()
     main, (stack, x_all, y_all) = measure_workload(args.workload, args.batch, args.steps, args.warmup, device,
                                                    dist, world, l2, l2_factor=args.l2_factor)
+    # secondary figures: flat scalars (one level), so that a record keeping
+    # only the line's scalar fields still holds them
+    secondary = {}
     extras = {}
     if not args.no_extras:
-        for name, b in (("70b_mlp_0.1bpw_single", 1), ("70b_mlp_0.1bpw_residual", 1),
-                        ("7b_layer_0.1bpw_residual", 1), ("7b_attn_0.1bpw_single", 1),
-                        ("7b_attn_0.1bpw_residual", 4), ("7b_attn_0.1bpw_residual", 16)):
+        for name, b in (("70b_mlp_0.1bpw_residual", 1), ("70b_mlp_0.1bpw_single", 1),
+                        ("7b_layer_0.1bpw_residual", 1), ("7b_attn_0.1bpw_residual", 1),
+                        ("7b_attn_0.1bpw_single", 1), ("7b_attn_0.1bpw_residual", 4),
+                        ("7b_attn_0.1bpw_residual", 16)):
             if name == args.workload and b == args.batch:
                 continue
-            r, held = measure_workload(name, b, max(5, args.steps // 2), args.warmup, device, dist, world, l2)
+            r, held = measure_workload(name, b, max(10, args.steps // 2), args.warmup, device, dist, world, l2)
             del held
             torch.cuda.empty_cache()
             r["roofline_frac_step"] = r["step_gbs"] / peak
             extras[f"{name}_b{b}"] = r
+            key = f"{name}_b{b}"
+            secondary[f"{key}_us_per_model_layer"] = round(r["us_per_model_layer"], 4)
+            secondary[f"{key}_step_hbm_frac"] = round(r["step_gbs"] / peak, 4)
+            dk = max(KERNELS, key=lambda k: r["kernels"][k]["ms"])
+            secondary[f"{key}_dominant_kernel_hbm_frac"] = round(r["kernels"][dk]["gbs"] / peak, 4)
         for b in (40, 130):
             extras[f"7b_attn_0.1bpw_residual_b{b}_mixed"] = measure_mixed(
                 "7b_attn_0.1bpw_residual", b, max(5, args.steps // 4), args.warmup, device, dist, l2)
         extras["latency_single_layer"] = measure_latency(device)
+        secondary["latency_single_layer_graph_us"] = extras["latency_single_layer"]["graph_us"]
     prefill = None
     if not args.no_prefill:
-        pms, pflops = measure_prefill(args.prefill_layers, 2048, max(3, args.steps // 20), 3, device, dist)
+        psteps = max(20, args.steps // 10)
+        pms, pflops = measure_prefill(args.prefill_layers, 2048, psteps, 3, device, dist)
         pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
             os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
         burst, sustained = float(pk.get("bf16_tflops", 1590.0)), float(pk.get("bf16_tflops_sustained", 1400.0))
         tf = pflops / (pms * 1e-3) / 1e12 * world
-        prefill = {"workload": f"Llama-2-7B full linear stack at 0.3 BPW residual (4x 4096^2 s=290; 4096<->11008 "
-                               f"s=431), {args.prefill_layers} layers, M=2048 bf16 tokens per matrix",
-                   "ms_per_step": round(pms, 4), "tflops": round(tf, 1), "unit": "TFLOP/s",
-                   "algorithmic_flops_per_step": pflops,
-                   "roofline": {"bound": "tensor", "achieved": round(tf / world, 1), "peak": burst,
-                                "unit": "TFLOP/s", "frac": round(tf / world / burst, 4),
-                                "frac_of_sustained": round(tf / world / sustained, 4),
-                                "peak_source": "measured (MEASURED_PEAKS.json bf16_tflops, burst)",
-                                "note": "step-level: operand preparation + both tcgen05 GEMMs"}}
+        prefill = {"workload": f"Llama-2-7B linear stack 0.3 BPW residual, {args.prefill_layers} layers, M=2048 bf16",
+                   "steps": psteps, "ms_per_step": round(pms, 4), "tflops": round(tf, 1), "unit": "TFLOP/s",
+                   "algorithmic_flops_per_step": pflops, "bound": "tensor",
+                   "peak_tflops": burst, "frac": round(tf / world / burst, 4),
+                   "frac_of_sustained": round(tf / world / sustained, 4),
+                   "peak_source": "measured (MEASURED_PEAKS.json bf16_tflops, burst)" if pk else "fallback",
+                   "note": "step-level: operand preparation + both tcgen05 GEMMs, fp16 operands, fp32 accumulate"}
     clocks = sampler.stop()
     # the end-to-end pass runs after the clock sampler has stopped: it is bound
     # by host-side driver calls and PCIe copies, which nvidia-smi's polling
     # slows down, and it carries no clock-sensitive kernel time of its own
-    e2e_ms, h2d, d2h = time_e2e(stack, x_all, y_all, max(3, args.steps // 4), 3, args.e2e_chunks)
+    e2e_steps = max(3, args.steps // 4)
+    e2e_ms, h2d, d2h = time_e2e(stack, x_all, y_all, e2e_steps, 3, args.e2e_chunks)
     e2e_ms = max_over_ranks([e2e_ms], device)[0]
     del stack, x_all, y_all
 
     n_layers = main["layers_per_step"]
+    model_layers = main["model_layers_per_step"]
     dom = max(KERNELS, key=lambda k: main["kernels"][k]["ms"])
     dom_bytes = main["kernels"][dom]["algorithmic_bytes"]
     dom_ms = main["kernels"][dom]["ms"]
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
-    traffic = traffic_record(dom, args.workload, main["model_layers_per_step"])
-    value = job_us_per_layer(main["ms_per_step"], n_layers, world)   # us per layer over all ranks' layers
+    traffic = traffic_record(dom, args.workload, model_layers)
+    value = job_us_per_layer(main["ms_per_step"], model_layers, world)   # us per model layer over all ranks
+    wl = WORKLOADS[args.workload]
     line = {
         "metric": METRIC,
         "value": round(value, 5),
@@ -491,12 +512,11 @@ def run_ours(args):
         "dtype_note": "int8 tensor-core products (u8 sign planes x s8 hi/lo bytes of the 16-bit quantised vector), "
                       "int32 accumulation, fp32 scaling; fp16 x and y",
         "data": "synthetic: fair random signs, scales ~U[0.5,1.5]/sqrt(s), x ~ N(0,1) fp16",
-        "config": {"workload": WORKLOADS[args.workload]["desc"] + f", decode batch {args.batch}, "
-                   f"stack of {n_layers} distinct layers per GPU ({main['stack_bytes'] / 1e6:.0f} MB packed, "
-                   f">= 4x L2; inputs larger than L2, no flush)",
-                   "d_in": WORKLOADS[args.workload]["mats"][0][0], "d_out": WORKLOADS[args.workload]["mats"][0][1],
-                   "s": WORKLOADS[args.workload]["mats"][0][2], "residual": WORKLOADS[args.workload]["mats"][0][3],
-                   "batch": args.batch, "layers_per_gpu": n_layers, "parallelism": f"replicas x{world}"},
+        "config": {"workload": f"{wl['desc']}, decode batch {args.batch}, {model_layers} model layers "
+                               f"({n_layers} matrices, {main['stack_bytes'] / 1e6:.0f} MB packed, inputs > L2, no flush)",
+                   "layer": f"{len(wl['mats'])} matrices per model layer",
+                   "batch": args.batch, "model_layers_per_gpu": model_layers, "matrices_per_gpu": n_layers,
+                   "us_per_matrix": round(main["us_per_matrix"], 5), "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
@@ -505,14 +525,16 @@ def run_ours(args):
                           "kernels": {k: {"ms_per_step": round(main["kernels"][k]["ms"], 5),
                                           "gbs": round(main["kernels"][k]["gbs"], 1)
                                           if main["kernels"][k]["gbs"] else None} for k in KERNELS}},
-        "e2e": {"value": round(job_us_per_layer(e2e_ms / max(3, args.steps // 4), n_layers, world), 5), "unit": "us/layer",
+        "step_hbm_frac": round(main["step_gbs"] / peak, 4),
+        "e2e": {"value": round(job_us_per_layer(e2e_ms / e2e_steps, model_layers, world), 5), "unit": "us/layer",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "api": "littlebit_linear_forward_many_host (pinned host buffers)", "chunks": args.e2e_chunks,
                 "note": "timed after the nvidia-smi clock sampler stopped"},
         "gpu_launches": 4 * args.steps,   # quantise, latent, finalize, output per step
         "clocks": clocks,
-        "extras": extras,
+        "secondary": secondary,
         "prefill": prefill,
+        "extras": extras,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload, args.batch, budget_s=args.cpu_seconds)
@@ -548,39 +570,49 @@ def _blas_threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(workload, batch, budget_s=10.0, n_distinct=4):
-    """Time the fp64 oracle (as it stands) on distinct layers of the workload
-    until about `budget_s` seconds of CPU work; returns us per layer."""
+def _oracle_model_layers(workload, batch, seed, n_distinct):
+    """n_distinct model layers of the workload (each a list of (paths, x) per
+    matrix), drawn with the shared input generator for the CPU oracle."""
     from latent_binary_factorization_b200 import synth
-    from oracle import littlebit_oracle as orc
     mats = WORKLOADS[workload]["mats"]
-    samples = []
+    out = []
     for i in range(n_distinct):
-        a, b, s, r = mats[i % len(mats)]
-        samples.append((synth.layer(a, b, s, r, seed=77, index=i), synth.activations(batch, a, seed=77, index=i)))
-    orc.factored_forward(samples[0][1], samples[0][0])   # warm
+        out.append([(synth.layer(a, b, s, r, seed=seed, index=len(mats) * i + k),
+                     synth.activations(batch, a, seed=seed, index=len(mats) * i + k))
+                    for k, (a, b, s, r) in enumerate(mats)])
+    return out
+
+
+def cpu_baseline(workload, batch, budget_s=10.0, n_distinct=2):
+    """Time the fp64 oracle (as it stands) on distinct model layers of the
+    workload until about `budget_s` seconds of CPU work; returns us per model
+    layer."""
+    from oracle import littlebit_oracle as orc
+    samples = _oracle_model_layers(workload, batch, 77, n_distinct)
+    for paths, x in samples[0]:
+        orc.factored_forward(x, paths)   # warm
 
     def timed(seconds):
         t0 = time.perf_counter()
         n = 0
         while True:
-            paths, x = samples[n % n_distinct]
-            orc.factored_forward(x, paths)
+            for paths, x in samples[n % n_distinct]:
+                orc.factored_forward(x, paths)
             n += 1
-            if time.perf_counter() - t0 >= seconds and n >= 3:
+            if time.perf_counter() - t0 >= seconds and n >= 2:
                 break
         return n, time.perf_counter() - t0
 
     n, dt = timed(budget_s)
     out = {"value": round(1e6 * dt / n, 3), "unit": "us/layer", "cores": _blas_threads(), "kind": "oracle",
-           "sample": f"{n} forwards of {n_distinct} distinct {WORKLOADS[workload]['desc']} layers, batch {batch}, "
-                     f"fp64 numpy, {dt:.1f} s", "nproc": os.cpu_count(), "cpu_model": _cpu_model()}
+           "sample": f"{n} forwards of {n_distinct} distinct model layers ({WORKLOADS[workload]['desc']}), "
+                     f"batch {batch}, fp64 numpy, {dt:.1f} s", "nproc": os.cpu_count(), "cpu_model": _cpu_model()}
     try:   # the same oracle with its BLAS held to one thread
         from threadpoolctl import threadpool_limits
         with threadpool_limits(limits=1, user_api="blas"):
             n1, dt1 = timed(budget_s / 4)
         out["single_thread"] = {"value": round(1e6 * dt1 / n1, 3), "unit": "us/layer", "cores": 1,
-                                "sample": f"{n1} forwards, {dt1:.1f} s"}
+                                "sample": f"{n1} model-layer forwards, {dt1:.1f} s"}
     except ImportError:
         pass
     return out
@@ -591,35 +623,31 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    from latent_binary_factorization_b200 import synth
     from oracle import littlebit_oracle as orc
-    mats = WORKLOADS[args.workload]["mats"]
-    per_step = 4
-    samples = []
-    for i in range(per_step):
-        a, b, s, r = mats[i % len(mats)]
-        samples.append((synth.layer(a, b, s, r, seed=88, index=i), synth.activations(args.batch, a, seed=88, index=i)))
+    n_distinct = 2
+    samples = _oracle_model_layers(args.workload, args.batch, 88, n_distinct)
 
-    def step():
-        for paths, x in samples:
+    def step(k):
+        for paths, x in samples[k % n_distinct]:
             orc.factored_forward(x, paths)
 
-    for _ in range(args.warmup):
-        step()
+    for k in range(args.warmup):
+        step(k)
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
+    for k in range(args.steps):
+        step(k)
     dt = time.perf_counter() - t0
-    value = 1e6 * dt / (args.steps * per_step)
+    value = 1e6 * dt / args.steps
+    wl = WORKLOADS[args.workload]
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "us/layer", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(1e3 * dt / args.steps, 3), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOADS[args.workload]["desc"] + f", decode batch {args.batch}; each step = "
-                   f"{per_step} distinct layers on the CPU oracle", "batch": args.batch},
+        "config": {"workload": f"{wl['desc']}, decode batch {args.batch}; each step = one model layer "
+                               f"({len(wl['mats'])} matrices) on the CPU oracle", "batch": args.batch},
         "impl": "reference",
         "cpu_baseline": {"value": round(value, 3), "unit": "us/layer", "kind": "oracle", "cores": _blas_threads(),
-                         "sample": f"{per_step} layers per step x {args.steps} steps"},
+                         "sample": f"one model layer per step x {args.steps} steps, {n_distinct} distinct layers"},
         "e2e": {"value": round(value, 3), "unit": "us/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -631,7 +659,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="7b_attn_0.1bpw_residual")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -48,7 +48,8 @@ typedef enum {
   LB_ERR_SHAPE = 3,       /* a dimension is outside what the kernels accept */
   LB_ERR_CUDA = 4,        /* a CUDA runtime call failed (see littlebit_last_cuda_error) */
   LB_ERR_TIMEOUT = 5,     /* a bounded device wait ran out (littlebit_device_status) */
-  LB_ERR_UNSUPPORTED = 6  /* a valid request this build does not implement */
+  LB_ERR_UNSUPPORTED = 6, /* a valid request this build does not implement */
+  LB_ERR_RANGE = 7        /* a value left the range of the format it is held in (littlebit_device_status) */
 } lb_status;
 
 typedef enum { LB_F16 = 0, LB_BF16 = 1, LB_F32 = 2, LB_I8 = 3 } lb_dtype;
@@ -226,12 +227,15 @@ lb_status littlebit_linear_forward_many_host(const lb_layer* layers, int n, cons
  *     4096*r bytes, 4*ceil(n/4) * batch * 16*ceil(s/16) fp32 partial sums,
  *     and the t' bytes (about 2*r*s).
  *   - The first call on a device, with that device current, looks up the
- *     array's device address (cudaGetSymbolAddress); make that first call
- *     before any stream capture.
+ *     array's device address (cudaGetSymbolAddress) and zeroes its status
+ *     word on `stream`; make that first call before any stream capture.
  *   - Every call shares the array and the array keeps the last call's
- *     contents; the call clears what must start at zero itself.  Calls whose
- *     work overlaps on the GPU (other streams, other host threads) race on it
- *     and give wrong results: serialise them.
+ *     contents; each call writes every region its kernels read before they
+ *     read it.  Calls whose work overlaps on the GPU (other streams, other
+ *     host threads) race on it and give wrong results: serialise them.
+ *   - Device-side error bits (a bounded wait that gave up, a non-finite
+ *     input) collect in the array's status word until littlebit_device_status
+ *     reads and clears them.
  * Arguments, alignment and other errors as littlebit_linear_forward.
  */
 lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_dev, void* y_dev,
@@ -243,6 +247,13 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
  * the forward kernels enqueued on it have raised since the last call, and
  * clears them.  Bit (1 << LB_ERR_TIMEOUT) means a bounded wait for a bulk copy
  * into shared memory gave up (the outputs of that call are not valid).
+ * Bit (1 << LB_ERR_RANGE) means a value could not be held in the format the
+ * kernels keep it in, so the outputs of that call hold inf or NaN: an input
+ * x that is inf or NaN (decode and prefill), a bf16 input beyond fp16's
+ * finite range (|x| > 65504; prefill converts x to fp16), or a latent value
+ * t' = l (.) t, or an fp16 output y, beyond fp16's range (prefill).
+ * The word of littlebit_linear_forward_noalloc on the current device is read
+ * and cleared too (its calls may be on any stream: synchronise them first).
  * *status is 0 when nothing was raised.  Errors: LB_ERR_ARG, LB_ERR_CUDA.
  */
 lb_status littlebit_device_status(void* stream, unsigned int* status);

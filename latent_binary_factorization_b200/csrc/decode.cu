@@ -179,6 +179,7 @@ __global__ void __launch_bounds__(kQWarps * 32) quantise_input_kernel(const Deco
   const int nchunk = min(kVSlice, d_in - k0) / 8;
   const size_t blk_off = (size_t)sl * xq_slice_bytes(B);
 
+  unsigned bad = 0;   // an input x that is inf or NaN (LB_ERR_RANGE)
   {
     const PathDesc& P = L.p[p];
     unsigned char* blk = P.ws.xq + blk_off;
@@ -199,6 +200,7 @@ __global__ void __launch_bounds__(kQWarps * 32) quantise_input_kernel(const Deco
         const uint32_t* gw = &gq.x;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
+          bad |= half2_nonfinite(xw[e]);
           const float2 xf = h2x2(xw[e]), gf = h2x2(gw[e]);
           u[j][2 * e] = xf.x * gf.x;
           u[j][2 * e + 1] = xf.y * gf.y;
@@ -247,6 +249,7 @@ __global__ void __launch_bounds__(kQWarps * 32) quantise_input_kernel(const Deco
       }
     }
   }
+  if (__any_sync(0xffffffffu, bad != 0) && lane == 0) atomicOr(a.status, kStatusRange);
 }
 
 // ---------------------------------------------------------------------------
@@ -1092,19 +1095,16 @@ cudaError_t launch_latent(const DecodeArgs& a, int num_sms, cudaStream_t st) {
   constexpr size_t smem = latent_smem<NB, RB, W>();
   static_assert(smem <= 227 * 1024, "latent pass shared memory");
   auto kern = latent_pass_kernel<NB, RB, W>;
-  static bool attr_set = false;
-  cudaError_t e;
-  if (!attr_set) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  static int per_sm = 0;
-  if (per_sm == 0) {
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, W * 32, smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  }
+  // the shared-memory attribute and the occupancy it allows, once per device
+  static PerDevice cache;
+  int per_sm = 0;
+  const int err = cache.get(current_device(), per_sm, [&](int& v) -> int {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kern, W * 32, smem);
+    if (e == cudaSuccess && v < 1) e = cudaErrorInvalidConfiguration;
+    return (int)e;
+  });
+  if (err != 0) return (cudaError_t)err;
   const int grid = max(1, min(a.v_items, per_sm * num_sms));
   return launch_dependent(kern, grid, W * 32, smem, st, a);
 }
@@ -1112,18 +1112,18 @@ cudaError_t launch_latent(const DecodeArgs& a, int num_sms, cudaStream_t st) {
 template <int NB>
 cudaError_t launch_output(const DecodeArgs& a, int num_sms, cudaStream_t st) {
   const size_t smem = output_smem<NB>(a.batch);
-  const size_t smem_max = output_smem<NB>(4 * NB);
-  static bool attr_set = false;
-  cudaError_t e;
-  if (!attr_set) {
-    e = cudaFuncSetAttribute(output_pass_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  // the shared-memory attribute and the occupancy it allows, once per device
+  static PerDevice cache;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, output_pass_kernel<NB>, kUWarps * 32, smem);
-  if (e != cudaSuccess) return e;
-  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const int err = cache.get(current_device(), per_sm, [&](int& v) -> int {
+    cudaError_t e = cudaFuncSetAttribute(output_pass_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, output_pass_kernel<NB>, kUWarps * 32, smem);
+    if (e == cudaSuccess && v < 1) e = cudaErrorInvalidConfiguration;
+    return (int)e;
+  });
+  if (err != 0) return (cudaError_t)err;
   const int grid = max(1, min((a.u_items + kUWarps - 1) / kUWarps, per_sm * num_sms));
   return launch_dependent(output_pass_kernel<NB>, grid, kUWarps * 32, smem, st, a);
 }
@@ -1164,19 +1164,17 @@ cudaError_t launch_finalize_pass(const DecodeArgs& a, int max_s16, cudaStream_t 
 
 cudaError_t launch_output_packed(const DecodeArgs& a, int num_sms, cudaStream_t st) {
   const size_t smem = (size_t)kUWarps * kPkStages * kPkStageBytes + (size_t)kUWarps * kPkStages * 8;
-  static bool attr_set = false;
-  cudaError_t e;
-  if (!attr_set) {
-    e = cudaFuncSetAttribute(output_packed_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  static int per_sm = 0;
-  if (per_sm == 0) {
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, output_packed_kernel, kUWarps * 32, smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  }
+  // the shared-memory attribute and the occupancy it allows, once per device
+  static PerDevice cache;
+  int per_sm = 0;
+  const int err = cache.get(current_device(), per_sm, [&](int& v) -> int {
+    cudaError_t e = cudaFuncSetAttribute(output_packed_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, output_packed_kernel, kUWarps * 32, smem);
+    if (e == cudaSuccess && v < 1) e = cudaErrorInvalidConfiguration;
+    return (int)e;
+  });
+  if (err != 0) return (cudaError_t)err;
   const int grid = max(1, min((a.u_items + kUWarps - 1) / kUWarps, per_sm * num_sms));
   return launch_dependent(output_packed_kernel, grid, kUWarps * 32, smem, st, a);
 }

@@ -8,8 +8,15 @@
 #include <vector>
 
 #include "littlebit.h"
+#include "per_device.h"
 
 namespace lb {
+
+// The device ordinal that is current on this thread (-1 if it cannot be read).
+inline int current_device() {
+  int d = -1;
+  return cudaGetDevice(&d) == cudaSuccess ? d : -1;
+}
 
 constexpr int kMaxBatchDecode = 16;   // decode kernels: 1..16 rows
 constexpr int kMaxRank = 1024;        // latent rank s accepted by the kernels
@@ -71,6 +78,16 @@ constexpr int kUWarps = 4;
 // Quantisation of the int8 B operand: v = 256*hi + lo with hi, lo in [-128, 127]
 // needs |v| <= 32639.
 constexpr float kQMax = 32639.f;
+
+// Device status word bits raised by the kernels (littlebit_device_status).
+constexpr unsigned kStatusTimeout = 1u << LB_ERR_TIMEOUT;
+constexpr unsigned kStatusRange = 1u << LB_ERR_RANGE;
+
+// Non-zero when either fp16 of the pair in `w` is inf or NaN (exponent field
+// all ones): adding 1 to an all-ones exponent carries into the sign position.
+__host__ __device__ inline unsigned half2_nonfinite(unsigned w) {
+  return ((w & 0x7c007c00u) + 0x04000400u) & 0x80008000u;
+}
 
 // Bounded waits: polls of mbarrier.try_wait (each may suspend up to ~1 us)
 // before a wait gives up (a few seconds in total).
@@ -179,9 +196,27 @@ void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const*
                         unsigned char* bufs, int num_sms, std::vector<unsigned char>& img, PrefillPlan& plan);
 // A chunk's operand preparation (three grouped launches), then its two
 // grouped GEMM launches; both read the table image uploaded at table_dev.
-cudaError_t launch_prefill_prep(const PrefillPlan& plan, const unsigned char* table_dev, cudaStream_t st);
+cudaError_t launch_prefill_prep(const PrefillPlan& plan, const unsigned char* table_dev, unsigned int* status,
+                                cudaStream_t st);
 cudaError_t launch_prefill_gemms(const PrefillPlan& plan, const unsigned char* table_dev, unsigned int* status,
                                  cudaStream_t st);
+
+// littlebit_capi.cu: helpers shared by the entry points.
+// Records `e` as this thread's last CUDA error text and returns LB_ERR_CUDA.
+lb_status cuda_fail(cudaError_t e);
+// Shape, pointer and alignment checks of one layer (not of x and y).
+lb_status check_layer(const lb_layer& L);
+// Bytes of each per-path decode scratch region of a layer at this batch
+// (every region a multiple of 256 bytes; PathScratch order).
+size_t xq_bytes(const lb_layer& L, int batch);
+size_t partial_bytes(const lb_layer& L, int batch);
+size_t planes_bytes(const lb_layer& L, int batch);
+size_t tstat_bytes(int batch);
+size_t path_scratch_bytes(const lb_layer& L, int batch);
+
+// noalloc.cu: device address of the allocation-free forward's status word on
+// device `dev`, or null before that entry point's first call on the device.
+unsigned int* noalloc_status_word(int dev);
 
 // pack.cu
 cudaError_t launch_unpack(const void* src, int n_long, int s, lb_role role, int8_t* dst, cudaStream_t st);

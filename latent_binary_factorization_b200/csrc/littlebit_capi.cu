@@ -18,15 +18,62 @@ namespace {
 
 thread_local char g_last_cuda_error[256] = "";
 
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace
+
+namespace lb {
+
 lb_status cuda_fail(cudaError_t e) {
   std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
                 cudaGetErrorString(e));
   return LB_ERR_CUDA;
 }
 
-bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+lb_status check_layer(const lb_layer& L) {
+  if (L.d_in < 256 || L.d_in % 256 != 0) return LB_ERR_SHAPE;
+  if (L.d_out < 128 || L.d_out % 128 != 0) return LB_ERR_SHAPE;
+  if (L.s < 1 || L.s > kMaxRank) return LB_ERR_SHAPE;
+  if (L.residual != 0 && L.residual != 1) return LB_ERR_ARG;
+  for (int p = 0; p <= L.residual; ++p) {
+    const lb_path& P = L.path[p];
+    if (!P.V_bits || !P.U_bits || !P.h || !P.g || !P.l) return LB_ERR_ARG;
+    if (!aligned(P.V_bits, 16) || !aligned(P.U_bits, 16)) return LB_ERR_ALIGN;
+    if (!aligned(P.h, 16) || !aligned(P.g, 16) || !aligned(P.l, 2)) return LB_ERR_ALIGN;
+  }
+  return LB_OK;
+}
 
-size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+size_t xq_bytes(const lb_layer& L, int batch) {
+  return align_up((size_t)ceil_div(L.d_in, kVSlice) * xq_slice_bytes(batch), 256);
+}
+size_t partial_bytes(const lb_layer& L, int batch) {
+  const size_t ns4 = (size_t)ceil_div(ceil_div(L.d_in, kVSlice), 4) * 4;
+  return align_up(ns4 * batch * s16(L.s) * sizeof(float), 256);
+}
+// t' planes and stats are padded to whole groups of four batch rows; at batch
+// 1 path 0's planes hold the combined K range of both paths (packed output pass)
+size_t planes_bytes(const lb_layer& L, int batch) {
+  return align_up((size_t)ceil_div(batch, 4) * 4 * 2 * s32(L.s) * (batch == 1 ? 2 : 1), 256);
+}
+size_t tstat_bytes(int batch) { return align_up((size_t)ceil_div(batch, 4) * 4 * sizeof(TStat), 256); }
+size_t path_scratch_bytes(const lb_layer& L, int batch) {
+  return xq_bytes(L, batch) + partial_bytes(L, batch) + planes_bytes(L, batch) + tstat_bytes(batch);
+}
+
+}  // namespace lb
+
+namespace {
+
+using lb::check_layer;
+using lb::cuda_fail;
+using lb::partial_bytes;
+using lb::path_scratch_bytes;
+using lb::planes_bytes;
+using lb::tstat_bytes;
+using lb::xq_bytes;
 
 struct Workspace {
   void* buf = nullptr;
@@ -93,37 +140,6 @@ int num_sms(int dev) {
   return g_num_sms[dev];
 }
 
-lb_status check_layer(const lb_layer& L) {
-  if (L.d_in < 256 || L.d_in % 256 != 0) return LB_ERR_SHAPE;
-  if (L.d_out < 128 || L.d_out % 128 != 0) return LB_ERR_SHAPE;
-  if (L.s < 1 || L.s > lb::kMaxRank) return LB_ERR_SHAPE;
-  if (L.residual != 0 && L.residual != 1) return LB_ERR_ARG;
-  for (int p = 0; p <= L.residual; ++p) {
-    const lb_path& P = L.path[p];
-    if (!P.V_bits || !P.U_bits || !P.h || !P.g || !P.l) return LB_ERR_ARG;
-    if (!aligned(P.V_bits, 16) || !aligned(P.U_bits, 16)) return LB_ERR_ALIGN;
-    if (!aligned(P.h, 16) || !aligned(P.g, 16) || !aligned(P.l, 2)) return LB_ERR_ALIGN;
-  }
-  return LB_OK;
-}
-
-// Bytes of per-path scratch for one layer at this batch.
-size_t xq_bytes(const lb_layer& L, int batch) {
-  return align_up((size_t)lb::ceil_div(L.d_in, lb::kVSlice) * lb::xq_slice_bytes(batch), 256);
-}
-size_t partial_bytes(const lb_layer& L, int batch) {
-  const size_t ns4 = (size_t)lb::ceil_div(lb::ceil_div(L.d_in, lb::kVSlice), 4) * 4;
-  return align_up(ns4 * batch * lb::s16(L.s) * sizeof(float), 256);
-}
-// t' planes and stats are padded to whole groups of four batch rows; at batch
-// 1 path 0's planes hold the combined K range of both paths (packed output pass)
-size_t planes_bytes(const lb_layer& L, int batch) {
-  return align_up((size_t)lb::ceil_div(batch, 4) * 4 * 2 * lb::s32(L.s) * (batch == 1 ? 2 : 1), 256);
-}
-size_t tstat_bytes(int batch) { return align_up((size_t)lb::ceil_div(batch, 4) * 4 * sizeof(lb::TStat), 256); }
-size_t path_scratch_bytes(const lb_layer& L, int batch) {
-  return xq_bytes(L, batch) + partial_bytes(L, batch) + planes_bytes(L, batch) + tstat_bytes(batch);
-}
 
 constexpr size_t kStatusBytes = 256;   // device status word at the start of a workspace
 constexpr int kMaxHostChunks = 64;     // chunks of one host-buffer stack call
@@ -413,7 +429,7 @@ lb_status prefill_launch(Workspace& ws, cudaStream_t st) {
   const int n_chunks = (int)ws.p_plans.size();
   cudaError_t e;
   if (n_chunks == 1) {
-    e = lb::launch_prefill_prep(ws.p_plans[0], table_dev, st);
+    e = lb::launch_prefill_prep(ws.p_plans[0], table_dev, status, st);
     if (e != cudaSuccess) return cuda_fail(e);
     e = lb::launch_prefill_gemms(ws.p_plans[0], table_dev, status, st);
     return e == cudaSuccess ? LB_OK : cuda_fail(e);
@@ -428,7 +444,7 @@ lb_status prefill_launch(Workspace& ws, cudaStream_t st) {
     const int h = c & 1;
     // the half was last used by chunk c - 2's GEMMs
     if (c >= 2) e = cudaStreamWaitEvent(ws.side, ws.gemm_done[h], 0);
-    if (e == cudaSuccess) e = lb::launch_prefill_prep(ws.p_plans[c], table_dev, ws.side);
+    if (e == cudaSuccess) e = lb::launch_prefill_prep(ws.p_plans[c], table_dev, status, ws.side);
     if (e == cudaSuccess) e = cudaEventRecord(ws.prep_done[h], ws.side);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ws.prep_done[h], 0);
     if (e == cudaSuccess) e = lb::launch_prefill_gemms(ws.p_plans[c], table_dev, status, st);
@@ -646,6 +662,18 @@ lb_status littlebit_device_status(void* stream, unsigned int* status) {
     }
     *status |= bits;
   }
+  // the allocation-free forward's word on this device (any stream)
+  unsigned int* word = lb::noalloc_status_word(dev);
+  if (word) {
+    unsigned int bits = 0;
+    e = cudaMemcpy(&bits, word, sizeof(bits), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (bits) {
+      e = cudaMemset(word, 0, sizeof(unsigned int));
+      if (e != cudaSuccess) return cuda_fail(e);
+    }
+    *status |= bits;
+  }
   return LB_OK;
 }
 
@@ -782,6 +810,7 @@ const char* littlebit_status_string(lb_status st) {
     case LB_ERR_CUDA: return "LB_ERR_CUDA: CUDA runtime error";
     case LB_ERR_TIMEOUT: return "LB_ERR_TIMEOUT: device wait timed out";
     case LB_ERR_UNSUPPORTED: return "LB_ERR_UNSUPPORTED: not implemented for these arguments";
+    case LB_ERR_RANGE: return "LB_ERR_RANGE: a value left the range of its format";
   }
   return "unknown lb_status";
 }

@@ -10,6 +10,7 @@
 // holds until the process exits.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstring>
 
 #include "lb_internal.h"
@@ -29,66 +30,75 @@ constexpr size_t kTableOff = 256;
 constexpr size_t kPathOff = 512;
 static_assert(sizeof(lb::LayerDesc) <= kPathOff - kTableOff, "layer descriptor must fit its slot");
 
-constexpr int kMaxDevices = 64;
-unsigned char* g_scratch_dev[kMaxDevices] = {nullptr};   // device address per device, set once
-
-size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+// Device address of the array per device, set once by the first call on that
+// device (with the device current); read by littlebit_device_status too.
+std::atomic<unsigned char*> g_scratch_dev[lb::kMaxDevices];
 
 bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-lb_status check(const lb_layer& L, const void* x, const void* y, int batch, lb_dtype xdt) {
-  if (!x || !y) return LB_ERR_ARG;
-  if (L.d_in < 256 || L.d_in % 256 != 0 || L.d_out < 128 || L.d_out % 128 != 0) return LB_ERR_SHAPE;
-  if (L.s < 1 || L.s > lb::kMaxRank) return LB_ERR_SHAPE;
-  if (L.residual != 0 && L.residual != 1) return LB_ERR_ARG;
-  if (batch < 1 || batch > lb::kMaxBatchDecode) return batch < 1 ? LB_ERR_SHAPE : LB_ERR_UNSUPPORTED;
-  if (xdt != LB_F16) return LB_ERR_UNSUPPORTED;
-  if (!aligned_to(x, 16) || !aligned_to(y, 16)) return LB_ERR_ALIGN;
-  for (int p = 0; p <= L.residual; ++p) {
-    const lb_path& P = L.path[p];
-    if (!P.V_bits || !P.U_bits || !P.h || !P.g || !P.l) return LB_ERR_ARG;
-    if (!aligned_to(P.V_bits, 16) || !aligned_to(P.U_bits, 16)) return LB_ERR_ALIGN;
-    if (!aligned_to(P.h, 16) || !aligned_to(P.g, 16) || !aligned_to(P.l, 2)) return LB_ERR_ALIGN;
+// Writes the call's layer descriptor into the array.  The descriptor travels
+// as a kernel argument, so no host buffer has to outlive the call.
+__global__ void write_desc_kernel(const lb::LayerDesc d, lb::LayerDesc* dst) { *dst = d; }
+
+// The array's device address on the current device `dev`, looked up (and its
+// status word zeroed on `st`) by the first call on that device.
+lb_status scratch_base(int dev, cudaStream_t st, unsigned char** base) {
+  unsigned char* b = g_scratch_dev[dev].load(std::memory_order_acquire);
+  if (!b) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return lb::cuda_fail(e);
+    if (!ptr) return lb::cuda_fail(cudaErrorInvalidSymbol);
+    e = cudaMemsetAsync(static_cast<unsigned char*>(ptr) + kStatusOff, 0, kTableOff - kStatusOff, st);
+    if (e != cudaSuccess) return lb::cuda_fail(e);
+    b = static_cast<unsigned char*>(ptr);
+    g_scratch_dev[dev].store(b, std::memory_order_release);
   }
+  *base = b;
   return LB_OK;
 }
 
 }  // namespace
 
+namespace lb {
+
+unsigned int* noalloc_status_word(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  unsigned char* b = g_scratch_dev[dev].load(std::memory_order_acquire);
+  return b ? reinterpret_cast<unsigned int*>(b + kStatusOff) : nullptr;
+}
+
+}  // namespace lb
+
 extern "C" {
 
 lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_dev, void* y_dev, int batch,
                                            lb_dtype xdt, void* stream) {
-  if (!layer) return LB_ERR_ARG;
+  if (!layer || !x_dev || !y_dev) return LB_ERR_ARG;
   const lb_layer& L = *layer;
-  lb_status chk = check(L, x_dev, y_dev, batch, xdt);
+  lb_status chk = lb::check_layer(L);
   if (chk != LB_OK) return chk;
+  if (batch < 1) return LB_ERR_SHAPE;
+  if (batch > lb::kMaxBatchDecode || xdt != LB_F16) return LB_ERR_UNSUPPORTED;
+  if (!aligned_to(x_dev, 16) || !aligned_to(y_dev, 16)) return LB_ERR_ALIGN;
 
-  // scratch needed by this layer at this batch
-  const int n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
-  const int S16 = lb::s16(L.s), S32 = lb::s32(L.s);
-  const size_t xq_b = round256((size_t)n_slices * lb::xq_slice_bytes(batch));
-  const size_t part_b = round256((size_t)lb::ceil_div(n_slices, 4) * 4 * batch * S16 * sizeof(float));
-  const int bpad = lb::ceil_div(batch, 4) * 4;   // t' planes and stats padded to groups of 4 rows
-  // at batch 1 path 0's planes hold the combined K range of both paths
-  const size_t planes_b = round256((size_t)bpad * 2 * S32 * (batch == 1 ? 2 : 1));
-  const size_t tstat_b = round256((size_t)bpad * sizeof(lb::TStat));
+  // scratch needed by this layer at this batch (the regular workspace's sizes)
   const int npaths = L.residual + 1;
+  const size_t xq_b = lb::xq_bytes(L, batch), part_b = lb::partial_bytes(L, batch);
+  const size_t planes_b = lb::planes_bytes(L, batch), tstat_b = lb::tstat_bytes(batch);
   if (kPathOff + (size_t)npaths * (xq_b + part_b + planes_b + tstat_b) > kNoAllocScratchBytes) return LB_ERR_SHAPE;
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LB_ERR_CUDA;
-  if (!g_scratch_dev[dev]) {
-    // once per device, with that device current
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess || !ptr) return LB_ERR_CUDA;
-    g_scratch_dev[dev] = static_cast<unsigned char*>(ptr);
-  }
-  unsigned char* base = g_scratch_dev[dev];
+  if (e != cudaSuccess) return lb::cuda_fail(e);
+  if (dev < 0 || dev >= lb::kMaxDevices) return LB_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned char* base = nullptr;
+  lb_status r = scratch_base(dev, st, &base);
+  if (r != LB_OK) return r;
 
+  const int n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
+  const int S16 = lb::s16(L.s);
   lb::LayerDesc D;
   std::memset(&D, 0, sizeof(D));
   D.x = static_cast<const uint16_t*>(x_dev);
@@ -103,10 +113,6 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
     w = 1.0;
   });
   D.n_rchunks = lb::ceil_div(S16 / 16, 2 * vw);
-  D.v_begin = 0;
-  D.u_begin = 0;
-  D.p_begin = 0;
-  D.x_begin = 0;
   size_t off = kPathOff;
   for (int p = 0; p < npaths; ++p) {
     lb::PathDesc& P = D.p[p];
@@ -124,12 +130,11 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
     P.ws.tstat = reinterpret_cast<lb::TStat*>(base + off);
     off += tstat_b;
   }
-  // every call shares the array: the status word must start at zero, whatever
-  // the previous call left there (every other region is written before it is read)
-  e = cudaMemsetAsync(base + kStatusOff, 0, kTableOff - kStatusOff, st);
-  if (e != cudaSuccess) return LB_ERR_CUDA;
-  e = cudaMemcpyAsync(base + kTableOff, &D, sizeof(D), cudaMemcpyHostToDevice, st);
-  if (e != cudaSuccess) return LB_ERR_CUDA;
+  // every region the kernels read is written earlier in the same call; the
+  // status word keeps its bits until littlebit_device_status reads them
+  write_desc_kernel<<<1, 1, 0, st>>>(D, reinterpret_cast<lb::LayerDesc*>(base + kTableOff));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return lb::cuda_fail(e);
 
   lb::DecodeArgs a;
   a.layers = reinterpret_cast<const lb::LayerDesc*>(base + kTableOff);
@@ -145,16 +150,13 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
   a.packed = batch == 1 && L.residual ? 1 : 0;
   int sms = 0;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess || sms <= 0) return LB_ERR_CUDA;
+  if (e != cudaSuccess) return lb::cuda_fail(e);
+  if (sms <= 0) return lb::cuda_fail(cudaErrorInvalidDevice);
   e = lb::launch_quantise_pass(a, st);
-  if (e != cudaSuccess) return LB_ERR_CUDA;
-  e = lb::launch_latent_pass(a, S16, sms, st);
-  if (e != cudaSuccess) return LB_ERR_CUDA;
-  e = lb::launch_finalize_pass(a, S16, st);
-  if (e != cudaSuccess) return LB_ERR_CUDA;
-  e = lb::launch_output_pass(a, sms, st);
-  if (e != cudaSuccess) return LB_ERR_CUDA;
-  return LB_OK;
+  if (e == cudaSuccess) e = lb::launch_latent_pass(a, S16, sms, st);
+  if (e == cudaSuccess) e = lb::launch_finalize_pass(a, S16, st);
+  if (e == cudaSuccess) e = lb::launch_output_pass(a, sms, st);
+  return e == cudaSuccess ? LB_OK : lb::cuda_fail(e);
 }
 
 }  // extern "C"

@@ -159,8 +159,12 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
 // The three preparation steps below each run as one grouped launch over all
 // layers of a chunk: a layer owns a contiguous range of blocks (PrepJob) and
 // its step runs with block `bid` of `nblk` in place of blockIdx/gridDim.
+// An fp16 value that is inf or NaN after the conversion (a bf16 input beyond
+// fp16's finite range, or a non-finite input) raises LB_ERR_RANGE in *status.
 __device__ __forceinline__ void prep_x(const uint16_t* __restrict__ x, int is_bf16, int M, int K,
-                                       unsigned char* __restrict__ out, unsigned bid, unsigned nblk) {
+                                       unsigned char* __restrict__ out, unsigned bid, unsigned nblk,
+                                       unsigned int* status) {
+  unsigned bad = 0;
   const unsigned n16 = (unsigned)((size_t)M * K / 8);   // < 2^32 for the shapes accepted
   const unsigned rgs = (unsigned)M >> 3;
   const unsigned stride = nblk * blockDim.x;
@@ -179,10 +183,14 @@ __device__ __forceinline__ void prep_x(const uint16_t* __restrict__ x, int is_bf
     }
 #pragma unroll
     for (int u = 0; u < kXUnroll; ++u) {
-      if (t0 + u * stride < n16)
-        *reinterpret_cast<uint4*>(out + dst[u]) = is_bf16 ? bf16x8_to_f16x8(v[u]) : v[u];
+      if (t0 + u * stride < n16) {
+        const uint4 h = is_bf16 ? bf16x8_to_f16x8(v[u]) : v[u];
+        bad |= half2_nonfinite(h.x) | half2_nonfinite(h.y) | half2_nonfinite(h.z) | half2_nonfinite(h.w);
+        *reinterpret_cast<uint4*>(out + dst[u]) = h;
+      }
     }
   }
+  if (bad) atomicOr(status, kStatusRange);
 }
 
 // B1 (P*Sp rows x d_in): row p*Sp + j holds V_p[i][j] * g_p[i].  Work unit =
@@ -302,13 +310,14 @@ __device__ __forceinline__ int prep_job_of(const PrepJob* jobs, int n, int k, un
 }
 
 template <int KIND>
-__global__ void __launch_bounds__(256) prep_group_kernel(const PrepJob* __restrict__ jobs, int n) {
+__global__ void __launch_bounds__(256) prep_group_kernel(const PrepJob* __restrict__ jobs, int n,
+                                                         unsigned int* status) {
   const int j = prep_job_of(jobs, n, KIND, blockIdx.x);
   const PrepJob& J = jobs[j];
   const unsigned b0 = (unsigned)J.first[KIND];
   const unsigned b1 = j + 1 < n ? (unsigned)jobs[j + 1].first[KIND] : gridDim.x;
   const unsigned bid = blockIdx.x - b0, nblk = b1 - b0;
-  if (KIND == 0) prep_x(J.x, J.x_bf16, J.M, J.L.d_in, J.X16, bid, nblk);
+  if (KIND == 0) prep_x(J.x, J.x_bf16, J.M, J.L.d_in, J.X16, bid, nblk, status);
   else if (KIND == 1) prep_b1(J.L, J.Sp, J.B1, bid, nblk);
   else prep_b2(J.L, J.Sp, J.B2, bid, nblk);
 }
@@ -450,6 +459,7 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
     // ---- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
     const int quarter = warp & 3;
     uint32_t nt = 0;
+    unsigned bad = 0;   // a t' (or fp16 y) beyond fp16's range: LB_ERR_RANGE
     for (int k = ga.begin[blockIdx.x]; k < ga.begin[blockIdx.x + 1]; ++k, ++nt) {
       const TileInfo ti = tile_info(ga, ga.sched[k]);
       const int ab = nt & 1;
@@ -477,6 +487,7 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
               } else {
                 const __half2 hh = __floats2half2_rn(v[e], v[e + 1]);
                 w[e >> 1] = *reinterpret_cast<const uint32_t*>(&hh);
+                bad |= half2_nonfinite(w[e >> 1]);
               }
             }
             *reinterpret_cast<uint4*>(sy + lane * kYPitch + 32 * h) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -511,6 +522,7 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
             }
             const __half2 hh = __floats2half2_rn(lv[0] * v[e], lv[1] * v[e + 1]);
             w[e >> 1] = *reinterpret_cast<const uint32_t*>(&hh);
+            bad |= half2_nonfinite(w[e >> 1]);
           }
           *reinterpret_cast<uint4*>(P.T + tiled_off(row, ti.n0 + c0, P.M)) = make_uint4(w[0], w[1], w[2], w[3]);
           *reinterpret_cast<uint4*>(P.T + tiled_off(row, ti.n0 + c0 + 8, P.M)) =
@@ -521,7 +533,8 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
       __syncwarp();
       if (lane == 0) mbar_arrive(&acce[ab]);
     }
-    if (dead && lane == 0) atomicOr(ga.status, 1u << LB_ERR_TIMEOUT);
+    if (dead && lane == 0) atomicOr(ga.status, kStatusTimeout);
+    if (__any_sync(0xffffffffu, bad != 0) && lane == 0) atomicOr(ga.status, kStatusRange);
   }
   if ((threadIdx.x == 0 || threadIdx.x == 32) && dead) atomicOr(ga.status, 1u << LB_ERR_TIMEOUT);
   __syncwarp();
@@ -609,11 +622,12 @@ static void prep_blocks(const LayerDesc& L, int M, int Sp, int (&blocks)[3]) {
 
 // Operand preparation of a planned chunk: three grouped launches (x, B1, B2)
 // over all its layers, arguments in the chunk's table at table_dev.
-cudaError_t launch_prefill_prep(const PrefillPlan& plan, const unsigned char* table_dev, cudaStream_t st) {
+cudaError_t launch_prefill_prep(const PrefillPlan& plan, const unsigned char* table_dev, unsigned int* status,
+                                cudaStream_t st) {
   const PrepJob* jobs = reinterpret_cast<const PrepJob*>(table_dev + plan.table_off + plan.jobs_off);
-  prep_group_kernel<0><<<plan.prep_grid[0], 256, 0, st>>>(jobs, plan.n);
-  prep_group_kernel<1><<<plan.prep_grid[1], 256, 0, st>>>(jobs, plan.n);
-  prep_group_kernel<2><<<plan.prep_grid[2], 256, 0, st>>>(jobs, plan.n);
+  prep_group_kernel<0><<<plan.prep_grid[0], 256, 0, st>>>(jobs, plan.n, status);
+  prep_group_kernel<1><<<plan.prep_grid[1], 256, 0, st>>>(jobs, plan.n, status);
+  prep_group_kernel<2><<<plan.prep_grid[2], 256, 0, st>>>(jobs, plan.n, status);
   return cudaGetLastError();
 }
 
@@ -716,13 +730,15 @@ void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const*
 // launch each.
 cudaError_t launch_prefill_gemms(const PrefillPlan& plan, const unsigned char* table_dev, unsigned int* status,
                                  cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(umma_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)group_smem());
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  // the shared-memory attribute, once per device
+  static PerDevice cache;
+  int done = 0;
+  const int err = cache.get(current_device(), done, [](int& v) -> int {
+    v = 1;
+    return (int)cudaFuncSetAttribute(umma_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)group_smem());
+  });
+  if (err != 0) return (cudaError_t)err;
   const unsigned char* base = table_dev + plan.table_off;
   const size_t prob_b = (size_t)2 * plan.n * sizeof(GemmProblem);
   const GemmProblem* probs = reinterpret_cast<const GemmProblem*>(base);

@@ -28,7 +28,7 @@ LB_F16, LB_BF16, LB_F32, LB_I8 = 0, 1, 2, 3
 LB_ROLE_V, LB_ROLE_U = 0, 1
 ROLE = {"V": LB_ROLE_V, "U": LB_ROLE_U}
 STATUS = {0: "LB_OK", 1: "LB_ERR_ARG", 2: "LB_ERR_ALIGN", 3: "LB_ERR_SHAPE", 4: "LB_ERR_CUDA",
-          5: "LB_ERR_TIMEOUT", 6: "LB_ERR_UNSUPPORTED"}
+          5: "LB_ERR_TIMEOUT", 6: "LB_ERR_UNSUPPORTED", 7: "LB_ERR_RANGE"}
 _DTYPE = {torch.float16: LB_F16, torch.bfloat16: LB_BF16, torch.float32: LB_F32, torch.int8: LB_I8}
 
 

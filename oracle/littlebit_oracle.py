@@ -29,7 +29,7 @@ What it computes, and where each piece is defined
 * ``rotation_residual``: the gauge freedom the LittleBit-2 column (chapter 2,
   "solution 1", Joint-ITQ) relies on: (U R)(R^T V^T) = U V^T for orthogonal R.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 * sign(0) is taken as +1 (bit = [v < 0]); the pages only say "binarise to +-1".
 * the residual path uses the same rank s as the main path (the cost formula's
   factor 2 multiplies every term).

@@ -44,10 +44,22 @@ def test_worked_example_7b_attention_residual():
 def test_stacks_exceed_l2(name):
     l2 = 126 * 2 ** 20
     mats = bench.WORKLOADS[name]["mats"]
-    reps = bench.stack_reps_for_l2(mats, 1, l2)
+    model_layers = bench.WORKLOADS[name].get("model_layers", 1)
+    reps = bench.stack_reps_for_l2(mats, 1, l2, 4.0, model_layers)
     per = sum(bench.algorithmic_bytes(*m, 1) for m in mats)
     assert reps * per >= 4 * l2
-    assert (reps - 1) * per < 4 * l2
+    # the model's own depth, or the fewest copies that reach 4x L2
+    assert reps == model_layers or (reps - 1) * per < 4 * l2
+
+
+def test_headline_is_the_70b_mlp_stack():
+    """The default (headline) workload is the 80-layer Llama-2-70B MLP stack at
+    0.1 BPW, whose packed bytes are several times the L2 cache."""
+    wl = bench.WORKLOADS[bench.DEFAULT_WORKLOAD]
+    assert wl["mats"] == [(8192, 28672, 620, False), (8192, 28672, 620, False), (28672, 8192, 620, False)]
+    assert wl["model_layers"] == 80
+    per = sum(bench.algorithmic_bytes(*m, 1) for m in wl["mats"])
+    assert 80 * per > 5 * 126 * 2 ** 20
 
 
 def test_traffic_record_only_for_the_captured_source(tmp_path, monkeypatch):

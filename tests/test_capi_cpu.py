@@ -152,3 +152,45 @@ def test_binding_rejects_buffers_the_library_would_misread():
         lb.Layer(256, 128, 4, []).c_struct()                   # no path
     with pytest.raises(ValueError):
         lb.HostStack([layer], 1)                               # path tensors on the CPU
+
+
+PER_DEVICE_CHECK = r"""
+#include <cstdio>
+#include "per_device.h"
+int main() {
+  lb::PerDevice cache;
+  int runs = 0, v = 0;
+  auto init = [&](int dev) { return [&, dev](int& out) { ++runs; out = 100 + dev; return 0; }; };
+  // first use on device 0 runs the set-up; device 1 has its own slot
+  if (cache.get(0, v, init(0)) || v != 100 || runs != 1) return 1;
+  if (cache.get(1, v, init(1)) || v != 101 || runs != 2) return 2;
+  // later uses return each device's own value without running it again
+  if (cache.get(0, v, init(0)) || v != 100 || runs != 2) return 3;
+  if (cache.get(1, v, init(1)) || v != 101 || runs != 2) return 4;
+  // a failed set-up is reported and leaves nothing cached
+  int fails = 0;
+  if (cache.get(2, v, [&](int& out) { ++fails; out = 7; return 9; }) != 9) return 5;
+  if (cache.get(2, v, [&](int& out) { ++fails; out = 7; return 0; }) || v != 7 || fails != 2) return 6;
+  // an ordinal outside the table runs the set-up every time
+  if (cache.get(lb::kMaxDevices, v, init(0)) || cache.get(lb::kMaxDevices, v, init(0)) || runs != 4) return 7;
+  std::puts("ok");
+  return 0;
+}
+"""
+
+
+def test_kernel_attribute_caches_are_per_device(tmp_path):
+    """The launch set-up caches (shared-memory attribute, occupancy) are kept
+    per device ordinal: a process driving two GPUs sets each one up."""
+    import shutil
+    import subprocess
+    gxx = shutil.which("g++")
+    if gxx is None:
+        pytest.skip("no g++")
+    src = tmp_path / "per_device_check.cc"
+    src.write_text(PER_DEVICE_CHECK)
+    exe = tmp_path / "per_device_check"
+    csrc = os.path.join(ROOT, "latent_binary_factorization_b200", "csrc")
+    subprocess.run([gxx, "-std=c++17", "-O1", "-I", csrc, str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", out.returncode

@@ -310,3 +310,95 @@ def test_batches_between_decode_and_prefill(lbm, batch):
     y = lb.forward(layer, torch.from_numpy(x).cuda())
     torch.cuda.synchronize()
     _check(y, orc.factored_forward(x, paths), f"B={batch}")
+
+
+@pytest.mark.parametrize("d_in,d_out,s,residual,batch", [
+    (28672, 8192, 620, False, 1),     # 70B MLP down projection, single path
+    (28672, 8192, 620, False, 4),
+    (28672, 8192, 302, True, 1),      # 70B MLP down projection, residual
+    (28672, 8192, 302, True, 4),
+    (8192, 28672, 302, True, 1),      # 70B MLP gate/up, residual
+    (8192, 28672, 302, True, 4),
+])
+def test_full_size_70b_mlp_matrices_sampled_rows(lbm, d_in, d_out, s, residual, batch):
+    """Every full-size matrix shape of the 70B MLP stack (14 input slices on
+    the down projection; the residual rank s = 302 with both paths), at batch
+    1 and 4, in the launch configuration of the stack benchmark: the oracle
+    computes 512 sampled output rows of every batch row."""
+    lb, layers = lbm
+    gen = torch.Generator(device="cuda").manual_seed(d_in + s + batch)
+    layer, host = layers.random_layer(d_in, d_out, s, residual, gen, keep_signs=True)
+    x = torch.randn(batch, d_in, generator=gen, device="cuda").half()
+    y = lb.forward(layer, x)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(d_in).choice(d_out, 512, replace=False))
+    y_ref = orc.factored_forward(x.cpu().numpy(), host, rows=rows)
+    _check(y[:, rows], y_ref, f"{d_in}->{d_out} s={s} res={residual} B={batch}")
+    assert lb.device_status() == 0
+
+
+def _outlier_activations(batch, d_in, seed, frac=0.01):
+    """x ~ N(0,1) with a fraction `frac` of the entries scaled by 10^2..10^3
+    (log-uniform): the heavy-tailed activations of real LLM layers."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((batch, d_in))
+    mask = rng.random((batch, d_in)) < frac
+    x[mask] *= 10.0 ** rng.uniform(2.0, 3.0, size=int(mask.sum()))
+    return x.astype(np.float16)
+
+
+@pytest.mark.parametrize("d_in,d_out,s,residual", [(4096, 4096, 86, True), (11008, 4096, 133, True),
+                                                   (4096, 4096, 188, False)])
+@pytest.mark.parametrize("batch", [1, 16])
+def test_outlier_activations(lbm, d_in, d_out, s, residual, batch):
+    """Outlier activations (1 % of the entries 100-1000x the rest): the 16-bit
+    fixed point of g*x per input slice and batch row keeps the result within
+    the forward's tolerances."""
+    lb, layers = lbm
+    paths = synth.layer(d_in, d_out, s, residual, seed=s + batch)
+    x = _outlier_activations(batch, d_in, seed=s + batch)
+    layer = layers.upload(paths, d_in, d_out, s)
+    y = lb.forward(layer, torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    _check(y, orc.factored_forward(x, paths), f"outliers B={batch}")
+
+
+@pytest.mark.parametrize("batch", [1, 4])
+def test_single_outlier_per_slice_and_small_rows(lbm, batch):
+    """The worst case for a per-slice step: one entry per 2048-input slice at
+    4000x the rest, and batch rows of very different magnitude (each row has
+    its own step)."""
+    lb, layers = lbm
+    d_in, d_out, s = 8192, 2048, 150
+    paths = synth.layer(d_in, d_out, s, True, seed=77)
+    rng = np.random.default_rng(77)
+    x = rng.standard_normal((batch, d_in))
+    for sl in range(d_in // 2048):
+        x[:, sl * 2048 + rng.integers(0, 2048)] = 4000.0
+    x *= (10.0 ** -np.arange(batch))[:, None]          # rows 1, 0.1, 0.01, ...
+    x = x.astype(np.float16)
+    layer = layers.upload(paths, d_in, d_out, s)
+    y = lb.forward(layer, torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    y_ref = orc.factored_forward(x, paths)
+    for b in range(batch):   # each row on its own scale
+        _check(y[b:b + 1], y_ref[b:b + 1], f"row {b}")
+
+
+def test_nonfinite_decode_input_is_reported(lbm):
+    """An inf or NaN in x cannot be quantised: the decode forward raises
+    LB_ERR_RANGE in the device status, and the next clean call raises nothing."""
+    lb, layers = lbm
+    range_bit = 1 << 7
+    d_in, d_out, s = 2048, 512, 64
+    paths = synth.layer(d_in, d_out, s, True, seed=23)
+    layer = layers.upload(paths, d_in, d_out, s)
+    xh = synth.activations(3, d_in, seed=23)
+    for bad in (float("inf"), float("nan")):
+        x = torch.from_numpy(xh).cuda()
+        x[1, 1000] = bad
+        lb.forward(layer, x)
+        assert lb.device_status() & range_bit
+    y = lb.forward(layer, torch.from_numpy(xh).cuda())
+    assert lb.device_status() == 0
+    _check(y, orc.factored_forward(xh, paths), "after a non-finite input")

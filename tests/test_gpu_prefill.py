@@ -157,3 +157,50 @@ def test_prefill_stack_in_cuda_graph(lbm):
     for i, (y, r) in enumerate(zip(Y, ref)):
         assert torch.equal(y, r), f"layer {i}"
     del g
+
+
+RANGE_BIT = 1 << 7   # LB_ERR_RANGE
+
+
+def test_prefill_range_errors_are_reported(lbm):
+    """Prefill holds x and t' in fp16.  A bf16 input beyond fp16's finite
+    range, and a latent value t' = l * t beyond it, cannot be held there: the
+    call raises LB_ERR_RANGE in the device status instead of returning inf
+    silently.  In-range inputs raise nothing."""
+    lb, layers = lbm
+    d_in, d_out, s, M = 512, 256, 40, 128
+    paths = synth.layer(d_in, d_out, s, True, seed=21)
+    layer = layers.upload(paths, d_in, d_out, s)
+    xt, _ = _x(M, d_in, seed=21, dtype=torch.bfloat16)
+    x = xt.cuda()
+    lb.forward(layer, x)
+    assert lb.device_status() == 0
+    # |x| = 1e5 is a finite bf16 value and an fp16 overflow
+    xb = x.clone()
+    xb[7, 100] = 1.0e5
+    lb.forward(layer, xb)
+    assert lb.device_status() & RANGE_BIT
+    assert lb.device_status() == 0            # read and cleared
+    # t' overflow: large latent scales make l * t exceed 65504
+    big = [dict(p) for p in paths]
+    for p in big:
+        p["l"] = np.full(s, 30000.0, np.float16)
+    big_layer = layers.upload(big, d_in, d_out, s)
+    lb.forward(big_layer, x)
+    assert lb.device_status() & RANGE_BIT
+    # the stream keeps working and in-range calls are exact again
+    y = lb.forward(layer, x)
+    assert lb.device_status() == 0
+    _check(y, orc.factored_forward(xt.float().numpy().astype(np.float64), paths), "after range errors")
+
+
+def test_prefill_nonfinite_fp16_input_is_reported(lbm):
+    lb, layers = lbm
+    d_in, d_out, s, M = 256, 128, 16, 128
+    paths = synth.layer(d_in, d_out, s, False, seed=22)
+    layer = layers.upload(paths, d_in, d_out, s)
+    xt, _ = _x(M, d_in, seed=22, dtype=torch.float16)
+    x = xt.cuda()
+    x[3, 5] = float("inf")
+    lb.forward(layer, x)
+    assert lb.device_status() & RANGE_BIT

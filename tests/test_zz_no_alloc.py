@@ -44,36 +44,65 @@ def _noalloc(env, layer, x):
     return y
 
 
-def _compare(y, y_ref):
-    a, b = y.float().cpu().numpy(), y_ref.float().cpu().numpy()
-    assert orc.rel_l2(a, b) <= REL_L2 and orc.max_abs_ratio(a, b) <= MAX_ABS
+def _compare_oracle(y, x_host, paths):
+    a = y.float().cpu().numpy()
+    ref = orc.factored_forward(x_host, paths)
+    assert orc.rel_l2(a, ref) <= REL_L2 and orc.max_abs_ratio(a, ref) <= MAX_ABS
+
+
+CASES = [(4096, 4096, 86, True, 1, 31),     # packed output pass (batch 1, two paths)
+         (8192, 2048, 300, False, 4, 32),
+         (4096, 4096, 86, True, 13, 33)]    # four groups of batch rows, both paths
 
 
 def test_noalloc_matches_regular_forward_twice_in_a_row(env):
+    """The same kernels on the same inputs as the regular forward: the outputs
+    are bitwise equal, and within the oracle's tolerance.  Calls follow one
+    another on different layers and on the same layer, so a region of the
+    shared scratch that kept the previous call's contents would show."""
     lb, layers, _ = env
-    cases = [(4096, 4096, 86, True, 1, 31), (8192, 2048, 300, False, 4, 32)]
     built = []
-    for d_in, d_out, s, res, batch, seed in cases:
+    for d_in, d_out, s, res, batch, seed in CASES:
         paths = synth.layer(d_in, d_out, s, res, seed=seed)
         layer = layers.upload(paths, d_in, d_out, s)
-        x = torch.from_numpy(synth.activations(batch, d_in, seed=seed)).cuda()
-        built.append((layer, x))
-    # two calls in a row, different layers: the second must not see the
-    # first call's leftovers in the shared scratch
-    for layer, x in built:
+        xh = synth.activations(batch, d_in, seed=seed)
+        built.append((layer, torch.from_numpy(xh).cuda(), xh, paths))
+    for layer, x, xh, paths in built:
         y_ref = lb.forward(layer, x).clone()
         y = _noalloc(env, layer, x)
         torch.cuda.synchronize()
-        _compare(y, y_ref)
-    # and the same layer twice in a row
-    layer, x = built[0]
-    y1 = _noalloc(env, layer, x).clone()
-    y2 = _noalloc(env, layer, x).clone()
+        assert torch.equal(y, y_ref)
+        _compare_oracle(y, xh, paths)
+    for layer, x, xh, paths in (built[0], built[2]):
+        y1 = _noalloc(env, layer, x).clone()
+        y2 = _noalloc(env, layer, x).clone()
+        torch.cuda.synchronize()
+        y_ref = lb.forward(layer, x)
+        torch.cuda.synchronize()
+        assert torch.equal(y1, y_ref) and torch.equal(y2, y_ref)
+    assert lb.device_status() == 0
+
+
+def test_noalloc_status_word_is_reported(env):
+    """The no-alloc calls keep their device error bits in the array's status
+    word, which littlebit_device_status reads and clears: a non-finite input
+    raises LB_ERR_RANGE there, and the next clean call raises nothing."""
+    lb, layers, _ = env
+    d_in, d_out, s, res, batch, seed = CASES[0]
+    paths = synth.layer(d_in, d_out, s, res, seed=seed)
+    layer = layers.upload(paths, d_in, d_out, s)
+    xh = synth.activations(batch, d_in, seed=seed)
+    x = torch.from_numpy(xh).cuda()
+    assert lb.device_status() == 0
+    xb = x.clone()
+    xb[0, 17] = float("inf")
+    _noalloc(env, layer, xb)
     torch.cuda.synchronize()
-    y_ref = lb.forward(layer, x)
+    assert lb.device_status() == 1 << 7          # LB_ERR_RANGE
+    y = _noalloc(env, layer, x)
     torch.cuda.synchronize()
-    _compare(y1, y_ref)
-    _compare(y2, y_ref)
+    assert lb.device_status() == 0
+    _compare_oracle(y, xh, paths)
 
 
 def test_noalloc_rejects_scratch_beyond_its_array(env):
