@@ -26,6 +26,9 @@ What it computes, and where each piece is defined
   only say the factors are binarised with sign() and stored at one bit each
   (the ``s(a+b)`` term of the cost formula); the bit layout is this library's
   own choice, restated here from its specification (tile shapes below).
+* ``latent_cache`` / ``expand``: the two halves of the forward, split where
+  the article (section 4, "KV cache" bullet) says a factorised K/V
+  projection can be cached: the r-wide latent t' instead of the d-wide row.
 * ``rotation_residual``: the gauge freedom the LittleBit-2 column (chapter 2,
   "solution 1", Joint-ITQ) relies on: (U R)(R^T V^T) = U V^T for orthogonal R.
 
@@ -213,6 +216,50 @@ def latent(x, path) -> np.ndarray:
     """t' = l (.) (V^T (g (.) x)) for one path, fp64 (batch x s)."""
     x = _f64(x)
     return ((x * _f64(path["g"])[None, :]) @ _f64(path["V"])) * _f64(path["l"])[None, :]
+
+
+# ---------------------------------------------------------------------------
+# the latent cache (Samsung LittleBit article, section 4, the KV-cache bullet)
+# ---------------------------------------------------------------------------
+#
+# Because a K or V projection is factorised, its output can be kept as the
+# latent t' (r numbers per token) instead of the d-wide projection; the
+# projection is rebuilt from the latent with the U pass when it is used.
+# A token's cache row holds the paths' latents side by side: path p's s values
+# at columns p*s .. p*s + s - 1 (the second half of the forward, written out).
+
+
+def latent_cache(x, paths) -> np.ndarray:
+    """Cache rows of x: [t'_1 | t'_2], t'_p = l_p (.) (V_p^T (g_p (.) x)), fp64
+    (batch x npaths*s)."""
+    return np.concatenate([latent(x, p) for p in paths], axis=1)
+
+
+def expand(t_cache, paths, rows=None) -> np.ndarray:
+    """The projection rebuilt from cache rows: y = sum_p h_p (.) (U_p t'_p),
+    fp64 (n x d_out); t_cache is n x npaths*s as written by latent_cache."""
+    t = _f64(t_cache)
+    s = np.asarray(paths[0]["l"]).shape[0]
+    y = None
+    for i, p in enumerate(paths):
+        tp = t[:, i * s:(i + 1) * s]
+        U = _f64(p["U"]) if rows is None else _f64(p["U"])[rows]
+        h = _f64(p["h"]) if rows is None else _f64(p["h"])[rows]
+        yp = (tp @ U.T) * h[None, :]
+        y = yp if y is None else y + yp
+    return y
+
+
+def cache_row_elems(s: int, npaths: int, align: int = 8) -> int:
+    """Elements of one cache row when rows are padded to whole 16-byte units
+    (8 fp16 values): npaths*s rounded up to a multiple of `align`."""
+    n = npaths * s
+    return -(-n // align) * align
+
+
+def kv_cache_ratio(d: int, s: int, npaths: int, align: int = 8) -> Fraction:
+    """Bytes of a d-wide fp16 K (or V) row over the bytes of its cache row."""
+    return Fraction(d, cache_row_elems(s, npaths, align))
 
 
 def dense_weight(path) -> np.ndarray:
