@@ -55,6 +55,8 @@ WORKLOADS = {
         "desc": "Llama-2-7B layer (4x 4096^2 s=86; 2x 4096->11008 and 11008->4096 s=133), 0.1 BPW residual",
         "mats": [(4096, 4096, 86, True)] * 4 + [(4096, 11008, 133, True)] * 2 + [(11008, 4096, 133, True)],
         "model_layers": 32,
+        # q, k, v read the block's normalised input; gate and up read the MLP's
+        "x_groups": [0, 0, 0, 1, 2, 2, 3],
     },
 }
 DEFAULT_WORKLOAD = "70b_mlp_0.1bpw_single"
@@ -167,23 +169,57 @@ def traffic_record(kernel: str, workload: str, model_layers: int):
 # our arm
 # ---------------------------------------------------------------------------
 
-def build_stack(mats, n_rep, batch, seed, device):
+def build_stack(mats, n_rep, batch, seed, device, x_groups=None):
+    """n_rep model layers of distinct random layers; within a model layer the
+    matrices of one x group read the same input tensor."""
     import torch
     from latent_binary_factorization_b200 import layers as lbl, littlebit as lb
     gen = torch.Generator(device=device).manual_seed(seed)
+    groups = x_groups or list(range(len(mats)))
     Ls = []
     for _ in range(n_rep):
         for (a, b, s, r) in mats:
             Ls.append(lbl.random_layer(a, b, s, r, gen, device=device)[0])
-    x_all = torch.randn(sum(L.d_in for L in Ls) * batch, generator=gen, device=device).half()
+    # one input per (model layer, group), back to back in x_all
+    first = {}
+    for k, g in enumerate(groups):
+        first.setdefault(g, k)
+    per_layer_x = sum(mats[k][0] for k in first.values())
+    x_all = torch.randn(n_rep * per_layer_x * batch, generator=gen, device=device).half()
     y_all = torch.empty(sum(L.d_out for L in Ls) * batch, dtype=torch.float16, device=device)
     xs, ys, xo, yo = [], [], 0, 0
+    for rep in range(n_rep):
+        gx = {}
+        for k, g in enumerate(groups):
+            if g not in gx:
+                a = mats[k][0]
+                gx[g] = x_all[xo:xo + batch * a].view(batch, a)
+                xo += batch * a
+            xs.append(gx[g])
     for L in Ls:
-        xs.append(x_all[xo:xo + batch * L.d_in].view(batch, L.d_in))
         ys.append(y_all[yo:yo + batch * L.d_out].view(batch, L.d_out))
-        xo += batch * L.d_in
         yo += batch * L.d_out
     return lb.Stack(Ls, xs, ys), Ls, x_all, y_all
+
+
+def shared_x_bytes(mats, x_groups, batch):
+    """Input bytes not read again because matrices of a model layer share
+    their x (one read per group instead of one per matrix)."""
+    if not x_groups:
+        return 0
+    seen, saved = set(), 0
+    for (a, _, _, _), g in zip(mats, x_groups):
+        if g in seen:
+            saved += 2 * batch * a
+        seen.add(g)
+    return saved
+
+
+def layer_bytes(name, batch):
+    """Algorithmic bytes of one model layer of a workload (shared inputs read once)."""
+    wl = WORKLOADS[name]
+    return (sum(algorithmic_bytes(*m, batch) for m in wl["mats"])
+            - shared_x_bytes(wl["mats"], wl.get("x_groups"), batch))
 
 
 def stack_reps_for_l2(mats, batch, l2_bytes, factor=4.0, model_layers=1):
@@ -340,8 +376,11 @@ def time_e2e(stack, x_all, y_all, steps, warmup, n_chunks):
     from latent_binary_factorization_b200 import littlebit as lb
     stream = torch.cuda.current_stream()
     hs = lb.HostStack(stack.layers, stack.batch, x_all.dtype)
-    xh = torch.empty(x_all.numel(), dtype=x_all.dtype, pin_memory=True)
-    xh.copy_(x_all.reshape(-1).cpu())
+    # the host call takes every layer's input back to back (a shared input is
+    # copied once per layer that reads it)
+    x_host = torch.cat([x.reshape(-1) for x in stack.xs]).cpu()
+    xh = torch.empty(x_host.numel(), dtype=x_all.dtype, pin_memory=True)
+    xh.copy_(x_host)
     yh = torch.empty(y_all.numel(), dtype=y_all.dtype, pin_memory=True)
 
     def step():
@@ -356,23 +395,26 @@ def time_e2e(stack, x_all, y_all, steps, warmup, n_chunks):
         step()
     t1.record(stream)
     torch.cuda.synchronize()
-    return t0.elapsed_time(t1), x_all.numel() * x_all.element_size(), y_all.numel() * y_all.element_size()
+    return t0.elapsed_time(t1), xh.numel() * xh.element_size(), y_all.numel() * y_all.element_size()
 
 
 def measure_workload(name, batch, steps, warmup, device, dist, world, l2, seed=1234, l2_factor=4.0):
     mats = WORKLOADS[name]["mats"]
+    x_groups = WORKLOADS[name].get("x_groups")
     model_layers = WORKLOADS[name].get("model_layers", 1) if l2_factor >= 4.0 else 1
     reps = stack_reps_for_l2(mats, batch, l2, l2_factor, model_layers)
-    stack, Ls, x_all, y_all = build_stack(mats, reps, batch, seed, device)
+    stack, Ls, x_all, y_all = build_stack(mats, reps, batch, seed, device, x_groups)
     n_layers = len(Ls)
     total_ms, per_ms = time_device(stack, steps, warmup, dist)
     red = max_over_ranks([total_ms] + [per_ms[k] for k in KERNELS], device)
     total_ms, per_ms = red[0], dict(zip(KERNELS, red[1:]))
-    alg = sum(algorithmic_bytes(*m, batch) for m in mats) * reps
+    alg = layer_bytes(name, batch) * reps
     kb = {k: sum(kernel_bytes(*m, batch)[k] for m in mats) * reps for k in KERNELS}
+    kb["quantise"] -= shared_x_bytes(mats, x_groups, batch) * reps
     ms_step = total_ms / steps
     res = {
         "workload": name, "desc": WORKLOADS[name]["desc"], "batch": batch, "layers_per_step": n_layers,
+        "shared_x_bytes_saved_per_step": shared_x_bytes(mats, x_groups, batch) * reps,
         "model_layers_per_step": reps, "stack_bytes": int(alg), "ms_per_step": ms_step,
         "us_per_matrix": 1e3 * ms_step / n_layers, "us_per_model_layer": 1e3 * ms_step / reps,
         "step_gbs": alg / (ms_step * 1e-3) / 1e9,

@@ -213,6 +213,85 @@ lb_status littlebit_linear_forward_many_host(const lb_layer* layers, int n, cons
                                              int batch, lb_dtype xdt, int n_chunks, void* stream);
 
 /*
+ * The latent cache (Samsung LittleBit article, section 4, the KV-cache bullet:
+ * because a K or V projection is factorised, the r-wide latent can be cached
+ * in place of the d-wide projection).  The forward splits at t'_p = l_p (.)
+ * V_p^T (g_p (.) x):
+ *   littlebit_latent_forward:  x rows -> cache rows [t'_1 | t'_2]
+ *   littlebit_latent_expand:   cache rows -> y = sum_p h_p (.) U_p t'_p
+ * so that latent_expand(latent_forward(x)) is the layer's output up to the
+ * rounding of the cache to fp16.
+ * A cache row holds npaths*s fp16 values, path p at columns p*s .. p*s+s-1;
+ * rows are littlebit_latent_row_elems(s, residual) elements apart (npaths*s
+ * rounded up to a multiple of 8, so every row starts on 16 bytes).  For the
+ * Llama-2-7B 4096x4096 projection at 0.1 BPW (s = 188, one path) a row is 192
+ * values against 4096 for the projection itself: 21.3x smaller.
+ */
+
+/* Elements between cache rows of a layer of rank s (0 for an invalid s). */
+int littlebit_latent_row_elems(int s, int residual);
+
+/*
+ * Cache rows of n layers' inputs: ts[i] (batch x littlebit_latent_row_elems
+ * fp16, 16-byte aligned, caller-owned) receives layer i's latents of xs[i]
+ * (batch x d_in, xdt).  Batch and dtype rules as littlebit_linear_forward_many
+ * (decode: the input quantisation, latent pass and finalize kernels; prefill:
+ * operand preparation and the first tcgen05 GEMM, whose epilogue writes the
+ * rows).  Errors as littlebit_linear_forward_many.
+ */
+lb_status littlebit_latent_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ts,
+                                   int batch, lb_dtype xdt, void* stream);
+
+/*
+ * Projections rebuilt from cache rows: ys[i] (rows x d_out, ydt) = sum_p h_p
+ * (.) U_p t'_p for the rows x littlebit_latent_row_elems fp16 cache rows at
+ * ts[i].  rows <= 16: the cache rows are quantised to the output pass's 16-bit
+ * operand (finalize kernel) and the output pass runs (ydt = LB_F16); rows a
+ * multiple of 128: the rows are laid out as the second tcgen05 GEMM's operand
+ * and that GEMM runs (ydt = LB_F16 or LB_BF16); other counts split as the
+ * forward does.  Errors as littlebit_linear_forward_many.
+ */
+lb_status littlebit_latent_expand(const lb_layer* layers, int n, const void* const* ts, void* const* ys, int rows,
+                                  lb_dtype ydt, void* stream);
+
+/*
+ * Initialisation of a path from real factors (the step before the forward).
+ * The caller supplies the rank-s truncated SVD of the weight (any library
+ * routine), split evenly: U' = U_s sqrt(S_s) (d_out x s) and V' = V_s sqrt(S_s)
+ * (d_in x s), fp32 row-major on the device.
+ *
+ * littlebit_init_dual_svid (Samsung LittleBit article, section 2, the
+ * Dual-SVID bullet: the factors' signs are the binary factors and rank-1
+ * approximations of their magnitudes give the scales):
+ *   U_bits_dev, V_bits_dev <- the packed signs of U', V' (sign(0) = +1; sizes
+ *     littlebit_packed_bytes(LB_ROLE_U, d_out, s) and (LB_ROLE_V, s, d_in));
+ *   |U'| ~ a_U b_U^T and |V'| ~ a_V b_V^T, the best rank-1 fits (top singular
+ *     pairs, non-negative), found by `iters` power steps (1..1000; 32 is
+ *     ample for factors of a truncated SVD);
+ *   h_dev <- a_U / mean(a_U) (d_out fp16), g_dev <- a_V / mean(a_V) (d_in fp16),
+ *   l_dev <- (mean(a_U) b_U) (.) (mean(a_V) b_V) (s fp16).
+ * Shapes as lb_layer; every pointer 16-byte aligned (l_dev 2).  Scratch is
+ * allocated and freed stream-ordered on `stream` (cudaMallocAsync).
+ * For residual compensation the second path is the same initialisation of
+ * the SVD of W - W_hat_1 (article section 2, residual-compensation bullet).
+ *
+ * littlebit_joint_itq (LittleBit-2 column, chapter 2, "solution 1"): X_dev
+ * holds the stacked factors [U'; V'] (n_rows = d_out + d_in rows of s fp32);
+ * `iters` (0..1000; the column's default is 50) alternations of
+ * B = sign(X R) and R = the orthogonal Procrustes solution (the polar factor
+ * of X^T B, by 30 Newton-Schulz steps) are run from R_dev (r_given = 1) or
+ * from the identity (r_given = 0); on return R_dev holds R (s x s fp32) and
+ * X_dev holds X R, i.e. U' R and V' R, whose product is U' V'^T.  Run it
+ * before littlebit_init_dual_svid.  fp32 products on the CUDA cores; scratch
+ * stream-ordered as above.
+ * Errors: LB_ERR_ARG, LB_ERR_SHAPE, LB_ERR_ALIGN, LB_ERR_CUDA.
+ */
+lb_status littlebit_init_dual_svid(const float* Uf_dev, const float* Vf_dev, int d_out, int d_in, int s, int iters,
+                                   void* U_bits_dev, void* V_bits_dev, uint16_t* h_dev, uint16_t* g_dev,
+                                   uint16_t* l_dev, void* stream);
+lb_status littlebit_joint_itq(float* X_dev, int n_rows, int s, int iters, float* R_dev, int r_given, void* stream);
+
+/*
  * The decode forward of littlebit_linear_forward (one layer, 1 <= batch <= 16,
  * fp16 x and y) for callers that cannot let the library allocate device
  * memory: for example a process whose device memory is reserved up front by

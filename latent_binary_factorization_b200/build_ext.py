@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "liblittlebit.so")
-SOURCES = ["littlebit_capi.cu", "pack.cu", "decode.cu", "prefill.cu", "noalloc.cu", "selfcheck.cu"]
+SOURCES = ["littlebit_capi.cu", "pack.cu", "decode.cu", "prefill.cu", "init.cu", "noalloc.cu", "selfcheck.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -23,7 +23,8 @@ def nvcc() -> str:
 
 def build(verbose: bool = False, force: bool = False) -> str:
     srcs = [os.path.join(CSRC, s) for s in SOURCES]
-    deps = srcs + [os.path.join(CSRC, "lb_internal.h"), os.path.join(INCLUDE, "littlebit.h")]
+    deps = srcs + [os.path.join(CSRC, "lb_internal.h"), os.path.join(CSRC, "per_device.h"),
+            os.path.join(INCLUDE, "littlebit.h")]
     if not force and os.path.exists(LIB):
         newest = max(os.path.getmtime(d) for d in deps)
         if os.path.getmtime(LIB) >= newest:

@@ -167,86 +167,105 @@ __device__ __forceinline__ uint32_t pack_byte(uint32_t a, uint32_t c, uint32_t d
   return __byte_perm(lo, hi, 0x5410);
 }
 
+// One (layer, path): u = g (.) x for one batch row from the lane's x chunks,
+// quantised and stored in the slice block at `blk`.
+__device__ __forceinline__ void quantise_row(const uint4 (&xq)[kQChunks], const uint16_t* __restrict__ g, int k0,
+                                             int nchunk, int row, int NC, int lane, unsigned char* blk, int B) {
+  uint32_t* frag = reinterpret_cast<uint32_t*>(blk + xq_stats_bytes(B));
+  float u[kQChunks][8];
+  float mx = 0.f;
+#pragma unroll
+  for (int j = 0; j < kQChunks; ++j) {
+    const int ch = lane + 32 * j;
+    const uint4 gq = ch < nchunk ? ld_nc(g + k0 + 8 * ch) : make_uint4(0, 0, 0, 0);
+    const uint32_t* xw = &xq[j].x;
+    const uint32_t* gw = &gq.x;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 xf = h2x2(xw[e]), gf = h2x2(gw[e]);
+      u[j][2 * e] = xf.x * gf.x;
+      u[j][2 * e + 1] = xf.y * gf.y;
+      mx = fmaxf(mx, fmaxf(fabsf(u[j][2 * e]), fabsf(u[j][2 * e + 1])));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const float inv = mx > 0.f ? kQMax / mx : 0.f;
+  int sum_hi = 0, sum_lo = 0;
+#pragma unroll
+  for (int j = 0; j < kQChunks; ++j) {
+    const int ch = lane + 32 * j;
+    uint32_t fb[8], fh[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      fb[e] = __float_as_uint(fmaf(u[j][e], inv, kRoundMagic));
+      fh[e] = fb[e] + 128u;
+    }
+    const uint32_t lw0 = pack_byte(fb[0], fb[1], fb[2], fb[3], 0), lw1 = pack_byte(fb[4], fb[5], fb[6], fb[7], 0);
+    const uint32_t hw0 = pack_byte(fh[0], fh[1], fh[2], fh[3], 1), hw1 = pack_byte(fh[4], fh[5], fh[6], fh[7], 1);
+    sum_hi = __dp4a((int)hw0, 0x01010101, __dp4a((int)hw1, 0x01010101, sum_hi));
+    sum_lo = __dp4a((int)lw0, 0x01010101, __dp4a((int)lw1, 0x01010101, sum_lo));
+    if (ch < nchunk) {
+      // inputs 8ch..8ch+7: K-block kb, offset kk0 (0, 8, 16, 24) inside it;
+      // kk < 16 -> b0 words of threads c = kk/4, else b1 words of c = (kk-16)/4
+      const int kb = ch >> 2, kk0 = (ch & 3) * 8;
+      const int cc = (kk0 & 15) >> 2, half = kk0 >> 4;
+      uint32_t* fhp = frag + ((size_t)kb * NC + 2 * row) * 8;   // column 2*row: 4 threads x (b0, b1)
+      uint32_t* flp = fhp + 8;                                  // column 2*row + 1
+      fhp[2 * cc + half] = hw0;
+      fhp[2 * (cc + 1) + half] = hw1;
+      flp[2 * cc + half] = lw0;
+      flp[2 * (cc + 1) + half] = lw1;
+    }
+  }
+  int vsum = 256 * sum_hi + sum_lo;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) vsum += __shfl_xor_sync(0xffffffffu, vsum, o);
+  if (lane == 0) {
+    TStat st;
+    st.step = mx > 0.f ? mx / kQMax : 0.f;
+    st.sum = vsum;
+    st.pad[0] = st.pad[1] = 0;
+    reinterpret_cast<TStat*>(blk)[row] = st;
+  }
+}
+
+// Work item = (group of layers that read the same x, 2048-input slice): the
+// item reads each batch row's x slice once and quantises g (.) x for every
+// path of every layer of the group (layers chained by x_next from the
+// group's first layer, whose x_begin numbers the group's items).
 __global__ void __launch_bounds__(kQWarps * 32) quantise_input_kernel(const DecodeArgs a) {
   grid_dep_launch();
   const int lane = threadIdx.x & 31;
   const int item = blockIdx.x * kQWarps + (threadIdx.x >> 5);
   if (item >= a.x_items) return;
   const int B = a.batch, NC = 2 * xq_rows(B);
-  const LayerDesc& L = a.layers[layer_of(a.item_layer.x, a.n_layers, item)];
-  const int p = (item - L.x_begin) / L.n_slices, sl = item - L.x_begin - p * L.n_slices;
-  const int d_in = L.d_in, k0 = sl * kVSlice;
+  const int first = layer_of(a.item_layer.x, a.n_layers, item);
+  const LayerDesc& L0 = a.layers[first];
+  const int sl = item - L0.x_begin;
+  const int d_in = L0.d_in, k0 = sl * kVSlice;
   const int nchunk = min(kVSlice, d_in - k0) / 8;
   const size_t blk_off = (size_t)sl * xq_slice_bytes(B);
 
   unsigned bad = 0;   // an input x that is inf or NaN (LB_ERR_RANGE)
-  {
-    const PathDesc& P = L.p[p];
-    unsigned char* blk = P.ws.xq + blk_off;
-    uint32_t* frag = reinterpret_cast<uint32_t*>(blk + xq_stats_bytes(B));
-    // rows B .. 4*nb-1 of the block are never read: their product columns are
-    // independent of the batch rows' and their sums are discarded
+  // rows B .. 4*nb-1 of a block are never read: their product columns are
+  // independent of the batch rows' and their sums are discarded
 #pragma unroll 1
-    for (int row = 0; row < B; ++row) {
-      float u[kQChunks][8];
-      float mx = 0.f;
+  for (int row = 0; row < B; ++row) {
+    uint4 xq[kQChunks];
 #pragma unroll
-      for (int j = 0; j < kQChunks; ++j) {
-        const int ch = lane + 32 * j;
-        const bool live = ch < nchunk;
-        const uint4 xq = live ? ld_nc(L.x + (size_t)row * d_in + k0 + 8 * ch) : make_uint4(0, 0, 0, 0);
-        const uint4 gq = live ? ld_nc(P.g + k0 + 8 * ch) : make_uint4(0, 0, 0, 0);
-        const uint32_t* xw = &xq.x;
-        const uint32_t* gw = &gq.x;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          bad |= half2_nonfinite(xw[e]);
-          const float2 xf = h2x2(xw[e]), gf = h2x2(gw[e]);
-          u[j][2 * e] = xf.x * gf.x;
-          u[j][2 * e + 1] = xf.y * gf.y;
-          mx = fmaxf(mx, fmaxf(fabsf(u[j][2 * e]), fabsf(u[j][2 * e + 1])));
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float inv = mx > 0.f ? kQMax / mx : 0.f;
-      int sum_hi = 0, sum_lo = 0;
-#pragma unroll
-      for (int j = 0; j < kQChunks; ++j) {
-        const int ch = lane + 32 * j;
-        uint32_t fb[8], fh[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          fb[e] = __float_as_uint(fmaf(u[j][e], inv, kRoundMagic));
-          fh[e] = fb[e] + 128u;
-        }
-        const uint32_t lw0 = pack_byte(fb[0], fb[1], fb[2], fb[3], 0), lw1 = pack_byte(fb[4], fb[5], fb[6], fb[7], 0);
-        const uint32_t hw0 = pack_byte(fh[0], fh[1], fh[2], fh[3], 1), hw1 = pack_byte(fh[4], fh[5], fh[6], fh[7], 1);
-        sum_hi = __dp4a((int)hw0, 0x01010101, __dp4a((int)hw1, 0x01010101, sum_hi));
-        sum_lo = __dp4a((int)lw0, 0x01010101, __dp4a((int)lw1, 0x01010101, sum_lo));
-        if (ch < nchunk) {
-          // inputs 8ch..8ch+7: K-block kb, offset kk0 (0, 8, 16, 24) inside it;
-          // kk < 16 -> b0 words of threads c = kk/4, else b1 words of c = (kk-16)/4
-          const int kb = ch >> 2, kk0 = (ch & 3) * 8;
-          const int cc = (kk0 & 15) >> 2, half = kk0 >> 4;
-          uint32_t* fhp = frag + ((size_t)kb * NC + 2 * row) * 8;   // column 2*row: 4 threads x (b0, b1)
-          uint32_t* flp = fhp + 8;                                  // column 2*row + 1
-          fhp[2 * cc + half] = hw0;
-          fhp[2 * (cc + 1) + half] = hw1;
-          flp[2 * cc + half] = lw0;
-          flp[2 * (cc + 1) + half] = lw1;
-        }
-      }
-      int vsum = 256 * sum_hi + sum_lo;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) vsum += __shfl_xor_sync(0xffffffffu, vsum, o);
-      if (lane == 0) {
-        TStat st;
-        st.step = mx > 0.f ? mx / kQMax : 0.f;
-        st.sum = vsum;
-        st.pad[0] = st.pad[1] = 0;
-        reinterpret_cast<TStat*>(blk)[row] = st;
-      }
+    for (int j = 0; j < kQChunks; ++j) {
+      const int ch = lane + 32 * j;
+      xq[j] = ch < nchunk ? ld_nc(L0.x + (size_t)row * d_in + k0 + 8 * ch) : make_uint4(0, 0, 0, 0);
+      bad |= half2_nonfinite(xq[j].x) | half2_nonfinite(xq[j].y) | half2_nonfinite(xq[j].z) |
+             half2_nonfinite(xq[j].w);
+    }
+#pragma unroll 1
+    for (int li = first; li >= 0; li = a.layers[li].x_next) {
+      const LayerDesc& L = a.layers[li];
+#pragma unroll 1
+      for (int p = 0; p < L.npaths; ++p)
+        quantise_row(xq, L.p[p].g, k0, nchunk, row, NC, lane, L.p[p].ws.xq + blk_off, B);
     }
   }
   if (__any_sync(0xffffffffu, bad != 0) && lane == 0) atomicOr(a.status, kStatusRange);
@@ -594,6 +613,7 @@ __global__ void __launch_bounds__(kFWarps * 32) finalize_kernel(const DecodeArgs
   const int s = L.s, S16 = (s + 15) & ~15, nkt = (s + 31) >> 5;
   const int ns = L.n_slices, ng = (ns + 3) >> 2;
   const bool packed = a.packed != 0;   // the output pass takes both paths as one K range
+  const int mode = a.mode;
 #pragma unroll 1
   for (int b = 0; b < B; ++b) {
     if (tid == 0) {
@@ -601,28 +621,36 @@ __global__ void __launch_bounds__(kFWarps * 32) finalize_kernel(const DecodeArgs
       s_sum = 0;
     }
     __syncthreads();
-    // a latent row's slice partials are contiguous float4s, summed in slice order
     float mx = 0.f;
 #pragma unroll 2
     for (int k = warp; k < nkt; k += kFWarps) {
       const int j = lane + 32 * k;
-      const int jc = min(j, S16 - 1);   // rows past S16 clamp (finite; zeroed below)
-      const float4* pp = reinterpret_cast<const float4*>(P.ws.partial) + ((size_t)b * S16 + jc) * ng;
-      float t = 0.f;
+      float v;
+      if (mode == kModeExpand) {
+        // t' from the caller's cache row (l already applied)
+        v = j < s ? h2f(L.x[(size_t)b * L.t_ld + pi * s + j]) : 0.f;
+      } else {
+        // a latent row's slice partials are contiguous float4s, summed in slice order
+        const int jc = min(j, S16 - 1);   // rows past S16 clamp (finite; zeroed below)
+        const float4* pp = reinterpret_cast<const float4*>(P.ws.partial) + ((size_t)b * S16 + jc) * ng;
+        float t = 0.f;
 #pragma unroll 4
-      for (int q4 = 0; q4 < ng; ++q4) {
-        const float4 f = pp[q4];
-        const int q = 4 * q4;
-        t += f.x;
-        if (q + 1 < ns) t += f.y;
-        if (q + 2 < ns) t += f.z;
-        if (q + 3 < ns) t += f.w;
+        for (int q4 = 0; q4 < ng; ++q4) {
+          const float4 f = pp[q4];
+          const int q = 4 * q4;
+          t += f.x;
+          if (q + 1 < ns) t += f.y;
+          if (q + 2 < ns) t += f.z;
+          if (q + 3 < ns) t += f.w;
+        }
+        const float l = h2f(P.l[min(j, s - 1)]);
+        v = j < s ? t * l : 0.f;
+        if (mode == kModeLatent && j < s) L.y[(size_t)b * L.t_ld + pi * s + j] = f2h(v);
       }
-      const float l = h2f(P.l[min(j, s - 1)]);
-      const float v = j < s ? t * l : 0.f;
       s_t[j] = v;
       mx = fmaxf(mx, fabsf(v));
     }
+    if (mode == kModeLatent) continue;   // the cache row is the result (mode is uniform over the CTA)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     if (lane == 0) atomicMax(&s_mx, __float_as_uint(mx));

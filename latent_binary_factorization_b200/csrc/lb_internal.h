@@ -127,17 +127,32 @@ struct PathDesc {
   PathScratch ws;
 };
 
+// What a forward call computes (Samsung LittleBit article, section 4, the
+// KV-cache bullet: a factorised K/V projection can be cached as its latent):
+//   kModeForward: y = layer(x)                       (all passes)
+//   kModeLatent:  t = [t'_1 | t'_2] cache rows of x    (no output pass; the
+//                 latent rows are written where y would go)
+//   kModeExpand:  y = sum_p h_p (.) U_p t'_p from cache rows (no input or
+//                 latent pass; the cache rows are read where x would be)
+// A cache row holds npaths*s fp16 values, path p at columns p*s .. p*s+s-1,
+// rows latent_row_elems(s, npaths) elements apart.
+enum CallMode { kModeForward = 0, kModeLatent = 1, kModeExpand = 2 };
+inline int latent_row_elems(int s, int npaths) { return (npaths * s + 7) / 8 * 8; }
+
 struct LayerDesc {
   PathDesc p[2];
-  const uint16_t* x;  // [batch][d_in] fp16
-  uint16_t* y;        // [batch][d_out] fp16
+  const uint16_t* x;  // [batch][d_in] fp16; kModeExpand: the cache rows [batch][t_ld]
+  uint16_t* y;        // [batch][d_out] fp16; kModeLatent: the cache rows [batch][t_ld]
+  int t_ld;           // elements between cache rows (latent_row_elems)
   int d_in, d_out, s, npaths;
   int n_slices;       // ceil(d_in / kVSlice)
   int n_rchunks;      // ceil(s16 / 16 / (2 * latent-pass warps))
   int v_begin;        // first latent-pass work item of this layer
   int u_begin;        // first output-pass work item of this layer
   int p_begin;        // first (layer, path) index of this layer
-  int x_begin;        // first quantise-pass item (layer, path, input slice) of this layer
+  int x_begin;        // first quantise-pass item (x group, input slice) of this layer's x group
+                      // (set on the group's first layer)
+  int x_next;         // next layer of the call that reads the same x (same pointer and d_in), or -1
 };
 
 // Layer index of every work item of each pass (device arrays built with the
@@ -158,9 +173,10 @@ struct DecodeArgs {
   int v_items;              // total latent-pass items
   int u_items;              // total output-pass items (layer, 128-row block)
   int p_items;              // total (layer, path) pairs
-  int x_items;              // total quantise-pass items (layer, path, input slice)
+  int x_items;              // total quantise-pass items (group of layers sharing x, input slice)
   int v_warps;              // latent-pass CTA width (3 or 4; latent_warps)
   int packed;               // batch 1 with a residual layer: paths share the output pass's product
+  int mode;                 // CallMode
 };
 
 // Launchers (decode.cu), in stream order quantise -> latent -> finalize ->
@@ -180,12 +196,13 @@ size_t prefill_layer_bytes(int M, int d_in, int d_out, int s, int npaths);
 long long prefill_layer_tiles(int M, int d_out, int s, int npaths);   // GEMM1 + GEMM2 tiles
 size_t prefill_table_bytes(int n_layers, long long tiles);
 constexpr int kPrefillMaxGroup = 4096;   // layers per chunk
+constexpr int kPrepKinds = 4;            // preparation steps: x, B1, B2, T' from cache rows
 // A chunk of layers: its table's place in the call's table image and the two
 // GEMMs' tile counts and grids.
 struct PrefillPlan {
   int n;
   int tiles1, tiles2, grid1, grid2;
-  int prep_grid[3];              // blocks of the grouped x, B1 and B2 preparation launches
+  int prep_grid[kPrepKinds];     // blocks of the grouped x, B1, B2 and cache-to-T' preparation launches
   size_t table_off, table_bytes;
   size_t jobs_off;               // preparation jobs, from table_off
 };
@@ -193,7 +210,8 @@ struct PrefillPlan {
 // per-layer preparation jobs) to img; its device pointers refer to the
 // chunk's operand buffers at `bufs`, the inputs xs and the outputs ys.
 void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const* ys, int n, int M, int x_bf16,
-                        unsigned char* bufs, int num_sms, std::vector<unsigned char>& img, PrefillPlan& plan);
+                        int mode, unsigned char* bufs, int num_sms, std::vector<unsigned char>& img,
+                        PrefillPlan& plan);
 // A chunk's operand preparation (three grouped launches), then its two
 // grouped GEMM launches; both read the table image uploaded at table_dev.
 cudaError_t launch_prefill_prep(const PrefillPlan& plan, const unsigned char* table_dev, unsigned int* status,
@@ -217,6 +235,14 @@ size_t path_scratch_bytes(const lb_layer& L, int batch);
 // noalloc.cu: device address of the allocation-free forward's status word on
 // device `dev`, or null before that entry point's first call on the device.
 unsigned int* noalloc_status_word(int dev);
+
+// init.cu: Dual-SVID and Joint-ITQ (scratch sizes in floats)
+size_t dual_svid_scratch_floats(int d_out, int d_in, int s);
+cudaError_t launch_dual_svid(const float* Uf, const float* Vf, int d_out, int d_in, int s, int iters, void* U_bits,
+                             void* V_bits, uint16_t* h, uint16_t* g, uint16_t* l, float* scratch, cudaStream_t st);
+size_t itq_scratch_floats(int n_rows, int s);
+cudaError_t launch_joint_itq(float* X, int n_rows, int s, int iters, int ns_steps, float* R, int r_given,
+                             float* scratch, cudaStream_t st);
 
 // pack.cu
 cudaError_t launch_unpack(const void* src, int n_long, int s, lb_role role, int8_t* dst, cudaStream_t st);

@@ -171,27 +171,32 @@ lb_status grow_workspace(Workspace& ws, size_t cap, cudaStream_t st) {
 
 // The four decode launches of a prepared call; events[i] (if given) is
 // recorded right after launch i.
+// The launches of a prepared call: all four for a forward, the first three
+// for a latent-only call, finalize and output for an expand call.
 lb_status decode_launch(const lb::DecodeArgs& a, int max_s16, int sms, cudaStream_t st, const cudaEvent_t* events,
                         int n_events) {
   auto mark = [&](int i) { return i < n_events && events[i] ? cudaEventRecord(events[i], st) : cudaSuccess; };
-  cudaError_t e = lb::launch_quantise_pass(a, st);
-  if (e == cudaSuccess) e = mark(0);
-  if (e == cudaSuccess) e = lb::launch_latent_pass(a, max_s16, sms, st);
-  if (e == cudaSuccess) e = mark(1);
+  cudaError_t e = cudaSuccess;
+  if (a.mode != lb::kModeExpand) {
+    e = lb::launch_quantise_pass(a, st);
+    if (e == cudaSuccess) e = mark(0);
+    if (e == cudaSuccess) e = lb::launch_latent_pass(a, max_s16, sms, st);
+    if (e == cudaSuccess) e = mark(1);
+  }
   if (e == cudaSuccess) e = lb::launch_finalize_pass(a, max_s16, st);
   if (e == cudaSuccess) e = mark(2);
-  if (e == cudaSuccess) e = lb::launch_output_pass(a, sms, st);
+  if (e == cudaSuccess && a.mode != lb::kModeLatent) e = lb::launch_output_pass(a, sms, st);
   return e == cudaSuccess ? LB_OK : cuda_fail(e);
 }
 
 lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
-                         cudaStream_t st, const cudaEvent_t* events, int n_events, int tag) {
+                         int mode, cudaStream_t st, const cudaEvent_t* events, int n_events, int tag) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
   std::lock_guard<std::mutex> lock(g_mu);
   Workspace& ws = g_ws[{dev, st, tag}];
-  std::vector<unsigned char> key = call_key('D', layers, n, xs, ys, batch, 0);
+  std::vector<unsigned char> key = call_key((char)('D' + 16 * mode), layers, n, xs, ys, batch, 0);
   if (ws.buf && ws.key == key) return decode_launch(ws.dargs, ws.d_max_s16, num_sms(dev), st, events, n_events);
   ws.key.clear();
 
@@ -200,13 +205,29 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
     n_rb = lb::s16(layers[i].s) / 16;
     w = (double)(layers[i].residual + 1) * n_rb * layers[i].d_in;
   });
+  // layers that read the same x (same pointer and width) form one quantise
+  // group: x_lead[i] is the group's first layer, x_next[i] the next member
+  std::vector<int> x_lead(n), x_next(n, -1);
+  {
+    std::map<std::pair<const void*, int>, int> last;   // (x, d_in) -> latest member
+    for (int i = 0; i < n; ++i) {
+      auto it = last.find({xs[i], layers[i].d_in});
+      if (it == last.end()) {
+        x_lead[i] = i;
+      } else {
+        x_lead[i] = x_lead[it->second];
+        x_next[it->second] = i;
+      }
+      last[{xs[i], layers[i].d_in}] = i;
+    }
+  }
   int x_items = 0, v_items = 0, p_items = 0, u_items = 0;
   int max_s16 = 16;
   size_t scratch = 0;
   for (int i = 0; i < n; ++i) {
     const lb_layer& L = layers[i];
     const int npaths = L.residual + 1, n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
-    x_items += npaths * n_slices;
+    if (x_lead[i] == i) x_items += n_slices;
     v_items += npaths * n_slices * lb::ceil_div(lb::s16(L.s) / 16, 2 * vw);
     p_items += npaths;
     u_items += L.d_out / lb::kUTileRows;
@@ -249,13 +270,16 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
     D.d_out = L.d_out;
     D.s = L.s;
     D.npaths = L.residual + 1;
+    D.t_ld = lb::latent_row_elems(L.s, D.npaths);
     D.n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
     D.n_rchunks = lb::ceil_div(lb::s16(L.s) / 16, 2 * vw);
-    D.x_begin = xi;
+    D.x_begin = x_lead[i] == i ? xi : -1;
+    D.x_next = x_next[i];
     D.v_begin = vi;
     D.p_begin = pi;
     D.u_begin = ui;
-    for (int k = 0; k < D.npaths * D.n_slices; ++k) xm[xi++] = i;
+    if (x_lead[i] == i)
+      for (int k = 0; k < D.n_slices; ++k) xm[xi++] = i;
     for (int k = 0; k < D.npaths * D.n_slices * D.n_rchunks; ++k) vm[vi++] = i;
     for (int k = 0; k < D.npaths; ++k) pm[pi++] = i;
     for (int k = 0; k < L.d_out / lb::kUTileRows; ++k) um[ui++] = i;
@@ -302,6 +326,7 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   a.p_items = p_items;
   a.x_items = x_items;
   a.v_warps = vw;
+  a.mode = mode;
   a.packed = 0;
   if (batch == 1)
     for (int i = 0; i < n; ++i) a.packed |= layers[i].residual;
@@ -337,13 +362,13 @@ cudaError_t ensure_side(Workspace& ws) {
 lb_status prefill_launch(Workspace& ws, cudaStream_t st);
 
 lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
-                          int x_bf16, cudaStream_t st, int tag) {
+                          int x_bf16, int mode, cudaStream_t st, int tag) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
   std::lock_guard<std::mutex> lock(g_mu);
   Workspace& ws = g_ws[{dev, st, tag}];
-  std::vector<unsigned char> key = call_key('P', layers, n, xs, ys, batch, x_bf16);
+  std::vector<unsigned char> key = call_key((char)('P' + 16 * mode), layers, n, xs, ys, batch, x_bf16);
   if (ws.buf && ws.key == key) return prefill_launch(ws, st);
   ws.key.clear();
   // plan the chunks: operand bytes per chunk (a workspace half) and table bytes
@@ -392,6 +417,7 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
     D.d_out = L.d_out;
     D.s = L.s;
     D.npaths = L.residual + 1;
+    D.t_ld = lb::latent_row_elems(L.s, D.npaths);
     for (int p = 0; p < D.npaths; ++p) {
       D.p[p].V = static_cast<const uint4*>(L.path[p].V_bits);
       D.p[p].U = static_cast<const uint4*>(L.path[p].U_bits);
@@ -408,7 +434,7 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
   std::vector<lb::PrefillPlan> plans(n_chunks);
   for (int c = 0; c < n_chunks; ++c)
     lb::plan_prefill_chunk(descs.data() + starts[c], xs + starts[c], ys + starts[c], starts[c + 1] - starts[c],
-                           batch, x_bf16, chunk_bufs(c), sms, img, plans[c]);
+                           batch, x_bf16, mode, chunk_bufs(c), sms, img, plans[c]);
   if (img.size() > tables) return LB_ERR_SHAPE;   // the plan above sized the tables
   if (ws.table.size() != img.size() || std::memcmp(ws.table.data(), img.data(), img.size()) != 0) {
     // pageable source: the copy is staged before the call returns
@@ -546,34 +572,60 @@ lb_status check_call(const lb_layer* layers, int n, int batch, lb_dtype xdt) {
 // `base`: batch <= 16 on the decode path, a multiple of 128 on the prefill
 // path, any other batch (fp16) the leading multiple of 128 rows through the
 // prefill path and the rest through the decode path in groups of at most 16
-// rows (rows are contiguous in x and y, so a group is an offset view).
+// rows (rows are contiguous in the inputs and outputs, so a group is an
+// offset view).  `mode` (CallMode) selects the whole forward or one of its
+// halves around the latent cache rows.
 lb_status forward_dispatch(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
-                           lb_dtype xdt, cudaStream_t st, const cudaEvent_t* evs, int n_events, int base) {
+                           lb_dtype xdt, int mode, cudaStream_t st, const cudaEvent_t* evs, int n_events,
+                           int base) {
   if (batch <= lb::kMaxBatchDecode)
-    return decode_forward(layers, n, xs, ys, batch, st, evs, n_events, ws_tag(base, 1));
+    return decode_forward(layers, n, xs, ys, batch, mode, st, evs, n_events, ws_tag(base, 1));
   if (batch % 128 == 0)
-    return prefill_forward(layers, n, xs, ys, batch, xdt == LB_BF16 ? 1 : 0, st, ws_tag(base, 0));
+    return prefill_forward(layers, n, xs, ys, batch, xdt == LB_BF16 ? 1 : 0, mode, st, ws_tag(base, 0));
   std::vector<const void*> xv(n);
   std::vector<void*> yv(n);
+  // bytes per row of each layer's input and output (2-byte elements)
+  auto in_row = [&](int i) -> size_t {
+    return 2 * (size_t)(mode == lb::kModeExpand ? lb::latent_row_elems(layers[i].s, layers[i].residual + 1)
+                                                : layers[i].d_in);
+  };
+  auto out_row = [&](int i) -> size_t {
+    return 2 * (size_t)(mode == lb::kModeLatent ? lb::latent_row_elems(layers[i].s, layers[i].residual + 1)
+                                                : layers[i].d_out);
+  };
   auto views = [&](int r0) {
     for (int i = 0; i < n; ++i) {
-      xv[i] = static_cast<const unsigned char*>(xs[i]) + (size_t)r0 * layers[i].d_in * 2;
-      yv[i] = static_cast<unsigned char*>(ys[i]) + (size_t)r0 * layers[i].d_out * 2;
+      xv[i] = static_cast<const unsigned char*>(xs[i]) + (size_t)r0 * in_row(i);
+      yv[i] = static_cast<unsigned char*>(ys[i]) + (size_t)r0 * out_row(i);
     }
   };
   const int m128 = batch / 128 * 128;
   if (m128 > 0) {
-    const lb_status r = prefill_forward(layers, n, xs, ys, m128, 0, st, ws_tag(base, 0));
+    const lb_status r = prefill_forward(layers, n, xs, ys, m128, 0, mode, st, ws_tag(base, 0));
     if (r != LB_OK) return r;
   }
   for (int r0 = m128, grp = 0; r0 < batch; r0 += lb::kMaxBatchDecode, ++grp) {
     views(r0);
     const int rows = std::min(lb::kMaxBatchDecode, batch - r0);
-    const lb_status r = decode_forward(layers, n, xv.data(), yv.data(), rows, st, r0 == m128 ? evs : nullptr,
-                                       r0 == m128 ? n_events : 0, ws_tag(base, 1 + grp));
+    const lb_status r = decode_forward(layers, n, xv.data(), yv.data(), rows, mode, st,
+                                       r0 == m128 ? evs : nullptr, r0 == m128 ? n_events : 0, ws_tag(base, 1 + grp));
     if (r != LB_OK) return r;
   }
   return LB_OK;
+}
+
+// Checks of a device-pointer call's buffers, then the dispatch.
+lb_status checked_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ys, int batch,
+                          lb_dtype xdt, int mode, void* stream, const cudaEvent_t* evs, int n_events) {
+  if (!layers || !xs || !ys || n < 1) return LB_ERR_ARG;
+  const lb_status chk = check_call(layers, n, batch, xdt);
+  if (chk != LB_OK) return chk;
+  for (int i = 0; i < n; ++i) {
+    if (!xs[i] || !ys[i]) return LB_ERR_ARG;
+    if (!aligned(xs[i], 16) || !aligned(ys[i], 16)) return LB_ERR_ALIGN;
+  }
+  return forward_dispatch(layers, n, xs, ys, batch, xdt, mode, static_cast<cudaStream_t>(stream), evs, n_events,
+                          0);
 }
 
 }  // namespace
@@ -618,15 +670,23 @@ lb_status littlebit_unpack_signs(const void* src_dev, lb_role role, int n_long, 
 lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, const void* const* xs,
                                               void* const* ys, int batch, lb_dtype xdt, void* stream,
                                               void* const* events, int n_events) {
-  if (!layers || !xs || !ys || n < 1) return LB_ERR_ARG;
-  const lb_status chk = check_call(layers, n, batch, xdt);
-  if (chk != LB_OK) return chk;
-  for (int i = 0; i < n; ++i) {
-    if (!xs[i] || !ys[i]) return LB_ERR_ARG;
-    if (!aligned(xs[i], 16) || !aligned(ys[i], 16)) return LB_ERR_ALIGN;
-  }
-  return forward_dispatch(layers, n, xs, ys, batch, xdt, static_cast<cudaStream_t>(stream),
-                          reinterpret_cast<const cudaEvent_t*>(events), n_events, 0);
+  return checked_forward(layers, n, xs, ys, batch, xdt, lb::kModeForward, stream,
+                         reinterpret_cast<const cudaEvent_t*>(events), n_events);
+}
+
+int littlebit_latent_row_elems(int s, int residual) {
+  if (s < 1 || s > lb::kMaxRank || (residual != 0 && residual != 1)) return 0;
+  return lb::latent_row_elems(s, residual + 1);
+}
+
+lb_status littlebit_latent_forward(const lb_layer* layers, int n, const void* const* xs, void* const* ts,
+                                   int batch, lb_dtype xdt, void* stream) {
+  return checked_forward(layers, n, xs, ts, batch, xdt, lb::kModeLatent, stream, nullptr, 0);
+}
+
+lb_status littlebit_latent_expand(const lb_layer* layers, int n, const void* const* ts, void* const* ys, int rows,
+                                  lb_dtype ydt, void* stream) {
+  return checked_forward(layers, n, ts, ys, rows, ydt, lb::kModeExpand, stream, nullptr, 0);
 }
 
 lb_status littlebit_linear_forward_many(const lb_layer* layers, int n, const void* const* xs, void* const* ys,
@@ -773,8 +833,8 @@ lb_status littlebit_linear_forward_many_host(const lb_layer* layers, int n, cons
       r = cuda_fail(e);
       break;
     }
-    r = forward_dispatch(layers + i0, i1 - i0, hp.xs.data() + i0, hp.ys.data() + i0, batch, xdt, st, nullptr, 0,
-                         c + 1);
+    r = forward_dispatch(layers + i0, i1 - i0, hp.xs.data() + i0, hp.ys.data() + i0, batch, xdt, lb::kModeForward,
+                         st, nullptr, 0, c + 1);
     if (r != LB_OK) break;
     e = cudaEventRecord(hp.fwd_done[c], st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(hp.d2h, hp.fwd_done[c], 0);

@@ -107,7 +107,9 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
   D.d_out = L.d_out;
   D.s = L.s;
   D.npaths = npaths;
+  D.t_ld = lb::latent_row_elems(L.s, npaths);
   D.n_slices = n_slices;
+  D.x_next = -1;
   const int vw = lb::latent_warps(1, batch, [&](int, int& n_rb, double& w) {
     n_rb = S16 / 16;
     w = 1.0;
@@ -145,9 +147,10 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
   a.v_items = npaths * D.n_slices * D.n_rchunks;
   a.u_items = L.d_out / lb::kUTileRows;
   a.p_items = npaths;
-  a.x_items = npaths * D.n_slices;
+  a.x_items = D.n_slices;
   a.v_warps = vw;
   a.packed = batch == 1 && L.residual ? 1 : 0;
+  a.mode = lb::kModeForward;
   int sms = 0;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return lb::cuda_fail(e);

@@ -292,11 +292,36 @@ __device__ __forceinline__ void prep_b2(const LayerDesc& L, int Sp, unsigned cha
 // the next layer's first[k], or the grid's end, belong to it).
 struct PrepJob {
   LayerDesc L;
-  const uint16_t* x;
-  unsigned char *X16, *B1, *B2;
+  const uint16_t* x;        // the activations, or (expand calls) the cache rows
+  unsigned char *X16, *B1, *B2, *T;
   int M, x_bf16, Sp;
-  int first[3];   // 0: x, 1: B1, 2: B2
+  int first[kPrepKinds];    // 0: x, 1: B1, 2: B2, 3: T' from cache rows
 };
+
+// T' (M x npaths*Sp core-matrix tiles, the A operand of GEMM2) from the
+// caller's cache rows: element (r, p*Sp + j) = cache[r * t_ld + p*s + j] for
+// j < s, else 0.  Work unit = one 16-byte piece (8 consecutive columns of one
+// row) of the tiles; the cache offsets need not be 16-byte aligned, so the
+// piece is gathered element by element.
+__device__ __forceinline__ void prep_t(const uint16_t* __restrict__ tc, const LayerDesc& L, int M, int Sp,
+                                       unsigned char* __restrict__ out, unsigned bid, unsigned nblk) {
+  const int NK = L.npaths * Sp;
+  const unsigned pieces = (unsigned)M * (unsigned)(NK / 8);
+  for (unsigned t = bid * blockDim.x + threadIdx.x; t < pieces; t += nblk * blockDim.x) {
+    const int r = (int)(t / (unsigned)(NK / 8)), k0 = (int)(t - (unsigned)r * (NK / 8)) * 8;
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      uint32_t lo = 0, hi = 0;
+      const int k = k0 + e;
+      const int p0 = k / Sp, j0 = k - p0 * Sp, p1 = (k + 1) / Sp, j1 = k + 1 - p1 * Sp;
+      if (j0 < L.s) lo = tc[(size_t)r * L.t_ld + p0 * L.s + j0];
+      if (j1 < L.s) hi = tc[(size_t)r * L.t_ld + p1 * L.s + j1];
+      w[e >> 1] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4*>(out + tiled_off(r, k0, M)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
 
 // The job that owns block b of launch k: the last one whose first[k] <= b.
 __device__ __forceinline__ int prep_job_of(const PrepJob* jobs, int n, int k, unsigned b) {
@@ -319,7 +344,8 @@ __global__ void __launch_bounds__(256) prep_group_kernel(const PrepJob* __restri
   const unsigned bid = blockIdx.x - b0, nblk = b1 - b0;
   if (KIND == 0) prep_x(J.x, J.x_bf16, J.M, J.L.d_in, J.X16, bid, nblk, status);
   else if (KIND == 1) prep_b1(J.L, J.Sp, J.B1, bid, nblk);
-  else prep_b2(J.L, J.Sp, J.B2, bid, nblk);
+  else if (KIND == 2) prep_b2(J.L, J.Sp, J.B2, bid, nblk);
+  else prep_t(J.x, J.L, J.M, J.Sp, J.T, bid, nblk);
 }
 
 // ------------------------------------------------------------------ grouped persistent tcgen05 GEMM
@@ -333,13 +359,14 @@ __global__ void __launch_bounds__(256) prep_group_kernel(const PrepJob* __restri
 struct GemmProblem {
   const unsigned char* A;   // core-matrix tiles, M rows x K
   const unsigned char* B;   // core-matrix tiles, N rows x K
-  int M, N, K, mode;        // mode 0: T' = l * acc -> fp16 tiles; 1: y = acc -> row-major
+  int M, N, K, mode;        // mode 0: T' = l * acc -> fp16 tiles; 1: y = acc -> row-major;
+                            // 2: T' = l * acc -> fp16 cache rows (latent-only calls)
   const uint16_t* l0;
   const uint16_t* l1;
   int s, Sp;
   unsigned char* T;         // mode 0 output, core-matrix tiles M x N
-  void* Y;                  // mode 1 output, row-major M x N
-  int y_bf16;
+  void* Y;                  // mode 1 output, row-major M x N; mode 2: cache rows, t_ld apart
+  int y_bf16, t_ld;
   int tiles_n, tile_begin;
 };
 
@@ -505,7 +532,7 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
           __syncwarp();
         }
       }
-      for (int c0 = 0; P.mode == 0 && c0 < ti.n_len; c0 += 16) {
+      for (int c0 = 0; P.mode != 1 && c0 < ti.n_len; c0 += 16) {
         float v[16];
         tmem_ld16(taddr + (uint32_t)c0, v);
         uint32_t w[8];
@@ -524,9 +551,20 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
             w[e >> 1] = *reinterpret_cast<const uint32_t*>(&hh);
             bad |= half2_nonfinite(w[e >> 1]);
           }
-          *reinterpret_cast<uint4*>(P.T + tiled_off(row, ti.n0 + c0, P.M)) = make_uint4(w[0], w[1], w[2], w[3]);
-          *reinterpret_cast<uint4*>(P.T + tiled_off(row, ti.n0 + c0 + 8, P.M)) =
-              make_uint4(w[4], w[5], w[6], w[7]);
+          if (P.mode == 0) {
+            *reinterpret_cast<uint4*>(P.T + tiled_off(row, ti.n0 + c0, P.M)) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(P.T + tiled_off(row, ti.n0 + c0 + 8, P.M)) =
+                make_uint4(w[4], w[5], w[6], w[7]);
+          } else {
+            // cache row: path p's t'_j at column p*s + j, j < s
+            uint16_t* yr = static_cast<uint16_t*>(P.Y) + (size_t)row * P.t_ld;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int n = ti.n0 + c0 + e;
+              const int p = n / P.Sp, j = n - p * P.Sp;
+              if (j < P.s) yr[p * P.s + j] = (uint16_t)(w[e >> 1] >> (16 * (e & 1)));
+            }
+          }
         }
       }
       tc_fence_before();
@@ -609,8 +647,9 @@ static LayerBufs layer_bufs(unsigned char*& buf, const LayerDesc& L, int M) {
 }
 
 // Blocks of one layer's preparation steps (x, B1, B2), as for a launch of its own.
-static void prep_blocks(const LayerDesc& L, int M, int Sp, int (&blocks)[3]) {
+static void prep_blocks(const LayerDesc& L, int M, int Sp, int mode, int (&blocks)[kPrepKinds]) {
   const int P = L.npaths;
+  blocks[3] = grid_for((long long)M * P * Sp / 8, 256);
   blocks[0] = grid_for((long long)M * L.d_in / 8 / kXUnroll, 256);
   const long long l1 = (long long)P * ((L.s + 15) >> 4) * (L.d_in / kVTileK) * 256 +
                        (long long)P * (Sp - 16 * ((L.s + 15) >> 4)) * (L.d_in / 8);
@@ -618,6 +657,10 @@ static void prep_blocks(const LayerDesc& L, int M, int Sp, int (&blocks)[3]) {
   const long long l2 = (long long)P * (L.d_out / kUTileRows) * ((L.s + 31) >> 5) * 256 +
                        (long long)P * L.d_out * ((Sp - 32 * ((L.s + 31) >> 5)) / 8);
   blocks[2] = grid_for(l2, 256);
+  // forward: x, B1, B2; latent-only: x, B1; expand: B2 and T' from the cache
+  if (mode == kModeLatent) blocks[2] = 0;
+  if (mode == kModeExpand) blocks[0] = blocks[1] = 0;
+  if (mode != kModeExpand) blocks[3] = 0;
 }
 
 // Operand preparation of a planned chunk: three grouped launches (x, B1, B2)
@@ -625,9 +668,11 @@ static void prep_blocks(const LayerDesc& L, int M, int Sp, int (&blocks)[3]) {
 cudaError_t launch_prefill_prep(const PrefillPlan& plan, const unsigned char* table_dev, unsigned int* status,
                                 cudaStream_t st) {
   const PrepJob* jobs = reinterpret_cast<const PrepJob*>(table_dev + plan.table_off + plan.jobs_off);
-  prep_group_kernel<0><<<plan.prep_grid[0], 256, 0, st>>>(jobs, plan.n, status);
-  prep_group_kernel<1><<<plan.prep_grid[1], 256, 0, st>>>(jobs, plan.n, status);
-  prep_group_kernel<2><<<plan.prep_grid[2], 256, 0, st>>>(jobs, plan.n, status);
+  // the kinds a call's mode needs (a kind with no blocks is not launched)
+  if (plan.prep_grid[0]) prep_group_kernel<0><<<plan.prep_grid[0], 256, 0, st>>>(jobs, plan.n, status);
+  if (plan.prep_grid[1]) prep_group_kernel<1><<<plan.prep_grid[1], 256, 0, st>>>(jobs, plan.n, status);
+  if (plan.prep_grid[2]) prep_group_kernel<2><<<plan.prep_grid[2], 256, 0, st>>>(jobs, plan.n, status);
+  if (plan.prep_grid[3]) prep_group_kernel<3><<<plan.prep_grid[3], 256, 0, st>>>(jobs, plan.n, status);
   return cudaGetLastError();
 }
 
@@ -666,7 +711,8 @@ static double tile_cost(int K, int n_len) { return (double)(K / kBK) * (double)m
 // to the chunk's buffers at `bufs` and to the image's own place at
 // table_dev + plan.table_off.
 void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const* ys, int n, int M, int x_bf16,
-                        unsigned char* bufs, int num_sms, std::vector<unsigned char>& img, PrefillPlan& plan) {
+                        int mode, unsigned char* bufs, int num_sms, std::vector<unsigned char>& img,
+                        PrefillPlan& plan) {
   const long long tiles_all = group_tiles(Ls, n, M);
   plan.n = n;
   plan.table_off = (img.size() + 1023) & ~(size_t)1023;
@@ -675,7 +721,7 @@ void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const*
   img.resize(plan.table_off + plan.table_bytes, 0);
   unsigned char* base = img.data() + plan.table_off;
   PrepJob* jobs = reinterpret_cast<PrepJob*>(base + plan.jobs_off);
-  plan.prep_grid[0] = plan.prep_grid[1] = plan.prep_grid[2] = 0;
+  for (int k = 0; k < kPrepKinds; ++k) plan.prep_grid[k] = 0;
   const size_t prob_b = (size_t)2 * n * sizeof(GemmProblem);
   GemmProblem* probs = reinterpret_cast<GemmProblem*>(base);
   int* begin1 = reinterpret_cast<int*>(base + prob_b);
@@ -692,37 +738,42 @@ void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const*
     std::memset(&J, 0, sizeof(J));
     J.L = L;
     J.x = static_cast<const uint16_t*>(xs[i]);
-    J.X16 = b.X16; J.B1 = b.B1; J.B2 = b.B2;
+    J.X16 = b.X16; J.B1 = b.B1; J.B2 = b.B2; J.T = b.T;
     J.M = M; J.x_bf16 = x_bf16; J.Sp = Sp;
-    int blocks[3];
-    prep_blocks(L, M, Sp, blocks);
-    for (int k = 0; k < 3; ++k) {
+    int blocks[kPrepKinds];
+    prep_blocks(L, M, Sp, mode, blocks);
+    for (int k = 0; k < kPrepKinds; ++k) {
       J.first[k] = plan.prep_grid[k];
       plan.prep_grid[k] += blocks[k];
     }
     GemmProblem& g1 = probs[i];
     g1 = GemmProblem{};
-    g1.A = b.X16; g1.B = b.B1; g1.M = M; g1.N = NK; g1.K = L.d_in; g1.mode = 0;
+    g1.A = b.X16; g1.B = b.B1; g1.M = M; g1.N = NK; g1.K = L.d_in; g1.mode = mode == kModeLatent ? 2 : 0;
     g1.l0 = L.p[0].l; g1.l1 = P == 2 ? L.p[1].l : L.p[0].l; g1.s = L.s; g1.Sp = Sp; g1.T = b.T;
+    g1.Y = mode == kModeLatent ? ys[i] : nullptr; g1.t_ld = L.t_ld;
     g1.tiles_n = ceil_div(NK, kBN); g1.tile_begin = tiles1;
-    tiles1 += (M / kBM) * g1.tiles_n;
-    for (int mt = 0; mt < M / kBM; ++mt)
-      for (int nt = 0; nt < g1.tiles_n; ++nt) cost1.push_back(tile_cost(g1.K, min(kBN, NK - nt * kBN)));
+    if (mode != kModeExpand) {
+      tiles1 += (M / kBM) * g1.tiles_n;
+      for (int mt = 0; mt < M / kBM; ++mt)
+        for (int nt = 0; nt < g1.tiles_n; ++nt) cost1.push_back(tile_cost(g1.K, min(kBN, NK - nt * kBN)));
+    }
     GemmProblem& g2 = probs[n + i];
     g2 = GemmProblem{};
     g2.A = b.T; g2.B = b.B2; g2.M = M; g2.N = L.d_out; g2.K = NK; g2.mode = 1; g2.Y = ys[i]; g2.y_bf16 = x_bf16;
     g2.tiles_n = ceil_div(L.d_out, kBN); g2.tile_begin = tiles2;
-    tiles2 += (M / kBM) * g2.tiles_n;
-    for (int mt = 0; mt < M / kBM; ++mt)
-      for (int nt = 0; nt < g2.tiles_n; ++nt) cost2.push_back(tile_cost(g2.K, min(kBN, L.d_out - nt * kBN)));
+    if (mode != kModeLatent) {
+      tiles2 += (M / kBM) * g2.tiles_n;
+      for (int mt = 0; mt < M / kBM; ++mt)
+        for (int nt = 0; nt < g2.tiles_n; ++nt) cost2.push_back(tile_cost(g2.K, min(kBN, L.d_out - nt * kBN)));
+    }
   }
   int* sched2 = sched1 + tiles1;
   plan.tiles1 = tiles1;
   plan.tiles2 = tiles2;
   plan.grid1 = min(min(tiles1, num_sms), kMaxGemmGrid);
   plan.grid2 = min(min(tiles2, num_sms), kMaxGemmGrid);
-  lpt_schedule(cost1, plan.grid1, sched1, begin1);
-  lpt_schedule(cost2, plan.grid2, sched2, begin2);
+  if (plan.grid1 > 0) lpt_schedule(cost1, plan.grid1, sched1, begin1);
+  if (plan.grid2 > 0) lpt_schedule(cost2, plan.grid2, sched2, begin2);
 }
 
 // GEMM1 and GEMM2 of a planned chunk (table uploaded at table_dev +
@@ -744,10 +795,11 @@ cudaError_t launch_prefill_gemms(const PrefillPlan& plan, const unsigned char* t
   const GemmProblem* probs = reinterpret_cast<const GemmProblem*>(base);
   const int* begin_dev = reinterpret_cast<const int*>(base + prob_b);
   const int* sched_dev = begin_dev + 2 * (kMaxGemmGrid + 1);
+  // GEMM1 (not in expand calls) and GEMM2 (not in latent-only calls)
   GroupArgs g1a{probs, sched_dev, begin_dev, plan.n, plan.tiles1, status};
-  umma_group_kernel<<<plan.grid1, kGroupThreads, group_smem(), st>>>(g1a);
+  if (plan.grid1 > 0) umma_group_kernel<<<plan.grid1, kGroupThreads, group_smem(), st>>>(g1a);
   GroupArgs g2a{probs + plan.n, sched_dev + plan.tiles1, begin_dev + kMaxGemmGrid + 1, plan.n, plan.tiles2, status};
-  umma_group_kernel<<<plan.grid2, kGroupThreads, group_smem(), st>>>(g2a);
+  if (plan.grid2 > 0) umma_group_kernel<<<plan.grid2, kGroupThreads, group_smem(), st>>>(g2a);
   return cudaGetLastError();
 }
 

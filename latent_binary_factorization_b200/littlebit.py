@@ -70,6 +70,19 @@ _lib.littlebit_linear_forward_many_host.restype = ctypes.c_int
 _lib.littlebit_linear_forward_many_host.argtypes = [ctypes.POINTER(LbLayer), ctypes.c_int, ctypes.c_void_p,
                                                     ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                     ctypes.c_void_p]
+_lib.littlebit_latent_row_elems.restype = ctypes.c_int
+_lib.littlebit_latent_row_elems.argtypes = [ctypes.c_int, ctypes.c_int]
+for _name in ("littlebit_latent_forward", "littlebit_latent_expand"):
+    getattr(_lib, _name).restype = ctypes.c_int
+    getattr(_lib, _name).argtypes = [ctypes.POINTER(LbLayer), ctypes.c_int, ctypes.POINTER(ctypes.c_void_p),
+                                     ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+_lib.littlebit_init_dual_svid.restype = ctypes.c_int
+_lib.littlebit_init_dual_svid.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+_lib.littlebit_joint_itq.restype = ctypes.c_int
+_lib.littlebit_joint_itq.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                     ctypes.c_int, ctypes.c_void_p]
 _lib.littlebit_device_status.restype = ctypes.c_int
 _lib.littlebit_device_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint)]
 _lib.littlebit_check_wait_timeout.restype = ctypes.c_int
@@ -271,6 +284,93 @@ class HostStack:
                                                        ctypes.c_void_p(y_host.data_ptr()), self.batch,
                                                        _DTYPE[self.dtype], int(n_chunks), _stream(stream)),
                "littlebit_linear_forward_many_host")
+
+
+def latent_row_elems(layer: Layer) -> int:
+    """fp16 elements between a layer's latent cache rows (npaths*s rounded up
+    to a multiple of 8)."""
+    return int(_lib.littlebit_latent_row_elems(layer.s, int(layer.residual)))
+
+
+def _ptrs(ts):
+    return (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+
+
+def latent_forward(layers: list, xs: list, ts: list | None = None, stream=None) -> list:
+    """Latent cache rows of each layer's input: ts[i] = [t'_1 | t'_2] of xs[i]
+    (fp16, batch x latent_row_elems), the K/V projection kept as its latent."""
+    batch = xs[0].shape[0]
+    for i, (L, x) in enumerate(zip(layers, xs)):
+        _activation(x, batch, L.d_in, f"xs[{i}]")
+    if ts is None:
+        ts = [torch.empty((batch, latent_row_elems(L)), dtype=torch.float16, device=x.device)
+              for L, x in zip(layers, xs)]
+    for i, (L, t) in enumerate(zip(layers, ts)):
+        _activation(t, batch, latent_row_elems(L), f"ts[{i}]")
+        if t.dtype != torch.float16:
+            raise ValueError("cache rows are fp16")
+    arr = (LbLayer * len(layers))(*[L.c_struct() for L in layers])
+    _check(_lib.littlebit_latent_forward(arr, len(layers), _ptrs(xs), _ptrs(ts), batch, _DTYPE[xs[0].dtype],
+                                         _stream(stream)), "littlebit_latent_forward")
+    return ts
+
+
+def latent_expand(layers: list, ts: list, ys: list | None = None, dtype=torch.float16, stream=None) -> list:
+    """Projections rebuilt from cache rows: ys[i] = sum_p h_p (.) U_p t'_p."""
+    rows = ts[0].shape[0]
+    for i, (L, t) in enumerate(zip(layers, ts)):
+        _activation(t, rows, latent_row_elems(L), f"ts[{i}]")
+        if t.dtype != torch.float16:
+            raise ValueError("cache rows are fp16")
+    if ys is None:
+        ys = [torch.empty((rows, L.d_out), dtype=dtype, device=t.device) for L, t in zip(layers, ts)]
+    for i, (L, y) in enumerate(zip(layers, ys)):
+        _activation(y, rows, L.d_out, f"ys[{i}]")
+    arr = (LbLayer * len(layers))(*[L.c_struct() for L in layers])
+    _check(_lib.littlebit_latent_expand(arr, len(layers), _ptrs(ts), _ptrs(ys), rows, _DTYPE[ys[0].dtype],
+                                        _stream(stream)), "littlebit_latent_expand")
+    return ys
+
+
+def _f32_rows(t: torch.Tensor, rows: int, cols: int, name: str) -> None:
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()
+            and tuple(t.shape) == (rows, cols)):
+        raise ValueError(f"{name} must be a contiguous CUDA float32 tensor of shape ({rows}, {cols})")
+
+
+def init_dual_svid(Uf: torch.Tensor, Vf: torch.Tensor, iters: int = 32, stream=None) -> Path:
+    """One path from real factors U' (d_out x s) and V' (d_in x s), fp32 CUDA:
+    packed signs and the rank-1 magnitude scales h, g, l (fp16)."""
+    d_out, s = Uf.shape
+    d_in = Vf.shape[0]
+    _f32_rows(Uf, d_out, s, "Uf")
+    _f32_rows(Vf, d_in, s, "Vf")
+    dev = Uf.device
+    p = Path(V_bits=torch.empty(packed_bytes("V", s, d_in), dtype=torch.uint8, device=dev),
+             U_bits=torch.empty(packed_bytes("U", d_out, s), dtype=torch.uint8, device=dev),
+             h=torch.empty(d_out, dtype=torch.float16, device=dev), g=torch.empty(d_in, dtype=torch.float16, device=dev),
+             l=torch.empty(s, dtype=torch.float16, device=dev))
+    _check(_lib.littlebit_init_dual_svid(ctypes.c_void_p(Uf.data_ptr()), ctypes.c_void_p(Vf.data_ptr()), d_out, d_in,
+                                         s, int(iters), ctypes.c_void_p(p.U_bits.data_ptr()),
+                                         ctypes.c_void_p(p.V_bits.data_ptr()), ctypes.c_void_p(p.h.data_ptr()),
+                                         ctypes.c_void_p(p.g.data_ptr()), ctypes.c_void_p(p.l.data_ptr()),
+                                         _stream(stream)), "littlebit_init_dual_svid")
+    return p
+
+
+def joint_itq(X: torch.Tensor, iters: int = 50, R: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Rotate the stacked factors X = [U'; V'] ((d_out + d_in) x s, fp32 CUDA)
+    in place by the Joint-ITQ rotation; returns R (s x s).  With R given, the
+    alternations start from it (and it is overwritten)."""
+    n_rows, s = X.shape
+    _f32_rows(X, n_rows, s, "X")
+    given = R is not None
+    if R is None:
+        R = torch.empty((s, s), dtype=torch.float32, device=X.device)
+    _f32_rows(R, s, s, "R")
+    _check(_lib.littlebit_joint_itq(ctypes.c_void_p(X.data_ptr()), n_rows, s, int(iters), ctypes.c_void_p(R.data_ptr()),
+                                    int(given), _stream(stream)), "littlebit_joint_itq")
+    return R
 
 
 def forward_many(layers: list, xs: list, ys: list, stream=None) -> None:

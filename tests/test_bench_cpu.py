@@ -89,3 +89,14 @@ def test_committed_traffic_records_name_a_source_hash():
         for kernel, r in kernels.items():
             if isinstance(r, dict) and "dram_bytes_per_model_layer" in r:
                 assert len(r["decode_cu_sha256_16"]) == 16, (workload, kernel)
+
+
+def test_shared_inputs_are_read_once_in_the_byte_model():
+    """The 7B full layer's q, k, v share one input and gate, up another: the
+    model layer's bytes count each shared input once."""
+    wl = bench.WORKLOADS["7b_layer_0.1bpw_residual"]
+    full = sum(bench.algorithmic_bytes(*m, 1) for m in wl["mats"])
+    saved = bench.shared_x_bytes(wl["mats"], wl["x_groups"], 1)
+    assert saved == 2 * (2 * 4096) + 1 * (2 * 4096)     # two extra reads for q,k,v; one for gate,up
+    assert bench.layer_bytes("7b_layer_0.1bpw_residual", 1) == full - saved
+    assert bench.shared_x_bytes([(4096, 4096, 86, True)], None, 1) == 0

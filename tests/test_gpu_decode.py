@@ -402,3 +402,37 @@ def test_nonfinite_decode_input_is_reported(lbm):
     y = lb.forward(layer, torch.from_numpy(xh).cuda())
     assert lb.device_status() == 0
     _check(y, orc.factored_forward(xh, paths), "after a non-finite input")
+
+
+@pytest.mark.parametrize("B", [1, 3, 16])
+def test_forward_many_shared_inputs(lbm, B):
+    """Layers of one call that read the same x (a block's q, k and v
+    projections; gate and up) are quantised from one read of x: every
+    layer's output still matches the oracle, and a layer listed twice with
+    the same input gives identical outputs."""
+    lb, layers = lbm
+    groups = [[(4096, 4096, 86, True)] * 3, [(4096, 4096, 86, True)], [(4096, 11008, 133, True)] * 2,
+              [(11008, 4096, 133, True)], [(1024, 512, 40, False), (1024, 768, 300, True)]]
+    L, X, Y, refs = [], [], [], []
+    k = 0
+    for g, members in enumerate(groups):
+        xh = synth.activations(B, members[0][0], seed=200 + g, index=g)
+        x = torch.from_numpy(xh).cuda()
+        for (a, b, s, r) in members:
+            paths = synth.layer(a, b, s, r, seed=400 + k, index=k)
+            L.append(layers.upload(paths, a, b, s))
+            X.append(x)
+            Y.append(torch.full((B, b), float("nan"), dtype=torch.float16, device="cuda"))
+            refs.append(orc.factored_forward(xh, paths))
+            k += 1
+    # the same layer twice on the same input
+    L.append(L[0])
+    X.append(X[0])
+    Y.append(torch.empty_like(Y[0]))
+    refs.append(refs[0])
+    lb.Stack(L, X, Y)()
+    torch.cuda.synchronize()
+    for i, (y, ref) in enumerate(zip(Y, refs)):
+        _check(y, ref, f"layer {i}")
+    assert torch.equal(Y[0], Y[-1])
+    assert lb.device_status() == 0
