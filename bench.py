@@ -45,11 +45,13 @@ WORKLOADS = {
         "desc": "Llama-2-70B MLP layer (8192->28672 gate, up; 28672->8192 down), 0.1 BPW single path s=620",
         "mats": [(8192, 28672, 620, False), (8192, 28672, 620, False), (28672, 8192, 620, False)],
         "model_layers": 80,
+        "x_groups": [0, 0, 1],   # gate and up read the MLP's input
     },
     "70b_mlp_0.1bpw_residual": {
         "desc": "Llama-2-70B MLP layer, 0.1 BPW residual s=302 x 2 paths",
         "mats": [(8192, 28672, 302, True), (8192, 28672, 302, True), (28672, 8192, 302, True)],
         "model_layers": 80,
+        "x_groups": [0, 0, 1],
     },
     "7b_layer_0.1bpw_residual": {
         "desc": "Llama-2-7B layer (4x 4096^2 s=86; 2x 4096->11008 and 11008->4096 s=133), 0.1 BPW residual",

@@ -172,7 +172,8 @@ __device__ __forceinline__ uint32_t pack_byte(uint32_t a, uint32_t c, uint32_t d
 __device__ __forceinline__ void quantise_row(const uint4 (&xq)[kQChunks], const uint16_t* __restrict__ g, int k0,
                                              int nchunk, int row, int NC, int lane, unsigned char* blk, int B) {
   uint32_t* frag = reinterpret_cast<uint32_t*>(blk + xq_stats_bytes(B));
-  float u[kQChunks][8];
+  // u = g * x is formed twice (for the max, then for the codes) rather than
+  // held: 64 more live registers would halve the resident warps
   float mx = 0.f;
 #pragma unroll
   for (int j = 0; j < kQChunks; ++j) {
@@ -183,9 +184,7 @@ __device__ __forceinline__ void quantise_row(const uint4 (&xq)[kQChunks], const 
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 xf = h2x2(xw[e]), gf = h2x2(gw[e]);
-      u[j][2 * e] = xf.x * gf.x;
-      u[j][2 * e + 1] = xf.y * gf.y;
-      mx = fmaxf(mx, fmaxf(fabsf(u[j][2 * e]), fabsf(u[j][2 * e + 1])));
+      mx = fmaxf(mx, fmaxf(fabsf(xf.x * gf.x), fabsf(xf.y * gf.y)));
     }
   }
 #pragma unroll
@@ -195,12 +194,18 @@ __device__ __forceinline__ void quantise_row(const uint4 (&xq)[kQChunks], const 
 #pragma unroll
   for (int j = 0; j < kQChunks; ++j) {
     const int ch = lane + 32 * j;
+    const uint4 gq = ch < nchunk ? ld_nc(g + k0 + 8 * ch) : make_uint4(0, 0, 0, 0);
+    const uint32_t* xw = &xq[j].x;
+    const uint32_t* gw = &gq.x;
     uint32_t fb[8], fh[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      fb[e] = __float_as_uint(fmaf(u[j][e], inv, kRoundMagic));
-      fh[e] = fb[e] + 128u;
+    for (int e = 0; e < 4; ++e) {
+      const float2 xf = h2x2(xw[e]), gf = h2x2(gw[e]);
+      fb[2 * e] = __float_as_uint(fmaf(xf.x * gf.x, inv, kRoundMagic));
+      fb[2 * e + 1] = __float_as_uint(fmaf(xf.y * gf.y, inv, kRoundMagic));
     }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) fh[e] = fb[e] + 128u;
     const uint32_t lw0 = pack_byte(fb[0], fb[1], fb[2], fb[3], 0), lw1 = pack_byte(fb[4], fb[5], fb[6], fb[7], 0);
     const uint32_t hw0 = pack_byte(fh[0], fh[1], fh[2], fh[3], 1), hw1 = pack_byte(fh[4], fh[5], fh[6], fh[7], 1);
     sum_hi = __dp4a((int)hw0, 0x01010101, __dp4a((int)hw1, 0x01010101, sum_hi));
@@ -307,6 +312,40 @@ __device__ __forceinline__ VItem decode_v(const DecodeArgs& a, int item, int& li
   return it;
 }
 
+// A latent-pass item's coordinates and its layer's constants, advanced one
+// item at a time by comparisons only (items run path-major, then slice, then
+// row chunk, layer after layer).
+struct VPos {
+  int item, li, p, sl, rc;
+  const LayerDesc* L;   // the layer's counts are read from its (cached) descriptor
+
+  __device__ __forceinline__ void load(const DecodeArgs& a) { L = a.layers + li; }
+  // position at `it`, whose layer is li0 or a later one
+  __device__ __forceinline__ void start(const DecodeArgs& a, int it, int li0) {
+    int l = li0;
+    const VItem v = decode_v(a, it, l);
+    item = it;
+    li = l;
+    p = v.p;
+    sl = v.sl;
+    rc = v.rc;
+    load(a);
+  }
+  __device__ __forceinline__ void next(const DecodeArgs& a) {
+    ++item;
+    if (++rc < L->n_rchunks) return;
+    rc = 0;
+    if (++sl < L->n_slices) return;
+    sl = 0;
+    if (++p < L->npaths) return;
+    p = 0;
+    if (li + 1 < a.n_layers) {
+      ++li;
+      load(a);
+    }
+  }
+};
+
 // Row blocks a warp processes at once: two share each B-fragment load; with
 // more than four batch rows the accumulators would not fit, so one.
 template <int NB>
@@ -334,36 +373,45 @@ __device__ __forceinline__ void x_issue(const DecodeArgs& a, int item, int li, u
 template <int NB, int W>
 struct VFeed {
   static constexpr int RPW = VCfg<NB>::kRPW;
-  int item, li, grp, kc;
+  VPos pos;
+  int item, grp, kc;
   int rb0, n_rb, n_kt_all, kt0, nkt;   // current item
   const unsigned char* V;
 
-  __device__ __forceinline__ void set(const DecodeArgs& a, int warp) {
+  // the current item's chunk parameters (from pos; no divisions)
+  __device__ __forceinline__ void set(int warp) {
     static_assert(W == 3 || W == 4, "latent-pass CTA width");
-    const VItem it = decode_v(a, item, li);
-    const LayerDesc& L = a.layers[li];
-    const int k0 = it.sl * kVSlice;
-    nkt = min(kVSliceTiles, (L.d_in - k0) / kVTileK);
-    n_kt_all = L.d_in / kVTileK;
+    item = pos.item;
+    const int k0 = pos.sl * kVSlice, d_in = pos.L->d_in;
+    nkt = min(kVSliceTiles, (d_in - k0) / kVTileK);
+    n_kt_all = d_in / kVTileK;
     kt0 = k0 / kVTileK;
-    n_rb = (L.s + 15) >> 4;
-    rb0 = it.rc * (2 * W) + 2 * warp;
-    V = reinterpret_cast<const unsigned char*>(L.p[it.p].V);
+    n_rb = (pos.L->s + 15) >> 4;
+    rb0 = pos.rc * (2 * W) + 2 * warp;
+    V = reinterpret_cast<const unsigned char*>(pos.L->p[pos.p].V);
     grp = 0;
     kc = 0;
+  }
+  __device__ __forceinline__ void start(const DecodeArgs& a, int warp, int it, int li0) {
+    pos.start(a, it, li0);
+    set(warp);
   }
   __device__ __forceinline__ int rb() const { return rb0 + grp * RPW; }
   __device__ __forceinline__ bool valid() const { return rb() < n_rb; }
   __device__ __forceinline__ void normalize(const DecodeArgs& a, int warp, int end) {
     while (item < end && !valid()) {
-      if (++item < end) set(a, warp);
+      pos.next(a);
+      if (pos.item < end) set(warp);
+      else item = pos.item;
     }
   }
   __device__ __forceinline__ void advance(const DecodeArgs& a, int warp, int end) {
     if (++kc * kChunkTiles >= nkt) {
       kc = 0;
       if (++grp * RPW >= 2) {
-        if (++item < end) set(a, warp);
+        pos.next(a);
+        if (pos.item < end) set(warp);
+        else item = pos.item;
       }
     }
     normalize(a, warp, end);
@@ -420,9 +468,7 @@ __global__ void __launch_bounds__(W * 32, NB == 1 ? 4 : 1) latent_pass_kernel(co
   grid_dep_launch();
   const int li0 = layer_of(a.item_layer.v, a.n_layers, i_begin);
   VFeed<NB, W> feed;
-  feed.item = i_begin;
-  feed.li = li0;
-  feed.set(a, warp);
+  feed.start(a, warp, i_begin, li0);
   feed.normalize(a, warp, i_end);
 #pragma unroll 1
   for (int st = 0; st < kVStages; ++st) {
@@ -451,13 +497,15 @@ __global__ void __launch_bounds__(W * 32, NB == 1 ? 4 : 1) latent_pass_kernel(co
 #pragma unroll
   for (int nb = 0; nb < NB; ++nb) boff[nb] = ((8 * nb + g) % NC) * 4 + c;
 
-  int li = li0;
   int prev_li = -1, prev_p = -1, prev_sl = -1;
   int seq = -1;   // index of the current slice in this CTA's sequence
 
-  for (int item = i_begin; item < i_end; ++item) {
-    const VItem it = decode_v(a, item, li);
-    const LayerDesc& L = a.layers[li];
+  VPos cur;
+  cur.start(a, i_begin, li0);
+  for (; cur.item < i_end; cur.next(a)) {
+    const int item = cur.item, li = cur.li;
+    const VItem it{cur.li, cur.p, cur.sl, cur.rc};
+    const LayerDesc& L = *cur.L;
     const PathDesc& P = L.p[it.p];
     const int s = L.s;
     const int S16 = (s + 15) & ~15, n_rb = S16 >> 4;
@@ -675,7 +723,9 @@ __global__ void __launch_bounds__(kFWarps * 32) finalize_kernel(const DecodeArgs
           pl[(1 - pi) * 64 + 32] = 0;
         }
       } else {
-        int8_t* pl = P.ws.planes + ((size_t)(k * 4 * NB + b) * 2) * 32 + lane;
+        // RS rows per K-tile: 1 at batch 1 (only row 0 is read), else 4*NB
+        const int RS = B == 1 ? 1 : 4 * NB;
+        int8_t* pl = P.ws.planes + ((size_t)(k * RS + b) * 2) * 32 + lane;
         pl[0] = (int8_t)((fb + 128u) >> 8);
         pl[32] = (int8_t)fb;
       }
@@ -707,8 +757,10 @@ struct OutCfg {
   static constexpr int kStages = 2;
 };
 
-// stage: [8 tiles: 4 KB][t' bytes: 8 K-tiles x 4NB x 64][h: 256][tstat: 16 B x 4NB]
-// (B below is the padded row count 4*NB)
+// stage: [8 tiles: 4 KB][t' bytes: 8 K-tiles x RS x 64][h: 256][tstat: 16 B x RS]
+// (B below is RS, the batch rows stored per K-tile of the t' planes: 1 at
+// batch 1, else 4*NB; at batch 1 the product's columns for rows 1..3 are
+// never read, so their zero planes are not stored or copied)
 __host__ __device__ __forceinline__ int out_planes_off() { return kUChunkBytes; }
 __host__ __device__ __forceinline__ int out_h_off(int B) { return kUChunkBytes + kUChunkTiles * B * 64; }
 __host__ __device__ __forceinline__ int out_tstat_off(int B) { return out_h_off(B) + kUTileRows * 2; }
@@ -772,17 +824,17 @@ __device__ __forceinline__ void out_issue(const OutCursor& cu, unsigned char* st
 }
 
 // One K-tile of one path: eight m16n8k32 products (row block q = 0..7).
-// `pl` points at this thread's t' bytes of tile t (batch row g/2, plane g%2);
-// `pl_step` = B * 64 bytes from one tile's t' bytes to the next.
-template <int NB, bool kFirst = false>
+// `pl` points at this thread's t' bytes of tile 0 (batch row 4nb + g/2,
+// plane g%2); RS * 64 bytes separate one tile's t' bytes from the next.
+template <int NB, int RS, bool kFirst = false>
 __device__ __forceinline__ void out_tile(int (&d)[8][NB][4], const unsigned char* stage, int t, int lane,
                                          const unsigned char* pl) {
   const uint4 cur = *reinterpret_cast<const uint4*>(stage + t * kTileBytes + lane * 16);
   uint32_t b0[NB], b1[NB];
 #pragma unroll
   for (int nb = 0; nb < NB; ++nb) {
-    b0[nb] = *reinterpret_cast<const uint32_t*>(pl + t * (256 * NB) + nb * 256);
-    b1[nb] = *reinterpret_cast<const uint32_t*>(pl + t * (256 * NB) + nb * 256 + 16);
+    b0[nb] = *reinterpret_cast<const uint32_t*>(pl + t * (64 * RS) + nb * 256);
+    b1[nb] = *reinterpret_cast<const uint32_t*>(pl + t * (64 * RS) + nb * 256 + 16);
   }
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
@@ -796,13 +848,14 @@ __device__ __forceinline__ void out_tile(int (&d)[8][NB][4], const unsigned char
   }
 }
 
-template <int NB>
+template <int NB, int RS>
 __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeArgs a) {
+  static_assert(RS == 4 * NB || (NB == 1 && RS == 1), "t' rows stored: 1 at batch 1, else 4 per n-block");
   constexpr int S = OutCfg<NB>::kStages;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
   const int B = a.batch;            // rows stored
-  constexpr int BP = 4 * NB;        // rows in the t' planes and stats (padded)
+  constexpr int BP = RS;            // rows in the t' planes and stats
   const int sb = out_stage_bytes(BP);
   unsigned char* my_ring = smem + (size_t)warp * S * sb;
   uint64_t* my_bar = reinterpret_cast<uint64_t*>(smem + (size_t)kUWarps * S * sb) + warp * S;
@@ -840,8 +893,9 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
   uint32_t consumed = 0;
   int slot = 0;
   bool dead = false;
-  // this thread's B-operand column: batch row 4nb + g/2, plane g%2
-  const int pl_off = out_planes_off() + g * 32 + 4 * c;
+  // this thread's B-operand column: batch row 4nb + g/2, plane g%2 (at batch
+  // 1, columns of rows 1..3 read row 0's bytes; their sums are not used)
+  const int pl_off = out_planes_off() + (RS == 1 ? (g & 1) : g) * 32 + 4 * c;
 
   while (cs.item < i_end) {
     if (!dead && !mbar_wait(&my_bar[slot], (consumed / S) & 1)) {
@@ -851,14 +905,14 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
     const unsigned char* stage = my_ring + slot * sb;
     const int nt = cs.ntile();
     const unsigned char* pl = stage + pl_off;
-    if (cs.kt0 == 0) out_tile<NB, true>(d, stage, 0, lane, pl);
-    else out_tile<NB>(d, stage, 0, lane, pl);
+    if (cs.kt0 == 0) out_tile<NB, RS, true>(d, stage, 0, lane, pl);
+    else out_tile<NB, RS>(d, stage, 0, lane, pl);
     if (nt == kUChunkTiles) {
 #pragma unroll
-      for (int t = 1; t < kUChunkTiles; ++t) out_tile<NB>(d, stage, t, lane, pl);
+      for (int t = 1; t < kUChunkTiles; ++t) out_tile<NB, RS>(d, stage, t, lane, pl);
     } else {
 #pragma unroll 1
-      for (int t = 1; t < nt; ++t) out_tile<NB>(d, stage, t, lane, pl);
+      for (int t = 1; t < nt; ++t) out_tile<NB, RS>(d, stage, t, lane, pl);
     }
     if (cs.path_end()) {
       // path finished: rows 128*ob + 16q + g (+8), batch row 4nb + c
@@ -1036,14 +1090,14 @@ __global__ void __launch_bounds__(kUWarps * 32) output_packed_kernel(const Decod
     const unsigned char* stage = my_ring + slot * kPkStageBytes;
     const int nt = cs.ntile();
     const unsigned char* pl = stage + pl_off;
-    if (cs.kv0 == 0) out_tile<1, true>(d, stage, 0, lane, pl);
-    else out_tile<1>(d, stage, 0, lane, pl);
+    if (cs.kv0 == 0) out_tile<1, 4, true>(d, stage, 0, lane, pl);
+    else out_tile<1, 4>(d, stage, 0, lane, pl);
     if (nt == kUChunkTiles) {
 #pragma unroll
-      for (int t = 1; t < kUChunkTiles; ++t) out_tile<1>(d, stage, t, lane, pl);
+      for (int t = 1; t < kUChunkTiles; ++t) out_tile<1, 4>(d, stage, t, lane, pl);
     } else {
 #pragma unroll 1
-      for (int t = 1; t < nt; ++t) out_tile<1>(d, stage, t, lane, pl);
+      for (int t = 1; t < nt; ++t) out_tile<1, 4>(d, stage, t, lane, pl);
     }
     if (cs.item_end()) {
       // rows 128*ob + 16q + g (+8); lane c < npaths scales path c, then c = 0
@@ -1112,9 +1166,9 @@ cudaError_t launch_finalize(const DecodeArgs& a, int, cudaStream_t st) {
   return launch_dependent(finalize_kernel<NB>, a.p_items, kFWarps * 32, 0, st, a);
 }
 
-template <int NB>
-size_t output_smem(int) {
-  return (size_t)kUWarps * OutCfg<NB>::kStages * out_stage_bytes(4 * NB) + (size_t)kUWarps * OutCfg<NB>::kStages * 8;
+template <int NB, int RS>
+size_t output_smem() {
+  return (size_t)kUWarps * OutCfg<NB>::kStages * out_stage_bytes(RS) + (size_t)kUWarps * OutCfg<NB>::kStages * 8;
 }
 
 template <int NB, int RB, int W>
@@ -1137,23 +1191,22 @@ cudaError_t launch_latent(const DecodeArgs& a, int num_sms, cudaStream_t st) {
   return launch_dependent(kern, grid, W * 32, smem, st, a);
 }
 
-template <int NB>
+template <int NB, int RS>
 cudaError_t launch_output(const DecodeArgs& a, int num_sms, cudaStream_t st) {
-  const size_t smem = output_smem<NB>(a.batch);
+  const size_t smem = output_smem<NB, RS>();
+  auto kern = output_pass_kernel<NB, RS>;
   // the shared-memory attribute and the occupancy it allows, once per device
   static PerDevice cache;
   int per_sm = 0;
   const int err = cache.get(current_device(), per_sm, [&](int& v) -> int {
-    cudaError_t e = cudaFuncSetAttribute(output_pass_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, output_pass_kernel<NB>, kUWarps * 32, smem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kern, kUWarps * 32, smem);
     if (e == cudaSuccess && v < 1) e = cudaErrorInvalidConfiguration;
     return (int)e;
   });
   if (err != 0) return (cudaError_t)err;
   const int grid = max(1, min((a.u_items + kUWarps - 1) / kUWarps, per_sm * num_sms));
-  return launch_dependent(output_pass_kernel<NB>, grid, kUWarps * 32, smem, st, a);
+  return launch_dependent(kern, grid, kUWarps * 32, smem, st, a);
 }
 
 }  // namespace
@@ -1209,11 +1262,12 @@ cudaError_t launch_output_packed(const DecodeArgs& a, int num_sms, cudaStream_t 
 
 cudaError_t launch_output_pass(const DecodeArgs& a, int num_sms, cudaStream_t st) {
   if (a.packed) return launch_output_packed(a, num_sms, st);
+  if (a.batch == 1) return launch_output<1, 1>(a, num_sms, st);
   switch ((a.batch + 3) / 4) {
-    case 1: return launch_output<1>(a, num_sms, st);
-    case 2: return launch_output<2>(a, num_sms, st);
-    case 3: return launch_output<3>(a, num_sms, st);
-    case 4: return launch_output<4>(a, num_sms, st);
+    case 1: return launch_output<1, 4>(a, num_sms, st);
+    case 2: return launch_output<2, 8>(a, num_sms, st);
+    case 3: return launch_output<3, 12>(a, num_sms, st);
+    case 4: return launch_output<4, 16>(a, num_sms, st);
   }
   return cudaErrorInvalidValue;
 }
