@@ -91,6 +91,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of phase `parity` of `bar`.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Plain arrival (no transaction bytes) on `bar`.
+__device__ __forceinline__ void mbar_arrive_one(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Bounded wait for phase `parity` of `bar`; false after kSpinLimit polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   for (int i = 0; i < kSpinLimit; ++i)
@@ -966,6 +984,244 @@ __global__ void __launch_bounds__(kUWarps * 32) output_pass_kernel(const DecodeA
 }
 
 // ---------------------------------------------------------------------------
+// output pass with a producer warp ("fed"): the same products and epilogue as
+// output_pass_kernel, but the bulk copies are issued by a ninth warp, so that
+// the eight consumer warps only wait, compute and release.  Lane w < 8 of the
+// producer warp runs consumer w's stream: its items are the CTA's items
+// w, w + 8, ..., each cut into chunks of up to 8 K-tiles per path; it writes
+// a 16-byte header into the stage (output pointer, tile count, flags) before
+// the stage's copies, and a final header that ends the stream.  A consumer
+// has kFedSlots stages; the lane refills a stage once its consumer has
+// released it (polled with test_wait, so a lane whose consumer is behind
+// does not hold up the others).
+// ---------------------------------------------------------------------------
+constexpr int kFedCons = 8;     // consumer warps per CTA
+constexpr int kFedSlots = 2;    // stages per consumer warp
+
+// stage: the per-warp pass's stage layout (out_*_off(RS)), then the header
+__host__ __device__ __forceinline__ int fed_hdr_off(int RS) { return out_tstat_off(RS) + 16 * RS; }
+__host__ __device__ __forceinline__ int fed_stage_bytes(int RS) { return (fed_hdr_off(RS) + 16 + 127) & ~127; }
+__host__ __device__ __forceinline__ size_t fed_smem(int RS) {
+  return (size_t)kFedCons * kFedSlots * fed_stage_bytes(RS) + (size_t)2 * kFedCons * kFedSlots * 8;
+}
+
+// header flags
+constexpr uint32_t kFedFirstTile = 1;   // the chunk starts a path: zero the accumulators
+constexpr uint32_t kFedPathEnd = 2;     // the chunk ends a path: scale it into the output
+constexpr uint32_t kFedFirstPath = 4;   // that path is the item's first (assign, not add)
+constexpr uint32_t kFedItemEnd = 8;     // store the item's 128 outputs
+constexpr uint32_t kFedEnd = 16;        // no more chunks for this consumer
+
+// A producer lane's position: item, path, first K-tile, and what it needs
+// to issue the chunk without further descriptor loads.
+struct FedCursor {
+  int item, p, kt0, n_kt, npaths, ob;
+  const LayerDesc* L;
+  const unsigned char* U;
+  const int8_t* planes;
+  const uint16_t* h;
+  const TStat* tstat;
+
+  __device__ __forceinline__ void set_path() {
+    const PathDesc& P = L->p[p];
+    U = reinterpret_cast<const unsigned char*>(P.U);
+    planes = P.ws.planes;
+    h = P.h;
+    tstat = P.ws.tstat;
+  }
+  __device__ __forceinline__ void enter(const DecodeArgs& a, int it) {
+    item = it;
+    L = a.layers + layer_of(a.item_layer.u, a.n_layers, it);
+    n_kt = (L->s + 31) >> 5;
+    npaths = L->npaths;
+    ob = it - L->u_begin;
+    p = 0;
+    kt0 = 0;
+    set_path();
+  }
+};
+
+template <int NB, int RS>
+__global__ void __launch_bounds__((kFedCons + 1) * 32, NB == 1 ? 2 : 1) output_fed_kernel(const DecodeArgs a) {
+  static_assert(RS == 4 * NB || (NB == 1 && RS == 1), "t' rows stored: 1 at batch 1, else 4 per n-block");
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int sb = fed_stage_bytes(RS);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kFedCons * kFedSlots * sb);
+  uint64_t* empty = full + kFedCons * kFedSlots;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  const int i_begin = (int)((long long)a.u_items * blockIdx.x / gridDim.x);
+  const int i_end = (int)((long long)a.u_items * (blockIdx.x + 1) / gridDim.x);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kFedCons * kFedSlots; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();   // the only CTA barrier
+
+  if (warp == kFedCons) {
+    // ---- producer: lane w feeds consumer w.  The first kFedSlots chunks'
+    //      sign tiles and h (weights) are issued before the wait for
+    //      finalize; their t' bytes and step records after it.
+    if (lane >= kFedCons) return;
+    FedCursor cu;
+    if (i_begin + lane < i_end) cu.enter(a, i_begin + lane);
+    else cu.item = i_end;
+    struct TCopy {
+      unsigned char* stage;
+      const int8_t* planes;
+      const TStat* tstat;
+      uint32_t pb;
+      bool path_end;
+      uint64_t* bar;
+    };
+    auto issue = [&](int s, TCopy& tc) -> bool {
+      unsigned char* stage = smem + (size_t)s * sb;
+      uint4* hdr = reinterpret_cast<uint4*>(stage + fed_hdr_off(RS));
+      if (cu.item >= i_end) {
+        *hdr = make_uint4(0u, 0u, kFedEnd << 8, 0u);
+        mbar_arrive_one(&full[s]);
+        tc.pb = 0;
+        return true;
+      }
+      const int nt = min(kUChunkTiles, cu.n_kt - cu.kt0);
+      const bool path_end = cu.kt0 + kUChunkTiles >= cu.n_kt;
+      const uint32_t flags = (cu.kt0 == 0 ? kFedFirstTile : 0u) | (path_end ? kFedPathEnd : 0u) |
+                             (cu.p == 0 ? kFedFirstPath : 0u) |
+                             (path_end && cu.p == cu.npaths - 1 ? kFedItemEnd : 0u);
+      const unsigned long long y = reinterpret_cast<unsigned long long>(cu.L->y + (size_t)cu.ob * kUTileRows);
+      *hdr = make_uint4((uint32_t)y, (uint32_t)(y >> 32), (uint32_t)nt | (flags << 8), (uint32_t)cu.L->d_out);
+      const uint32_t tb = (uint32_t)nt * kTileBytes, pb = (uint32_t)nt * RS * 64;
+      mbar_expect_tx(&full[s], tb + pb + (path_end ? kUTileRows * 2 + 16 * RS : 0));
+      bulk_g2s(stage, cu.U + ((size_t)cu.ob * cu.n_kt + cu.kt0) * kTileBytes, tb, &full[s]);
+      if (path_end) bulk_g2s(stage + out_h_off(RS), cu.h + (size_t)cu.ob * kUTileRows, kUTileRows * 2, &full[s]);
+      tc.stage = stage;
+      tc.planes = cu.planes + (size_t)cu.kt0 * RS * 64;
+      tc.tstat = cu.tstat;
+      tc.pb = pb;
+      tc.path_end = path_end;
+      tc.bar = &full[s];
+      // next chunk of this consumer's stream
+      cu.kt0 += kUChunkTiles;
+      if (cu.kt0 >= cu.n_kt) {
+        cu.kt0 = 0;
+        if (++cu.p == cu.npaths) {
+          if (cu.item + kFedCons < i_end) cu.enter(a, cu.item + kFedCons);
+          else cu.item = i_end;
+        } else {
+          cu.set_path();
+        }
+      }
+      return false;
+    };
+    auto issue_t = [&](const TCopy& tc) {
+      if (!tc.pb) return;
+      bulk_g2s(tc.stage + out_planes_off(), tc.planes, tc.pb, tc.bar);
+      if (tc.path_end) bulk_g2s(tc.stage + out_tstat_off(RS), tc.tstat, 16 * RS, tc.bar);
+    };
+    bool done = false, dead = false;
+    uint32_t n = 0, idle = 0;
+    TCopy pre[kFedSlots];
+    for (int k = 0; k < kFedSlots; ++k) pre[k].pb = 0;
+    for (; n < (uint32_t)kFedSlots && !done; ++n) done = issue(lane * kFedSlots + (int)n, pre[n]);
+    grid_dep_wait();   // finalize's t' planes and steps
+    for (int k = 0; k < kFedSlots; ++k) issue_t(pre[k]);
+    while (!done) {
+      const int s = lane * kFedSlots + (int)(n % kFedSlots);
+      if (!mbar_test_wait(&empty[s], ((n / kFedSlots) - 1) & 1)) {
+        if (++idle > (uint32_t)kSpinLimit) {   // the consumer stopped releasing stages
+          dead = true;
+          break;
+        }
+        __nanosleep(64);
+        continue;
+      }
+      idle = 0;
+      TCopy tc;
+      done = issue(s, tc);
+      issue_t(tc);
+      ++n;
+    }
+    if (dead) atomicOr(a.status, kStatusTimeout);
+    return;
+  }
+
+  // ---- consumer warp
+  const int B = a.batch;
+  float yacc[8][2][NB];
+  int d[8][NB][4];
+  bool dead = false;
+  const int pl_off = out_planes_off() + (RS == 1 ? (g & 1) : g) * 32 + 4 * c;
+#pragma unroll 1
+  for (uint32_t n = 0;; ++n) {
+    const int s = warp * kFedSlots + (int)(n % kFedSlots);
+    if (!mbar_wait(&full[s], (n / kFedSlots) & 1)) {
+      dead = true;
+      break;
+    }
+    const unsigned char* stage = smem + (size_t)s * sb;
+    const uint4 hdr = *reinterpret_cast<const uint4*>(stage + fed_hdr_off(RS));
+    const uint32_t flags = hdr.z >> 8;
+    if (flags & kFedEnd) break;
+    const int nt = (int)(hdr.z & 0xff);
+    const unsigned char* pl = stage + pl_off;
+    if (flags & kFedFirstTile) out_tile<NB, RS, true>(d, stage, 0, lane, pl);
+    else out_tile<NB, RS>(d, stage, 0, lane, pl);
+    if (nt == kUChunkTiles) {
+#pragma unroll
+      for (int t = 1; t < kUChunkTiles; ++t) out_tile<NB, RS>(d, stage, t, lane, pl);
+    } else {
+#pragma unroll 1
+      for (int t = 1; t < nt; ++t) out_tile<NB, RS>(d, stage, t, lane, pl);
+    }
+    if (flags & kFedPathEnd) {
+      // rows 16q + g (+8) of the item, batch row 4nb + c
+      const uint16_t* hs = reinterpret_cast<const uint16_t*>(stage + out_h_off(RS));
+      const TStat* tst = reinterpret_cast<const TStat*>(stage + out_tstat_off(RS));
+      const bool first_path = (flags & kFedFirstPath) != 0;
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        const int b = 4 * nb + c;
+        if (b < B) {
+          const float st = tst[b].step;
+          const float base = st * (float)tst[b].sum;
+          const float m2 = -2.f * st;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int c0 = ((d[q][nb][0] >> q) << 8) + (d[q][nb][1] >> q);
+            const int c1 = ((d[q][nb][2] >> q) << 8) + (d[q][nb][3] >> q);
+            const float y0 = first_path ? 0.f : yacc[q][0][nb], y1 = first_path ? 0.f : yacc[q][1][nb];
+            yacc[q][0][nb] = fmaf(h2f(hs[16 * q + g]), fmaf(m2, (float)c0, base), y0);
+            yacc[q][1][nb] = fmaf(h2f(hs[16 * q + g + 8]), fmaf(m2, (float)c1, base), y1);
+          }
+        }
+      }
+      if (flags & kFedItemEnd) {
+        uint16_t* y = reinterpret_cast<uint16_t*>((unsigned long long)hdr.x | ((unsigned long long)hdr.y << 32));
+        const int d_out = (int)hdr.w;
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          const int b = 4 * nb + c;
+          if (b < B) {
+            uint16_t* yr = y + (size_t)b * d_out + g;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              yr[16 * q] = f2h(yacc[q][0][nb]);
+              yr[16 * q + 8] = f2h(yacc[q][1][nb]);
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive_one(&empty[s]);
+  }
+  if (dead && lane == 0) atomicOr(a.status, kStatusTimeout);
+}
+
+// ---------------------------------------------------------------------------
 // output pass, batch 1 with residual layers ("packed"): the product's 8
 // columns hold 4 batch rows, of which batch 1 uses one, so the paths take the
 // spare ones instead.  Both
@@ -1166,6 +1422,10 @@ cudaError_t launch_finalize(const DecodeArgs& a, int, cudaStream_t st) {
   return launch_dependent(finalize_kernel<NB>, a.p_items, kFWarps * 32, 0, st, a);
 }
 
+// The non-packed output pass runs as the producer-fed kernel (true; up to 8
+// batch rows) or as the per-warp kernel that issues its own copies (false).
+constexpr bool kOutputFed = true;
+
 template <int NB, int RS>
 size_t output_smem() {
   return (size_t)kUWarps * OutCfg<NB>::kStages * out_stage_bytes(RS) + (size_t)kUWarps * OutCfg<NB>::kStages * 8;
@@ -1192,7 +1452,29 @@ cudaError_t launch_latent(const DecodeArgs& a, int num_sms, cudaStream_t st) {
 }
 
 template <int NB, int RS>
+cudaError_t launch_output_fed(const DecodeArgs& a, int num_sms, cudaStream_t st) {
+  const size_t smem = fed_smem(RS);
+  auto kern = output_fed_kernel<NB, RS>;
+  // the shared-memory attribute and the occupancy it allows, once per device
+  static PerDevice cache;
+  int per_sm = 0;
+  const int err = cache.get(current_device(), per_sm, [&](int& v) -> int {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kern, (kFedCons + 1) * 32, smem);
+    if (e == cudaSuccess && v < 1) e = cudaErrorInvalidConfiguration;
+    return (int)e;
+  });
+  if (err != 0) return (cudaError_t)err;
+  // at least two items per consumer warp where there are enough
+  const int grid = max(1, min((a.u_items + 2 * kFedCons - 1) / (2 * kFedCons), per_sm * num_sms));
+  return launch_dependent(kern, grid, (kFedCons + 1) * 32, smem, st, a);
+}
+
+template <int NB, int RS>
 cudaError_t launch_output(const DecodeArgs& a, int num_sms, cudaStream_t st) {
+  // (at three or four n-blocks the fed kernel's 288 threads leave too few
+  // registers for the accumulators; those batches keep the per-warp kernel)
+  if constexpr (kOutputFed && NB <= 2) return launch_output_fed<NB, RS>(a, num_sms, st);
   const size_t smem = output_smem<NB, RS>();
   auto kern = output_pass_kernel<NB, RS>;
   // the shared-memory attribute and the occupancy it allows, once per device
