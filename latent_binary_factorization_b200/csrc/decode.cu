@@ -1390,195 +1390,6 @@ __global__ void __launch_bounds__(kUWarps * 32) output_packed_kernel(const Decod
   }
 }
 
-// ---------------------------------------------------------------------------
-// packed output pass with a producer warp: output_packed_kernel's products and
-// epilogue (batch 1 with residual layers: both paths in one accumulator), fed
-// the way output_fed_kernel is: producer lane w issues consumer w's chunks of
-// up to 8 K-tiles of an item's combined K range, with a header, and the
-// consumers only wait, multiply, store at an item's end and release.
-// ---------------------------------------------------------------------------
-constexpr int kPkHdrOff = kPkTsOff + 2 * 16;
-constexpr int kPkFedStageBytes = (kPkHdrOff + 16 + 127) & ~127;
-constexpr size_t kPkFedSmem = (size_t)kFedCons * kFedSlots * kPkFedStageBytes + (size_t)2 * kFedCons * kFedSlots * 8;
-static_assert(2 * kPkFedSmem <= 227 * 1024, "two packed fed CTAs per SM");
-
-__global__ void __launch_bounds__((kFedCons + 1) * 32, 2) output_packed_fed_kernel(const DecodeArgs a) {
-  extern __shared__ __align__(1024) unsigned char smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kFedCons * kFedSlots * kPkFedStageBytes);
-  uint64_t* empty = full + kFedCons * kFedSlots;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-  const int i_begin = (int)((long long)a.u_items * blockIdx.x / gridDim.x);
-  const int i_end = (int)((long long)a.u_items * (blockIdx.x + 1) / gridDim.x);
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kFedCons * kFedSlots; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
-    }
-    fence_mbar_init();
-  }
-  __syncthreads();   // the only CTA barrier
-
-  if (warp == kFedCons) {
-    // ---- producer: lane w feeds consumer w.  The first kFedSlots chunks'
-    //      sign tiles and h (weights) go out before the wait for finalize.
-    if (lane >= kFedCons) return;
-    int item = i_begin + lane, kv0 = 0, n_kt = 0, npaths = 1, ob = 0;
-    const LayerDesc* L = nullptr;
-    auto enter = [&](int it) {
-      item = it;
-      L = a.layers + layer_of(a.item_layer.u, a.n_layers, it);
-      n_kt = (L->s + 31) >> 5;
-      npaths = L->npaths;
-      ob = it - L->u_begin;
-      kv0 = 0;
-    };
-    if (item < i_end) enter(item);
-    struct TCopy {
-      unsigned char* stage;
-      const int8_t* planes;
-      uint32_t pb;
-      bool last;
-      const LayerDesc* L;
-      uint64_t* bar;
-    };
-    auto issue = [&](int s, TCopy& tc) -> bool {
-      unsigned char* stage = smem + (size_t)s * kPkFedStageBytes;
-      uint4* hdr = reinterpret_cast<uint4*>(stage + kPkHdrOff);
-      if (item >= i_end) {
-        *hdr = make_uint4(0u, 0u, kFedEnd << 8, 0u);
-        mbar_arrive_one(&full[s]);
-        tc.pb = 0;
-        return true;
-      }
-      const int n_kv = npaths * n_kt;
-      const int nt = min(kUChunkTiles, n_kv - kv0);
-      const int t0 = max(0, min(nt, n_kt - kv0));   // tiles of path 0 in this chunk
-      const int t1 = nt - t0;                        // tiles of path 1
-      const bool last = kv0 + kUChunkTiles >= n_kv;
-      const uint32_t flags = (kv0 == 0 ? kFedFirstTile : 0u) | (last ? kFedItemEnd : 0u);
-      const unsigned long long y = reinterpret_cast<unsigned long long>(L->y + (size_t)ob * kUTileRows);
-      *hdr = make_uint4((uint32_t)y, (uint32_t)(y >> 32), (uint32_t)nt | (flags << 8), (uint32_t)npaths);
-      mbar_expect_tx(&full[s], (uint32_t)nt * (kTileBytes + 256) + (last ? npaths * (kUTileRows * 2 + 16) : 0));
-      const PathDesc& P0 = L->p[0];
-      const PathDesc& P1 = L->p[npaths - 1];
-      if (t0 > 0)
-        bulk_g2s(stage, reinterpret_cast<const unsigned char*>(P0.U) + ((size_t)ob * n_kt + kv0) * kTileBytes,
-                 (uint32_t)t0 * kTileBytes, &full[s]);
-      if (t1 > 0)
-        bulk_g2s(stage + t0 * kTileBytes,
-                 reinterpret_cast<const unsigned char*>(P1.U) + ((size_t)ob * n_kt + (kv0 + t0 - n_kt)) * kTileBytes,
-                 (uint32_t)t1 * kTileBytes, &full[s]);
-      if (last) {
-        bulk_g2s(stage + kPkHOff, P0.h + (size_t)ob * kUTileRows, kUTileRows * 2, &full[s]);
-        if (npaths == 2) bulk_g2s(stage + kPkHOff + kUTileRows * 2, P1.h + (size_t)ob * kUTileRows, kUTileRows * 2, &full[s]);
-      }
-      tc.stage = stage;
-      tc.planes = P0.ws.planes + (size_t)kv0 * 256;
-      tc.pb = (uint32_t)nt * 256;
-      tc.last = last;
-      tc.L = L;
-      tc.bar = &full[s];
-      // next chunk of this consumer's stream
-      kv0 += kUChunkTiles;
-      if (kv0 >= n_kv) {
-        if (item + kFedCons < i_end) enter(item + kFedCons);
-        else item = i_end;
-      }
-      return false;
-    };
-    auto issue_t = [&](const TCopy& tc) {
-      if (!tc.pb) return;
-      bulk_g2s(tc.stage + kPkPlanesOff, tc.planes, tc.pb, tc.bar);
-      if (tc.last) {
-        bulk_g2s(tc.stage + kPkTsOff, tc.L->p[0].ws.tstat, 16, tc.bar);
-        if (tc.L->npaths == 2) bulk_g2s(tc.stage + kPkTsOff + 16, tc.L->p[1].ws.tstat, 16, tc.bar);
-      }
-    };
-    bool done = false, dead = false;
-    uint32_t n = 0, idle = 0;
-    TCopy pre[kFedSlots];
-    for (int k = 0; k < kFedSlots; ++k) pre[k].pb = 0;
-    for (; n < (uint32_t)kFedSlots && !done; ++n) done = issue(lane * kFedSlots + (int)n, pre[n]);
-    grid_dep_wait();   // finalize's t' planes and steps
-    for (int k = 0; k < kFedSlots; ++k) issue_t(pre[k]);
-    while (!done) {
-      const int s = lane * kFedSlots + (int)(n % kFedSlots);
-      if (!mbar_test_wait(&empty[s], ((n / kFedSlots) - 1) & 1)) {
-        if (++idle > (uint32_t)kSpinLimit) {   // the consumer stopped releasing stages
-          dead = true;
-          break;
-        }
-        __nanosleep(64);
-        continue;
-      }
-      idle = 0;
-      TCopy tc;
-      done = issue(s, tc);
-      issue_t(tc);
-      ++n;
-    }
-    if (dead) atomicOr(a.status, kStatusTimeout);
-    return;
-  }
-
-  // ---- consumer warp
-  int d[8][1][4];
-  bool dead = false;
-  // this thread's B-operand column: row g/2 (path g/2 for g < 4), plane g%2
-  const int pl_off = kPkPlanesOff + g * 32 + 4 * c;
-  const int pc = min(c, 1);   // path whose sums this lane's columns 2c, 2c+1 hold (c < 2)
-#pragma unroll 1
-  for (uint32_t n = 0;; ++n) {
-    const int s = warp * kFedSlots + (int)(n % kFedSlots);
-    if (!mbar_wait(&full[s], (n / kFedSlots) & 1)) {
-      dead = true;
-      break;
-    }
-    const unsigned char* stage = smem + (size_t)s * kPkFedStageBytes;
-    const uint4 hdr = *reinterpret_cast<const uint4*>(stage + kPkHdrOff);
-    const uint32_t flags = hdr.z >> 8;
-    if (flags & kFedEnd) break;
-    const int nt = (int)(hdr.z & 0xff);
-    const unsigned char* pl = stage + pl_off;
-    if (flags & kFedFirstTile) out_tile<1, 4, true>(d, stage, 0, lane, pl);
-    else out_tile<1, 4>(d, stage, 0, lane, pl);
-    if (nt == kUChunkTiles) {
-#pragma unroll
-      for (int t = 1; t < kUChunkTiles; ++t) out_tile<1, 4>(d, stage, t, lane, pl);
-    } else {
-#pragma unroll 1
-      for (int t = 1; t < nt; ++t) out_tile<1, 4>(d, stage, t, lane, pl);
-    }
-    if (flags & kFedItemEnd) {
-      // rows 16q + g (+8) of the item; lane c < npaths scales path c, then
-      // c = 0 adds c = 1's value and stores
-      const int npaths = (int)hdr.w;
-      const bool live = c < npaths;
-      const uint16_t* hs = reinterpret_cast<const uint16_t*>(stage + kPkHOff + pc * kUTileRows * 2);
-      const TStat tsp = reinterpret_cast<const TStat*>(stage + kPkTsOff)[pc];
-      const float base = tsp.step * (float)tsp.sum, m2 = -2.f * tsp.step;
-      uint16_t* yr = reinterpret_cast<uint16_t*>((unsigned long long)hdr.x | ((unsigned long long)hdr.y << 32)) + g;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int c0 = ((d[q][0][0] >> q) << 8) + (d[q][0][1] >> q);
-        const int c1 = ((d[q][0][2] >> q) << 8) + (d[q][0][3] >> q);
-        float v0 = live ? h2f(hs[16 * q + g]) * fmaf(m2, (float)c0, base) : 0.f;
-        float v1 = live ? h2f(hs[16 * q + g + 8]) * fmaf(m2, (float)c1, base) : 0.f;
-        v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
-        v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
-        if (c == 0) {
-          yr[16 * q] = f2h(v0);
-          yr[16 * q + 8] = f2h(v1);
-        }
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive_one(&empty[s]);
-  }
-  if (dead && lane == 0) atomicOr(a.status, kStatusTimeout);
-}
-
 // ------------------------------------------------------------------ launchers
 
 // Launch `kern` on `st` with programmatic stream serialization: it may start
@@ -1714,25 +1525,7 @@ cudaError_t launch_finalize_pass(const DecodeArgs& a, int max_s16, cudaStream_t 
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_output_packed_fed(const DecodeArgs& a, int num_sms, cudaStream_t st) {
-  // the shared-memory attribute and the occupancy it allows, once per device
-  static PerDevice cache;
-  int per_sm = 0;
-  const int err = cache.get(current_device(), per_sm, [&](int& v) -> int {
-    cudaError_t e = cudaFuncSetAttribute(output_packed_fed_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kPkFedSmem);
-    if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, output_packed_fed_kernel, (kFedCons + 1) * 32, kPkFedSmem);
-    if (e == cudaSuccess && v < 1) e = cudaErrorInvalidConfiguration;
-    return (int)e;
-  });
-  if (err != 0) return (cudaError_t)err;
-  const int grid = max(1, min((a.u_items + 2 * kFedCons - 1) / (2 * kFedCons), per_sm * num_sms));
-  return launch_dependent(output_packed_fed_kernel, grid, (kFedCons + 1) * 32, kPkFedSmem, st, a);
-}
-
 cudaError_t launch_output_packed(const DecodeArgs& a, int num_sms, cudaStream_t st) {
-  if (kOutputFed) return launch_output_packed_fed(a, num_sms, st);
   const size_t smem = (size_t)kUWarps * kPkStages * kPkStageBytes + (size_t)kUWarps * kPkStages * 8;
   // the shared-memory attribute and the occupancy it allows, once per device
   static PerDevice cache;
