@@ -428,19 +428,25 @@ def measure_workload(name, batch, steps, warmup, device, dist, world, l2, seed=1
 
 
 PREFILL_MATS = [(4096, 4096, 290, True)] * 4 + [(4096, 11008, 431, True)] * 2 + [(11008, 4096, 431, True)]
+PREFILL_X_GROUPS = [0, 0, 0, 1, 2, 2, 3]   # q, k, v read one input; gate and up another
 
 
 def measure_prefill(n_layers, M, steps, warmup, device, dist, seed=4321):
     """Llama-2-7B full linear stack at 0.3 BPW residual (4096^2 at s=290;
-    4096<->11008 at s=431), M bf16 tokens per matrix, one forward_many per step."""
+    4096<->11008 at s=431), M bf16 tokens per matrix, one forward_many per step.
+    Within a model layer, q/k/v and gate/up read one input each, as in the
+    model (PREFILL_X_GROUPS)."""
     import torch
     from latent_binary_factorization_b200 import layers as lbl, littlebit as lb
     gen = torch.Generator(device=device).manual_seed(seed)
     Ls, X, Y = [], [], []
     for _ in range(n_layers):
-        for (a, b, s, r) in PREFILL_MATS:
+        xg = {}
+        for (a, b, s, r), g in zip(PREFILL_MATS, PREFILL_X_GROUPS):
             Ls.append(lbl.random_layer(a, b, s, r, gen, device=device)[0])
-            X.append(torch.randn(M, a, generator=gen, device=device).to(torch.bfloat16))
+            if g not in xg:
+                xg[g] = torch.randn(M, a, generator=gen, device=device).to(torch.bfloat16)
+            X.append(xg[g])
             Y.append(torch.empty(M, b, dtype=torch.bfloat16, device=device))
     stack = lb.Stack(Ls, X, Y)
     for _ in range(warmup):
@@ -516,7 +522,8 @@ def run_ours(args):
             os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
         burst, sustained = float(pk.get("bf16_tflops", 1590.0)), float(pk.get("bf16_tflops_sustained", 1400.0))
         tf = pflops / (pms * 1e-3) / 1e12 * world
-        prefill = {"workload": f"Llama-2-7B linear stack 0.3 BPW residual, {args.prefill_layers} layers, M=2048 bf16",
+        prefill = {"workload": f"Llama-2-7B linear stack 0.3 BPW residual, {args.prefill_layers} layers, M=2048 bf16; "
+                               "q/k/v and gate/up share their input",
                    "steps": psteps, "ms_per_step": round(pms, 4), "tflops": round(tf, 1), "unit": "TFLOP/s",
                    "algorithmic_flops_per_step": pflops, "bound": "tensor",
                    "peak_tflops": burst, "frac": round(tf / world / burst, 4),

@@ -201,6 +201,7 @@ constexpr int kPrepKinds = 4;            // preparation steps: x, B1, B2, T' fro
 // GEMMs' tile counts and grids.
 struct PrefillPlan {
   int n;
+  int pair;                      // 1: 256-row tiles on pairs of SMs (M a multiple of 256)
   int tiles1, tiles2, grid1, grid2;
   int prep_grid[kPrepKinds];     // blocks of the grouped x, B1, B2 and cache-to-T' preparation launches
   size_t table_off, table_bytes;
@@ -210,8 +211,11 @@ struct PrefillPlan {
 // per-layer preparation jobs) to img; its device pointers refer to the
 // chunk's operand buffers at `bufs`, the inputs xs and the outputs ys.
 void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const* ys, int n, int M, int x_bf16,
-                        int mode, unsigned char* bufs, int num_sms, std::vector<unsigned char>& img,
+                        int mode, unsigned char* bufs, int num_sms, int pair_slots, std::vector<unsigned char>& img,
                         PrefillPlan& plan);
+// Clusters of two CTAs of the 256-row GEMM that the current device holds at
+// once (0: none); a CUDA error code, 0 on success.
+int prefill_pair_slots(int* slots);
 // A chunk's operand preparation (three grouped launches), then its two
 // grouped GEMM launches; both read the table image uploaded at table_dev.
 cudaError_t launch_prefill_prep(const PrefillPlan& plan, const unsigned char* table_dev, unsigned int* status,

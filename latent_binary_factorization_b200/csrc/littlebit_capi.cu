@@ -430,11 +430,14 @@ lb_status prefill_forward(const lb_layer* layers, int n, const void* const* xs, 
   // table), so that a repeated call enqueues kernels and events only and can
   // be captured into a CUDA graph
   const int sms = num_sms(dev);
+  int pair_slots = 0;
+  const int perr = lb::prefill_pair_slots(&pair_slots);
+  if (perr != 0) return cuda_fail((cudaError_t)perr);
   std::vector<unsigned char> img;
   std::vector<lb::PrefillPlan> plans(n_chunks);
   for (int c = 0; c < n_chunks; ++c)
     lb::plan_prefill_chunk(descs.data() + starts[c], xs + starts[c], ys + starts[c], starts[c + 1] - starts[c],
-                           batch, x_bf16, mode, chunk_bufs(c), sms, img, plans[c]);
+                           batch, x_bf16, mode, chunk_bufs(c), sms, pair_slots, img, plans[c]);
   if (img.size() > tables) return LB_ERR_SHAPE;   // the plan above sized the tables
   if (ws.table.size() != img.size() || std::memcmp(ws.table.data(), img.data(), img.size()) != 0) {
     // pageable source: the copy is staged before the call returns

@@ -26,8 +26,10 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <array>
 #include <cstring>
 #include <functional>
+#include <map>
 #include <queue>
 #include <utility>
 #include <vector>
@@ -144,6 +146,9 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 // run of a row.  Each thread takes kXUnroll units spaced a grid apart and
 // issues all their loads before converting, so several loads are in flight.
 constexpr int kXUnroll = 4;
+// Preparation blocks (256 threads, <= 40 registers) per SM in one launch: three
+// leave room for a GEMM CTA beside them.
+constexpr int kPrepBlocksPerSm = 3;
 
 __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
   uint32_t* w = &v.x;
@@ -382,12 +387,19 @@ struct GroupArgs {
 
 constexpr int kGroupThreads = 192;
 
+// The pair kernel (below): 256-row tiles, each CTA of the pair holding 128
+// rows of A and half of B's rows per stage.
+constexpr int kPairStages = 6;
+constexpr int kPairBBytes = kBN / 2 * kBK * 2;   // 16 KB
+
 struct TileInfo {
   const GemmProblem* P;
   int m0, n0, n_len, nk;
 };
 
-__device__ __forceinline__ TileInfo tile_info(const GroupArgs& ga, int tile) {
+// Tile `tile` of the problem list; m-tiles are `rows` high (128, or 256 for
+// a pair of CTAs).
+__device__ __forceinline__ TileInfo tile_info(const GroupArgs& ga, int tile, int rows) {
   int lo = 0, hi = ga.n_probs - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -397,7 +409,7 @@ __device__ __forceinline__ TileInfo tile_info(const GroupArgs& ga, int tile) {
   ti.P = ga.probs + lo;
   const int local = tile - ti.P->tile_begin;
   const int mt = local / ti.P->tiles_n, nt = local - mt * ti.P->tiles_n;
-  ti.m0 = mt * kBM;
+  ti.m0 = mt * rows;
   ti.n0 = nt * kBN;
   ti.n_len = min(kBN, ti.P->N - ti.n0);
   ti.nk = ti.P->K / kBK;
@@ -406,6 +418,84 @@ __device__ __forceinline__ TileInfo tile_info(const GroupArgs& ga, int tile) {
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su(b)) : "memory");
+}
+
+// Drains one accumulator into the tile's output.  The calling warp reads TMEM
+// lanes 32*quarter .. +31 from taddr on, which hold output rows
+// row0 + 32*quarter + lane; `bad` collects fp16 values beyond range.
+__device__ __forceinline__ void epilogue_tile(const TileInfo& ti, uint32_t taddr, int row0, int quarter, int lane,
+                                              unsigned char* ystage, unsigned& bad) {
+  const GemmProblem& P = *ti.P;
+  const int row = row0 + 32 * quarter + lane;
+  if (P.mode == 1) {
+    // y: 64 columns at a time through shared memory, so that eight lanes
+    // write one row's 128 contiguous bytes
+    unsigned char* sy = ystage + (size_t)quarter * 32 * kYPitch;
+    for (int c0 = 0; c0 < ti.n_len; c0 += 64) {
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        float v[16];
+        tmem_ld16(taddr + (uint32_t)(c0 + 16 * h), v);
+        uint32_t w[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          if (P.y_bf16) {
+            const __nv_bfloat162 bb = __floats2bfloat162_rn(v[e], v[e + 1]);
+            w[e >> 1] = *reinterpret_cast<const uint32_t*>(&bb);
+          } else {
+            const __half2 hh = __floats2half2_rn(v[e], v[e + 1]);
+            w[e >> 1] = *reinterpret_cast<const uint32_t*>(&hh);
+            bad |= half2_nonfinite(w[e >> 1]);
+          }
+        }
+        *reinterpret_cast<uint4*>(sy + lane * kYPitch + 32 * h) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(sy + lane * kYPitch + 32 * h + 16) = make_uint4(w[4], w[5], w[6], w[7]);
+      }
+      __syncwarp();
+      const int cb = lane & 7;
+#pragma unroll
+      for (int r4 = 0; r4 < 32; r4 += 4) {
+        const int r = r4 + (lane >> 3);
+        const uint4 val = *reinterpret_cast<const uint4*>(sy + r * kYPitch + cb * 16);
+        uint16_t* yr = static_cast<uint16_t*>(P.Y) + (size_t)(row0 + 32 * quarter + r) * P.N + ti.n0 + c0;
+        *reinterpret_cast<uint4*>(yr + 8 * cb) = val;
+      }
+      __syncwarp();
+    }
+    return;
+  }
+  for (int c0 = 0; c0 < ti.n_len; c0 += 16) {
+    float v[16];
+    tmem_ld16(taddr + (uint32_t)c0, v);
+    uint32_t w[8];
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+      float lv[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int n = ti.n0 + c0 + e + u;
+        const int p = n / P.Sp, j = n - p * P.Sp;
+        const uint16_t* l = p == 0 ? P.l0 : P.l1;
+        lv[u] = j < P.s ? __half2float(__ushort_as_half(l[j])) : 0.f;
+      }
+      const __half2 hh = __floats2half2_rn(lv[0] * v[e], lv[1] * v[e + 1]);
+      w[e >> 1] = *reinterpret_cast<const uint32_t*>(&hh);
+      bad |= half2_nonfinite(w[e >> 1]);
+    }
+    if (P.mode == 0) {
+      *reinterpret_cast<uint4*>(P.T + tiled_off(row, ti.n0 + c0, P.M)) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4*>(P.T + tiled_off(row, ti.n0 + c0 + 8, P.M)) = make_uint4(w[4], w[5], w[6], w[7]);
+    } else {
+      // cache row: path p's t'_j at column p*s + j, j < s
+      uint16_t* yr = static_cast<uint16_t*>(P.Y) + (size_t)row * P.t_ld;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int n = ti.n0 + c0 + e;
+        const int p = n / P.Sp, j = n - p * P.Sp;
+        if (j < P.s) yr[p * P.s + j] = (uint16_t)(w[e >> 1] >> (16 * (e & 1)));
+      }
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const GroupArgs ga) {
@@ -448,7 +538,7 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
     // ---- producer
     uint32_t it = 0;
     for (int k = ga.begin[blockIdx.x]; k < ga.begin[blockIdx.x + 1]; ++k) {
-      const TileInfo ti = tile_info(ga, ga.sched[k]);
+      const TileInfo ti = tile_info(ga, ga.sched[k], kBM);
       const uint32_t bbytes = (uint32_t)ti.n_len * kBK * 2;
       const int Mg = ti.P->M >> 3, Ng = ti.P->N >> 3;
       for (int kb = 0; kb < ti.nk; ++kb, ++it) {
@@ -463,7 +553,7 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
     // ---- MMA issuer
     uint32_t it = 0, nt = 0;
     for (int k = ga.begin[blockIdx.x]; k < ga.begin[blockIdx.x + 1]; ++k, ++nt) {
-      const TileInfo ti = tile_info(ga, ga.sched[k]);
+      const TileInfo ti = tile_info(ga, ga.sched[k], kBM);
       const int ab = nt & 1;
       if (nt >= 2 && !dead && !mbar_wait(&acce[ab], ((nt >> 1) - 1) & 1)) dead = true;
       tc_fence_after();
@@ -488,85 +578,13 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
     uint32_t nt = 0;
     unsigned bad = 0;   // a t' (or fp16 y) beyond fp16's range: LB_ERR_RANGE
     for (int k = ga.begin[blockIdx.x]; k < ga.begin[blockIdx.x + 1]; ++k, ++nt) {
-      const TileInfo ti = tile_info(ga, ga.sched[k]);
+      const TileInfo ti = tile_info(ga, ga.sched[k], kBM);
       const int ab = nt & 1;
       if (!dead && !mbar_wait(&accf[ab], (nt >> 1) & 1)) dead = true;
       dead = __any_sync(0xffffffffu, dead);
       tc_fence_after();
-      const GemmProblem& P = *ti.P;
-      const int row = ti.m0 + 32 * quarter + lane;
-      const uint32_t taddr = tmem + (uint32_t)(ab * kBN) + ((uint32_t)(32 * quarter) << 16);
-      if (P.mode == 1) {
-        // y: 64 columns at a time through shared memory, so that eight lanes
-        // write one row's 128 contiguous bytes
-        unsigned char* sy = ystage + (size_t)quarter * 32 * kYPitch;
-        for (int c0 = 0; c0 < ti.n_len; c0 += 64) {
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            float v[16];
-            tmem_ld16(taddr + (uint32_t)(c0 + 16 * h), v);
-            uint32_t w[8];
-#pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              if (P.y_bf16) {
-                const __nv_bfloat162 bb = __floats2bfloat162_rn(v[e], v[e + 1]);
-                w[e >> 1] = *reinterpret_cast<const uint32_t*>(&bb);
-              } else {
-                const __half2 hh = __floats2half2_rn(v[e], v[e + 1]);
-                w[e >> 1] = *reinterpret_cast<const uint32_t*>(&hh);
-                bad |= half2_nonfinite(w[e >> 1]);
-              }
-            }
-            *reinterpret_cast<uint4*>(sy + lane * kYPitch + 32 * h) = make_uint4(w[0], w[1], w[2], w[3]);
-            *reinterpret_cast<uint4*>(sy + lane * kYPitch + 32 * h + 16) = make_uint4(w[4], w[5], w[6], w[7]);
-          }
-          __syncwarp();
-          const int cb = lane & 7;
-#pragma unroll
-          for (int r4 = 0; r4 < 32; r4 += 4) {
-            const int r = r4 + (lane >> 3);
-            const uint4 val = *reinterpret_cast<const uint4*>(sy + r * kYPitch + cb * 16);
-            uint16_t* yr = static_cast<uint16_t*>(P.Y) + (size_t)(ti.m0 + 32 * quarter + r) * P.N + ti.n0 + c0;
-            *reinterpret_cast<uint4*>(yr + 8 * cb) = val;
-          }
-          __syncwarp();
-        }
-      }
-      for (int c0 = 0; P.mode != 1 && c0 < ti.n_len; c0 += 16) {
-        float v[16];
-        tmem_ld16(taddr + (uint32_t)c0, v);
-        uint32_t w[8];
-        {
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            float lv[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int n = ti.n0 + c0 + e + u;
-              const int p = n / P.Sp, j = n - p * P.Sp;
-              const uint16_t* l = p == 0 ? P.l0 : P.l1;
-              lv[u] = j < P.s ? __half2float(__ushort_as_half(l[j])) : 0.f;
-            }
-            const __half2 hh = __floats2half2_rn(lv[0] * v[e], lv[1] * v[e + 1]);
-            w[e >> 1] = *reinterpret_cast<const uint32_t*>(&hh);
-            bad |= half2_nonfinite(w[e >> 1]);
-          }
-          if (P.mode == 0) {
-            *reinterpret_cast<uint4*>(P.T + tiled_off(row, ti.n0 + c0, P.M)) = make_uint4(w[0], w[1], w[2], w[3]);
-            *reinterpret_cast<uint4*>(P.T + tiled_off(row, ti.n0 + c0 + 8, P.M)) =
-                make_uint4(w[4], w[5], w[6], w[7]);
-          } else {
-            // cache row: path p's t'_j at column p*s + j, j < s
-            uint16_t* yr = static_cast<uint16_t*>(P.Y) + (size_t)row * P.t_ld;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int n = ti.n0 + c0 + e;
-              const int p = n / P.Sp, j = n - p * P.Sp;
-              if (j < P.s) yr[p * P.s + j] = (uint16_t)(w[e >> 1] >> (16 * (e & 1)));
-            }
-          }
-        }
-      }
+      epilogue_tile(ti, tmem + (uint32_t)(ab * kBN) + ((uint32_t)(32 * quarter) << 16), ti.m0, quarter, lane,
+                    ystage, bad);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acce[ab]);
@@ -574,7 +592,7 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
     if (dead && lane == 0) atomicOr(ga.status, kStatusTimeout);
     if (__any_sync(0xffffffffu, bad != 0) && lane == 0) atomicOr(ga.status, kStatusRange);
   }
-  if ((threadIdx.x == 0 || threadIdx.x == 32) && dead) atomicOr(ga.status, 1u << LB_ERR_TIMEOUT);
+  if ((threadIdx.x == 0 || threadIdx.x == 32) && dead) atomicOr(ga.status, kStatusTimeout);
   __syncwarp();
   tc_fence_before();
   __syncthreads();
@@ -584,7 +602,212 @@ __global__ void __launch_bounds__(kGroupThreads, 1) umma_group_kernel(const Grou
   }
 }
 
+// ---- helpers of the pair kernel
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of this CTA's variable p in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(su(p)), "r"(rank));
+  return a;
+}
+// arrive on a barrier of another CTA of the cluster (or this one), given its
+// shared::cluster address
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+// every thread of both CTAs
+__device__ __forceinline__ void pair_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void umma_f16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive on `bar` of both CTAs of the pair once every pair product issued so
+// far by this thread is done
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  const uint16_t both = 3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          su(bar)),
+      "h"(both)
+      : "memory");
+}
+
+// The grouped GEMM on pairs of SMs (clusters of two CTAs).  A tile is 256 rows:
+// CTA r of the pair holds rows 128r .. 128r+127 of A and rows
+// r*n_len/2 .. (r+1)*n_len/2 - 1 of B in its shared memory, and the even CTA
+// issues tcgen05.mma.cta_group::2 (M = 256), which reads both CTAs' operands
+// and writes each CTA's 128 accumulator rows into that CTA's tensor memory.
+// A K-block stage is 32 KB per CTA instead of 48, so shared memory moves a
+// third fewer bytes per product and each B tile leaves L2 once per pair.
+//
+// Synchronisation.  Each CTA's copies complete on its own full barrier; in the
+// odd CTA, warp 1 relays every completed stage to the even CTA's full barrier
+// (which counts two arrivals: its own copies' and the relay's).  The pair's
+// commits arrive on the empty and accumulator-full barriers of both CTAs.  The
+// epilogue warps of both CTAs free an accumulator on the even CTA's barrier
+// (eight arrivals).  Producers wait for the commits of their last stages, and
+// a cluster barrier precedes the exit, so nothing arrives on a CTA that has
+// left.  Every wait is bounded, as in the single-CTA kernel.
+__global__ void __launch_bounds__(kGroupThreads, 1) umma_pair_kernel(const GroupArgs ga) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  unsigned char* sA = smem;
+  unsigned char* sB = smem + kPairStages * kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kPairStages * kPairBBytes);
+  uint64_t* empty = full + kPairStages;
+  uint64_t* accf = empty + kPairStages;
+  uint64_t* acce = accf + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+  unsigned char* ystage = smem + kPairStages * (kABytes + kPairBBytes) + 1024;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su(tmem_slot)),
+                 "r"(2 * kBN)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  if (threadIdx.x == 32) {
+    for (int i = 0; i < kPairStages; ++i) {
+      mbar_init(&full[i], rank == 0 ? 2 : 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&accf[i], 1);
+      mbar_init(&acce[i], 8);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  pair_sync();   // both CTAs' barriers and tensor memory are set up before either uses the other's
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int t_begin = ga.begin[pair], t_end = ga.begin[pair + 1];
+  bool dead = false;
+
+  if (threadIdx.x == 0) {
+    // ---- producer: this CTA's half of every stage
+    uint32_t it = 0;
+    for (int k = t_begin; k < t_end; ++k) {
+      const TileInfo ti = tile_info(ga, ga.sched[k], 2 * kBM);
+      const int half = ti.n_len >> 1;
+      const uint32_t bbytes = (uint32_t)half * kBK * 2;
+      const int Mg = ti.P->M >> 3, Ng = ti.P->N >> 3;
+      const int ag = (ti.m0 + kBM * (int)rank) >> 3, bg = (ti.n0 + half * (int)rank) >> 3;
+      for (int kb = 0; kb < ti.nk; ++kb, ++it) {
+        const int st = it % kPairStages;
+        if (it >= kPairStages && !dead && !mbar_wait(&empty[st], ((it / kPairStages) - 1) & 1)) dead = true;
+        mbar_expect_tx(&full[st], kABytes + bbytes);
+        bulk_g2s(sA + st * kABytes, ti.P->A + ((size_t)kb * Mg + ag) * 1024, kABytes, &full[st]);
+        bulk_g2s(sB + st * kPairBBytes, ti.P->B + ((size_t)kb * Ng + bg) * 1024, bbytes, &full[st]);
+      }
+    }
+    // the commits that free the last stages
+    for (uint32_t i = it > kPairStages ? it - kPairStages : 0; i < it && !dead; ++i)
+      if (!mbar_wait(&empty[i % kPairStages], (i / kPairStages) & 1)) dead = true;
+  } else if (threadIdx.x == 32 && rank == 0) {
+    // ---- MMA issuer (even CTA)
+    uint32_t it = 0, nt = 0;
+    for (int k = t_begin; k < t_end; ++k, ++nt) {
+      const TileInfo ti = tile_info(ga, ga.sched[k], 2 * kBM);
+      const int ab = nt & 1;
+      if (nt >= 2 && !dead && !mbar_wait(&acce[ab], ((nt >> 1) - 1) & 1)) dead = true;
+      tc_fence_after();
+      const uint32_t d = tmem + (uint32_t)(ab * kBN);
+      const uint32_t idesc = umma_idesc_f16(2 * kBM, ti.n_len);
+      for (int kb = 0; kb < ti.nk; ++kb, ++it) {
+        const int st = it % kPairStages;
+        if (!dead && !mbar_wait(&full[st], (it / kPairStages) & 1)) dead = true;
+        tc_fence_after();
+        const uint32_t a0 = su(sA + st * kABytes), b0 = su(sB + st * kPairBBytes);
+#pragma unroll
+        for (int ks = 0; ks < kBK / 16; ++ks)
+          umma_f16_pair(d, umma_desc(a0 + ks * 256, 128, 1024), umma_desc(b0 + ks * 256, 128, 1024), idesc,
+                        (kb > 0 || ks > 0) ? 1u : 0u);
+        umma_commit_pair(&empty[st]);
+      }
+      umma_commit_pair(&accf[ab]);
+    }
+  } else if (threadIdx.x == 32) {
+    // ---- relay (odd CTA): each stage of this CTA, once landed, to the even CTA
+    uint32_t it = 0;
+    for (int k = t_begin; k < t_end; ++k) {
+      const TileInfo ti = tile_info(ga, ga.sched[k], 2 * kBM);
+      for (int kb = 0; kb < ti.nk; ++kb, ++it) {
+        const int st = it % kPairStages;
+        if (!dead && !mbar_wait(&full[st], (it / kPairStages) & 1)) dead = true;
+        if (!dead) mbar_arrive_remote(cluster_addr(&full[st], 0));
+      }
+    }
+  } else if (warp >= 2) {
+    // ---- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 of this CTA
+    const int quarter = warp & 3;
+    const uint32_t acce_even0 = cluster_addr(&acce[0], 0), acce_even1 = cluster_addr(&acce[1], 0);
+    uint32_t nt = 0;
+    unsigned bad = 0;
+    for (int k = t_begin; k < t_end; ++k, ++nt) {
+      const TileInfo ti = tile_info(ga, ga.sched[k], 2 * kBM);
+      const int ab = nt & 1;
+      if (!dead && !mbar_wait(&accf[ab], (nt >> 1) & 1)) dead = true;
+      dead = __any_sync(0xffffffffu, dead);
+      tc_fence_after();
+      epilogue_tile(ti, tmem + (uint32_t)(ab * kBN) + ((uint32_t)(32 * quarter) << 16), ti.m0 + kBM * (int)rank,
+                    quarter, lane, ystage, bad);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(ab ? acce_even1 : acce_even0);
+    }
+    if (dead && lane == 0) atomicOr(ga.status, kStatusTimeout);
+    if (__any_sync(0xffffffffu, bad != 0) && lane == 0) atomicOr(ga.status, kStatusRange);
+  }
+  if ((threadIdx.x == 0 || threadIdx.x == 32) && dead) atomicOr(ga.status, kStatusTimeout);
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  pair_sync();   // neither CTA leaves while the pair's products or arrivals may still reach it
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kBN) : "memory");
+  }
+}
+
 size_t group_smem() { return (size_t)kStages * (kABytes + kBBytes) + 1024 + (size_t)4 * 32 * kYPitch; }
+size_t pair_smem() { return (size_t)kPairStages * (kABytes + kPairBBytes) + 1024 + (size_t)4 * 32 * kYPitch; }
+
+cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kGroupThreads, 1, 1);
+  cfg.dynamicSmemBytes = pair_smem();
+  cfg.stream = st;
+  attr->id = cudaLaunchAttributeClusterDimension;
+  attr->val.clusterDim.x = 2;
+  attr->val.clusterDim.y = 1;
+  attr->val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+// `clusters` pairs of CTAs over the tile lists of ga
+cudaError_t launch_pair(const GroupArgs& ga, int clusters, cudaStream_t st) {
+  cudaLaunchAttribute attr;
+  const cudaLaunchConfig_t cfg = pair_config(clusters, st, &attr);
+  return cudaLaunchKernelEx(&cfg, umma_pair_kernel, ga);
+}
 
 int grid_for(long long work, int per_block) {
   long long b = (work + per_block - 1) / per_block;
@@ -593,6 +816,29 @@ int grid_for(long long work, int per_block) {
 }
 
 }  // namespace
+
+// Pairs of CTAs of the pair kernel that can be resident at once on the
+// current device (its shared-memory attribute set on first use); 0 when the
+// device runs none.  Returns a CUDA error code, 0 on success.
+int prefill_pair_slots(int* slots) {
+  static PerDevice cache;
+  int v = 0;
+  const int err = cache.get(current_device(), v, [](int& out) -> int {
+    cudaError_t e = cudaFuncSetAttribute(umma_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)pair_smem());
+    if (e != cudaSuccess) return (int)e;
+    cudaLaunchAttribute attr;
+    const cudaLaunchConfig_t cfg = pair_config(1, nullptr, &attr);
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, umma_pair_kernel, &cfg);
+    if (e != cudaSuccess) return (int)e;
+    out = n > 0 ? n : -1;   // -1: cached "none"
+    return 0;
+  });
+  if (err != 0) return err;
+  *slots = v > 0 ? v : 0;
+  return 0;
+}
 
 int prefill_sp(int s, int npaths) { return npaths == 2 ? s32(s) : ceil_div(s, 64) * 64; }
 
@@ -647,7 +893,7 @@ static LayerBufs layer_bufs(unsigned char*& buf, const LayerDesc& L, int M) {
 }
 
 // Blocks of one layer's preparation steps (x, B1, B2), as for a launch of its own.
-static void prep_blocks(const LayerDesc& L, int M, int Sp, int mode, int (&blocks)[kPrepKinds]) {
+static void prep_blocks(const LayerDesc& L, int M, int Sp, int mode, std::array<int, kPrepKinds>& blocks) {
   const int P = L.npaths;
   blocks[3] = grid_for((long long)M * P * Sp / 8, 256);
   blocks[0] = grid_for((long long)M * L.d_in / 8 / kXUnroll, 256);
@@ -711,10 +957,13 @@ static double tile_cost(int K, int n_len) { return (double)(K / kBK) * (double)m
 // to the chunk's buffers at `bufs` and to the image's own place at
 // table_dev + plan.table_off.
 void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const* ys, int n, int M, int x_bf16,
-                        int mode, unsigned char* bufs, int num_sms, std::vector<unsigned char>& img,
+                        int mode, unsigned char* bufs, int num_sms, int pair_slots, std::vector<unsigned char>& img,
                         PrefillPlan& plan) {
   const long long tiles_all = group_tiles(Ls, n, M);
   plan.n = n;
+  // 256-row tiles on pairs of SMs when M allows them and pairs can be resident
+  plan.pair = (M % (2 * kBM) == 0 && pair_slots > 0) ? 1 : 0;
+  const int rows = plan.pair ? 2 * kBM : kBM;
   plan.table_off = (img.size() + 1023) & ~(size_t)1023;
   plan.table_bytes = prefill_table_bytes(n, tiles_all);
   plan.jobs_off = prep_jobs_off(n, tiles_all);
@@ -730,22 +979,31 @@ void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const*
   std::vector<double> cost1, cost2;
   int tiles1 = 0, tiles2 = 0;
   unsigned char* buf = bufs;
+  std::vector<std::array<int, kPrepKinds>> blocks(n);
+  // layers of the chunk that read the same x (same pointer and width; a
+  // block's q, k and v projections, gate and up) share one converted X16
+  std::map<std::pair<const void*, int>, unsigned char*> x16_of;
   for (int i = 0; i < n; ++i) {
     const LayerDesc& L = Ls[i];
     const int P = L.npaths, Sp = prefill_sp(L.s, P), NK = P * Sp;
-    const LayerBufs b = layer_bufs(buf, L, M);
+    LayerBufs b = layer_bufs(buf, L, M);
     PrepJob& J = jobs[i];
     std::memset(&J, 0, sizeof(J));
     J.L = L;
     J.x = static_cast<const uint16_t*>(xs[i]);
+    prep_blocks(L, M, Sp, mode, blocks[i]);
+    if (mode != kModeExpand) {
+      const auto key = std::make_pair(xs[i], L.d_in);
+      const auto it = x16_of.find(key);
+      if (it == x16_of.end()) {
+        x16_of.emplace(key, b.X16);
+      } else {
+        b.X16 = it->second;   // converted by the first layer that reads this x
+        blocks[i][0] = 0;
+      }
+    }
     J.X16 = b.X16; J.B1 = b.B1; J.B2 = b.B2; J.T = b.T;
     J.M = M; J.x_bf16 = x_bf16; J.Sp = Sp;
-    int blocks[kPrepKinds];
-    prep_blocks(L, M, Sp, mode, blocks);
-    for (int k = 0; k < kPrepKinds; ++k) {
-      J.first[k] = plan.prep_grid[k];
-      plan.prep_grid[k] += blocks[k];
-    }
     GemmProblem& g1 = probs[i];
     g1 = GemmProblem{};
     g1.A = b.X16; g1.B = b.B1; g1.M = M; g1.N = NK; g1.K = L.d_in; g1.mode = mode == kModeLatent ? 2 : 0;
@@ -753,8 +1011,8 @@ void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const*
     g1.Y = mode == kModeLatent ? ys[i] : nullptr; g1.t_ld = L.t_ld;
     g1.tiles_n = ceil_div(NK, kBN); g1.tile_begin = tiles1;
     if (mode != kModeExpand) {
-      tiles1 += (M / kBM) * g1.tiles_n;
-      for (int mt = 0; mt < M / kBM; ++mt)
+      tiles1 += (M / rows) * g1.tiles_n;
+      for (int mt = 0; mt < M / rows; ++mt)
         for (int nt = 0; nt < g1.tiles_n; ++nt) cost1.push_back(tile_cost(g1.K, min(kBN, NK - nt * kBN)));
     }
     GemmProblem& g2 = probs[n + i];
@@ -762,16 +1020,34 @@ void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const*
     g2.A = b.T; g2.B = b.B2; g2.M = M; g2.N = L.d_out; g2.K = NK; g2.mode = 1; g2.Y = ys[i]; g2.y_bf16 = x_bf16;
     g2.tiles_n = ceil_div(L.d_out, kBN); g2.tile_begin = tiles2;
     if (mode != kModeLatent) {
-      tiles2 += (M / kBM) * g2.tiles_n;
-      for (int mt = 0; mt < M / kBM; ++mt)
+      tiles2 += (M / rows) * g2.tiles_n;
+      for (int mt = 0; mt < M / rows; ++mt)
         for (int nt = 0; nt < g2.tiles_n; ++nt) cost2.push_back(tile_cost(g2.K, min(kBN, L.d_out - nt * kBN)));
+    }
+  }
+  // The preparation of the next chunk runs beside this chunk's GEMM (one CTA
+  // per SM, 192 threads x 128 registers).  Each preparation launch is
+  // therefore held to kPrepBlocksPerSm blocks per SM in total, so that a GEMM
+  // CTA still fits on an SM next to them; a layer's share stays proportional
+  // to its work.
+  for (int k = 0; k < kPrepKinds; ++k) {
+    long long total = 0;
+    for (int i = 0; i < n; ++i) total += blocks[i][k];
+    const long long cap = (long long)kPrepBlocksPerSm * num_sms;
+    for (int i = 0; i < n; ++i) {
+      int b = blocks[i][k];
+      if (total > cap && b > 0) b = (int)std::max<long long>(1, (long long)b * cap / total);
+      jobs[i].first[k] = plan.prep_grid[k];
+      plan.prep_grid[k] += b;
     }
   }
   int* sched2 = sched1 + tiles1;
   plan.tiles1 = tiles1;
   plan.tiles2 = tiles2;
-  plan.grid1 = min(min(tiles1, num_sms), kMaxGemmGrid);
-  plan.grid2 = min(min(tiles2, num_sms), kMaxGemmGrid);
+  // CTAs (or, for pairs, clusters) of the persistent launches
+  const int slots = plan.pair ? min(pair_slots, kMaxGemmGrid / 2) : min(num_sms, kMaxGemmGrid);
+  plan.grid1 = min(tiles1, slots);
+  plan.grid2 = min(tiles2, slots);
   if (plan.grid1 > 0) lpt_schedule(cost1, plan.grid1, sched1, begin1);
   if (plan.grid2 > 0) lpt_schedule(cost2, plan.grid2, sched2, begin2);
 }
@@ -790,6 +1066,10 @@ cudaError_t launch_prefill_gemms(const PrefillPlan& plan, const unsigned char* t
                                      (int)group_smem());
   });
   if (err != 0) return (cudaError_t)err;
+  if (plan.pair) {
+    const int perr = prefill_pair_slots(&done);
+    if (perr != 0) return (cudaError_t)perr;
+  }
   const unsigned char* base = table_dev + plan.table_off;
   const size_t prob_b = (size_t)2 * plan.n * sizeof(GemmProblem);
   const GemmProblem* probs = reinterpret_cast<const GemmProblem*>(base);
@@ -797,10 +1077,16 @@ cudaError_t launch_prefill_gemms(const PrefillPlan& plan, const unsigned char* t
   const int* sched_dev = begin_dev + 2 * (kMaxGemmGrid + 1);
   // GEMM1 (not in expand calls) and GEMM2 (not in latent-only calls)
   GroupArgs g1a{probs, sched_dev, begin_dev, plan.n, plan.tiles1, status};
-  if (plan.grid1 > 0) umma_group_kernel<<<plan.grid1, kGroupThreads, group_smem(), st>>>(g1a);
   GroupArgs g2a{probs + plan.n, sched_dev + plan.tiles1, begin_dev + kMaxGemmGrid + 1, plan.n, plan.tiles2, status};
-  if (plan.grid2 > 0) umma_group_kernel<<<plan.grid2, kGroupThreads, group_smem(), st>>>(g2a);
-  return cudaGetLastError();
+  if (!plan.pair) {
+    if (plan.grid1 > 0) umma_group_kernel<<<plan.grid1, kGroupThreads, group_smem(), st>>>(g1a);
+    if (plan.grid2 > 0) umma_group_kernel<<<plan.grid2, kGroupThreads, group_smem(), st>>>(g2a);
+    return cudaGetLastError();
+  }
+  cudaError_t e = cudaSuccess;
+  if (plan.grid1 > 0) e = launch_pair(g1a, plan.grid1, st);
+  if (e == cudaSuccess && plan.grid2 > 0) e = launch_pair(g2a, plan.grid2, st);
+  return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 }  // namespace lb

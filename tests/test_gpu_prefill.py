@@ -101,19 +101,53 @@ def test_prefill_forward_many(lbm):
         _check(y, ref, f"layer {i}")
 
 
-def test_prefill_chunked_stack_matches_single_layer_calls(lbm):
+@pytest.mark.parametrize("M", [256, 384])
+def test_prefill_forward_many_shared_inputs(lbm, M):
+    """Layers of one prefill call that read the same x (q, k and v; gate and
+    up) share one converted operand: every output matches the oracle and is
+    bit-identical to its one-layer call.  M = 256 runs the GEMMs on pairs of
+    SMs, M = 384 on single SMs."""
+    lb, layers = lbm
+    groups = [[(1024, 1024, 64, True)] * 3, [(1024, 2048, 100, False)] * 2, [(2048, 512, 77, True)],
+              [(1024, 768, 45, True)]]
+    L, X, Y, refs = [], [], [], []
+    k = 0
+    for g, members in enumerate(groups):
+        xt, x64 = _x(M, members[0][0], seed=60 + g, dtype=torch.bfloat16)
+        x = xt.cuda()
+        for (a, b, s, r) in members:
+            paths = synth.layer(a, b, s, r, seed=70 + k, index=k)
+            L.append(layers.upload(paths, a, b, s))
+            X.append(x)
+            Y.append(torch.full((M, b), float("nan"), dtype=torch.bfloat16, device="cuda"))
+            refs.append(orc.factored_forward(x64, paths))
+            k += 1
+    lb.Stack(L, X, Y)()
+    torch.cuda.synchronize()
+    for i, (y, ref) in enumerate(zip(Y, refs)):
+        _check(y, ref, f"layer {i}")
+        assert torch.equal(y, lb.forward(L[i], X[i])), f"layer {i} differs from its one-layer call"
+    assert lb.device_status() == 0
+
+
+@pytest.mark.parametrize("shared", [False, True])
+def test_prefill_chunked_stack_matches_single_layer_calls(lbm, shared):
     """A stack whose operand buffers span several chunks (preparation of one
     chunk overlapped with the GEMMs of the previous one, two workspace halves
     reused in turn) gives, layer by layer, exactly what one-layer calls give;
     a second call in a row, after the halves hold the last call's operands,
-    gives it again."""
+    gives it again.  With `shared`, layers read their inputs in groups of three
+    (as q, k and v do), and some groups straddle a chunk boundary."""
     lb, layers = lbm
     gen = torch.Generator(device="cuda").manual_seed(11)
     M, n = 2048, 40   # ~29 MB of operands per layer: three chunks
     L, X, Y = [], [], []
     for i in range(n):
         L.append(layers.random_layer(4096, 4096, 290, True, gen)[0])
-        X.append(torch.randn(M, 4096, generator=gen, device="cuda").to(torch.bfloat16))
+        if shared and i % 3:
+            X.append(X[-1])
+        else:
+            X.append(torch.randn(M, 4096, generator=gen, device="cuda").to(torch.bfloat16))
         Y.append(torch.full((M, 4096), float("nan"), dtype=torch.bfloat16, device="cuda"))
     st = lb.Stack(L, X, Y)
     st()
