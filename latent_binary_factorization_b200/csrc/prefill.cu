@@ -198,97 +198,109 @@ __device__ __forceinline__ void prep_x(const uint16_t* __restrict__ x, int is_bf
   if (bad) atomicOr(status, kStatusRange);
 }
 
-// B1 (P*Sp rows x d_in): row p*Sp + j holds V_p[i][j] * g_p[i].  Work unit =
-// (16-byte lane of a packed role-V tile, word r, half qh of the eight
-// products): for each of its four q the word gives four consecutive i of one
-// row, i.e. one 8-byte piece of B1.  Units with the same tile, r and qh are 32
-// consecutive threads (one per lane), so a warp's stores cover whole 128-byte
-// core-matrix rows.  Rows j >= s inside the packed tiles get +-g (finite;
-// GEMM1's epilogue zeroes them through l); rows from the tiles' end up to Sp
-// are zero.
+// The bit of word w (of a packed tile's 16-byte lane) for product q, as the
+// fp16 sign bits of four consecutive elements: byte m of (w >> q) & 0x01010101
+// is element m's sign.
+__device__ __forceinline__ uint2 sign_bits4(uint32_t w, int q) {
+  const uint32_t bits = (w >> q) & 0x01010101u;
+  return make_uint2(((bits & 1u) << 15) | (((bits >> 8) & 1u) << 31),
+                    (((bits >> 16) & 1u) << 15) | (((bits >> 24) & 1u) << 31));
+}
+
+// B1 (P*Sp rows x d_in): row p*Sp + j holds V_p[i][j] * g_p[i].  One warp per
+// packed role-V tile (16 rows j x 256 inputs i): each lane loads its 16-byte
+// lane of the tile once; word r, product q gives four consecutive i of one row,
+// i.e. one 8-byte piece of B1, for 32 pieces per lane.  For each (q, r) the
+// warp's pieces cover two whole 128-byte core-matrix rows.  g is read through
+// L1 (8 bytes per lane and q, shared by the tile's rows).  Rows j >= s inside
+// the packed tiles get +-g (finite; GEMM1's epilogue zeroes them through l);
+// rows from the tiles' end up to Sp are zero, written by the same threads in
+// 16-byte pieces after the tiles.
 __device__ __forceinline__ void prep_b1(const LayerDesc& L, int Sp, unsigned char* __restrict__ out, unsigned bid,
                                         unsigned nblk) {
   const int R = L.npaths * Sp, K = L.d_in;
   const int n_kt = K / kVTileK, n_rb = (L.s + 15) >> 4;
   const unsigned tiles_p = (unsigned)(n_rb * n_kt);
-  const unsigned units = (unsigned)L.npaths * tiles_p * 256;
-  const unsigned zrow16 = (unsigned)(K / 8);                    // 16-byte pieces per zero row
-  const unsigned zeros = (unsigned)(L.npaths * (Sp - 16 * n_rb)) * zrow16;
-  for (unsigned t = bid * blockDim.x + threadIdx.x; t < units + zeros; t += nblk * blockDim.x) {
-    if (t < units) {
-      const int lane = t & 31, r = (t >> 5) & 3, qh = (t >> 7) & 1;
-      const unsigned tile = t >> 8;
-      const int p = tile >= tiles_p ? 1 : 0;
-      const int tt = (int)(tile - p * tiles_p);
-      const int rb = tt / n_kt, kt = tt - rb * n_kt;
-      const uint32_t w = reinterpret_cast<const uint32_t*>(reinterpret_cast<const unsigned char*>(L.p[p].V) +
-                                                           (size_t)tt * kTileBytes + 16 * lane)[r];
-      const uint16_t* g = L.p[p].g;
-      const int gg = lane >> 2, c = lane & 3;
-      const int jr = p * Sp + 16 * rb + gg + 8 * (r & 1);
+  const unsigned tiles = (unsigned)L.npaths * tiles_p;
+  const int lane = threadIdx.x & 31, gg = lane >> 2, c = lane & 3;
+  const unsigned nwarps = nblk * (blockDim.x >> 5);
+  for (unsigned tile = bid * (blockDim.x >> 5) + (threadIdx.x >> 5); tile < tiles; tile += nwarps) {
+    const int p = tile >= tiles_p ? 1 : 0;
+    const int tt = (int)(tile - p * tiles_p);
+    const int rb = tt / n_kt, kt = tt - rb * n_kt;
+    const uint4 wv = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned char*>(L.p[p].V) +
+                                                          (size_t)tt * kTileBytes) + lane);
+    const uint32_t w[4] = {wv.x, wv.y, wv.z, wv.w};
+    const uint16_t* g = L.p[p].g;
+    const int j0 = p * Sp + 16 * rb + gg;
 #pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
-        const int q = 4 * qh + qq;
-        const int i0 = 256 * kt + 32 * q + 16 * (r >> 1) + 4 * c;
-        const uint2 gv = *reinterpret_cast<const uint2*>(g + i0);
-        const uint32_t bits = (w >> q) & 0x01010101u;   // byte m: bit of i0 + m
-        const uint32_t s0 = (bits & 1u) << 15, s1 = ((bits >> 8) & 1u) << 31;
-        const uint32_t s2 = ((bits >> 16) & 1u) << 15, s3 = ((bits >> 24) & 1u) << 31;
-        *reinterpret_cast<uint2*>(out + tiled_off(jr, i0, R)) = make_uint2(gv.x ^ (s0 | s1), gv.y ^ (s2 | s3));
+    for (int q = 0; q < 8; ++q) {
+#pragma unroll
+      for (int rh = 0; rh < 2; ++rh) {
+        const int i0 = 256 * kt + 32 * q + 16 * rh + 4 * c;
+        const uint2 gv = __ldg(reinterpret_cast<const uint2*>(g + i0));
+#pragma unroll
+        for (int rl = 0; rl < 2; ++rl) {
+          const uint2 sg = sign_bits4(w[2 * rh + rl], q);
+          *reinterpret_cast<uint2*>(out + tiled_off(j0 + 8 * rl, i0, R)) = make_uint2(gv.x ^ sg.x, gv.y ^ sg.y);
+        }
       }
-    } else {
-      const unsigned z = t - units;
-      const unsigned row_i = z / zrow16;
-      const int k = (int)(z - row_i * zrow16) * 8;
-      const int per = Sp - 16 * n_rb;
-      const int p = (int)row_i / per, jr = p * Sp + 16 * n_rb + ((int)row_i - p * per);
-      *reinterpret_cast<uint4*>(out + tiled_off(jr, k, R)) = make_uint4(0u, 0u, 0u, 0u);
     }
+  }
+  const unsigned zrow16 = (unsigned)(K / 8);                    // 16-byte pieces per zero row
+  const int per = Sp - 16 * n_rb;
+  const unsigned zeros = (unsigned)(L.npaths * per) * zrow16;
+  for (unsigned z = bid * blockDim.x + threadIdx.x; z < zeros; z += nblk * blockDim.x) {
+    const unsigned row_i = z / zrow16;
+    const int k = (int)(z - row_i * zrow16) * 8;
+    const int p = (int)row_i / per, jr = p * Sp + 16 * n_rb + ((int)row_i - p * per);
+    *reinterpret_cast<uint4*>(out + tiled_off(jr, k, R)) = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
-// B2 (d_out rows x P*Sp): row o, column p*Sp + j holds U_p[o][j] * h_p[o].  Work
-// unit = (16-byte lane of a packed role-U tile, word r, half qh of the eight
-// products): for each of its four q the word gives four consecutive j of one
-// row.  Columns from the tiles' end up to Sp are zero.
+// B2 (d_out rows x P*Sp): row o, column p*Sp + j holds U_p[o][j] * h_p[o].  One
+// warp per packed role-U tile (128 rows o x 32 latent j), as prep_b1: word r,
+// product q of a lane gives four consecutive j of row o = 128*ob + 16*q + gg +
+// 8*(r&1).  Columns from the tiles' end up to Sp are zero.
 __device__ __forceinline__ void prep_b2(const LayerDesc& L, int Sp, unsigned char* __restrict__ out, unsigned bid,
                                         unsigned nblk) {
   const int R = L.d_out;
   const int n_kt = (L.s + 31) >> 5, n_ob = R / kUTileRows;
   const unsigned tiles_p = (unsigned)(n_ob * n_kt);
-  const unsigned units = (unsigned)L.npaths * tiles_p * 256;
+  const unsigned tiles = (unsigned)L.npaths * tiles_p;
+  const int lane = threadIdx.x & 31, gg = lane >> 2, c = lane & 3;
+  const unsigned nwarps = nblk * (blockDim.x >> 5);
+  for (unsigned tile = bid * (blockDim.x >> 5) + (threadIdx.x >> 5); tile < tiles; tile += nwarps) {
+    const int p = tile >= tiles_p ? 1 : 0;
+    const int tt = (int)(tile - p * tiles_p);
+    const int ob = tt / n_kt, kt = tt - ob * n_kt;
+    const uint4 wv = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned char*>(L.p[p].U) +
+                                                          (size_t)tt * kTileBytes) + lane);
+    const uint32_t w[4] = {wv.x, wv.y, wv.z, wv.w};
+    const uint16_t* h = L.p[p].h;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+#pragma unroll
+      for (int rl = 0; rl < 2; ++rl) {
+        const int o = kUTileRows * ob + 16 * q + gg + 8 * rl;
+        const uint32_t hv = (uint32_t)__ldg(h + o) * 0x00010001u;
+#pragma unroll
+        for (int rh = 0; rh < 2; ++rh) {
+          const int j0 = p * Sp + 32 * kt + 16 * rh + 4 * c;
+          const uint2 sg = sign_bits4(w[2 * rh + rl], q);
+          *reinterpret_cast<uint2*>(out + tiled_off(o, j0, R)) = make_uint2(hv ^ sg.x, hv ^ sg.y);
+        }
+      }
+    }
+  }
   const int zc8 = (Sp - 32 * n_kt) / 8;                    // zero 16-byte pieces per row and path
   const unsigned per = (unsigned)(R * zc8);
   const unsigned zeros = (unsigned)L.npaths * per;
-  for (unsigned t = bid * blockDim.x + threadIdx.x; t < units + zeros; t += nblk * blockDim.x) {
-    if (t < units) {
-      const int lane = t & 31, r = (t >> 5) & 3, qh = (t >> 7) & 1;
-      const unsigned tile = t >> 8;
-      const int p = tile >= tiles_p ? 1 : 0;
-      const int tt = (int)(tile - p * tiles_p);
-      const int ob = tt / n_kt, kt = tt - ob * n_kt;
-      const uint32_t w = reinterpret_cast<const uint32_t*>(reinterpret_cast<const unsigned char*>(L.p[p].U) +
-                                                           (size_t)tt * kTileBytes + 16 * lane)[r];
-      const uint16_t* h = L.p[p].h;
-      const int gg = lane >> 2, c = lane & 3;
-      const int j0 = p * Sp + 32 * kt + 16 * (r >> 1) + 4 * c;
-#pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
-        const int q = 4 * qh + qq;
-        const int o = kUTileRows * ob + 16 * q + gg + 8 * (r & 1);
-        const uint32_t hv = (uint32_t)h[o] * 0x00010001u;
-        const uint32_t bits = (w >> q) & 0x01010101u;
-        const uint32_t s0 = (bits & 1u) << 15, s1 = ((bits >> 8) & 1u) << 31;
-        const uint32_t s2 = ((bits >> 16) & 1u) << 15, s3 = ((bits >> 24) & 1u) << 31;
-        *reinterpret_cast<uint2*>(out + tiled_off(o, j0, R)) = make_uint2(hv ^ (s0 | s1), hv ^ (s2 | s3));
-      }
-    } else {
-      const unsigned z = t - units;
-      const int p = (int)(z / per);
-      const int zz = (int)(z - (unsigned)p * per);
-      const int o = zz / zc8, j = p * Sp + 32 * n_kt + (zz - o * zc8) * 8;
-      *reinterpret_cast<uint4*>(out + tiled_off(o, j, R)) = make_uint4(0u, 0u, 0u, 0u);
-    }
+  for (unsigned z = bid * blockDim.x + threadIdx.x; z < zeros; z += nblk * blockDim.x) {
+    const int p = (int)(z / per);
+    const int zz = (int)(z - (unsigned)p * per);
+    const int o = zz / zc8, j = p * Sp + 32 * n_kt + (zz - o * zc8) * 8;
+    *reinterpret_cast<uint4*>(out + tiled_off(o, j, R)) = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
@@ -372,7 +384,8 @@ struct GemmProblem {
   unsigned char* T;         // mode 0 output, core-matrix tiles M x N
   void* Y;                  // mode 1 output, row-major M x N; mode 2: cache rows, t_ld apart
   int y_bf16, t_ld;
-  int tiles_n, tile_begin;
+  int tiles_n, tile_w;      // N is cut into tiles_n column tiles of tile_w (the last may be narrower)
+  int tile_begin;
 };
 
 // Tiles of CTA b: sched[begin[b] .. begin[b+1]), built on the host (longest
@@ -410,8 +423,8 @@ __device__ __forceinline__ TileInfo tile_info(const GroupArgs& ga, int tile, int
   const int local = tile - ti.P->tile_begin;
   const int mt = local / ti.P->tiles_n, nt = local - mt * ti.P->tiles_n;
   ti.m0 = mt * rows;
-  ti.n0 = nt * kBN;
-  ti.n_len = min(kBN, ti.P->N - ti.n0);
+  ti.n0 = nt * ti.P->tile_w;
+  ti.n_len = min(ti.P->tile_w, ti.P->N - ti.n0);
   ti.nk = ti.P->K / kBK;
   return ti;
 }
@@ -897,12 +910,13 @@ static void prep_blocks(const LayerDesc& L, int M, int Sp, int mode, std::array<
   const int P = L.npaths;
   blocks[3] = grid_for((long long)M * P * Sp / 8, 256);
   blocks[0] = grid_for((long long)M * L.d_in / 8 / kXUnroll, 256);
-  const long long l1 = (long long)P * ((L.s + 15) >> 4) * (L.d_in / kVTileK) * 256 +
-                       (long long)P * (Sp - 16 * ((L.s + 15) >> 4)) * (L.d_in / 8);
-  blocks[1] = grid_for(l1, 256);
-  const long long l2 = (long long)P * (L.d_out / kUTileRows) * ((L.s + 31) >> 5) * 256 +
-                       (long long)P * L.d_out * ((Sp - 32 * ((L.s + 31) >> 5)) / 8);
-  blocks[2] = grid_for(l2, 256);
+  // B1, B2: a warp per packed tile, then a thread per zero 16-byte piece
+  const long long v_tiles = (long long)P * ((L.s + 15) >> 4) * (L.d_in / kVTileK);
+  const long long v_zeros = (long long)P * (Sp - 16 * ((L.s + 15) >> 4)) * (L.d_in / 8);
+  blocks[1] = grid_for(std::max(v_tiles * 32, v_zeros), 256);
+  const long long u_tiles = (long long)P * (L.d_out / kUTileRows) * ((L.s + 31) >> 5);
+  const long long u_zeros = (long long)P * L.d_out * ((Sp - 32 * ((L.s + 31) >> 5)) / 8);
+  blocks[2] = grid_for(std::max(u_tiles * 32, u_zeros), 256);
   // forward: x, B1, B2; latent-only: x, B1; expand: B2 and T' from the cache
   if (mode == kModeLatent) blocks[2] = 0;
   if (mode == kModeExpand) blocks[0] = blocks[1] = 0;
@@ -922,14 +936,18 @@ cudaError_t launch_prefill_prep(const PrefillPlan& plan, const unsigned char* ta
   return cudaGetLastError();
 }
 
-// Longest-first schedule of `cost` over `grid` CTAs: every tile, in order of
-// decreasing cost, goes to the CTA with the least work so far.  Writes the
-// CTA lists to sched (tile indices) and their offsets to begin[0..grid].
-static void lpt_schedule(const std::vector<double>& cost, int grid, int* sched, int* begin) {
+// Longest-first schedule of `cost` over `grid` CTAs: every tile goes to the
+// CTA with the least work so far.  Tiles are taken in order of decreasing
+// `key`, ties in list order; the key is the cost of the tile's row panel (its
+// first tile), so the tiles of one panel stay together and run at about the
+// same time.  Writes the CTA lists to sched (tile indices) and their offsets
+// to begin[0..grid].
+static void lpt_schedule(const std::vector<double>& cost, const std::vector<double>& key, int grid, int* sched,
+                         int* begin) {
   const int T = (int)cost.size();
   std::vector<int> order(T);
   for (int i = 0; i < T; ++i) order[i] = i;
-  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return key[a] > key[b]; });
   using Slot = std::pair<double, int>;   // (load, cta)
   std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
   for (int b = 0; b < grid; ++b) heap.push({0.0, b});
@@ -946,6 +964,18 @@ static void lpt_schedule(const std::vector<double>& cost, int grid, int* sched, 
     for (int t : lists[b]) sched[k++] = t;
   }
   begin[grid] = k;
+}
+
+// Column tiles of an N-wide product: as few as UMMA's N <= 256 allows, of
+// equal width rounded up to `gran` (16; 64 for GEMM2, whose epilogue stores
+// 64 columns at a time).  Equal widths keep a row panel's tiles in one cost
+// class of the schedule, so they run at about the same time and the panel
+// leaves DRAM once; a narrow last tile would be scheduled much later and read
+// it again.
+static void split_n(int N, int gran, int& tiles, int& width) {
+  tiles = ceil_div(N, kBN);
+  width = ceil_div(ceil_div(N, tiles), gran) * gran;
+  tiles = ceil_div(N, width);
 }
 
 // Tile cost for the schedule: K-blocks times the tile's share of a full-width
@@ -976,7 +1006,7 @@ void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const*
   int* begin1 = reinterpret_cast<int*>(base + prob_b);
   int* begin2 = begin1 + kMaxGemmGrid + 1;
   int* sched1 = begin2 + kMaxGemmGrid + 1;
-  std::vector<double> cost1, cost2;
+  std::vector<double> cost1, cost2, key1, key2;
   int tiles1 = 0, tiles2 = 0;
   unsigned char* buf = bufs;
   std::vector<std::array<int, kPrepKinds>> blocks(n);
@@ -1009,20 +1039,28 @@ void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const*
     g1.A = b.X16; g1.B = b.B1; g1.M = M; g1.N = NK; g1.K = L.d_in; g1.mode = mode == kModeLatent ? 2 : 0;
     g1.l0 = L.p[0].l; g1.l1 = P == 2 ? L.p[1].l : L.p[0].l; g1.s = L.s; g1.Sp = Sp; g1.T = b.T;
     g1.Y = mode == kModeLatent ? ys[i] : nullptr; g1.t_ld = L.t_ld;
-    g1.tiles_n = ceil_div(NK, kBN); g1.tile_begin = tiles1;
+    split_n(NK, 16, g1.tiles_n, g1.tile_w);
+    g1.tile_begin = tiles1;
     if (mode != kModeExpand) {
       tiles1 += (M / rows) * g1.tiles_n;
       for (int mt = 0; mt < M / rows; ++mt)
-        for (int nt = 0; nt < g1.tiles_n; ++nt) cost1.push_back(tile_cost(g1.K, min(kBN, NK - nt * kBN)));
+        for (int nt = 0; nt < g1.tiles_n; ++nt) {
+          cost1.push_back(tile_cost(g1.K, min(g1.tile_w, NK - nt * g1.tile_w)));
+          key1.push_back(tile_cost(g1.K, g1.tile_w));
+        }
     }
     GemmProblem& g2 = probs[n + i];
     g2 = GemmProblem{};
     g2.A = b.T; g2.B = b.B2; g2.M = M; g2.N = L.d_out; g2.K = NK; g2.mode = 1; g2.Y = ys[i]; g2.y_bf16 = x_bf16;
-    g2.tiles_n = ceil_div(L.d_out, kBN); g2.tile_begin = tiles2;
+    split_n(L.d_out, 64, g2.tiles_n, g2.tile_w);
+    g2.tile_begin = tiles2;
     if (mode != kModeLatent) {
       tiles2 += (M / rows) * g2.tiles_n;
       for (int mt = 0; mt < M / rows; ++mt)
-        for (int nt = 0; nt < g2.tiles_n; ++nt) cost2.push_back(tile_cost(g2.K, min(kBN, L.d_out - nt * kBN)));
+        for (int nt = 0; nt < g2.tiles_n; ++nt) {
+          cost2.push_back(tile_cost(g2.K, min(g2.tile_w, L.d_out - nt * g2.tile_w)));
+          key2.push_back(tile_cost(g2.K, g2.tile_w));
+        }
     }
   }
   // The preparation of the next chunk runs beside this chunk's GEMM (one CTA
@@ -1048,8 +1086,8 @@ void plan_prefill_chunk(const LayerDesc* Ls, const void* const* xs, void* const*
   const int slots = plan.pair ? min(pair_slots, kMaxGemmGrid / 2) : min(num_sms, kMaxGemmGrid);
   plan.grid1 = min(tiles1, slots);
   plan.grid2 = min(tiles2, slots);
-  if (plan.grid1 > 0) lpt_schedule(cost1, plan.grid1, sched1, begin1);
-  if (plan.grid2 > 0) lpt_schedule(cost2, plan.grid2, sched2, begin2);
+  if (plan.grid1 > 0) lpt_schedule(cost1, key1, plan.grid1, sched1, begin1);
+  if (plan.grid2 > 0) lpt_schedule(cost2, key2, plan.grid2, sched2, begin2);
 }
 
 // GEMM1 and GEMM2 of a planned chunk (table uploaded at table_dev +
