@@ -164,9 +164,10 @@ __device__ __forceinline__ int layer_of(const int* map, int n_layers, int item) 
 // quantise pass:  u = g_p (.) x on one 2048-input slice of one layer, for each
 // path p, quantised per batch row to 16 bits, v = step * (256*hi + lo), and
 // stored as the latent pass's int8 B fragments (slice block layout in
-// lb_internal.h).  One warp per (layer, path, slice): lane i holds the 8-input
-// chunks i + 32j (j < 8) of one batch row; max and sum are warp reductions, so
-// the kernel has no CTA barrier.
+// lb_internal.h).  One warp per (group of layers reading one x, slice, up to
+// kQRows batch rows): lane i holds the 8-input chunks i + 32j (j < 8) of one
+// batch row at a time; max and sum are warp reductions, so the kernel has no
+// CTA barrier.
 //
 // Arithmetic per value: u = g*x in fp32 (exact for fp16 operands); v =
 // round(u * 32639 / max|u|) by adding 1.5*2^23 in fp32, which leaves v in the
@@ -253,10 +254,11 @@ __device__ __forceinline__ void quantise_row(const uint4 (&xq)[kQChunks], const 
   }
 }
 
-// Work item = (group of layers that read the same x, 2048-input slice): the
-// item reads each batch row's x slice once and quantises g (.) x for every
-// path of every layer of the group (layers chained by x_next from the
-// group's first layer, whose x_begin numbers the group's items).
+// Work item = (group of layers that read the same x, 2048-input slice, group
+// of kQRows batch rows): the item reads each of its batch rows' x slice once
+// and quantises g (.) x for every path of every layer of the group (layers
+// chained by x_next from the group's first layer, whose x_begin numbers the
+// group's items, slice-major).
 __global__ void __launch_bounds__(kQWarps * 32) quantise_input_kernel(const DecodeArgs a) {
   grid_dep_launch();
   const int lane = threadIdx.x & 31;
@@ -265,7 +267,8 @@ __global__ void __launch_bounds__(kQWarps * 32) quantise_input_kernel(const Deco
   const int B = a.batch, NC = 2 * xq_rows(B);
   const int first = layer_of(a.item_layer.x, a.n_layers, item);
   const LayerDesc& L0 = a.layers[first];
-  const int sl = item - L0.x_begin;
+  const int n_rg = (B + kQRows - 1) / kQRows, rel = item - L0.x_begin;
+  const int sl = rel / n_rg, rg = rel - sl * n_rg;
   const int d_in = L0.d_in, k0 = sl * kVSlice;
   const int nchunk = min(kVSlice, d_in - k0) / 8;
   const size_t blk_off = (size_t)sl * xq_slice_bytes(B);
@@ -273,8 +276,9 @@ __global__ void __launch_bounds__(kQWarps * 32) quantise_input_kernel(const Deco
   unsigned bad = 0;   // an input x that is inf or NaN (LB_ERR_RANGE)
   // rows B .. 4*nb-1 of a block are never read: their product columns are
   // independent of the batch rows' and their sums are discarded
+  const int row_end = min(B, kQRows * (rg + 1));
 #pragma unroll 1
-  for (int row = 0; row < B; ++row) {
+  for (int row = kQRows * rg; row < row_end; ++row) {
     uint4 xq[kQChunks];
 #pragma unroll
     for (int j = 0; j < kQChunks; ++j) {

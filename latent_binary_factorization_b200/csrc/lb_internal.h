@@ -33,6 +33,10 @@ constexpr int kTileBytes = 512;
 // buffer copy and wait, and finalize sums more partials: at batch 16 on a
 // 28672-input layer, 512-input slices ran 4x slower.)
 constexpr int kVSliceTiles = 8;
+// Batch rows per quantise-pass item: a batch of B rows is quantised by
+// ceil(B / kQRows) warps per input slice.
+constexpr int kQRows = 4;
+inline int q_row_groups(int batch) { return (batch + kQRows - 1) / kQRows; }
 constexpr int kVSlice = kVSliceTiles * kVTileK;          // 2048 inputs
 constexpr int kVStages = 2;                              // bulk-copy ring per warp
 
@@ -150,7 +154,7 @@ struct LayerDesc {
   int v_begin;        // first latent-pass work item of this layer
   int u_begin;        // first output-pass work item of this layer
   int p_begin;        // first (layer, path) index of this layer
-  int x_begin;        // first quantise-pass item (x group, input slice) of this layer's x group
+  int x_begin;        // first quantise-pass item (x group, input slice, row group) of this layer's x group
                       // (set on the group's first layer)
   int x_next;         // next layer of the call that reads the same x (same pointer and d_in), or -1
 };
@@ -173,7 +177,7 @@ struct DecodeArgs {
   int v_items;              // total latent-pass items
   int u_items;              // total output-pass items (layer, 128-row block)
   int p_items;              // total (layer, path) pairs
-  int x_items;              // total quantise-pass items (group of layers sharing x, input slice)
+  int x_items;              // total quantise-pass items (group of layers sharing x, input slice, row group)
   int v_warps;              // latent-pass CTA width (3 or 4; latent_warps)
   int packed;               // batch 1 with a residual layer: paths share the output pass's product
   int mode;                 // CallMode

@@ -227,7 +227,7 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
   for (int i = 0; i < n; ++i) {
     const lb_layer& L = layers[i];
     const int npaths = L.residual + 1, n_slices = lb::ceil_div(L.d_in, lb::kVSlice);
-    if (x_lead[i] == i) x_items += n_slices;
+    if (x_lead[i] == i) x_items += n_slices * lb::q_row_groups(batch);
     v_items += npaths * n_slices * lb::ceil_div(lb::s16(L.s) / 16, 2 * vw);
     p_items += npaths;
     u_items += L.d_out / lb::kUTileRows;
@@ -279,7 +279,7 @@ lb_status decode_forward(const lb_layer* layers, int n, const void* const* xs, v
     D.p_begin = pi;
     D.u_begin = ui;
     if (x_lead[i] == i)
-      for (int k = 0; k < D.n_slices; ++k) xm[xi++] = i;
+      for (int k = 0; k < D.n_slices * lb::q_row_groups(batch); ++k) xm[xi++] = i;
     for (int k = 0; k < D.npaths * D.n_slices * D.n_rchunks; ++k) vm[vi++] = i;
     for (int k = 0; k < D.npaths; ++k) pm[pi++] = i;
     for (int k = 0; k < L.d_out / lb::kUTileRows; ++k) um[ui++] = i;

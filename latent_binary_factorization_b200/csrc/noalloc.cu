@@ -147,7 +147,7 @@ lb_status littlebit_linear_forward_noalloc(const lb_layer* layer, const void* x_
   a.v_items = npaths * D.n_slices * D.n_rchunks;
   a.u_items = L.d_out / lb::kUTileRows;
   a.p_items = npaths;
-  a.x_items = D.n_slices;
+  a.x_items = D.n_slices * lb::q_row_groups(batch);
   a.v_warps = vw;
   a.packed = batch == 1 && L.residual ? 1 : 0;
   a.mode = lb::kModeForward;

@@ -84,6 +84,32 @@ def test_prefill_matches_decode_on_same_rows(lbm):
     assert orc.rel_l2(a, b) <= 2 * REL_L2
 
 
+@pytest.mark.parametrize("d_in,d_out,s,residual", [(1024, 640, 290, True), (2048, 768, 133, True),
+                                                   (1024, 384, 188, False)])
+def test_pair_and_single_sm_gemms_agree(lbm, d_in, d_out, s, residual):
+    """The same 384 rows through the pair-of-SMs GEMMs (M = 256: rows 0..255)
+    and the single-SM GEMMs (M = 384 and M = 128): every row matches the
+    oracle, and the two kernels agree row by row within fp16 rounding of t'
+    and y.  The shapes give unequal column tiles (640 = 224 + 224 + 192 and a
+    path boundary inside a tile)."""
+    lb, layers = lbm
+    paths = synth.layer(d_in, d_out, s, residual, seed=s + 5)
+    layer = layers.upload(paths, d_in, d_out, s)
+    xt, x64 = _x(384, d_in, seed=s, dtype=torch.bfloat16)
+    xd = xt.cuda()
+    y_all = lb.forward(layer, xd)                 # M = 384: single-SM tiles
+    y_pair = lb.forward(layer, xd[:256].contiguous())   # M = 256: pairs of SMs
+    y_tail = lb.forward(layer, xd[256:].contiguous())   # M = 128: single-SM
+    torch.cuda.synchronize()
+    ref = orc.factored_forward(x64, paths)
+    _check(y_pair, ref[:256], "pair GEMM")
+    _check(y_all, ref, "single-SM GEMM")
+    assert torch.equal(y_tail, y_all[256:])
+    a, b = y_pair.float().cpu().numpy(), y_all[:256].float().cpu().numpy()
+    assert orc.rel_l2(a, b) <= REL_L2
+    assert lb.device_status() == 0
+
+
 def test_prefill_forward_many(lbm):
     lb, layers = lbm
     specs = [(1024, 1024, 64, True), (1024, 2048, 100, False), (2048, 512, 77, True)]
