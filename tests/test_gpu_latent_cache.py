@@ -51,6 +51,7 @@ def test_row_size_matches_the_oracle(lbm):
     (2048, 1024, 100, True, 16, torch.float16),
     (4096, 4096, 188, False, 256, torch.bfloat16),  # prefill: a prompt's K/V rows
     (1024, 768, 90, True, 128, torch.float16),
+    (1024, 768, 90, True, 512, torch.bfloat16),     # pairs of SMs, both paths in one column tile
     (1024, 768, 45, True, 130, torch.float16),      # prefill 128 + decode group of 2
 ])
 def test_latent_forward_and_expand(lbm, d_in, d_out, s, residual, batch, dtype):
