@@ -456,7 +456,7 @@ struct VFeed {
 };
 
 template <int NB, int RB, int W>
-__global__ void __launch_bounds__(W * 32, NB == 1 ? 4 : 1) latent_pass_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(W * 32, NB == 1 ? 3 : 1) latent_pass_kernel(const DecodeArgs a) {
   constexpr int NC = 2 * RB;                      // B-fragment columns stored per K-block
   constexpr int RPW = VCfg<NB>::kRPW;
   constexpr int kStageBytes = RPW * kChunkBytes;
