@@ -301,11 +301,12 @@ __global__ void __launch_bounds__(kQWarps * 32) quantise_input_kernel(const Deco
 // ---------------------------------------------------------------------------
 // latent pass:  t_j (partial over one slice) = sum_i V[i][j] g_i x_i
 // ---------------------------------------------------------------------------
-// CTA item = (layer, path, 2048-input slice, 8 latent row blocks).  The slice's
-// quantised input (B fragments and per-row step) arrives by one bulk copy into
-// one of two shared buffers; warp w takes row blocks 2w, 2w+1 and accumulates
-// their eight products per K-block over the whole slice (one B fragment load
-// feeds both blocks), then folds the 2^q factors once and writes one fp32
+// CTA item = (layer, path, 2048-input slice, 8 latent row blocks; 6 with three
+// warps).  The slice's quantised input (B fragments and per-row step) arrives
+// by one bulk copy into one of two shared buffers; warp w takes row blocks 2w,
+// 2w+1 (w alone in the eight-warp CTAs of batches 9-16) and accumulates their
+// eight products per K-block over the whole slice (at batch 1-4 one B fragment
+// load feeds both blocks), then folds the 2^q factors once and writes one fp32
 // partial per latent row.
 //
 // Buffer hand-over without CTA barriers: the CTA's items are walked by every
@@ -375,6 +376,10 @@ struct VCfg {
   static constexpr int kRPW = NB == 1 ? 2 : 1;
 };
 
+// Row blocks of a latent-pass item per warp: an item is 8 row blocks (6 with
+// three warps), two per warp, or one per warp in the eight-warp CTAs.
+__host__ __device__ constexpr int latent_rows_per_warp(int W) { return W == 8 ? 1 : 2; }
+
 // Bytes of one quantised input slice buffer (shared memory and global stride).
 __host__ __device__ constexpr int xq_buf_bytes(int nb, int rb) { return (64 * nb + kVSlice * 2 * rb + 127) & ~127; }
 
@@ -395,6 +400,7 @@ __device__ __forceinline__ void x_issue(const DecodeArgs& a, int item, int li, u
 template <int NB, int W>
 struct VFeed {
   static constexpr int RPW = VCfg<NB>::kRPW;
+  static constexpr int kRW = latent_rows_per_warp(W);
   VPos pos;
   int item, grp, kc;
   int rb0, n_rb, n_kt_all, kt0, nkt;   // current item
@@ -402,14 +408,14 @@ struct VFeed {
 
   // the current item's chunk parameters (from pos; no divisions)
   __device__ __forceinline__ void set(int warp) {
-    static_assert(W == 3 || W == 4, "latent-pass CTA width");
+    static_assert(W == 3 || W == 4 || W == 8, "latent-pass CTA width");
     item = pos.item;
     const int k0 = pos.sl * kVSlice, d_in = pos.L->d_in;
     nkt = min(kVSliceTiles, (d_in - k0) / kVTileK);
     n_kt_all = d_in / kVTileK;
     kt0 = k0 / kVTileK;
     n_rb = (pos.L->s + 15) >> 4;
-    rb0 = pos.rc * (2 * W) + 2 * warp;
+    rb0 = pos.rc * (W * kRW) + kRW * warp;
     V = reinterpret_cast<const unsigned char*>(pos.L->p[pos.p].V);
     grp = 0;
     kc = 0;
@@ -430,7 +436,7 @@ struct VFeed {
   __device__ __forceinline__ void advance(const DecodeArgs& a, int warp, int end) {
     if (++kc * kChunkTiles >= nkt) {
       kc = 0;
-      if (++grp * RPW >= 2) {
+      if (++grp * RPW >= kRW) {
         pos.next(a);
         if (pos.item < end) set(warp);
         else item = pos.item;
@@ -459,6 +465,7 @@ template <int NB, int RB, int W>
 __global__ void __launch_bounds__(W * 32, NB == 1 ? 3 : 1) latent_pass_kernel(const DecodeArgs a) {
   constexpr int NC = 2 * RB;                      // B-fragment columns stored per K-block
   constexpr int RPW = VCfg<NB>::kRPW;
+  constexpr int kRW = latent_rows_per_warp(W);    // row blocks of an item per warp
   constexpr int kStageBytes = RPW * kChunkBytes;
   constexpr int kXBuf = xq_buf_bytes(NB, RB);
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -568,8 +575,8 @@ __global__ void __launch_bounds__(W * 32, NB == 1 ? 3 : 1) latent_pass_kernel(co
     const int ns4 = (L.n_slices + 3) & ~3;
     float* part = P.ws.partial + it.sl;
 #pragma unroll 1
-    for (int grp = 0; grp * RPW < 2; ++grp) {
-      const int rbA = it.rc * (2 * W) + 2 * warp + grp * RPW;
+    for (int grp = 0; grp * RPW < kRW; ++grp) {
+      const int rbA = it.rc * (W * kRW) + kRW * warp + grp * RPW;
       if (rbA >= n_rb) break;
       const int nvalid = min(RPW, n_rb - rbA);
       constexpr int R = RPW;
@@ -1513,8 +1520,11 @@ cudaError_t launch_latent_pass(const DecodeArgs& a, int, int num_sms, cudaStream
   switch ((a.batch + 3) / 4) {
     case 1: return launch_latent<1, 4, 4>(a, num_sms, st);
     case 2: return launch_latent<2, 8, 4>(a, num_sms, st);
-    case 3: return launch_latent<3, 12, 4>(a, num_sms, st);
-    case 4: return launch_latent<4, 16, 4>(a, num_sms, st);
+    // 9-16 rows: the two slice buffers fill most of shared memory, so one CTA
+    // per SM runs; eight warps of one row block each (instead of four of two)
+    // keep the same items with twice the resident warps
+    case 3: return launch_latent<3, 12, 8>(a, num_sms, st);
+    case 4: return launch_latent<4, 16, 8>(a, num_sms, st);
   }
   return cudaErrorInvalidValue;
 }
