@@ -205,7 +205,12 @@ lb_status littlebit_linear_forward_many_timed(const lb_layer* layers, int n, con
  * until littlebit_release().  Both copy streams start after the work already
  * enqueued on `stream`, and `stream` continues only after the last output
  * copy, so y_host is complete once `stream` has been synchronised (the host
- * buffers must stay untouched until then).  Not for CUDA-graph capture.
+ * buffers must stay untouched until then).  Not for CUDA-graph capture by the
+ * caller.  With page-locked buffers, the second of consecutive calls with the
+ * same layers, batch, dtype, chunk count and host buffers captures the call's
+ * copies and kernels as a CUDA graph, and later such calls replay it with one
+ * launch; a host-buffer call with other arguments on `stream`, or
+ * littlebit_release(), drops it.
  * Batch, dtype and layer rules, and errors, as littlebit_linear_forward_many;
  * LB_ERR_ARG also for NULL host pointers or n_chunks < 1.
  */

@@ -101,6 +101,37 @@ def test_host_stack_equals_device_stack_and_follows_new_inputs(lbm):
         _check(y, orc.factored_forward(x2, p), f"new inputs, layer {i}")
 
 
+@pytest.mark.parametrize("batch,dtype", [(1, torch.float16), (3, torch.float16), (128, torch.bfloat16)])
+def test_host_stack_repeated_calls_replay_with_new_inputs(lbm, batch, dtype):
+    """Consecutive identical calls (the second captures the pipeline as a CUDA
+    graph, the later ones replay it) read the host inputs as they are at each
+    call: three input sets at the same pinned addresses, called in turn, give
+    the oracle's outputs every time and bitwise the outputs of the first
+    (eager) calls on the same inputs; a call with another chunk count in
+    between drops the graph, and the calls after it are again exact."""
+    lb, _ = lbm
+    L, _, paths = _stack(lbm, SPECS, batch, seed=650 + batch)
+    sets = [[synth.activations(batch, a, seed=900 + 10 * k + i, index=i) for i, (a, _, _, _) in enumerate(SPECS)]
+            for k in range(3)]
+    xh = _host(sets[0], dtype, True)
+    yh = torch.empty(batch * sum(b for _, b, _, _ in SPECS), dtype=dtype).pin_memory()
+    hs = lb.HostStack(L, batch, dtype)
+    first = {}
+    for call, (k, chunks) in enumerate([(0, 3), (1, 3), (2, 3), (0, 3), (1, 3), (2, 2), (0, 3), (1, 3), (2, 3)]):
+        xh.copy_(_host(sets[k], dtype, False))
+        hs(xh, yh, n_chunks=chunks)
+        torch.cuda.synchronize()
+        got = yh.clone()
+        if chunks == 3:
+            if k in first:
+                assert torch.equal(got, first[k]), f"call {call}: input set {k} differs from its first call"
+            else:
+                first[k] = got
+        for i, (y, x, p) in enumerate(zip(_split(got, SPECS, batch), _split_in(xh, SPECS, batch), paths)):
+            _check(y, orc.factored_forward(x, p), f"call {call}, layer {i}")
+    assert lb.device_status() == 0
+
+
 def test_host_stack_prefill_bf16(lbm):
     lb, _ = lbm
     batch = 128
