@@ -890,7 +890,9 @@ lb_status littlebit_linear_forward_many_host(const lb_layer* layers, int n, cons
   e = ensure_pipe_objects(hp, chunks);
   if (e != cudaSuccess) return cuda_fail(e);
 
-  if (hp.key_changed_this_call || hp.g_x != x_host || hp.g_y != y_host) {
+  // the graph's copies need the same, still page-locked, host buffers
+  const bool locked = pinned(x_host) && pinned(y_host);
+  if (hp.key_changed_this_call || hp.g_x != x_host || hp.g_y != y_host || !locked) {
     drop_graph(hp);
     hp.g_x = x_host;
     hp.g_y = y_host;
@@ -904,7 +906,7 @@ lb_status littlebit_linear_forward_many_host(const lb_layer* layers, int n, cons
   // workspace and table, so the enqueue allocates and uploads nothing), with
   // page-locked buffers and a stream that is not already being captured
   ++hp.repeats;
-  if (hp.repeats >= 2 && !hp.no_graph && pinned(x_host) && pinned(y_host)) {
+  if (hp.repeats >= 2 && !hp.no_graph && locked) {
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     e = cudaStreamIsCapturing(st, &cs);
     if (e == cudaSuccess && cs == cudaStreamCaptureStatusNone) {
